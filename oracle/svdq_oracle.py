@@ -1,0 +1,345 @@
+"""Plain, slow, fp64 CPU oracle of the SVDQuant linear layer.
+
+TEST INFRASTRUCTURE: only tests/, __graft_entry__.smoke() and bench.py's CPU
+baseline may use it; the C-ABI library never does.  It shares no code with
+the CUDA path (no kernels, headers, tables or helpers); only the seeded input
+generator in `synth` serves both.
+
+What it computes follows "SVDQuant: How a Small High-Precision Branch Makes
+4-Bit Diffusion Practical" (technical review of arXiv:2411.05007v4):
+
+  * smoothing  X~ = X D^-1, W~ = D W, D = diag(lambda)        (section 3.1, eq. 3)
+  * lambda_i = max|X_:,i|^a / max|W_i,:|^(1-a)                 (section 3.1, eq. 4)
+  * rank-r SVD  L1 = U_r S_r, L2 = V_r^T, R = W~ - L1 L2       (section 5, eq. 10)
+  * symmetric INT4 group quantiser s = max|Z|/7,
+    Q(Z) = s round(Z/s)                                        (section 2.2, eq. 1)
+  * two-branch output  Y = (X~ L1) L2 + Q(X~) Q(R)            (section 4.2, eq. 7)
+  * LoRA in smoothed coordinates  [L1 | D A] [L2 ; B]          (section 7, eq. 13)
+  * MAC and storage ratios                                     (section 6, eqs. 11-12)
+
+Readings taken where the pages leave a step open (each is listed in the
+design notes of the repository):
+  * group size 64 along K on both operands, scales stored as fp32
+    s = fl32(max|z| / 7); codes round-half-even of the exact quotient z/s,
+    then clamped to [-8, 7] (the clamp only acts when s is subnormal);
+    an all-zero group, or one whose scale underflows to 0, has s = 0, codes 0;
+  * lambda_k = 1 when either statistic is zero;  inv_lambda = fl32(1/lambda);
+  * x~ = fl32(x * inv_lambda) (one fp32 rounding of the exact product);
+  * the 16-bit branch is bf16: L1, L2 stored as bf16, Z = bf16(bf16(x~) L1)
+    with exact (fp64) accumulation;
+  * R is taken against the stored bf16 factors, summed j = 0..r-1 in order;
+  * Y = bf16(sum_g s_x s_w P_g + Z L2 + b), optional exact-erf GELU before
+    the final rounding.
+Every function is pinned by the tests in tests/test_oracle_*.py; none is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+__all__ = [
+    "GROUP", "bf16_bits_to_f64", "round_bf16_bits", "round_bf16", "round_f32",
+    "smoothing_lambda", "quantize_groups", "pack_nibbles", "unpack_nibbles",
+    "calib_absmax", "pack_weights", "quantize_act", "group_partials",
+    "linear", "gelu", "layer_forward", "mac_ratio", "storage_ratio",
+    "two_branch_unquantized", "dequantize_groups", "residual_quantize",
+]
+
+GROUP = 64
+
+
+# --------------------------------------------------------------------------
+# number formats
+# --------------------------------------------------------------------------
+def bf16_bits_to_f64(b):
+    """bf16 bit patterns -> exactly equal float64 values."""
+    u = np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def round_bf16(x):
+    """Round float64 values to the nearest bf16 value, ties to even, in ONE
+    rounding (no detour through fp32).  Returns float64 values.
+
+    bf16 keeps 8 significant bits and fp32's exponent range; its subnormal
+    quantum is 2^-133.  Values whose rounded magnitude reaches 2^128
+    overflow to +-inf."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.array(x, copy=True)
+    fin = np.isfinite(x) & (x != 0)
+    xf = x[fin]
+    _, e = np.frexp(xf)                     # xf = m 2^e, 0.5 <= |m| < 1
+    qexp = np.maximum(e - 8, -133)          # quantum exponent
+    y = np.ldexp(np.rint(np.ldexp(xf, -qexp)), qexp)
+    y[np.abs(y) >= 2.0 ** 128] = np.copysign(np.inf, y[np.abs(y) >= 2.0 ** 128])
+    out[fin] = y
+    return out
+
+
+def round_bf16_bits(x):
+    """Round float64 values to bf16 (one rounding) and return the bits."""
+    y = round_bf16(x).astype(np.float32)    # exact: y is a bf16 value
+    return (np.ascontiguousarray(y).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def round_f32(x):
+    """Round float64 values to fp32 (IEEE round-to-nearest-even), as float64."""
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# eq. 4: smoothing factors
+# --------------------------------------------------------------------------
+def calib_absmax(X):
+    """Calibration statistic max_i |X_ik| per input channel k (eq. 4's
+    max|X_:,i|), over the rows of X (float64 values)."""
+    return np.max(np.abs(np.asarray(X, dtype=np.float64)), axis=0)
+
+
+def smoothing_lambda(act_absmax, w_absmax, alpha=0.5):
+    """lambda_k = a_k^alpha / w_k^(1-alpha) (eq. 4); lambda_k = 1 where either
+    statistic is zero (the pages name no safeguard; this is the reading).
+    alpha = 0.5 is evaluated as sqrt(a)/sqrt(w) (correctly rounded)."""
+    a = np.asarray(act_absmax, dtype=np.float64)
+    w = np.asarray(w_absmax, dtype=np.float64)
+    lam = np.ones_like(a)
+    ok = (a > 0) & (w > 0)
+    if alpha == 0.5:
+        lam[ok] = np.sqrt(a[ok]) / np.sqrt(w[ok])
+    else:
+        lam[ok] = np.power(a[ok], alpha) / np.power(w[ok], 1.0 - alpha)
+    return lam
+
+
+# --------------------------------------------------------------------------
+# eq. 1: symmetric INT4 group quantiser
+# --------------------------------------------------------------------------
+def quantize_groups(z):
+    """Quantise groups of fp32 values (given as float64, last axis = one
+    group of 64) with eq. 1: s = fl32(max|z| / 7), q = round(z / s).
+
+    The rounding is round-half-even of the EXACT real quotient z/s, decided
+    by exact fp64 comparisons of z with (q +- 1/2) s: q*s has at most 28
+    significant bits and z - q*s at most 29, so every quantity below is
+    exact.  fl32(m/7) is taken as the fp64 quotient rounded to fp32, which
+    equals the correctly rounded fp32 quotient (53 >= 2*24 + 2).
+    Codes are clamped to [-8, 7]; with a normal s they already lie in
+    [-7, 7].  s = 0 (all-zero group, or a scale that underflows) gives
+    codes 0.  Returns (codes int64 like z, scales float64 [..., G])."""
+    z = np.asarray(z, dtype=np.float64)
+    m = np.max(np.abs(z), axis=-1)
+    s = round_f32(m / 7.0)
+    codes = np.zeros(z.shape, dtype=np.int64)
+    nz = s > 0
+    if np.any(nz):
+        zz = z[nz]
+        ss = np.broadcast_to(s[nz][..., None], zz.shape)
+        q = np.rint(zz / ss)
+        for _ in range(3):                  # converges in one pass
+            d = zz - q * ss                 # exact
+            two_d = 2.0 * d
+            q = np.where(two_d > ss, q + 1, np.where(two_d < -ss, q - 1, q))
+        d = zz - q * ss
+        tie = (2.0 * np.abs(d) == ss) & (np.mod(q, 2) != 0)
+        q = np.where(tie, q + np.sign(d), q)
+        codes[nz] = np.clip(q, -8, 7).astype(np.int64)
+    return codes, s
+
+
+def dequantize_groups(codes, scales):
+    """codes [rows, K], scales [G, rows] -> float64 [rows, K] = q * s."""
+    codes = np.asarray(codes)
+    rows, K = codes.shape
+    G = K // GROUP
+    s = np.asarray(scales, dtype=np.float64).T.reshape(rows, G, 1)
+    return (codes.reshape(rows, G, GROUP) * s).reshape(rows, K)
+
+
+def pack_nibbles(codes):
+    """Two's-complement nibbles, two per byte: byte b of a row holds
+    k = 2b in the low nibble and k = 2b+1 in the high nibble (the review's
+    companion explainer describes packing two 4-bit values per byte)."""
+    c = np.asarray(codes, dtype=np.int64) & 0xF
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_nibbles(packed):
+    p = np.asarray(packed, dtype=np.int64)
+    lo = p & 0xF
+    hi = (p >> 4) & 0xF
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), dtype=np.int64)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return np.where(out >= 8, out - 16, out)
+
+
+def _quantize_rows(v):
+    """v float64 [rows, K] of fp32 values -> codes [rows, K], scales [G, rows]."""
+    rows, K = v.shape
+    if K % GROUP:
+        raise ValueError("K must be a multiple of the group size 64")
+    codes, s = quantize_groups(v.reshape(rows, K // GROUP, GROUP))
+    return codes.reshape(rows, K), np.ascontiguousarray(s.T)
+
+
+# --------------------------------------------------------------------------
+# offline pack: eqs. 3, 4, 10, 13 and eq. 1 on the residual
+# --------------------------------------------------------------------------
+def residual_quantize(Wt, L1b, L2b):
+    """R = W~ - L1b L2b (fp64; the product of two bf16 values is exact and the
+    rank-one terms are subtracted j = 0..r-1 in order, each step rounded),
+    then eq. 1 per group of 64 input channels of each output column.
+    Wt is the smoothed weight [K, N].  Returns (R, codes [N, K], s_w [G, N])."""
+    R = np.array(Wt, dtype=np.float64, copy=True)
+    for j in range(L1b.shape[1]):
+        R -= np.outer(L1b[:, j], L2b[j, :])
+    codes, s_w = _quantize_rows(round_f32(R.T))
+    return R, codes, s_w
+
+
+def pack_weights(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None,
+                 lora_A_bits=None, lora_B_bits=None, lora_scale=1.0,
+                 smooth=True, svd=None):
+    """Offline transform of one linear layer (review Algorithm 1, steps 2-5
+    and 9, with alpha fixed and no refinement / GPTQ).
+
+    W_bits: bf16 bits [N, K] (nn.Linear layout; the math weight W is its
+    transpose, K x N, rows = input channels).  act_absmax: [K] calibration
+    statistic.  smooth=False uses lambda = 1 (plain W4A4, for ablations).
+    `svd` may pass a precomputed (U, S, Vt) of W~ to skip the SVD."""
+    Wl = bf16_bits_to_f64(W_bits)                      # [N, K]
+    N, K = Wl.shape
+    W = Wl.T                                           # [K, N]
+    w_absmax = np.max(np.abs(W), axis=1)
+    if smooth:
+        lam = smoothing_lambda(act_absmax, w_absmax, alpha)
+    else:
+        lam = np.ones(K)
+    inv_lam = round_f32(1.0 / lam)
+    Wt = lam[:, None] * W                              # eq. 3, W~ = D W
+    if svd is None:
+        U, S, Vt = np.linalg.svd(Wt, full_matrices=False)
+    else:
+        U, S, Vt = svd
+    r = int(rank)
+    L1 = U[:, :r] * S[None, :r]                        # eq. 10
+    L2 = Vt[:r, :]
+    L1b = round_bf16(L1)
+    L2b = round_bf16(L2)
+    R, codes, s_w = residual_quantize(Wt, L1b, L2b)
+    if lora_A_bits is not None and lora_A_bits.shape[1] > 0:
+        A = bf16_bits_to_f64(lora_A_bits)              # [K, k]
+        B = bf16_bits_to_f64(lora_B_bits)              # [k, N]
+        DA = (lam[:, None] * A) * float(np.float32(lora_scale))
+        L1b = np.hstack([L1b, round_bf16(DA)])         # eq. 13: [L1 | D A]
+        L2b = np.vstack([L2b, B])                      #          [L2 ; B]
+    bias = (np.zeros(N) if bias_bits is None else bf16_bits_to_f64(bias_bits))
+    return dict(lam=lam, inv_lambda=inv_lam, Wt=Wt, U=U, S=S, Vt=Vt,
+                L1=L1, L2=L2, L1b=L1b, L2b=L2b, R=R, wcodes=codes,
+                wq=pack_nibbles(codes), s_w=s_w, sigma=S[:r + 1].copy(),
+                bias=bias, rank=L1b.shape[1], K=K, N=N)
+
+
+# --------------------------------------------------------------------------
+# runtime: activation quantise + down-projection, then the two-branch product
+# --------------------------------------------------------------------------
+def quantize_act(X_bits, inv_lambda, L1b):
+    """Review Algorithm 2 steps 1-3: x~ = fl32(x * inv_lambda) (eq. 3),
+    eq. 1 per (token, group of 64), and the 16-bit down-projection
+    Z = bf16(bf16(x~) L1) with exact accumulation.
+    Returns (codes [M, K], s_x [G, M], Z [M, r] float64 bf16 values, xhat)."""
+    X = bf16_bits_to_f64(X_bits)
+    xhat = round_f32(X * np.asarray(inv_lambda, dtype=np.float64)[None, :])
+    codes, s_x = _quantize_rows(xhat)
+    r = L1b.shape[1]
+    if r:
+        Z = round_bf16(round_bf16(xhat) @ L1b)
+    else:
+        Z = np.zeros((X.shape[0], 0))
+    return codes, s_x, Z, xhat
+
+
+def group_partials(xcodes, wcodes, rows=None, cols=None):
+    """P_g[i, n] = sum_{k in group g} q_x[i, k] q_w[n, k] for every group g.
+    Computed as an fp64 matmul of integer-valued arrays: every product and
+    partial sum is an integer below 2^13, so the result is exact.
+    Returns int64 [G, len(rows), len(cols)]."""
+    xc = np.asarray(xcodes)
+    wc = np.asarray(wcodes)
+    if rows is not None:
+        xc = xc[rows]
+    if cols is not None:
+        wc = wc[cols]
+    m, K = xc.shape
+    n = wc.shape[0]
+    G = K // GROUP
+    xg = xc.reshape(m, G, GROUP).astype(np.float64)
+    wg = wc.reshape(n, G, GROUP).astype(np.float64)
+    P = np.empty((G, m, n), dtype=np.int64)
+    for g in range(G):
+        P[g] = np.rint(xg[:, g, :] @ wg[:, g, :].T).astype(np.int64)
+    return P
+
+
+def gelu(y):
+    """GELU with the exact error function: 0.5 y (1 + erf(y / sqrt 2))."""
+    y = np.asarray(y, dtype=np.float64)
+    return 0.5 * y * (1.0 + _erf(y / math.sqrt(2.0)))
+
+
+def linear(xcodes, s_x, Z, wcodes, s_w, L2b, bias, apply_gelu=False,
+           rows=None, cols=None):
+    """Review Algorithm 2 steps 4-8 / eq. 7:
+    Y = sum_g s_x[g, i] s_w[g, n] P_g[i, n] + Z L2 + b (fp64), optional GELU,
+    then one bf16 rounding.  Returns (Y float64, Y_bf16 float64 values)."""
+    xc = np.asarray(xcodes)
+    M = xc.shape[0]
+    N = np.asarray(wcodes).shape[0]
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    cols = np.arange(N) if cols is None else np.asarray(cols)
+    P = group_partials(xc, wcodes, rows, cols)
+    sx = np.asarray(s_x, dtype=np.float64)[:, rows]
+    sw = np.asarray(s_w, dtype=np.float64)[:, cols]
+    Y = np.zeros((len(rows), len(cols)))
+    for g in range(P.shape[0]):
+        Y += (sx[g][:, None] * sw[g][None, :]) * P[g]
+    if np.asarray(L2b).shape[0]:
+        Y += np.asarray(Z)[rows] @ np.asarray(L2b)[:, cols]
+    Y += np.asarray(bias, dtype=np.float64)[cols][None, :]
+    if apply_gelu:
+        Y = gelu(Y)
+    return Y, round_bf16(Y)
+
+
+def layer_forward(X_bits, packed, apply_gelu=False, rows=None, cols=None):
+    """quantize_act then linear for one packed layer (oracle end to end)."""
+    xc, s_x, Z, _ = quantize_act(X_bits, packed["inv_lambda"], packed["L1b"])
+    Y, Yb = linear(xc, s_x, Z, packed["wcodes"], packed["s_w"], packed["L2b"],
+                   packed["bias"], apply_gelu, rows, cols)
+    return dict(xcodes=xc, s_x=s_x, Z=Z, Y=Y, Ybf16=Yb)
+
+
+def two_branch_unquantized(X, lam, L1, L2, R, bias):
+    """Eq. 7 with quantisation switched off, all in fp64:
+    (X~ L1) L2 + X~ R + b with X~ = X D^-1 (exact-lambda smoothing)."""
+    Xt = np.asarray(X, dtype=np.float64) / np.asarray(lam)[None, :]
+    out = Xt @ R + np.asarray(bias)[None, :]
+    if np.asarray(L1).shape[1]:
+        out += (Xt @ L1) @ L2
+    return out
+
+
+# --------------------------------------------------------------------------
+# eqs. 11-12: cost accounting of the protected branch
+# --------------------------------------------------------------------------
+def mac_ratio(m, n, r):
+    """Low-rank MACs over dense MACs: (b m r + b r n) / (b m n) (eq. 11)."""
+    return (m * r + r * n) / (m * n)
+
+
+def storage_ratio(m, n, r):
+    """(m n / 2 + 2 r (m + n)) / (2 m n) bytes vs bf16 (eq. 12)."""
+    return (m * n / 2 + 2 * r * (m + n)) / (2 * m * n)
