@@ -1,0 +1,196 @@
+/*
+ * svdq.h -- C ABI of the SVDQuant W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (SVDQuant technical review of arXiv:2411.05007v4, section 4.2,
+ * eq. 7; section 6.1, Algorithm 2):
+ *
+ *     Y = Q(X~) Q(R) + (X~ L1) L2 + b,   X~ = X diag(lambda)^-1,
+ *     R = diag(lambda) W - L1 L2                       (section 5, eq. 10)
+ *
+ * Math shapes: X is M x K (tokens x input channels), W is K x N.  Arrays
+ * cross this ABI in row-major order; the weight is passed in nn.Linear
+ * layout [N][K] (its transpose).
+ *
+ * Number formats (section 2.2, eq. 1; section 8 for group 64):
+ *   - INT4 codes: symmetric, per group of 64 consecutive K, scale
+ *     s = fl32(max|z| / 7), code = clamp(round_half_even(z / s), -8, 7)
+ *     of the exact quotient; s = 0 and codes 0 for an all-zero group.
+ *   - Packed codes: two's-complement nibbles, two per byte; byte b of a row
+ *     holds k = 2b in the low nibble and k = 2b+1 in the high nibble.
+ *   - Scales: fp32, group-major: s_x[g][m] (K/64 x M), s_w[g][n] (K/64 x N).
+ *   - 16-bit branch: bf16 (uint16_t bit patterns) with fp32 accumulation.
+ *
+ * Conventions for every call:
+ *   - Calls return svdq_status; nothing is thrown across the ABI.
+ *   - Argument checks (null, shape, alignment) are synchronous and happen
+ *     before any launch; a failed check launches nothing.
+ *   - Device pointers must be 16-byte aligned, leading dimensions must keep
+ *     every row 16-byte aligned, else SVDQ_ERR_ALIGNMENT.
+ *   - K must be a multiple of 64, else SVDQ_ERR_SHAPE.  Any M >= 0, N >= 1.
+ *   - Hot-path calls are asynchronous on `stream`; the caller owns every
+ *     device buffer it passes.  A launch failure returns SVDQ_ERR_CUDA.
+ *   - A device-side wait that exceeds its bound sets a sticky error word in
+ *     the weights handle instead of hanging; read it with
+ *     svdq_get_device_error.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;   /* same type as CUDA's own */
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,     /* null pointer, bad enum, bad rank          */
+  SVDQ_ERR_SHAPE = 2,           /* K % 64 != 0, negative sizes, ld too small */
+  SVDQ_ERR_ALIGNMENT = 3,       /* device pointer or row not 16-byte aligned */
+  SVDQ_ERR_UNSUPPORTED = 4,     /* no sm_100 device, group != 64, rank > 128 */
+  SVDQ_ERR_NUMERIC = 5,         /* non-finite weights or statistics          */
+  SVDQ_ERR_CUDA = 6,            /* a CUDA runtime call or launch failed      */
+  SVDQ_ERR_DEVICE_TIMEOUT = 7,  /* a bounded device wait expired             */
+  SVDQ_ERR_OOM = 8,             /* device or host allocation failed          */
+  SVDQ_ERR_IO = 9               /* file could not be read or written         */
+} svdq_status;
+
+enum { SVDQ_EPI_NONE = 0, SVDQ_EPI_GELU = 1 };
+
+#define SVDQ_GROUP 64
+#define SVDQ_MAX_RANK 128
+
+/* Opaque packed layer, immutable after svdq_pack_weights / svdq_weights_load.
+ * Holds device copies of every operand plus host copies for export. */
+typedef struct svdq_weights svdq_weights;
+
+const char* svdq_status_string(int status);
+int svdq_version(void);
+
+/*
+ * Calibration statistic of eq. 4 (section 3.1): absmax[k] = max(absmax[k],
+ * max_i |X[i][k]|) over the M rows of a host bf16 matrix X [M][ldx].
+ * Call it once per calibration batch on an array that starts at zero.
+ * Host only; K need not be a multiple of 64 here.
+ */
+svdq_status svdq_calib_absmax(int M, int K, const uint16_t* X, int ldx,
+                              float* absmax);
+
+/*
+ * Offline transform of one layer (review Algorithm 1, steps 2-5 and 9 with a
+ * fixed alpha and no refinement).  Host inputs, device result.
+ *   lambda_k = act_absmax[k]^alpha / max_n|W[n][k]|^(1-alpha)   (eq. 4);
+ *              lambda_k = 1 if either statistic is 0;
+ *   W~ = diag(lambda) W (fp64)                                   (eq. 3);
+ *   top-`rank` SVD of W~ in fp64: L1 = U S, L2 = V^T             (eq. 10),
+ *   stored as bf16;  R = W~ - L1 L2 against the stored factors, quantised
+ *   per group of 64 input channels of each output column       (eq. 1);
+ *   optional LoRA (eq. 13): L1 <- [L1 | bf16(diag(lambda) A lora_scale)],
+ *   L2 <- [L2 ; B]; R is not recomputed.
+ * Arguments:
+ *   K, N        input / output channels, K % 64 == 0;
+ *   rank        SVD rank, 0 <= rank <= min(K, N), rank + lora_rank <= 128;
+ *   group       must be 64;
+ *   W           host bf16 [N][K];  act_absmax  host fp32 [K], finite, >= 0;
+ *   alpha       migration strength in (0, 1) (0.5 in every workload);
+ *   bias        host bf16 [N] or NULL (zero bias);
+ *   lora_rank   0 or the adapter rank; lora_A host bf16 [K][lora_rank],
+ *               lora_B host bf16 [lora_rank][N] (both required if > 0);
+ *   stream      stream for the upload (the call synchronises it);
+ *   out         receives the handle; *out is NULL on error.
+ * The current CUDA device at the time of the call owns the handle.
+ */
+svdq_status svdq_pack_weights(int K, int N, int rank, int group,
+                              const uint16_t* W, const float* act_absmax,
+                              double alpha, const uint16_t* bias,
+                              int lora_rank, const uint16_t* lora_A,
+                              const uint16_t* lora_B, float lora_scale,
+                              cudaStream_t stream, svdq_weights** out);
+
+/*
+ * Same transform as svdq_pack_weights, without touching a GPU: the handle
+ * holds host copies only (export / save work; the hot-path calls reject it
+ * with SVDQ_ERR_INVALID_ARG).  Lets a machine without a GPU pack a layer and
+ * save it for svdq_weights_load elsewhere.
+ */
+svdq_status svdq_pack_weights_host(int K, int N, int rank, int group,
+                                   const uint16_t* W, const float* act_absmax,
+                                   double alpha, const uint16_t* bias,
+                                   int lora_rank, const uint16_t* lora_A,
+                                   const uint16_t* lora_B, float lora_scale,
+                                   svdq_weights** out);
+
+/* Sizes of a handle; any output pointer may be NULL.  `rank` is the total
+ * branch rank (svd_rank + lora_rank). */
+svdq_status svdq_weights_info(const svdq_weights* w, int* K, int* N, int* rank,
+                              int* svd_rank, int* lora_rank);
+
+/*
+ * Host copies of the packed operands (for checking against an oracle).  Any
+ * output may be NULL.  inv_lambda fp32 [K] (= fl32(1/lambda)); wq uint8
+ * [N][K/2] (weight codes, layout as above); s_w fp32 [K/64][N];
+ * L1 bf16 [K][rank]; L2 bf16 [rank][N]; bias bf16 [N]; sigma fp64
+ * [svd_rank + 1] (leading singular values of W~).
+ */
+svdq_status svdq_weights_export(const svdq_weights* w, float* inv_lambda,
+                                uint8_t* wq, float* s_w, uint16_t* L1,
+                                uint16_t* L2, uint16_t* bias, double* sigma);
+
+/* Store / restore a packed layer (Algorithm 1 step 9): versioned header and
+ * raw host arrays.  load uploads to the current device on `stream`. */
+svdq_status svdq_weights_save(const svdq_weights* w, const char* path);
+svdq_status svdq_weights_load(const char* path, cudaStream_t stream,
+                              svdq_weights** out);
+void svdq_weights_free(svdq_weights* w);
+
+/*
+ * Fused activation pass (review section 6.1, Algorithm 2 steps 1-3): one
+ * kernel reads X once and writes
+ *   xq  [M][K/2]   packed INT4 codes of x~ = fl32(x * inv_lambda_k);
+ *   s_x [K/64][M]  fp32 scales, fl32(max|x~| / 7) per token and group;
+ *   Z   [M][rank]  bf16 down-projection bf16(bf16(x~) L1), fp32 accumulation
+ *                  (ignored, may be NULL, when rank == 0).
+ * X is device bf16 [M][ldx], ldx >= K.  All device pointers, 16-byte
+ * aligned.  M == 0 is a no-op.
+ */
+svdq_status svdq_quantize_act(const svdq_weights* w, int M, const uint16_t* X,
+                              int ldx, uint8_t* xq, float* s_x, uint16_t* Z,
+                              cudaStream_t stream);
+
+/*
+ * Fused W4A4 product (Algorithm 2 steps 4-8): one kernel computes
+ *   P_g = sum_{k in g} q_x q_w       (int32, per group, on the tensor cores)
+ *   acc = sum_g s_x[g][m] s_w[g][n] P_g            (fp32)
+ *   Y   = bf16(epi(acc + Z L2 + b))                 written once
+ * with epi = identity or GELU (exact-erf form in fp32).  Y is device bf16
+ * [M][ldy], ldy >= N.  xq, s_x, Z as produced by svdq_quantize_act.
+ */
+svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq,
+                        const float* s_x, const uint16_t* Z, uint16_t* Y,
+                        int ldy, int epilogue, cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the handle's sticky device
+ * error word: SVDQ_OK, or SVDQ_ERR_DEVICE_TIMEOUT if a bounded wait in a
+ * kernel of this handle expired since the last read.
+ */
+svdq_status svdq_get_device_error(const svdq_weights* w, cudaStream_t stream);
+
+/*
+ * Test hook, not on the measured path: runs svdq_linear's tensor-core main
+ * loop over the output block [row0, row0+nrows) x [col0, col0+ncols) and
+ * writes its int32 group partials instead of rescaling them:
+ *   P[g][i][j] = sum_{k in group g} q_x[row0+i][k] q_w[col0+j][k]
+ * P is device int32 [K/64][nrows][ncols].
+ */
+svdq_status svdq_debug_partials(const svdq_weights* w, int M, const uint8_t* xq,
+                                int row0, int nrows, int col0, int ncols,
+                                int32_t* P, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SVDQ_H_ */

@@ -46,6 +46,7 @@ __all__ = [
     "calib_absmax", "pack_weights", "quantize_act", "group_partials",
     "linear", "gelu", "layer_forward", "mac_ratio", "storage_ratio",
     "two_branch_unquantized", "dequantize_groups", "residual_quantize",
+    "leading_svd",
 ]
 
 GROUP = 64
@@ -200,6 +201,16 @@ def residual_quantize(Wt, L1b, L2b):
     return R, codes, s_w
 
 
+def leading_svd(Wt, k):
+    """Leading k singular triplets of W~ (fp64) with ARPACK (scipy's svds),
+    returned like np.linalg.svd's truncated output (descending order)."""
+    from scipy.sparse.linalg import svds
+    k = min(k, min(Wt.shape) - 1)
+    U, S, Vt = svds(Wt, k=k, tol=0, which="LM", random_state=0)
+    order = np.argsort(S)[::-1]
+    return U[:, order], S[order], Vt[order]
+
+
 def pack_weights(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None,
                  lora_A_bits=None, lora_B_bits=None, lora_scale=1.0,
                  smooth=True, svd=None):
@@ -209,7 +220,9 @@ def pack_weights(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None,
     W_bits: bf16 bits [N, K] (nn.Linear layout; the math weight W is its
     transpose, K x N, rows = input channels).  act_absmax: [K] calibration
     statistic.  smooth=False uses lambda = 1 (plain W4A4, for ablations).
-    `svd` may pass a precomputed (U, S, Vt) of W~ to skip the SVD."""
+    svd=None runs the full LAPACK SVD (np.linalg.svd); svd="leading" takes
+    only the leading rank+1 triplets from ARPACK (same definition, for large
+    layers)."""
     Wl = bf16_bits_to_f64(W_bits)                      # [N, K]
     N, K = Wl.shape
     W = Wl.T                                           # [K, N]
@@ -222,8 +235,10 @@ def pack_weights(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None,
     Wt = lam[:, None] * W                              # eq. 3, W~ = D W
     if svd is None:
         U, S, Vt = np.linalg.svd(Wt, full_matrices=False)
+    elif svd == "leading":
+        U, S, Vt = leading_svd(Wt, int(rank) + 1)
     else:
-        U, S, Vt = svd
+        raise ValueError(svd)
     r = int(rank)
     L1 = U[:, :r] * S[None, :r]                        # eq. 10
     L2 = Vt[:r, :]

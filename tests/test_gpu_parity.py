@@ -1,0 +1,186 @@
+"""GPU parity: the C-ABI library (pack, svdq_quantize_act, svdq_linear,
+svdq_debug_partials) against the fp64 oracle on the same seeded inputs.
+
+Bar (SVDQuant layer contract): INT4 codes, fp32 scales and int32 group
+partials bit-exact; weight codes and scales bit-exact; Z within one bf16 ulp
+plus the fp32 accumulation bound; Y within 2e-3 relative Frobenius error of
+the oracle's bf16 Y.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import w4a4_quantized_gemm_smooth_b200 as S
+from helpers import Y_REL_FRO, check_z, column_signs, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+def to_dev(bits, ld=None):
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    if ld is not None and ld != bits.shape[1]:
+        full = torch.zeros((bits.shape[0], ld), dtype=torch.bfloat16)
+        full[:, :bits.shape[1]] = t
+        return full.cuda()[:, :bits.shape[1]]
+    return t.cuda()
+
+
+def to_bits(t):
+    return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "gpu tests need a CUDA device"
+    S.lib()
+
+
+def check_layer(spec, epilogue=S.EPI_NONE, rows_sample=None, partial_blocks=None,
+                svd=None, X_bits=None, ldy=None):
+    L = synth.make_layer(spec)
+    Xb = L.X if X_bits is None else X_bits
+    a = S.svdq_calib_absmax(Xb)
+    w = S.svdq_pack_weights(L.W, a, spec.rank, bias_bits=L.b, lora_A_bits=L.A,
+                            lora_B_bits=L.B)
+    p = oracle.pack_weights(L.W, a.astype(np.float64), spec.rank, bias_bits=L.b,
+                            lora_A_bits=L.A, lora_B_bits=L.B, svd=svd)
+    e = w.export()
+    # weights
+    assert np.array_equal(e["inv_lambda"].astype(np.float64), p["inv_lambda"])
+    assert np.array_equal(e["wq"], p["wq"])
+    assert np.array_equal(e["s_w"].astype(np.float64), p["s_w"])
+    signs = column_signs(e["L1"], p["L1b"]) if w.rank else np.zeros(0)
+    # activation pass
+    M, K, N = Xb.shape[0], spec.K, spec.N
+    X = to_dev(Xb)
+    lin = S.SVDQLinear(w, epilogue)
+    xq, s_x, Z, Y = lin.buffers(M)
+    if ldy is not None:
+        Yfull = torch.empty((M, ldy), dtype=torch.bfloat16, device="cuda")
+        Y = Yfull[:, :N]
+    lin.forward(X, out=Y)
+    torch.cuda.synchronize()
+    S.svdq_get_device_error(w)
+    xc, sxo, Zo, xhat = oracle.quantize_act(Xb, p["inv_lambda"], p["L1b"])
+    assert np.array_equal(xq.cpu().numpy(), oracle.pack_nibbles(xc)), "activation codes"
+    assert np.array_equal(s_x.cpu().numpy().astype(np.float64), sxo), "activation scales"
+    if w.rank:
+        check_z(to_bits(Z), Zo, xhat, p["L1b"], signs)
+    # output
+    rows = np.arange(M) if rows_sample is None else rows_sample
+    _, Yo = oracle.linear(xc, sxo, Zo, p["wcodes"], p["s_w"], p["L2b"], p["bias"],
+                          apply_gelu=(epilogue == S.EPI_GELU), rows=rows)
+    Yg = oracle.bf16_bits_to_f64(to_bits(Y))[rows]
+    err = rel_fro(Yg, Yo)
+    assert err <= Y_REL_FRO, err
+    # int32 partials from the tensor-core path
+    blocks = partial_blocks or [(0, min(M, 256), 0, min(N, 256))]
+    for (r0, nr, c0, nc) in blocks:
+        P = torch.empty((K // 64, nr, nc), dtype=torch.int32, device="cuda")
+        S.svdq_debug_partials(w, M, xq, r0, nr, c0, nc, P)
+        torch.cuda.synchronize()
+        Po = oracle.group_partials(xc, p["wcodes"], np.arange(r0, r0 + nr), np.arange(c0, c0 + nc))
+        assert np.array_equal(P.cpu().numpy().astype(np.int64), Po), f"partials {r0},{c0}"
+    S.svdq_get_device_error(w)
+    w.free()
+    return err
+
+
+def test_tiny_layer():
+    spec = synth.WORKLOADS["tiny"]
+    err = check_layer(spec, partial_blocks=[(0, 256, 0, 512)])
+    assert err < 1e-3
+
+
+def test_tiny_layer_gelu_epilogue():
+    check_layer(synth.WORKLOADS["tiny"], epilogue=S.EPI_GELU)
+
+
+@pytest.mark.parametrize("M,K,N,r", [
+    (200, 512, 384, 16),     # ragged M
+    (130, 320, 136, 24),     # ragged M, K not a multiple of 256, N not of 128, r not of 16
+    (1, 64, 128, 8),         # one token, one group
+    (333, 1152, 256, 64),    # PixArt width, rank 64
+    (128, 256, 128, 0),      # no low-rank branch
+])
+def test_ragged_and_small_shapes(M, K, N, r):
+    spec = synth.layer_spec(f"e{M}_{K}_{N}_{r}", M, K, N, r, 100 + M + K + N + r, tiny=True)
+    check_layer(spec, partial_blocks=[(0, M, 0, N), (M - 1, 1, N - 1, 1)])
+
+
+def test_ragged_output_stride():
+    spec = synth.layer_spec("ldy", 96, 256, 196, 16, 7, tiny=True)
+    check_layer(spec, ldy=200)
+
+
+def test_lora_branch():
+    spec = synth.layer_spec("lora", 256, 512, 384, 16, 21, lora_rank=16)
+    check_layer(spec)
+
+
+def test_zero_rows_and_groups():
+    spec = synth.layer_spec("zeros", 160, 256, 128, 8, 9, tiny=True)
+    L = synth.make_layer(spec)
+    X = L.X.copy()
+    X[5] = 0                    # an all-zero token
+    X[7, 64:128] = 0            # one all-zero group
+    X[9, :64] = 0x8000          # negative zeros
+    check_layer(spec, X_bits=X)
+
+
+def test_argument_errors_launch_nothing():
+    spec = synth.layer_spec("args", 64, 128, 64, 8, 3, tiny=True)
+    L = synth.make_layer(spec)
+    w = S.svdq_pack_weights(L.W, S.svdq_calib_absmax(L.X), 8, bias_bits=L.b)
+    lib = S.lib()
+    X = to_dev(L.X)
+    xq = torch.empty((64, 64), dtype=torch.uint8, device="cuda")
+    s_x = torch.empty((2, 64), dtype=torch.float32, device="cuda")
+    Z = torch.empty((64, 8), dtype=torch.bfloat16, device="cuda")
+    Y = torch.empty((64, 64), dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    import ctypes
+    vp = ctypes.c_void_p
+    # misaligned X (offset by one element)
+    assert lib.svdq_quantize_act(w.handle, 63, vp(X.data_ptr() + 2), 128, vp(xq.data_ptr()),
+                                 vp(s_x.data_ptr()), vp(Z.data_ptr()), vp(st)) == 3
+    # ldx too small
+    assert lib.svdq_quantize_act(w.handle, 64, vp(X.data_ptr()), 64, vp(xq.data_ptr()),
+                                 vp(s_x.data_ptr()), vp(Z.data_ptr()), vp(st)) == 2
+    # missing Z with rank > 0
+    assert lib.svdq_linear(w.handle, 64, vp(xq.data_ptr()), vp(s_x.data_ptr()), None,
+                           vp(Y.data_ptr()), 64, 0, vp(st)) == 1
+    # bad epilogue
+    assert lib.svdq_linear(w.handle, 64, vp(xq.data_ptr()), vp(s_x.data_ptr()),
+                           vp(Z.data_ptr()), vp(Y.data_ptr()), 64, 7, vp(st)) == 1
+    # M == 0 is a no-op
+    assert lib.svdq_linear(w.handle, 0, None, None, None, None, 64, 0, vp(st)) == 0
+    # partial block outside the output
+    assert lib.svdq_debug_partials(w.handle, 64, vp(xq.data_ptr()), 60, 8, 0, 4,
+                                   vp(Y.data_ptr()), vp(st)) == 2
+    torch.cuda.synchronize()
+    S.svdq_get_device_error(w)
+    w.free()
+
+
+def test_save_load_roundtrip(tmp_path):
+    spec = synth.layer_spec("sl", 128, 256, 192, 16, 31, lora_rank=4)
+    L = synth.make_layer(spec)
+    w = S.svdq_pack_weights(L.W, S.svdq_calib_absmax(L.X), 16, bias_bits=L.b,
+                            lora_A_bits=L.A, lora_B_bits=L.B)
+    path = str(tmp_path / "l.svdq")
+    w.save(path)
+    w2 = S.svdq_weights_load(path)
+    e1, e2 = w.export(), w2.export()
+    for k in e1:
+        assert np.array_equal(e1[k], e2[k]), k
+    X = to_dev(L.X)
+    Y1 = S.SVDQLinear(w)(X).clone()
+    Y2 = S.SVDQLinear(w2)(X).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+    w.free()
+    w2.free()

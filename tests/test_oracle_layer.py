@@ -212,3 +212,12 @@ def test_lora_identity_eq13():
     y = Xt @ (p["Wt"] - p["L1"] @ p["L2"]) + (Xt @ np.hstack([p["L1"], lam[:, None] * A])) @ \
         np.vstack([p["L2"], B]) + b
     assert _rel(y, X @ (W + A @ B) + b) < 1e-12
+
+
+def test_leading_svd_matches_full_svd(tiny):
+    """The ARPACK path used for large layers agrees with LAPACK's full SVD."""
+    L, X, a, p = tiny
+    q = oracle.pack_weights(L.W, a, 16, bias_bits=L.b, svd="leading")
+    assert np.max(np.abs(q["sigma"] - p["sigma"]) / p["sigma"]) < 1e-12
+    assert np.array_equal(np.abs(q["L1b"]), np.abs(p["L1b"]))
+    assert np.array_equal(q["wq"], p["wq"]) and np.array_equal(q["s_w"], p["s_w"])

@@ -1,0 +1,272 @@
+"""Python binding of the SVDQuant W4A4 linear-layer library (libsvdq.so).
+
+Argument marshalling only: every step of the layer runs in the C-ABI
+library (host pack code and sm_100a kernels).  PyTorch supplies device
+memory and the current CUDA stream.  The binding never falls back to another
+implementation: if the library is missing it raises.
+
+The call names follow include/svdq.h:
+    svdq_calib_absmax, svdq_pack_weights, svdq_pack_weights_host,
+    svdq_weights_export, svdq_weights_save, svdq_weights_load,
+    svdq_quantize_act, svdq_linear, svdq_get_device_error,
+    svdq_debug_partials
+and SVDQLinear bundles one packed layer with its two hot-path calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+__all__ = [
+    "lib", "SVDQError", "Weights", "SVDQLinear", "svdq_calib_absmax",
+    "svdq_pack_weights", "svdq_pack_weights_host", "svdq_weights_load",
+    "svdq_quantize_act", "svdq_linear", "svdq_get_device_error",
+    "svdq_debug_partials", "EPI_NONE", "EPI_GELU", "LIB_PATH",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libsvdq.so")
+EPI_NONE = 0
+EPI_GELU = 1
+
+_STATUS = {
+    0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_SHAPE",
+    3: "SVDQ_ERR_ALIGNMENT", 4: "SVDQ_ERR_UNSUPPORTED", 5: "SVDQ_ERR_NUMERIC",
+    6: "SVDQ_ERR_CUDA", 7: "SVDQ_ERR_DEVICE_TIMEOUT", 8: "SVDQ_ERR_OOM",
+    9: "SVDQ_ERR_IO",
+}
+
+
+class SVDQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsvdq.so (built in-tree by `python -m
+    w4a4_quantized_gemm_smooth_b200.build`).  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m w4a4_quantized_gemm_smooth_b200.build` (no fallback exists)")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "svdq_status_string": (ctypes.c_char_p, [_i]),
+        "svdq_version": (_i, []),
+        "svdq_calib_absmax": (_i, [_i, _i, _vp, _i, _vp]),
+        "svdq_pack_weights": (_i, [_i, _i, _i, _i, _vp, _vp, ctypes.c_double, _vp, _i,
+                                   _vp, _vp, ctypes.c_float, _vp, _vp]),
+        "svdq_pack_weights_host": (_i, [_i, _i, _i, _i, _vp, _vp, ctypes.c_double, _vp,
+                                        _i, _vp, _vp, ctypes.c_float, _vp]),
+        "svdq_weights_info": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
+        "svdq_weights_export": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+        "svdq_weights_save": (_i, [_vp, ctypes.c_char_p]),
+        "svdq_weights_load": (_i, [ctypes.c_char_p, _vp, _vp]),
+        "svdq_weights_free": (None, [_vp]),
+        "svdq_quantize_act": (_i, [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp]),
+        "svdq_linear": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _vp]),
+        "svdq_get_device_error": (_i, [_vp, _vp]),
+        "svdq_debug_partials": (_i, [_vp, _i, _vp, _i, _i, _i, _i, _vp, _vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise SVDQError(status, where)
+
+
+def _np_ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(_vp)
+
+
+def _stream_ptr(stream=None):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return _vp(stream.cuda_stream)
+
+
+def _dev_ptr(t):
+    return None if t is None else _vp(t.data_ptr())
+
+
+class Weights:
+    """Owns one packed layer handle (svdq_weights*)."""
+
+    def __init__(self, handle: ctypes.c_void_p):
+        self._h = handle
+        K, N, r, sr, lr = (ctypes.c_int() for _ in range(5))
+        _check(lib().svdq_weights_info(handle, ctypes.byref(K), ctypes.byref(N),
+                                       ctypes.byref(r), ctypes.byref(sr),
+                                       ctypes.byref(lr)), "svdq_weights_info")
+        self.K, self.N, self.rank = K.value, N.value, r.value
+        self.svd_rank, self.lora_rank = sr.value, lr.value
+
+    @property
+    def handle(self):
+        return self._h
+
+    def export(self) -> dict:
+        K, N, r = self.K, self.N, self.rank
+        out = dict(
+            inv_lambda=np.empty(K, np.float32), wq=np.empty((N, K // 2), np.uint8),
+            s_w=np.empty((K // 64, N), np.float32), L1=np.empty((K, r), np.uint16),
+            L2=np.empty((r, N), np.uint16), bias=np.empty(N, np.uint16),
+            sigma=np.empty(self.svd_rank + 1, np.float64))
+        _check(lib().svdq_weights_export(
+            self._h, _np_ptr(out["inv_lambda"]), _np_ptr(out["wq"]), _np_ptr(out["s_w"]),
+            _np_ptr(out["L1"]), _np_ptr(out["L2"]), _np_ptr(out["bias"]),
+            _np_ptr(out["sigma"])), "svdq_weights_export")
+        return out
+
+    def save(self, path: str):
+        _check(lib().svdq_weights_save(self._h, path.encode()), "svdq_weights_save")
+
+    def free(self):
+        if self._h:
+            lib().svdq_weights_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def svdq_calib_absmax(X_bits: np.ndarray, absmax: np.ndarray | None = None) -> np.ndarray:
+    """Running per-channel max|X| of a host bf16 matrix (uint16 bits [M, K])."""
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    M, K = X_bits.shape
+    if absmax is None:
+        absmax = np.zeros(K, np.float32)
+    _check(lib().svdq_calib_absmax(M, K, _np_ptr(X_bits), K, _np_ptr(absmax)),
+           "svdq_calib_absmax")
+    return absmax
+
+
+def _pack_args(W_bits, act_absmax, bias_bits, lora_A_bits, lora_B_bits):
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    act_absmax = np.ascontiguousarray(act_absmax, dtype=np.float32)
+    bias_bits = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    A = None if lora_A_bits is None else np.ascontiguousarray(lora_A_bits, dtype=np.uint16)
+    B = None if lora_B_bits is None else np.ascontiguousarray(lora_B_bits, dtype=np.uint16)
+    lr = 0 if A is None else A.shape[1]
+    return W_bits, act_absmax, bias_bits, A, B, lr
+
+
+def svdq_pack_weights(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None,
+                      lora_A_bits=None, lora_B_bits=None, lora_scale=1.0,
+                      stream=None) -> Weights:
+    """Offline pack onto the current CUDA device (see include/svdq.h)."""
+    W_bits, act_absmax, bias_bits, A, B, lr = _pack_args(
+        W_bits, act_absmax, bias_bits, lora_A_bits, lora_B_bits)
+    N, K = W_bits.shape
+    h = _vp()
+    _check(lib().svdq_pack_weights(K, N, int(rank), 64, _np_ptr(W_bits), _np_ptr(act_absmax),
+                                   float(alpha), _np_ptr(bias_bits), lr, _np_ptr(A),
+                                   _np_ptr(B), float(lora_scale), _stream_ptr(stream),
+                                   ctypes.byref(h)), "svdq_pack_weights")
+    return Weights(h)
+
+
+def svdq_pack_weights_host(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None,
+                           lora_A_bits=None, lora_B_bits=None, lora_scale=1.0) -> Weights:
+    """Same transform without a GPU (host copies only)."""
+    W_bits, act_absmax, bias_bits, A, B, lr = _pack_args(
+        W_bits, act_absmax, bias_bits, lora_A_bits, lora_B_bits)
+    N, K = W_bits.shape
+    h = _vp()
+    _check(lib().svdq_pack_weights_host(K, N, int(rank), 64, _np_ptr(W_bits),
+                                        _np_ptr(act_absmax), float(alpha), _np_ptr(bias_bits),
+                                        lr, _np_ptr(A), _np_ptr(B), float(lora_scale),
+                                        ctypes.byref(h)), "svdq_pack_weights_host")
+    return Weights(h)
+
+
+def svdq_weights_load(path: str, stream=None) -> Weights:
+    h = _vp()
+    _check(lib().svdq_weights_load(path.encode(), _stream_ptr(stream), ctypes.byref(h)),
+           "svdq_weights_load")
+    return Weights(h)
+
+
+def svdq_quantize_act(w: Weights, X, xq, s_x, Z=None, stream=None):
+    """X: cuda bf16 [M, K] (row stride X.stride(0)); xq uint8 [M, K/2];
+    s_x float32 [K/64, M]; Z bf16 [M, rank] or None when rank == 0."""
+    M = X.shape[0]
+    _check(lib().svdq_quantize_act(w.handle, M, _dev_ptr(X), X.stride(0), _dev_ptr(xq),
+                                   _dev_ptr(s_x), _dev_ptr(Z), _stream_ptr(stream)),
+           "svdq_quantize_act")
+
+
+def svdq_linear(w: Weights, xq, s_x, Z, Y, epilogue=EPI_NONE, stream=None):
+    """Y: cuda bf16 [M, N] (row stride Y.stride(0))."""
+    M = Y.shape[0]
+    _check(lib().svdq_linear(w.handle, M, _dev_ptr(xq), _dev_ptr(s_x), _dev_ptr(Z),
+                             _dev_ptr(Y), Y.stride(0), int(epilogue), _stream_ptr(stream)),
+           "svdq_linear")
+
+
+def svdq_get_device_error(w: Weights, stream=None):
+    _check(lib().svdq_get_device_error(w.handle, _stream_ptr(stream)), "device")
+
+
+def svdq_debug_partials(w: Weights, M, xq, row0, nrows, col0, ncols, P, stream=None):
+    """P: cuda int32 [K/64, nrows, ncols]."""
+    _check(lib().svdq_debug_partials(w.handle, int(M), _dev_ptr(xq), int(row0), int(nrows),
+                                     int(col0), int(ncols), _dev_ptr(P), _stream_ptr(stream)),
+           "svdq_debug_partials")
+
+
+class SVDQLinear:
+    """One packed layer plus the buffers of its two hot-path calls.
+
+    forward(X) runs svdq_quantize_act then svdq_linear on the current stream
+    and returns Y (bf16 [M, N]).  Buffers are reallocated only when M grows.
+    """
+
+    def __init__(self, weights: Weights, epilogue: int = EPI_NONE):
+        self.w = weights
+        self.epilogue = epilogue
+        self._M = -1
+        self.xq = self.s_x = self.Z = self.Y = None
+
+    def buffers(self, M: int, device="cuda"):
+        import torch
+        if M != self._M:
+            K, N, r = self.w.K, self.w.N, self.w.rank
+            self.xq = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+            self.s_x = torch.empty((K // 64, M), dtype=torch.float32, device=device)
+            self.Z = torch.empty((M, max(r, 1)), dtype=torch.bfloat16, device=device) if r else None
+            self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            self._M = M
+        return self.xq, self.s_x, self.Z, self.Y
+
+    def forward(self, X, out=None):
+        M = X.shape[0]
+        xq, s_x, Z, Y = self.buffers(M, X.device)
+        if out is not None:
+            Y = out
+        svdq_quantize_act(self.w, X, xq, s_x, Z)
+        svdq_linear(self.w, xq, s_x, Z, Y, self.epilogue)
+        return Y
+
+    __call__ = forward

@@ -1,0 +1,239 @@
+// Fused activation pass (SVDQuant review section 6.1, Algorithm 2 steps 1-3):
+// read X once, smooth it (eq. 3), quantise it per token and group of 64
+// (eq. 1) and, from the same tile, compute the 16-bit down-projection
+// Z = bf16(x~) L1 on the tensor cores (mma.sync bf16, fp32 accumulation).
+//
+// Layout: one CTA of 8 warps owns 32 consecutive tokens and walks K in
+// chunks of 256 channels.  A warp instruction loads one token's 256 channels
+// (512 contiguous bytes, 16 bytes per lane); the 8 lanes holding one group of
+// 64 find its absmax with three xor-shuffles.  The next chunk is loaded
+// before the current one is processed.  bf16(x~) is staged in shared memory
+// for the MMA; the scale tile is staged so that s_x[g][m] is written with
+// contiguous stores.
+//
+// Bit-exact quantiser: x~ = fl32(x * inv_lambda) (one IEEE multiply),
+// s = fl32(m / 7) (IEEE division), and the code is round-half-even of the
+// exact quotient x~/s: a first guess from the correctly rounded reciprocal
+// is corrected with the exact residual x~ - q s computed by an fma.
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "svdq_internal.h"
+
+namespace svdq {
+namespace {
+
+constexpr int AQ_ROWS = 32;
+constexpr int AQ_CH = 256;
+constexpr int AQ_THREADS = 256;
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Round-half-even of the exact quotient x / s, clamped to [-8, 7]; s > 0.
+// `ss`, `rcp` are s (possibly scaled by 2^64 when s is tiny) and its
+// correctly rounded reciprocal; `scale` is the same power of two for x.
+__device__ __forceinline__ int quant_code(float x, float ss, float rcp, float scale) {
+  const float xx = __fmul_rn(x, scale);              // exact (power of two)
+  float q = rintf(__fmul_rn(xx, rcp));
+  const float d2 = 2.0f * __fmaf_rn(-q, ss, xx);     // exact residual, doubled
+  if (d2 > ss) {
+    q += 1.0f;
+  } else if (d2 < -ss) {
+    q -= 1.0f;
+  } else if (fabsf(d2) == ss) {                      // exact tie: go to even
+    const int qi = (int)q;
+    if (qi & 1) q += (d2 > 0.0f) ? 1.0f : -1.0f;
+  }
+  q = fminf(fmaxf(q, -8.0f), 7.0f);
+  return (int)q;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(AQ_THREADS)
+act_quant_kernel(const uint16_t* __restrict__ X, int ldx,
+                 const float* __restrict__ inv_lambda,
+                 const uint16_t* __restrict__ L1T,   // [NT*8][K] bf16
+                 int M, int K, int rank,
+                 uint8_t* __restrict__ xq, float* __restrict__ s_x,
+                 uint16_t* __restrict__ Z) {
+  __shared__ __align__(16) uint16_t xs[AQ_ROWS][AQ_CH + 8];
+  __shared__ float ss_tile[AQ_CH / 64][AQ_ROWS];
+  extern __shared__ float red[];   // [8][AQ_ROWS][NT*8], NT > 0 only
+
+  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+  const int row0 = blockIdx.x * AQ_ROWS;
+  const int G = K / 64;
+  const int nchunks = (K + AQ_CH - 1) / AQ_CH;
+
+  float zacc[2][NT > 0 ? NT : 1][4];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < (NT > 0 ? NT : 1); ++b)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) zacc[a][b][c] = 0.0f;
+
+  uint4 cur[4], nxt[4];
+  auto load_chunk = [&](int c, uint4 (&v)[4]) {
+    const int col = c * AQ_CH + l * 8;
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int row = row0 + w + 8 * rr;
+      if (col < K && row < M)
+        v[rr] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)row * ldx + col));
+      else
+        v[rr] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  load_chunk(0, cur);
+
+  for (int c = 0; c < nchunks; ++c) {
+    if (c + 1 < nchunks) load_chunk(c + 1, nxt);
+    const int col = c * AQ_CH + l * 8;
+    const bool colok = col < K;
+    float il[8];
+    if (colok) {
+      const float4 i0 = __ldg(reinterpret_cast<const float4*>(inv_lambda + col));
+      const float4 i1 = __ldg(reinterpret_cast<const float4*>(inv_lambda + col + 4));
+      il[0] = i0.x; il[1] = i0.y; il[2] = i0.z; il[3] = i0.w;
+      il[4] = i1.x; il[5] = i1.y; il[6] = i1.z; il[7] = i1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) il[j] = 0.0f;
+    }
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int lr = w + 8 * rr;
+      const int row = row0 + lr;
+      const uint32_t u[4] = {cur[rr].x, cur[rr].y, cur[rr].z, cur[rr].w};
+      float xh[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        xh[2 * j] = __fmul_rn(bf16lo(u[j]), il[2 * j]);
+        xh[2 * j + 1] = __fmul_rn(bf16hi(u[j]), il[2 * j + 1]);
+      }
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(xh[j]));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+      const float s = __fdiv_rn(m, 7.0f);
+      uint32_t packed = 0u;
+      if (s > 0.0f) {
+        const bool tiny = s < 0x1p-64f;
+        const float scale = tiny ? 0x1p64f : 1.0f;
+        const float ssc = __fmul_rn(s, scale);
+        const float rcp = __frcp_rn(ssc);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          packed |= (uint32_t)(quant_code(xh[j], ssc, rcp, scale) & 0xF) << (4 * j);
+      }
+      if (colok && row < M)
+        *reinterpret_cast<uint32_t*>(xq + (size_t)row * (K / 2) + col / 2) = packed;
+      if ((l & 7) == 0) ss_tile[l >> 3][lr] = s;
+      uint4 hv;
+      hv.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[0])) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[1])) << 16);
+      hv.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[2])) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[3])) << 16);
+      hv.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[4])) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[5])) << 16);
+      hv.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[6])) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[7])) << 16);
+      *reinterpret_cast<uint4*>(&xs[lr][l * 8]) = hv;
+    }
+    __syncthreads();
+    if (tid < (AQ_CH / 64) * AQ_ROWS) {
+      const int g = c * (AQ_CH / 64) + (tid >> 5);
+      const int row = row0 + (tid & 31);
+      if (g < G && row < M) s_x[(size_t)g * M + row] = ss_tile[tid >> 5][tid & 31];
+    }
+    if constexpr (NT > 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int kc = (w + 8 * h) * 16;          // k16 step inside the chunk
+        const int kglob = c * AQ_CH + kc;
+        if (kglob < K) {
+          uint32_t a[2][4];
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+            ldmatrix_x4(smem_u32(&xs[mt * 16 + (l & 15)][kc + (l >> 4) * 8]), a[mt]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint16_t* bp = L1T + (size_t)(nt * 8 + (l >> 2)) * K + kglob + 2 * (l & 3);
+            const uint32_t b0 = __ldg(reinterpret_cast<const uint32_t*>(bp));
+            const uint32_t b1 = __ldg(reinterpret_cast<const uint32_t*>(bp + 8));
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) mma_bf16_16816(zacc[mt][nt], a[mt], b0, b1);
+          }
+        }
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) cur[rr] = nxt[rr];
+  }
+
+  if constexpr (NT > 0) {
+    constexpr int RP = NT * 8;
+    float* rw = red + (size_t)w * AQ_ROWS * RP;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int r = mt * 16 + (l >> 2);
+        const int cc = nt * 8 + 2 * (l & 3);
+        rw[r * RP + cc] = zacc[mt][nt][0];
+        rw[r * RP + cc + 1] = zacc[mt][nt][1];
+        rw[(r + 8) * RP + cc] = zacc[mt][nt][2];
+        rw[(r + 8) * RP + cc + 1] = zacc[mt][nt][3];
+      }
+    __syncthreads();
+    for (int idx = tid; idx < AQ_ROWS * rank; idx += AQ_THREADS) {
+      const int r = idx / rank, j = idx % rank;
+      float sum = 0.0f;
+#pragma unroll
+      for (int ww = 0; ww < 8; ++ww) sum += red[(size_t)ww * AQ_ROWS * RP + r * RP + j];
+      if (row0 + r < M)
+        Z[(size_t)(row0 + r) * rank + j] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+    }
+  }
+}
+
+template <int NT>
+cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                      uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
+  const size_t red_bytes = NT > 0 ? (size_t)8 * AQ_ROWS * NT * 8 * sizeof(float) : 0;
+  if (red_bytes > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<NT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)red_bytes);
+    if (e != cudaSuccess) return e;
+  }
+  const dim3 grid((M + AQ_ROWS - 1) / AQ_ROWS);
+  act_quant_kernel<NT><<<grid, AQ_THREADS, red_bytes, st>>>(
+      X, ldx, w->d_inv_lambda, w->d_L1T, M, w->K, w->rank, xq, s_x, Z);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                             uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
+  switch (w->rank_pad / 8) {
+    case 0: return launch_aq<0>(w, M, X, ldx, xq, s_x, Z, st);
+    case 2: return launch_aq<2>(w, M, X, ldx, xq, s_x, Z, st);
+    case 4: return launch_aq<4>(w, M, X, ldx, xq, s_x, Z, st);
+    case 6: return launch_aq<6>(w, M, X, ldx, xq, s_x, Z, st);
+    case 8: return launch_aq<8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 10: return launch_aq<10>(w, M, X, ldx, xq, s_x, Z, st);
+    case 12: return launch_aq<12>(w, M, X, ldx, xq, s_x, Z, st);
+    case 14: return launch_aq<14>(w, M, X, ldx, xq, s_x, Z, st);
+    case 16: return launch_aq<16>(w, M, X, ldx, xq, s_x, Z, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace svdq

@@ -1,0 +1,65 @@
+// C ABI of the hot path: argument checks, then one kernel launch per call.
+#include <cstdint>
+
+#include "svdq_internal.h"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+svdq_status check_handle(const svdq_weights* w) {
+  if (!w || !w->d_wq || !w->d_err) return SVDQ_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
+  return SVDQ_OK;
+}
+
+svdq_status from_launch(cudaError_t e) { return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+svdq_status svdq_quantize_act(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                              uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t stream) {
+  svdq_status s = check_handle(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || ldx < w->K) return SVDQ_ERR_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !xq || !s_x || (w->rank > 0 && !Z)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(xq) || !aligned16(s_x) || (ldx % 8) != 0 ||
+      (w->rank > 0 && !aligned16(Z)))
+    return SVDQ_ERR_ALIGNMENT;
+  return from_launch(svdq::launch_act_quant(w, M, X, ldx, xq, s_x, Z, stream));
+}
+
+svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
+                        const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
+                        cudaStream_t stream) {
+  svdq_status s = check_handle(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || ldy < w->N) return SVDQ_ERR_SHAPE;
+  if (epilogue != SVDQ_EPI_NONE && epilogue != SVDQ_EPI_GELU) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!xq || !s_x || !Y || (w->rank > 0 && !Z)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(s_x) || !aligned16(Y) || (ldy % 8) != 0 ||
+      (w->rank > 0 && !aligned16(Z)))
+    return SVDQ_ERR_ALIGNMENT;
+  return from_launch(svdq::launch_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, stream));
+}
+
+svdq_status svdq_debug_partials(const svdq_weights* w, int M, const uint8_t* xq, int row0,
+                                int nrows, int col0, int ncols, int32_t* P,
+                                cudaStream_t stream) {
+  svdq_status s = check_handle(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 1 || nrows < 1 || ncols < 1 || row0 < 0 || col0 < 0 || row0 + nrows > M ||
+      col0 + ncols > w->N)
+    return SVDQ_ERR_SHAPE;
+  if (!xq || !P) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(P)) return SVDQ_ERR_ALIGNMENT;
+  return from_launch(svdq::launch_partials(w, M, xq, row0, nrows, col0, ncols, P, stream));
+}
+
+}  // extern "C"

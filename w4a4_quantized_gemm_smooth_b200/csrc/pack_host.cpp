@@ -1,0 +1,392 @@
+// Host side of the C ABI: the offline pack (SVDQuant review Algorithm 1,
+// steps 2-5 and 9), handle management, export, save/load.
+//
+// Exactness contract with the checks: every rounding below is a single IEEE
+// rounding of a value that both sides define the same way, so the codes and
+// scales of the quantised residual are reproducible bit for bit:
+//   lambda (eq. 4, alpha = 0.5) = sqrt(a) / sqrt(w)   (fp64, correctly rounded)
+//   inv_lambda = fl32(1 / lambda)
+//   W~ = lambda_k * W[k][n]                           (fp64, eq. 3)
+//   R = W~ - sum_j L1b[k][j] L2b[j][n], j ascending   (fp64; the products of
+//       two bf16 values are exact, each subtraction is rounded once)
+//   s = fl32(max|fl32(R)| / 7), codes = rne of the exact quotient  (eq. 1)
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "svdq_internal.h"
+
+namespace {
+
+uint32_t f32_bits(float f) { uint32_t u; std::memcpy(&u, &f, 4); return u; }
+float bits_f32(uint32_t u) { float f; std::memcpy(&f, &u, 4); return f; }
+
+double bf16_to_f64(uint16_t b) { return (double)bits_f32((uint32_t)b << 16); }
+
+// One round-to-nearest-even rounding of an fp64 value to bf16 (8 significant
+// bits, fp32's exponent range, subnormal quantum 2^-133).
+uint16_t f64_to_bf16(double x) {
+  if (std::isnan(x)) return 0x7FC0;
+  const double ax = std::fabs(x);
+  if (ax == 0.0) return std::signbit(x) ? 0x8000 : 0x0000;
+  double y;
+  if (ax < 0x1p-126) {
+    y = std::nearbyint(x * 0x1p133) * 0x1p-133;   // exact scalings
+  } else {
+    uint64_t u;
+    std::memcpy(&u, &x, 8);
+    const uint64_t keep = (u >> 45) & 1u;          // lsb of the kept part
+    u += ((uint64_t)1 << 44) - 1 + keep;
+    u &= ~(((uint64_t)1 << 45) - 1);
+    std::memcpy(&y, &u, 8);
+    if (std::fabs(y) >= 0x1p128) return std::signbit(x) ? 0xFF80 : 0x7F80;
+  }
+  return (uint16_t)(f32_bits((float)y) >> 16);     // exact conversion
+}
+
+// Eq. 1 on one group of 64 fp32 values: scale and codes.
+float quantize_group(const float* z, int stride, int8_t* q) {
+  float m = 0.0f;
+  for (int i = 0; i < 64; ++i) m = std::fmax(m, std::fabs(z[(long)i * stride]));
+  const float s = m / 7.0f;    // IEEE fp32 division
+  if (s == 0.0f) {
+    for (int i = 0; i < 64; ++i) q[i] = 0;
+    return 0.0f;
+  }
+  const double sd = s;
+  for (int i = 0; i < 64; ++i) {
+    const double zd = z[(long)i * stride];
+    double c = std::nearbyint(zd / sd);
+    for (int it = 0; it < 2; ++it) {
+      const double d2 = 2.0 * (zd - c * sd);          // exact
+      if (d2 > sd) c += 1.0;
+      else if (d2 < -sd) c -= 1.0;
+    }
+    const double d2 = 2.0 * (zd - c * sd);
+    if (std::fabs(d2) == sd && std::fmod(c, 2.0) != 0.0) c += (d2 > 0 ? 1.0 : -1.0);
+    if (c > 7.0) c = 7.0;
+    if (c < -8.0) c = -8.0;
+    q[i] = (int8_t)c;
+  }
+  return s;
+}
+
+template <class T>
+svdq_status dev_alloc_copy(T** dst, const T* src, size_t n, cudaStream_t st) {
+  if (n == 0) n = 1;
+  if (cudaMalloc((void**)dst, n * sizeof(T)) != cudaSuccess) return SVDQ_ERR_OOM;
+  if (src && cudaMemcpyAsync(*dst, src, n * sizeof(T), cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  return SVDQ_OK;
+}
+
+void free_device(svdq_weights* w) {
+  cudaFree(w->d_inv_lambda); cudaFree(w->d_wq); cudaFree(w->d_sw);
+  cudaFree(w->d_L1T); cudaFree(w->d_L2); cudaFree(w->d_bias); cudaFree(w->d_err);
+  w->d_inv_lambda = nullptr; w->d_wq = nullptr; w->d_sw = nullptr;
+  w->d_L1T = nullptr; w->d_L2 = nullptr; w->d_bias = nullptr; w->d_err = nullptr;
+}
+
+}  // namespace
+
+namespace svdq {
+
+svdq_status upload(svdq_weights* w, cudaStream_t st) {
+  if (cudaGetDevice(&w->device) != cudaSuccess) return SVDQ_ERR_CUDA;
+  const int K = w->K, N = w->N, G = w->G, rp = w->rank_pad;
+  std::vector<uint16_t> L1T((size_t)rp * K, 0), L2p((size_t)rp * N, 0);
+  for (int j = 0; j < w->rank; ++j)
+    for (int k = 0; k < K; ++k) L1T[(size_t)j * K + k] = w->L1[(size_t)k * w->rank + j];
+  for (int j = 0; j < w->rank; ++j)
+    std::memcpy(&L2p[(size_t)j * N], &w->L2[(size_t)j * N], (size_t)N * 2);
+  svdq_status s;
+  if ((s = dev_alloc_copy(&w->d_inv_lambda, w->inv_lambda.data(), (size_t)K, st))) return s;
+  if ((s = dev_alloc_copy(&w->d_wq, w->wq.data(), (size_t)N * K / 2, st))) return s;
+  if ((s = dev_alloc_copy(&w->d_sw, w->sw.data(), (size_t)G * N, st))) return s;
+  if ((s = dev_alloc_copy(&w->d_L1T, L1T.data(), L1T.size(), st))) return s;
+  if ((s = dev_alloc_copy(&w->d_L2, L2p.data(), L2p.size(), st))) return s;
+  if ((s = dev_alloc_copy(&w->d_bias, w->bias.data(), (size_t)N, st))) return s;
+  if ((s = dev_alloc_copy<int>(&w->d_err, nullptr, 1, st))) return s;
+  if (cudaMemsetAsync(w->d_err, 0, sizeof(int), st) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SVDQ_ERR_CUDA;
+  return SVDQ_OK;
+}
+
+}  // namespace svdq
+
+extern "C" {
+
+const char* svdq_status_string(int status) {
+  switch (status) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_SHAPE: return "unsupported shape (K must be a multiple of 64)";
+    case SVDQ_ERR_ALIGNMENT: return "pointer or row not 16-byte aligned";
+    case SVDQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SVDQ_ERR_NUMERIC: return "non-finite input";
+    case SVDQ_ERR_CUDA: return "CUDA runtime error";
+    case SVDQ_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case SVDQ_ERR_OOM: return "out of memory";
+    case SVDQ_ERR_IO: return "file I/O error";
+    default: return "unknown status";
+  }
+}
+
+int svdq_version(void) { return 100; }
+
+svdq_status svdq_calib_absmax(int M, int K, const uint16_t* X, int ldx, float* absmax) {
+  if (M < 0 || K < 1 || ldx < K) return SVDQ_ERR_SHAPE;
+  if ((M > 0 && !X) || !absmax) return SVDQ_ERR_INVALID_ARG;
+  for (int i = 0; i < M; ++i)
+    for (int k = 0; k < K; ++k) {
+      const float v = std::fabs(bits_f32((uint32_t)X[(size_t)i * ldx + k] << 16));
+      if (std::isnan(v)) return SVDQ_ERR_NUMERIC;
+      if (v > absmax[k]) absmax[k] = v;
+    }
+  return SVDQ_OK;
+}
+
+static svdq_status pack_impl(int K, int N, int rank, int group, const uint16_t* W,
+                             const float* act_absmax, double alpha, const uint16_t* bias,
+                             int lora_rank, const uint16_t* lora_A, const uint16_t* lora_B,
+                             float lora_scale, bool to_device, cudaStream_t stream,
+                             svdq_weights** out) {
+  if (!out) return SVDQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!W || !act_absmax) return SVDQ_ERR_INVALID_ARG;
+  if (group != SVDQ_GROUP) return SVDQ_ERR_UNSUPPORTED;
+  if (K < SVDQ_GROUP || N < 1 || K % SVDQ_GROUP) return SVDQ_ERR_SHAPE;
+  if (rank < 0 || lora_rank < 0 || rank > (K < N ? K : N)) return SVDQ_ERR_INVALID_ARG;
+  if (rank + lora_rank > SVDQ_MAX_RANK) return SVDQ_ERR_UNSUPPORTED;
+  if (lora_rank > 0 && (!lora_A || !lora_B)) return SVDQ_ERR_INVALID_ARG;
+  if (!(alpha > 0.0 && alpha < 1.0)) return SVDQ_ERR_INVALID_ARG;
+  if (!std::isfinite(lora_scale)) return SVDQ_ERR_NUMERIC;
+
+  svdq_weights* w = new (std::nothrow) svdq_weights();
+  if (!w) return SVDQ_ERR_OOM;
+  w->K = K; w->N = N; w->G = K / SVDQ_GROUP;
+  w->svd_rank = rank; w->lora_rank = lora_rank; w->rank = rank + lora_rank;
+  w->rank_pad = (w->rank + 15) / 16 * 16;
+
+  // eq. 4 statistics and lambda
+  std::vector<double> lam(K), Wt((size_t)K * N);
+  for (int k = 0; k < K; ++k) {
+    const double a = act_absmax[k];
+    if (!std::isfinite(a) || a < 0) { delete w; return SVDQ_ERR_NUMERIC; }
+  }
+  std::vector<double> wmax(K, 0.0);
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      const double v = bf16_to_f64(W[(size_t)n * K + k]);
+      if (!std::isfinite(v)) { delete w; return SVDQ_ERR_NUMERIC; }
+      wmax[k] = std::fmax(wmax[k], std::fabs(v));
+    }
+  w->inv_lambda.resize(K);
+  for (int k = 0; k < K; ++k) {
+    const double a = act_absmax[k], m = wmax[k];
+    double l = 1.0;
+    if (a > 0.0 && m > 0.0)
+      l = (alpha == 0.5) ? std::sqrt(a) / std::sqrt(m)
+                         : std::pow(a, alpha) / std::pow(m, 1.0 - alpha);
+    lam[k] = l;
+    w->inv_lambda[k] = (float)(1.0 / l);
+  }
+  // eq. 3: W~ = diag(lambda) W in the math layout [K][N]
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k)
+      Wt[(size_t)k * N + n] = lam[k] * bf16_to_f64(W[(size_t)n * K + k]);
+
+  // eq. 10: leading rank+1 singular triplets (sigma exported for checks)
+  const int nsv = std::min(rank + 1, std::min(K, N));
+  std::vector<double> sig(nsv), L1((size_t)K * (rank > 0 ? rank : 1)),
+      L2((size_t)(rank > 0 ? rank : 1) * N);
+  if (svdq::top_singular(Wt.data(), K, N, nsv, rank, sig.data(), L1.data(), L2.data())) {
+    delete w;
+    return SVDQ_ERR_NUMERIC;
+  }
+  w->sigma.assign(rank + 1, 0.0);
+  for (int j = 0; j < nsv; ++j) w->sigma[j] = sig[j];
+
+  const int rt = w->rank;
+  w->L1.assign((size_t)K * rt, 0);
+  w->L2.assign((size_t)rt * N, 0);
+  for (int k = 0; k < K; ++k)
+    for (int j = 0; j < rank; ++j) w->L1[(size_t)k * rt + j] = f64_to_bf16(L1[(size_t)k * rank + j]);
+  for (int j = 0; j < rank; ++j)
+    for (int n = 0; n < N; ++n) w->L2[(size_t)j * N + n] = f64_to_bf16(L2[(size_t)j * N + n]);
+
+  // residual against the stored factors, then fp32
+  std::vector<float> R32((size_t)K * N);
+#pragma omp parallel for schedule(static)
+  for (int k = 0; k < K; ++k) {
+    double* row = &Wt[(size_t)k * N];
+    for (int j = 0; j < rank; ++j) {
+      const double a = bf16_to_f64(w->L1[(size_t)k * rt + j]);
+      const uint16_t* l2 = &w->L2[(size_t)j * N];
+      for (int n = 0; n < N; ++n) row[n] -= a * bf16_to_f64(l2[n]);
+    }
+    for (int n = 0; n < N; ++n) R32[(size_t)k * N + n] = (float)row[n];
+  }
+  // eq. 1 per (output column, group of 64 input channels)
+  const int G = w->G;
+  w->sw.assign((size_t)G * N, 0.0f);
+  w->wq.assign((size_t)N * K / 2, 0);
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; ++n) {
+    int8_t q[64];
+    for (int g = 0; g < G; ++g) {
+      w->sw[(size_t)g * N + n] = quantize_group(&R32[(size_t)g * 64 * N + n], N, q);
+      uint8_t* dst = &w->wq[(size_t)n * (K / 2) + g * 32];
+      for (int b = 0; b < 32; ++b)
+        dst[b] = (uint8_t)((q[2 * b] & 0xF) | ((q[2 * b + 1] & 0xF) << 4));
+    }
+  }
+  // eq. 13: LoRA joins the 16-bit branch in smoothed coordinates
+  for (int k = 0; k < K; ++k)
+    for (int j = 0; j < lora_rank; ++j) {
+      const double a = bf16_to_f64(lora_A[(size_t)k * lora_rank + j]);
+      w->L1[(size_t)k * rt + rank + j] = f64_to_bf16((lam[k] * a) * (double)lora_scale);
+    }
+  for (int j = 0; j < lora_rank; ++j)
+    std::memcpy(&w->L2[(size_t)(rank + j) * N], &lora_B[(size_t)j * N], (size_t)N * 2);
+  w->bias.assign(N, 0);
+  if (bias) std::memcpy(w->bias.data(), bias, (size_t)N * 2);
+
+  if (to_device) {
+    const svdq_status st = svdq::upload(w, stream);
+    if (st != SVDQ_OK) { free_device(w); delete w; return st; }
+  }
+  *out = w;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_pack_weights(int K, int N, int rank, int group, const uint16_t* W,
+                              const float* act_absmax, double alpha, const uint16_t* bias,
+                              int lora_rank, const uint16_t* lora_A, const uint16_t* lora_B,
+                              float lora_scale, cudaStream_t stream, svdq_weights** out) {
+  return pack_impl(K, N, rank, group, W, act_absmax, alpha, bias, lora_rank, lora_A,
+                   lora_B, lora_scale, true, stream, out);
+}
+
+svdq_status svdq_pack_weights_host(int K, int N, int rank, int group, const uint16_t* W,
+                                   const float* act_absmax, double alpha,
+                                   const uint16_t* bias, int lora_rank,
+                                   const uint16_t* lora_A, const uint16_t* lora_B,
+                                   float lora_scale, svdq_weights** out) {
+  return pack_impl(K, N, rank, group, W, act_absmax, alpha, bias, lora_rank, lora_A,
+                   lora_B, lora_scale, false, nullptr, out);
+}
+
+svdq_status svdq_weights_info(const svdq_weights* w, int* K, int* N, int* rank,
+                              int* svd_rank, int* lora_rank) {
+  if (!w) return SVDQ_ERR_INVALID_ARG;
+  if (K) *K = w->K;
+  if (N) *N = w->N;
+  if (rank) *rank = w->rank;
+  if (svd_rank) *svd_rank = w->svd_rank;
+  if (lora_rank) *lora_rank = w->lora_rank;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_weights_export(const svdq_weights* w, float* inv_lambda, uint8_t* wq,
+                                float* s_w, uint16_t* L1, uint16_t* L2, uint16_t* bias,
+                                double* sigma) {
+  if (!w) return SVDQ_ERR_INVALID_ARG;
+  if (inv_lambda) std::memcpy(inv_lambda, w->inv_lambda.data(), w->inv_lambda.size() * 4);
+  if (wq) std::memcpy(wq, w->wq.data(), w->wq.size());
+  if (s_w) std::memcpy(s_w, w->sw.data(), w->sw.size() * 4);
+  if (L1 && !w->L1.empty()) std::memcpy(L1, w->L1.data(), w->L1.size() * 2);
+  if (L2 && !w->L2.empty()) std::memcpy(L2, w->L2.data(), w->L2.size() * 2);
+  if (bias) std::memcpy(bias, w->bias.data(), w->bias.size() * 2);
+  if (sigma) std::memcpy(sigma, w->sigma.data(), w->sigma.size() * 8);
+  return SVDQ_OK;
+}
+
+static const char kMagic[8] = {'S', 'V', 'D', 'Q', 'W', '0', '0', '1'};
+
+svdq_status svdq_weights_save(const svdq_weights* w, const char* path) {
+  if (!w || !path) return SVDQ_ERR_INVALID_ARG;
+  FILE* f = std::fopen(path, "wb");
+  if (!f) return SVDQ_ERR_IO;
+  int32_t hdr[6] = {w->K, w->N, w->svd_rank, w->lora_rank, SVDQ_GROUP, 0};
+  bool ok = std::fwrite(kMagic, 1, 8, f) == 8 && std::fwrite(hdr, 4, 6, f) == 6;
+  auto put = [&](const void* p, size_t bytes) {
+    if (ok && bytes) ok = std::fwrite(p, 1, bytes, f) == bytes;
+  };
+  put(w->inv_lambda.data(), w->inv_lambda.size() * 4);
+  put(w->wq.data(), w->wq.size());
+  put(w->sw.data(), w->sw.size() * 4);
+  put(w->L1.data(), w->L1.size() * 2);
+  put(w->L2.data(), w->L2.size() * 2);
+  put(w->bias.data(), w->bias.size() * 2);
+  put(w->sigma.data(), w->sigma.size() * 8);
+  ok = (std::fclose(f) == 0) && ok;
+  return ok ? SVDQ_OK : SVDQ_ERR_IO;
+}
+
+svdq_status svdq_weights_load(const char* path, cudaStream_t stream, svdq_weights** out) {
+  if (!path || !out) return SVDQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  FILE* f = std::fopen(path, "rb");
+  if (!f) return SVDQ_ERR_IO;
+  char magic[8];
+  int32_t hdr[6];
+  if (std::fread(magic, 1, 8, f) != 8 || std::memcmp(magic, kMagic, 8) != 0 ||
+      std::fread(hdr, 4, 6, f) != 6) {
+    std::fclose(f);
+    return SVDQ_ERR_IO;
+  }
+  const int K = hdr[0], N = hdr[1], r = hdr[2], lr = hdr[3];
+  if (hdr[4] != SVDQ_GROUP || K < 64 || K % 64 || N < 1 || r < 0 || lr < 0 ||
+      r + lr > SVDQ_MAX_RANK || K > (1 << 20) || N > (1 << 20)) {
+    std::fclose(f);
+    return SVDQ_ERR_IO;
+  }
+  svdq_weights* w = new (std::nothrow) svdq_weights();
+  if (!w) { std::fclose(f); return SVDQ_ERR_OOM; }
+  w->K = K; w->N = N; w->G = K / 64; w->svd_rank = r; w->lora_rank = lr;
+  w->rank = r + lr; w->rank_pad = (w->rank + 15) / 16 * 16;
+  w->inv_lambda.resize(K); w->wq.resize((size_t)N * K / 2); w->sw.resize((size_t)w->G * N);
+  w->L1.resize((size_t)K * w->rank); w->L2.resize((size_t)w->rank * N);
+  w->bias.resize(N); w->sigma.resize(r + 1);
+  bool ok = true;
+  auto get = [&](void* p, size_t bytes) {
+    if (ok && bytes) ok = std::fread(p, 1, bytes, f) == bytes;
+  };
+  get(w->inv_lambda.data(), (size_t)K * 4);
+  get(w->wq.data(), w->wq.size());
+  get(w->sw.data(), w->sw.size() * 4);
+  get(w->L1.data(), w->L1.size() * 2);
+  get(w->L2.data(), w->L2.size() * 2);
+  get(w->bias.data(), w->bias.size() * 2);
+  get(w->sigma.data(), w->sigma.size() * 8);
+  std::fclose(f);
+  if (!ok) { delete w; return SVDQ_ERR_IO; }
+  const svdq_status st = svdq::upload(w, stream);
+  if (st != SVDQ_OK) { free_device(w); delete w; return st; }
+  *out = w;
+  return SVDQ_OK;
+}
+
+void svdq_weights_free(svdq_weights* w) {
+  if (!w) return;
+  free_device(w);
+  delete w;
+}
+
+svdq_status svdq_get_device_error(const svdq_weights* w, cudaStream_t stream) {
+  if (!w || !w->d_err) return SVDQ_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SVDQ_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, w->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  if (h != SVDQ_DEVERR_NONE) {
+    if (cudaMemset(w->d_err, 0, sizeof(int)) != cudaSuccess) return SVDQ_ERR_CUDA;
+    return SVDQ_ERR_DEVICE_TIMEOUT;
+  }
+  return SVDQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// Internal declarations shared by the host pack code and the device launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "svdq.h"
+
+struct svdq_weights {
+  int K = 0, N = 0, G = 0;
+  int rank = 0;        // total branch rank = svd_rank + lora_rank
+  int svd_rank = 0, lora_rank = 0;
+  int rank_pad = 0;    // rank rounded up to a multiple of 16 (zero rows)
+  int device = 0;
+  // device copies (owned)
+  float* d_inv_lambda = nullptr;   // [K]
+  uint8_t* d_wq = nullptr;         // [N][K/2] packed residual codes
+  float* d_sw = nullptr;           // [G][N]
+  uint16_t* d_L1T = nullptr;       // [rank_pad][K] bf16, transposed L1
+  uint16_t* d_L2 = nullptr;        // [rank_pad][N] bf16
+  uint16_t* d_bias = nullptr;      // [N] bf16
+  int* d_err = nullptr;            // sticky device error word
+  // host copies (export / save)
+  std::vector<float> inv_lambda;
+  std::vector<uint8_t> wq;
+  std::vector<float> sw;
+  std::vector<uint16_t> L1;        // [K][rank]
+  std::vector<uint16_t> L2;        // [rank][N]
+  std::vector<uint16_t> bias;      // [N]
+  std::vector<double> sigma;       // [svd_rank + 1]
+};
+
+// Device error word values.
+enum { SVDQ_DEVERR_NONE = 0, SVDQ_DEVERR_TIMEOUT = 1 };
+
+namespace svdq {
+
+// Upload the host copies of `w` to the current device (allocates).
+svdq_status upload(svdq_weights* w, cudaStream_t stream);
+
+// Kernel launchers (capi_device.cu validates, these only launch).
+cudaError_t launch_act_quant(const svdq_weights* w, int M, const uint16_t* X,
+                             int ldx, uint8_t* xq, float* s_x, uint16_t* Z,
+                             cudaStream_t stream);
+cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq,
+                          const float* s_x, const uint16_t* Z, uint16_t* Y,
+                          int ldy, int epilogue, cudaStream_t stream);
+cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq,
+                            int row0, int nrows, int col0, int ncols,
+                            int32_t* P, cudaStream_t stream);
+
+// Host linear algebra for the pack (svd_host.cpp).
+// Leading `nsv` singular triplets of the K x N row-major matrix A:
+// sigma[0..nsv), L1 = U S as K x r row-major, L2 = V^T as r x N row-major,
+// for r = min(nsv, r_out) columns/rows.  Returns 0 on success.
+int top_singular(const double* A, int K, int N, int nsv, int r_out,
+                 double* sigma, double* L1, double* L2);
+
+}  // namespace svdq
