@@ -206,7 +206,9 @@ template <int NT>
 cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
                       uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
   const size_t red_bytes = NT > 0 ? (size_t)8 * AQ_ROWS * NT * 8 * sizeof(float) : 0;
-  if (red_bytes > 48 * 1024) {
+  // static (about 17 KB) + dynamic shared memory may exceed the 48 KB that
+  // needs no opt-in; opting in costs nothing when it does not.
+  if (red_bytes > 0) {
     cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)red_bytes);
