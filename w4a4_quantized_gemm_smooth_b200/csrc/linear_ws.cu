@@ -1,0 +1,530 @@
+// W4A4 product with the 16-bit up-projection fused (SVDQuant review section
+// 6.1, Algorithm 2 steps 4-8; eq. 7), warp-specialised for sm_100a.
+//
+// sm_100a tensor cores have no 4-bit integer kind, so the packed codes are
+// streamed by TMA into shared memory, expanded there to int8 and multiplied
+// with tcgen05.mma.kind::i8 into int32 TMEM accumulators, one per group of
+// 64 K.  Every group's int32 partial P_g is read back with tcgen05.ld and
+// folded into an fp32 register accumulator with the group's scales
+// s_x[g][m] * s_w[g][n].  The low-rank term Z L2 is one more tensor-core
+// stage (kind::f16, bf16 operands, fp32 in TMEM) added unscaled; then the
+// bias (and GELU) are applied and Y is written once, as bf16, by TMA.
+//
+// Persistent CTAs (one per SM, 128 x BN output tiles, static round-robin
+// schedule); 12 warps:
+//   warp 0      TMA producer: packed A (128 rows x 32 B) and B (BN x 32 B)
+//               per group into a 4-stage ring;
+//   warp 1      TMEM owner and MMA issuer (one thread);
+//   warps 2-3   expanders: packed nibbles -> int8 in the UMMA K-major
+//               layout (2-stage ring), and the Z / L2 slices of the
+//               low-rank stage;
+//   warps 4-11  rescale + epilogue: warp w owns TMEM lanes 32 (w % 4).. and
+//               BN/2 columns; double-buffered TMEM lets group g+1 run on
+//               the tensor cores while group g is rescaled.
+// Every wait is bounded: an expired wait raises the handle's error word and
+// the CTA drains and exits instead of hanging.
+//
+// Expanded operand layout (no swizzle): a 64-byte K row of a group is four
+// 16-byte core-matrix rows; core matrix (row r/8, chunk c) is stored at
+// (r/8)*512 + c*128, row r%8 at +16*(r%8).  Inside every 8 codes the
+// expansion places the even-k codes before the odd-k codes; A and B use the
+// same order, so each group's dot product is unchanged.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "ptx.cuh"
+#include "svdq_internal.h"
+
+namespace svdq {
+namespace {
+
+constexpr int BM = 128;
+constexpr int NP = 4;            // packed-code stages
+constexpr int NE = 2;            // expanded-operand stages
+constexpr int THREADS = 384;
+constexpr int N_EXP = 64;        // expander threads (warps 2-3)
+constexpr int N_RES_WARPS = 8;   // rescale / epilogue warps (4-11)
+constexpr uint64_t LIMIT_NS = 2000000000ull;
+
+struct LinArgs {
+  const float* s_x;
+  const float* s_w;
+  const uint16_t* Z;
+  const uint16_t* L2T;     // [N_pad][rank_pad32]
+  const uint16_t* bias;
+  int M, N, K, G;
+  int rank, rank_pad32, n_lr;
+  int epilogue;
+  int tiles_n, num_tiles, tile_m0, tile_n0;
+  int* err;
+  int32_t* P;              // partial dump (MODE 1)
+  int row0, nrows, col0, ncols;
+};
+
+template <int BN>
+struct Lay {
+  static constexpr int CW = BN / 2;                      // columns per rescale warp
+  static constexpr int Y_BOX = 32 * 64 * 2;              // 32 rows x 64 bf16 (4 KB)
+  static constexpr int Y_WARP = (CW / 64) * Y_BOX;
+  static constexpr int PK_A = BM * 32, PK_B = BN * 32, PK_STAGE = PK_A + PK_B;
+  static constexpr int EX_A = BM * 64, EX_B = BN * 64, EX_STAGE = EX_A + EX_B;
+  static constexpr int OFF_Y = 0;
+  static constexpr int OFF_PK = OFF_Y + N_RES_WARPS * Y_WARP;
+  static constexpr int OFF_EX = OFF_PK + NP * PK_STAGE;
+  static constexpr int OFF_SW = OFF_EX + NE * EX_STAGE;
+  static constexpr int OFF_BAR = OFF_SW + N_RES_WARPS * 2 * CW * 4;
+  // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[2], tm_empty[2]
+  static constexpr int N_BARS = 2 * NP + 2 * NE + 4;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;              // slack for 1024-B alignment
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
+                                              volatile int* abort_flag, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 63u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > LIMIT_NS) {
+        *abort_flag = 1;
+        atomicExch(err, SVDQ_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// 16 packed bytes (32 codes of one row) -> two 16-byte core-matrix rows.
+__device__ __forceinline__ void expand16(const uint8_t* src, uint8_t* dst_base, int row,
+                                         int half) {
+  const uint4 p = *reinterpret_cast<const uint4*>(src);
+  uint4 o0, o1;
+  o0.x = sext_nibbles(p.x & 0x0F0F0F0Fu);
+  o0.y = sext_nibbles((p.x >> 4) & 0x0F0F0F0Fu);
+  o0.z = sext_nibbles(p.y & 0x0F0F0F0Fu);
+  o0.w = sext_nibbles((p.y >> 4) & 0x0F0F0F0Fu);
+  o1.x = sext_nibbles(p.z & 0x0F0F0F0Fu);
+  o1.y = sext_nibbles((p.z >> 4) & 0x0F0F0F0Fu);
+  o1.z = sext_nibbles(p.w & 0x0F0F0F0Fu);
+  o1.w = sext_nibbles((p.w >> 4) & 0x0F0F0F0Fu);
+  uint8_t* d = dst_base + (row >> 3) * 512 + (row & 7) * 16 + half * 256;
+  *reinterpret_cast<uint4*>(d) = o0;
+  *reinterpret_cast<uint4*>(d + 128) = o1;
+}
+
+__device__ __forceinline__ float gelu_f(float y) {
+  return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a)) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
+}
+
+// MODE 0: the layer (rescale, low-rank stage, epilogue, TMA store of Y).
+// MODE 1: dump the int32 group partials of the tiles covering the requested
+//         block instead of rescaling them (test hook).
+template <int BN, int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
+                 const __grid_constant__ CUtensorMap tm_b,
+                 const __grid_constant__ CUtensorMap tm_y, const LinArgs p) {
+  using L = Lay<BN>;
+  constexpr int CW = L::CW;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::OFF_BAR;
+  auto pk_full = [&](int s) { return bar0 + 8u * s; };
+  auto pk_empty = [&](int s) { return bar0 + 8u * (NP + s); };
+  auto ex_full = [&](int s) { return bar0 + 8u * (2 * NP + s); };
+  auto ex_empty = [&](int s) { return bar0 + 8u * (2 * NP + NE + s); };
+  auto tm_full = [&](int b) { return bar0 + 8u * (2 * NP + 2 * NE + b); };
+  auto tm_empty = [&](int b) { return bar0 + 8u * (2 * NP + 2 * NE + 2 + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = p.G;
+
+  if (tid == 0) {
+    for (int s = 0; s < NP; ++s) { mbar_init(pk_full(s), 1); mbar_init(pk_empty(s), N_EXP); }
+    for (int s = 0; s < NE; ++s) { mbar_init(ex_full(s), N_EXP); mbar_init(ex_empty(s), 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(tm_full(b), 1); mbar_init(tm_empty(b), N_RES_WARPS); }
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 2 * BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+        const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
+        const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
+        for (int g = 0; g < G; ++g, ++it) {
+          const int s = it % NP;
+          if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err)) goto producer_done;
+          mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE);
+          const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
+          tma_load_2d(dst, &tm_a, g * 32, m0, pk_full(s));
+          tma_load_2d(dst + L::PK_A, &tm_b, g * 32, n0, pk_full(s));
+        }
+      }
+    producer_done:
+      // drain: every issued load has landed before the CTA exits
+      for (uint32_t k = (it > NP ? it - NP : 0); k < it; ++k)
+        mbar_wait_bounded(pk_full(k % NP), (k / NP) & 1, LIMIT_NS);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_i8 = idesc_i8(BM, BN), id_bf = idesc_bf16(BM, BN);
+      uint32_t ite = 0, tb = 0;
+      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+        for (int g = 0; g < G + (p.n_lr > 0 ? 1 : 0); ++g) {
+          const int b = tb & 1;
+          if (!wait_or_abort(tm_empty(b), ((tb >> 1) & 1) ^ 1, abort_flag, p.err)) goto mma_done;
+          const uint32_t d = tmem + b * BN;
+          const int nsub = (g < G) ? 1 : p.n_lr;
+          for (int j = 0; j < nsub; ++j, ++ite) {
+            const int s = ite % NE;
+            if (!wait_or_abort(ex_full(s), (ite / NE) & 1, abort_flag, p.err)) goto mma_done;
+            tc_fence_after();
+            const uint32_t ea = sbase + L::OFF_EX + s * L::EX_STAGE;
+            const uint64_t ad = sdesc_kmajor_noswizzle(ea, 128, 512);
+            const uint64_t bd = sdesc_kmajor_noswizzle(ea + L::EX_A, 128, 512);
+            if (g < G) {
+              mma_i8(d, ad, bd, id_i8, 0u);
+              mma_i8(d, ad + 16, bd + 16, id_i8, 1u);
+            } else {
+              mma_bf16(d, ad, bd, id_bf, j > 0 ? 1u : 0u);
+              mma_bf16(d, ad + 16, bd + 16, id_bf, 1u);
+            }
+            mma_commit(ex_empty(s));
+          }
+          mma_commit(tm_full(b));
+          ++tb;
+        }
+      }
+    mma_done:;
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------ expanders
+    const int et = tid - 64;
+    uint32_t itp = 0, ite = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+      const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
+      const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
+      for (int g = 0; g < G + p.n_lr; ++g, ++ite) {
+        const int se = ite % NE;
+        if (!wait_or_abort(ex_empty(se), ((ite / NE) & 1) ^ 1, abort_flag, p.err)) goto exp_done;
+        uint8_t* ea = smem + L::OFF_EX + se * L::EX_STAGE;
+        uint8_t* eb = ea + L::EX_A;
+        if (g < G) {
+          const int sp = itp % NP;
+          if (!wait_or_abort(pk_full(sp), (itp / NP) & 1, abort_flag, p.err)) goto exp_done;
+          const uint8_t* pa = smem + L::OFF_PK + sp * L::PK_STAGE;
+          const uint8_t* pb = pa + L::PK_A;
+#pragma unroll
+          for (int i = et; i < BM * 2; i += N_EXP) expand16(pa + i * 16, ea, i >> 1, i & 1);
+#pragma unroll
+          for (int i = et; i < BN * 2; i += N_EXP) expand16(pb + i * 16, eb, i >> 1, i & 1);
+          mbar_arrive(pk_empty(sp));
+          ++itp;
+        } else {
+          // low-rank slice j: Z[:, 32j:32j+32] and L2T[:, 32j:32j+32] (bf16)
+          const int k0 = (g - G) * 32;
+          for (int i = et; i < BM * 4; i += N_EXP) {
+            const int r = i >> 2, c = i & 3, row = m0 + r, col = k0 + 8 * c;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (row < p.M) {
+              const uint16_t* src = p.Z + (size_t)row * p.rank + col;
+              if ((p.rank & 7) == 0) {
+                if (col < p.rank) v = __ldg(reinterpret_cast<const uint4*>(src));
+              } else {
+                uint16_t e[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) e[q] = (col + q < p.rank) ? src[q] : (uint16_t)0;
+                v.x = e[0] | ((uint32_t)e[1] << 16); v.y = e[2] | ((uint32_t)e[3] << 16);
+                v.z = e[4] | ((uint32_t)e[5] << 16); v.w = e[6] | ((uint32_t)e[7] << 16);
+              }
+            }
+            *reinterpret_cast<uint4*>(ea + (r >> 3) * 512 + c * 128 + (r & 7) * 16) = v;
+          }
+          for (int i = et; i < BN * 4; i += N_EXP) {
+            const int r = i >> 2, c = i & 3;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+                p.L2T + (size_t)(n0 + r) * p.rank_pad32 + k0 + 8 * c));
+            *reinterpret_cast<uint4*>(eb + (r >> 3) * 512 + c * 128 + (r & 7) * 16) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(ex_full(se));
+      }
+    }
+  exp_done:;
+  } else {
+    // ------------------------------------------------------ rescale + epilogue
+    const int rw = warp - 4, q = warp & 3, h = rw >> 2;
+    float* swb = reinterpret_cast<float*>(smem + L::OFF_SW) + rw * 2 * CW;
+    uint8_t* ystage = smem + L::OFF_Y + rw * L::Y_WARP;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    uint32_t tb = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
+      const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
+      const int row = m0 + 32 * q + lane;
+      const int ncol0 = n0 + h * CW;           // first column of this warp
+      float acc[CW];
+#pragma unroll
+      for (int j = 0; j < CW; ++j) acc[j] = 0.0f;
+      // scales of group 0
+      constexpr int PER = CW / 32;             // sw values loaded per lane
+      float sx_n = (MODE == 0 && row < p.M) ? __ldg(p.s_x + row) : 0.0f;
+      float sw_n[PER];
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int n = ncol0 + lane * PER + e;
+        sw_n[e] = (MODE == 0 && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
+      }
+      for (int g = 0; g < G; ++g, ++tb) {
+        const float sx = sx_n;
+        float* swg = swb + (g & 1) * CW;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) swg[lane * PER + e] = sw_n[e];
+        __syncwarp();
+        if (MODE == 0 && g + 1 < G) {
+          sx_n = (row < p.M) ? __ldg(p.s_x + (size_t)(g + 1) * p.M + row) : 0.0f;
+#pragma unroll
+          for (int e = 0; e < PER; ++e) {
+            const int n = ncol0 + lane * PER + e;
+            sw_n[e] = (n < p.N) ? __ldg(p.s_w + (size_t)(g + 1) * p.N + n) : 0.0f;
+          }
+        }
+        const int b = tb & 1;
+        if (!wait_or_abort(tm_full(b), (tb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ta = tmem + b * BN + h * CW + lane_off;
+#pragma unroll
+        for (int c = 0; c < CW / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(ta + 16 * c, r);
+          tmem_wait_ld();
+          if (MODE == 0) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              acc[16 * c + j] = fmaf(sx * swg[16 * c + j], (float)(int32_t)r[j], acc[16 * c + j]);
+          } else {
+            const int i = row - p.row0;
+            if (i >= 0 && i < p.nrows) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int jj = ncol0 + 16 * c + j - p.col0;
+                if (jj >= 0 && jj < p.ncols)
+                  p.P[((size_t)g * p.nrows + i) * p.ncols + jj] = (int32_t)r[j];
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tm_empty(b));
+      }
+      if (!ok || MODE != 0) continue;
+      if (p.n_lr > 0) {
+        const int b = tb & 1;
+        if (!wait_or_abort(tm_full(b), (tb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ta = tmem + b * BN + h * CW + lane_off;
+#pragma unroll
+        for (int c = 0; c < CW / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(ta + 16 * c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc[16 * c + j] += __uint_as_float(r[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tm_empty(b));
+        ++tb;
+      }
+      // epilogue: bias, GELU, bf16, swizzled staging, TMA store
+      float* bb = swb + (G & 1) * CW;          // not the buffer read last
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int n = ncol0 + lane * PER + e;
+        bb[lane * PER + e] = (n < p.N) ? __uint_as_float((uint32_t)__ldg(p.bias + n) << 16) : 0.0f;
+      }
+      if (lane == 0) tma_store_wait_read0();
+      __syncwarp();
+#pragma unroll
+      for (int box = 0; box < CW / 64; ++box) {
+        uint8_t* yb = ystage + box * L::Y_BOX + lane * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int j = box * 64 + ch * 8 + e;
+            float y = acc[j] + bb[j];
+            if (p.epilogue == SVDQ_EPI_GELU) y = gelu_f(y);
+            v[e] = y;
+          }
+          uint4 o;
+          o.x = pack_bf16x2(v[0], v[1]); o.y = pack_bf16x2(v[2], v[3]);
+          o.z = pack_bf16x2(v[4], v[5]); o.w = pack_bf16x2(v[6], v[7]);
+          *reinterpret_cast<uint4*>(yb + ((ch ^ (lane & 7)) * 16)) = o;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int box = 0; box < CW / 64; ++box)
+          tma_store_2d(&tm_y, ncol0 + box * 64, m0 + 32 * q,
+                       smem_u32(ystage + box * L::Y_BOX));
+        tma_store_commit();
+      }
+      __syncwarp();
+    }
+    if (MODE == 0 && lane == 0) tma_store_wait0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * BN);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2D map over a row-major [rows][cols] array with a row pitch in bytes.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols,
+              uint64_t rows, uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows,
+              CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int BN, int MODE>
+cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtensorMap& tb,
+                      const CUtensorMap& ty, LinArgs a, int tiles_m, cudaStream_t st) {
+  using L = Lay<BN>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(linear_ws_kernel<BN, MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  a.num_tiles = tiles_m * a.tiles_n;
+  const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
+  linear_ws_kernel<BN, MODE><<<grid, THREADS, L::ALLOC, st>>>(ta, tb, ty, a);
+  return cudaGetLastError();
+}
+
+int pick_bn(int N) {
+  if (N <= 128) return 128;
+  const int r = N % 256;
+  return (r != 0 && r <= 128) ? 128 : 256;
+}
+
+}  // namespace
+
+cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
+                          const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
+                          cudaStream_t st) {
+  const int BN = pick_bn(w->N);
+  CUtensorMap ta, tb, ty;
+  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 32, BM,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 32, BN,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  LinArgs a{};
+  a.s_x = s_x; a.s_w = w->d_sw; a.Z = Z; a.L2T = w->d_L2T; a.bias = w->d_bias;
+  a.M = M; a.N = w->N; a.K = w->K; a.G = w->G;
+  a.rank = w->rank; a.rank_pad32 = w->rank_pad32; a.n_lr = w->rank_pad32 / 32;
+  a.epilogue = epilogue;
+  a.tiles_n = (w->N + BN - 1) / BN;
+  a.tile_m0 = 0; a.tile_n0 = 0;
+  a.err = w->d_err;
+  const int tiles_m = (M + BM - 1) / BM;
+  return BN == 256 ? launch_ws<256, 0>(w, ta, tb, ty, a, tiles_m, st)
+                   : launch_ws<128, 0>(w, ta, tb, ty, a, tiles_m, st);
+}
+
+cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int row0,
+                            int nrows, int col0, int ncols, int32_t* P, cudaStream_t st) {
+  const int BN = pick_bn(w->N);
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 32, BM,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 32, BN,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  LinArgs a{};
+  a.M = M; a.N = w->N; a.K = w->K; a.G = w->G;
+  a.rank = 0; a.rank_pad32 = 0; a.n_lr = 0; a.epilogue = 0;
+  a.err = w->d_err;
+  a.P = P; a.row0 = row0; a.nrows = nrows; a.col0 = col0; a.ncols = ncols;
+  const int tm0 = row0 / BM, tm1 = (row0 + nrows - 1) / BM;
+  const int tn0 = col0 / BN, tn1 = (col0 + ncols - 1) / BN;
+  a.tile_m0 = tm0; a.tile_n0 = tn0; a.tiles_n = tn1 - tn0 + 1;
+  return BN == 256 ? launch_ws<256, 1>(w, ta, tb, ta, a, tm1 - tm0 + 1, st)
+                   : launch_ws<128, 1>(w, ta, tb, ta, a, tm1 - tm0 + 1, st);
+}
+
+}  // namespace svdq

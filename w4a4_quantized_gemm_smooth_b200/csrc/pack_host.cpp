@@ -84,9 +84,10 @@ svdq_status dev_alloc_copy(T** dst, const T* src, size_t n, cudaStream_t st) {
 
 void free_device(svdq_weights* w) {
   cudaFree(w->d_inv_lambda); cudaFree(w->d_wq); cudaFree(w->d_sw);
-  cudaFree(w->d_L1T); cudaFree(w->d_L2); cudaFree(w->d_bias); cudaFree(w->d_err);
-  w->d_inv_lambda = nullptr; w->d_wq = nullptr; w->d_sw = nullptr;
-  w->d_L1T = nullptr; w->d_L2 = nullptr; w->d_bias = nullptr; w->d_err = nullptr;
+  cudaFree(w->d_L1T); cudaFree(w->d_L2); cudaFree(w->d_L2T); cudaFree(w->d_bias);
+  cudaFree(w->d_err);
+  w->d_inv_lambda = nullptr; w->d_wq = nullptr; w->d_sw = nullptr; w->d_L1T = nullptr;
+  w->d_L2 = nullptr; w->d_L2T = nullptr; w->d_bias = nullptr; w->d_err = nullptr;
 }
 
 }  // namespace
@@ -96,7 +97,13 @@ namespace svdq {
 svdq_status upload(svdq_weights* w, cudaStream_t st) {
   if (cudaGetDevice(&w->device) != cudaSuccess) return SVDQ_ERR_CUDA;
   const int K = w->K, N = w->N, G = w->G, rp = w->rank_pad;
-  std::vector<uint16_t> L1T((size_t)rp * K, 0), L2p((size_t)rp * N, 0);
+  w->rank_pad32 = (w->rank + 31) / 32 * 32;
+  w->N_pad = (N + 255) / 256 * 256;
+  const int rp32 = w->rank_pad32;
+  std::vector<uint16_t> L1T((size_t)rp * K, 0), L2p((size_t)rp * N, 0),
+      L2T((size_t)w->N_pad * (rp32 > 0 ? rp32 : 1), 0);
+  for (int j = 0; j < w->rank; ++j)
+    for (int n = 0; n < N; ++n) L2T[(size_t)n * rp32 + j] = w->L2[(size_t)j * N + n];
   for (int j = 0; j < w->rank; ++j)
     for (int k = 0; k < K; ++k) L1T[(size_t)j * K + k] = w->L1[(size_t)k * w->rank + j];
   for (int j = 0; j < w->rank; ++j)
@@ -107,6 +114,7 @@ svdq_status upload(svdq_weights* w, cudaStream_t st) {
   if ((s = dev_alloc_copy(&w->d_sw, w->sw.data(), (size_t)G * N, st))) return s;
   if ((s = dev_alloc_copy(&w->d_L1T, L1T.data(), L1T.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_L2, L2p.data(), L2p.size(), st))) return s;
+  if ((s = dev_alloc_copy(&w->d_L2T, L2T.data(), L2T.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_bias, w->bias.data(), (size_t)N, st))) return s;
   if ((s = dev_alloc_copy<int>(&w->d_err, nullptr, 1, st))) return s;
   if (cudaMemsetAsync(w->d_err, 0, sizeof(int), st) != cudaSuccess) return SVDQ_ERR_CUDA;

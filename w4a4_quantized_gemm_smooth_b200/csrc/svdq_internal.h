@@ -13,6 +13,8 @@ struct svdq_weights {
   int rank = 0;        // total branch rank = svd_rank + lora_rank
   int svd_rank = 0, lora_rank = 0;
   int rank_pad = 0;    // rank rounded up to a multiple of 16 (zero rows)
+  int rank_pad32 = 0;  // rank rounded up to a multiple of 32
+  int N_pad = 0;       // N rounded up to a multiple of 256
   int device = 0;
   // device copies (owned)
   float* d_inv_lambda = nullptr;   // [K]
@@ -20,6 +22,7 @@ struct svdq_weights {
   float* d_sw = nullptr;           // [G][N]
   uint16_t* d_L1T = nullptr;       // [rank_pad][K] bf16, transposed L1
   uint16_t* d_L2 = nullptr;        // [rank_pad][N] bf16
+  uint16_t* d_L2T = nullptr;       // [N_pad][rank_pad32] bf16, transposed L2
   uint16_t* d_bias = nullptr;      // [N] bf16
   int* d_err = nullptr;            // sticky device error word
   // host copies (export / save)
