@@ -50,7 +50,7 @@ typedef enum {
   SVDQ_ERR_INVALID_ARG = 1,     /* null pointer, bad enum, bad rank          */
   SVDQ_ERR_SHAPE = 2,           /* K % 64 != 0, negative sizes, ld too small */
   SVDQ_ERR_ALIGNMENT = 3,       /* device pointer or row not 16-byte aligned */
-  SVDQ_ERR_UNSUPPORTED = 4,     /* no sm_100 device, group != 64, rank > 128 */
+  SVDQ_ERR_UNSUPPORTED = 4,     /* group != 64, branch rank > 128 or % 8     */
   SVDQ_ERR_NUMERIC = 5,         /* non-finite weights or statistics          */
   SVDQ_ERR_CUDA = 6,            /* a CUDA runtime call or launch failed      */
   SVDQ_ERR_DEVICE_TIMEOUT = 7,  /* a bounded device wait expired             */
@@ -92,7 +92,10 @@ svdq_status svdq_calib_absmax(int M, int K, const uint16_t* X, int ldx,
  *   L2 <- [L2 ; B]; R is not recomputed.
  * Arguments:
  *   K, N        input / output channels, K % 64 == 0;
- *   rank        SVD rank, 0 <= rank <= min(K, N), rank + lora_rank <= 128;
+ *   rank        SVD rank, 0 <= rank <= min(K, N); the branch rank
+ *               rank + lora_rank must be a multiple of 8 and <= 128 (the
+ *               low-rank operands move in 16-byte units), else
+ *               SVDQ_ERR_UNSUPPORTED;
  *   group       must be 64;
  *   W           host bf16 [N][K];  act_absmax  host fp32 [K], finite, >= 0;
  *   alpha       migration strength in (0, 1) (0.5 in every workload);

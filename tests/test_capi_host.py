@@ -49,20 +49,22 @@ def test_pack_argument_validation():
                                     1.0, ctypes.byref(h)) == 4       # group != 64
     assert L.svdq_pack_weights_host(128, 64, 65, 64, p(W), p(a), 0.5, None, 0, None, None,
                                     1.0, ctypes.byref(h)) == 1       # rank > min(K, N)
-    assert L.svdq_pack_weights_host(128, 64, 4, 64, None, p(a), 0.5, None, 0, None, None,
+    assert L.svdq_pack_weights_host(128, 64, 12, 64, p(W), p(a), 0.5, None, 0, None, None,
+                                    1.0, ctypes.byref(h)) == 4       # branch rank % 8 != 0
+    assert L.svdq_pack_weights_host(128, 64, 8, 64, None, p(a), 0.5, None, 0, None, None,
                                     1.0, ctypes.byref(h)) == 1       # null weight
     a_bad = a.copy()
     a_bad[3] = np.inf
-    assert L.svdq_pack_weights_host(128, 64, 4, 64, p(W), p(a_bad), 0.5, None, 0, None,
+    assert L.svdq_pack_weights_host(128, 64, 8, 64, p(W), p(a_bad), 0.5, None, 0, None,
                                     None, 1.0, ctypes.byref(h)) == 5
     assert not h.value
 
 
 def test_host_only_handle_is_rejected_by_hot_path_calls():
-    spec = synth.layer_spec("v", 16, 128, 64, 4, 5, tiny=True)
+    spec = synth.layer_spec("v", 16, 128, 64, 8, 5, tiny=True)
     L = synth.make_layer(spec)
     a = S.svdq_calib_absmax(L.X)
-    w = S.svdq_pack_weights_host(L.W, a, 4, bias_bits=L.b)
+    w = S.svdq_pack_weights_host(L.W, a, 8, bias_bits=L.b)
     lib = S.lib()
     assert lib.svdq_quantize_act(w.handle, 16, None, 128, None, None, None, None) == 1
     assert lib.svdq_linear(w.handle, 16, None, None, None, None, 64, 0, None) == 1
@@ -112,9 +114,9 @@ def test_host_pack_matches_oracle(case):
 
 
 def test_save_writes_a_versioned_file():
-    spec = synth.layer_spec("s", 16, 128, 64, 4, 6, tiny=True)
+    spec = synth.layer_spec("s", 16, 128, 64, 8, 6, tiny=True)
     L = synth.make_layer(spec)
-    w = S.svdq_pack_weights_host(L.W, S.svdq_calib_absmax(L.X), 4, bias_bits=L.b)
+    w = S.svdq_pack_weights_host(L.W, S.svdq_calib_absmax(L.X), 8, bias_bits=L.b)
     with tempfile.TemporaryDirectory() as d:
         path = os.path.join(d, "layer.svdq")
         w.save(path)
@@ -122,6 +124,6 @@ def test_save_writes_a_versioned_file():
             blob = f.read()
     assert blob[:8] == b"SVDQW001"
     hdr = np.frombuffer(blob[8:32], np.int32)
-    assert list(hdr[:5]) == [128, 64, 4, 0, 64]
-    expect = 32 + 128 * 4 + 64 * 64 + 2 * 64 * 4 + 128 * 4 * 2 + 4 * 64 * 2 + 64 * 2 + 5 * 8
+    assert list(hdr[:5]) == [128, 64, 8, 0, 64]
+    expect = 32 + 128 * 4 + 64 * 64 + 2 * 64 * 4 + 128 * 8 * 2 + 8 * 64 * 2 + 64 * 2 + 9 * 8
     assert len(blob) == expect

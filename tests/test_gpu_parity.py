@@ -167,7 +167,7 @@ def test_argument_errors_launch_nothing():
 
 
 def test_save_load_roundtrip(tmp_path):
-    spec = synth.layer_spec("sl", 128, 256, 192, 16, 31, lora_rank=4)
+    spec = synth.layer_spec("sl", 128, 256, 192, 16, 31, lora_rank=8)
     L = synth.make_layer(spec)
     w = S.svdq_pack_weights(L.W, S.svdq_calib_absmax(L.X), 16, bias_bits=L.b,
                             lora_A_bits=L.A, lora_B_bits=L.B)

@@ -4,18 +4,21 @@
 // Z = bf16(x~) L1 on the tensor cores (mma.sync bf16, fp32 accumulation).
 //
 // Layout: one CTA of 8 warps owns 32 consecutive tokens and walks K in
-// chunks of 256 channels.  A warp instruction loads one token's 256 channels
-// (512 contiguous bytes, 16 bytes per lane); the 8 lanes holding one group of
-// 64 find its absmax with three xor-shuffles.  The next chunk is loaded
-// before the current one is processed.  bf16(x~) is staged in shared memory
-// for the MMA; the scale tile is staged so that s_x[g][m] is written with
-// contiguous stores.
+// chunks of 256 channels.  TMA streams 32 x 256 bf16 tiles of X into a
+// 4-stage shared-memory ring (64 KB in flight per SM), so X is read from HBM
+// exactly once with full-width transactions.  A warp reads one token's 256
+// channels from the ring (16 bytes per lane); the 8 lanes holding one group
+// of 64 find its absmax with three xor-shuffles.  bf16(x~) is staged in
+// shared memory for the MMA; the scale tile is staged so that s_x[g][m] is
+// written with contiguous stores.
 //
 // Bit-exact quantiser: x~ = fl32(x * inv_lambda) (one IEEE multiply),
 // s = fl32(m / 7) (IEEE division), and the code is round-half-even of the
 // exact quotient x~/s: a first guess from the correctly rounded reciprocal
 // is corrected with the exact residual x~ - q s computed by an fma.
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 
 #include "ptx.cuh"
 #include "svdq_internal.h"
@@ -26,6 +29,9 @@ namespace {
 constexpr int AQ_ROWS = 32;
 constexpr int AQ_CH = 256;
 constexpr int AQ_THREADS = 256;
+constexpr int AQ_STAGES = 4;
+constexpr int AQ_STAGE_BYTES = AQ_ROWS * AQ_CH * 2;     // 16 KB
+constexpr uint64_t AQ_LIMIT_NS = 2000000000ull;
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
@@ -51,15 +57,23 @@ __device__ __forceinline__ int quant_code(float x, float ss, float rcp, float sc
 
 template <int NT>
 __global__ void __launch_bounds__(AQ_THREADS)
-act_quant_kernel(const uint16_t* __restrict__ X, int ldx,
+act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
                  const float* __restrict__ inv_lambda,
                  const uint16_t* __restrict__ L1T,   // [NT*8][K] bf16
                  int M, int K, int rank,
                  uint8_t* __restrict__ xq, float* __restrict__ s_x,
-                 uint16_t* __restrict__ Z) {
+                 uint16_t* __restrict__ Z, int* __restrict__ err) {
   __shared__ __align__(16) uint16_t xs[AQ_ROWS][AQ_CH + 8];
   __shared__ float ss_tile[AQ_CH / 64][AQ_ROWS];
-  extern __shared__ float red[];   // [8][AQ_ROWS][NT*8], NT > 0 only
+  __shared__ __align__(8) uint64_t full_bar[AQ_STAGES];
+  __shared__ int abort_sh;
+  // dynamic: [AQ_STAGES][32 rows][box_cols] bf16 ring (1024-B aligned),
+  // then [8][AQ_ROWS][NT*8] fp32 reduction buffer when NT > 0
+  extern __shared__ uint8_t aq_dyn_raw[];
+  uint8_t* aq_dyn = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(aq_dyn_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = aq_dyn;
+  float* red = reinterpret_cast<float*>(aq_dyn + AQ_STAGES * AQ_STAGE_BYTES);
 
   const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
   const int row0 = blockIdx.x * AQ_ROWS;
@@ -74,22 +88,36 @@ act_quant_kernel(const uint16_t* __restrict__ X, int ldx,
 #pragma unroll
       for (int c = 0; c < 4; ++c) zacc[a][b][c] = 0.0f;
 
-  uint4 cur[4], nxt[4];
-  auto load_chunk = [&](int c, uint4 (&v)[4]) {
-    const int col = c * AQ_CH + l * 8;
-#pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
-      const int row = row0 + w + 8 * rr;
-      if (col < K && row < M)
-        v[rr] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)row * ldx + col));
-      else
-        v[rr] = make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t stage_bytes = (uint32_t)box_cols * AQ_ROWS * 2;
+  if (tid == 0) {
+    for (int s = 0; s < AQ_STAGES; ++s) mbar_init(smem_u32(&full_bar[s]), 1);
+    abort_sh = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int c = 0; c < AQ_STAGES && c < nchunks; ++c) {
+      mbar_arrive_expect_tx(smem_u32(&full_bar[c]), stage_bytes);
+      tma_load_2d(smem_u32(ring + c * AQ_STAGE_BYTES), &tm_x, c * AQ_CH, row0,
+                  smem_u32(&full_bar[c]));
     }
-  };
-  load_chunk(0, cur);
+  }
 
   for (int c = 0; c < nchunks; ++c) {
-    if (c + 1 < nchunks) load_chunk(c + 1, nxt);
+    const int st = c % AQ_STAGES;
+    if (!mbar_wait_bounded(smem_u32(&full_bar[st]), (c / AQ_STAGES) & 1, AQ_LIMIT_NS)) {
+      atomicExch(err, SVDQ_DEVERR_TIMEOUT);
+      abort_sh = 1;
+    }
+    __syncthreads();
+    if (abort_sh) break;
+    uint4 cur[4];
+    const uint8_t* stage = ring + st * AQ_STAGE_BYTES;
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr)
+      cur[rr] = (l * 8 < box_cols)
+                    ? *reinterpret_cast<const uint4*>(stage + (w + 8 * rr) * box_cols * 2 + l * 16)
+                    : make_uint4(0u, 0u, 0u, 0u);
     const int col = c * AQ_CH + l * 8;
     const bool colok = col < K;
     float il[8];
@@ -172,8 +200,18 @@ act_quant_kernel(const uint16_t* __restrict__ X, int ldx,
       }
     }
     __syncthreads();
-#pragma unroll
-    for (int rr = 0; rr < 4; ++rr) cur[rr] = nxt[rr];
+    if (tid == 0 && c + AQ_STAGES < nchunks) {
+      mbar_arrive_expect_tx(smem_u32(&full_bar[st]), stage_bytes);
+      tma_load_2d(smem_u32(ring + st * AQ_STAGE_BYTES), &tm_x, (c + AQ_STAGES) * AQ_CH, row0,
+                  smem_u32(&full_bar[st]));
+    }
+  }
+  if (abort_sh) {
+    // let every issued copy land before the CTA exits
+    if (tid == 0)
+      for (int c = 0; c < AQ_STAGES && c < nchunks; ++c)
+        mbar_wait_bounded(smem_u32(&full_bar[c]), 0, AQ_LIMIT_NS);
+    return;
   }
 
   if constexpr (NT > 0) {
@@ -202,21 +240,45 @@ act_quant_kernel(const uint16_t* __restrict__ X, int ldx,
   }
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 aq_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
 template <int NT>
 cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
                       uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
   const size_t red_bytes = NT > 0 ? (size_t)8 * AQ_ROWS * NT * 8 * sizeof(float) : 0;
-  // static (about 17 KB) + dynamic shared memory may exceed the 48 KB that
-  // needs no opt-in; opting in costs nothing when it does not.
-  if (red_bytes > 0) {
+  const size_t dyn = (size_t)AQ_STAGES * AQ_STAGE_BYTES + red_bytes + 1024;
+  static bool attr = false;
+  if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<NT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)red_bytes);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess) return e;
+    attr = true;
   }
+  auto fn = aq_encode_fn();
+  if (!fn) return cudaErrorInvalidValue;
+  const int box_cols = w->K < AQ_CH ? w->K : AQ_CH;
+  CUtensorMap tm;
+  const cuuint64_t dims[2] = {(cuuint64_t)w->K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)AQ_ROWS};
+  const cuuint32_t estr[2] = {1, 1};
+  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
+         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   const dim3 grid((M + AQ_ROWS - 1) / AQ_ROWS);
-  act_quant_kernel<NT><<<grid, AQ_THREADS, red_bytes, st>>>(
-      X, ldx, w->d_inv_lambda, w->d_L1T, M, w->K, w->rank, xq, s_x, Z);
+  act_quant_kernel<NT><<<grid, AQ_THREADS, dyn, st>>>(
+      tm, box_cols, w->d_inv_lambda, w->d_L1T, M, w->K, w->rank, xq, s_x, Z, w->d_err);
   return cudaGetLastError();
 }
 

@@ -11,16 +11,17 @@
 // bias (and GELU) are applied and Y is written once, as bf16, by TMA.
 //
 // Persistent CTAs (one per SM, 128 x BN output tiles, static round-robin
-// schedule); 12 warps:
+// schedule); 16 warps:
 //   warp 0      TMA producer: packed A (128 rows x 32 B) and B (BN x 32 B)
-//               per group into a 4-stage ring;
+//               per group into a 4-stage ring, and the bf16 Z / L2 slices
+//               of the low-rank stage (loaded straight into UMMA layout);
 //   warp 1      TMEM owner and MMA issuer (one thread);
-//   warps 2-3   expanders: packed nibbles -> int8 in the UMMA K-major
-//               layout (2-stage ring), and the Z / L2 slices of the
-//               low-rank stage;
-//   warps 4-11  rescale + epilogue: warp w owns TMEM lanes 32 (w % 4).. and
+//   warps 2-7   expanders: packed nibbles -> int8 in the UMMA K-major
+//               layout (2-stage ring);
+//   warps 8-15  rescale + epilogue: warp w owns TMEM lanes 32 (w % 4).. and
 //               BN/2 columns; double-buffered TMEM lets group g+1 run on
 //               the tensor cores while group g is rescaled.
+// The first two warpgroups hand registers to the last two (setmaxnreg).
 // Every wait is bounded: an expired wait raises the handle's error word and
 // the CTA drains and exits instead of hanging.
 //
@@ -28,7 +29,9 @@
 // 16-byte core-matrix rows; core matrix (row r/8, chunk c) is stored at
 // (r/8)*512 + c*128, row r%8 at +16*(r%8).  Inside every 8 codes the
 // expansion places the even-k codes before the odd-k codes; A and B use the
-// same order, so each group's dot product is unchanged.
+// same order, so each group's dot product is unchanged.  The low-rank
+// slices use the other legal arrangement of the same core matrices, chunk c
+// at c*rows*16 and row r at r*16, which a 16-byte-wide TMA box produces.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -42,10 +45,20 @@ namespace {
 constexpr int BM = 128;
 constexpr int NP = 4;            // packed-code stages
 constexpr int NE = 2;            // expanded-operand stages
-constexpr int THREADS = 384;
-constexpr int N_EXP = 64;        // expander threads (warps 2-3)
-constexpr int N_RES_WARPS = 8;   // rescale / epilogue warps (4-11)
+constexpr int THREADS = 512;
+constexpr int EXP_WARP0 = 2;     // expanders: warps 2-7
+constexpr int N_EXP = 192;
+constexpr int RES_WARP0 = 8;     // rescale / epilogue: warps 8-15
+constexpr int N_RES_WARPS = 8;
 constexpr uint64_t LIMIT_NS = 2000000000ull;
+// Register split after launch: the first two warpgroups (producer, MMA,
+// expanders) give registers to the two rescale warpgroups.
+// 256 * REG_LO + 256 * REG_HI
+// must not exceed the launch allotment (THREADS x the kernel's register
+// count); the launcher checks the compiled count before every launch.
+constexpr int REG_LO = 56;
+constexpr int REG_HI = 200;
+constexpr int REG_NEED = (256 * REG_LO + 256 * REG_HI + THREADS - 1) / THREADS;
 
 struct LinArgs {
   const float* s_x;
@@ -72,10 +85,13 @@ struct Lay {
   static constexpr int OFF_Y = 0;
   static constexpr int OFF_PK = OFF_Y + N_RES_WARPS * Y_WARP;
   static constexpr int OFF_EX = OFF_PK + NP * PK_STAGE;
-  static constexpr int OFF_SW = OFF_EX + NE * EX_STAGE;
+  static constexpr int LR_A = BM * 64, LR_B = BN * 64;     // 4 chunks x rows x 16 B
+  static constexpr int OFF_LR = OFF_EX + NE * EX_STAGE;
+  static constexpr int OFF_SW = OFF_LR + LR_A + LR_B;
   static constexpr int OFF_BAR = OFF_SW + N_RES_WARPS * 2 * CW * 4;
-  // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[2], tm_empty[2]
-  static constexpr int N_BARS = 2 * NP + 2 * NE + 4;
+  // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[2],
+  // tm_empty[2], lr_full, lr_empty
+  static constexpr int N_BARS = 2 * NP + 2 * NE + 6;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;              // slack for 1024-B alignment
@@ -132,7 +148,9 @@ template <int BN, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_b,
-                 const __grid_constant__ CUtensorMap tm_y, const LinArgs p) {
+                 const __grid_constant__ CUtensorMap tm_y,
+                 const __grid_constant__ CUtensorMap tm_z,
+                 const __grid_constant__ CUtensorMap tm_l2, const LinArgs p) {
   using L = Lay<BN>;
   constexpr int CW = L::CW;
   extern __shared__ uint8_t smem_raw[];
@@ -146,6 +164,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
   auto ex_empty = [&](int s) { return bar0 + 8u * (2 * NP + NE + s); };
   auto tm_full = [&](int b) { return bar0 + 8u * (2 * NP + 2 * NE + b); };
   auto tm_empty = [&](int b) { return bar0 + 8u * (2 * NP + 2 * NE + 2 + b); };
+  const uint32_t lr_full = bar0 + 8u * (2 * NP + 2 * NE + 4);
+  const uint32_t lr_empty = bar0 + 8u * (2 * NP + 2 * NE + 5);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -156,6 +176,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     for (int s = 0; s < NP; ++s) { mbar_init(pk_full(s), 1); mbar_init(pk_empty(s), N_EXP); }
     for (int s = 0; s < NE; ++s) { mbar_init(ex_full(s), N_EXP); mbar_init(ex_empty(s), 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(tm_full(b), 1); mbar_init(tm_empty(b), N_RES_WARPS); }
+    mbar_init(lr_full, 1);
+    mbar_init(lr_empty, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -168,120 +190,109 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-        const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
-        const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
-        for (int g = 0; g < G; ++g, ++it) {
-          const int s = it % NP;
-          if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err)) goto producer_done;
-          mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE);
-          const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
-          tma_load_2d(dst, &tm_a, g * 32, m0, pk_full(s));
-          tma_load_2d(dst + L::PK_A, &tm_b, g * 32, n0, pk_full(s));
+  if (warp < RES_WARP0) {
+    regs_dec<REG_LO>();
+    if (warp == 0) {
+      // ---------------------------------------------------- TMA producer
+      if (lane == 0) {
+        uint32_t it = 0, il = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+          const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
+          const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
+          for (int g = 0; g < G; ++g, ++it) {
+            const int s = it % NP;
+            if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err)) goto producer_done;
+            mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE);
+            const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
+            tma_load_2d(dst, &tm_a, g * 32, m0, pk_full(s));
+            tma_load_2d(dst + L::PK_A, &tm_b, g * 32, n0, pk_full(s));
+          }
+          for (int j = 0; j < p.n_lr; ++j, ++il) {
+            if (!wait_or_abort(lr_empty, (il & 1) ^ 1, abort_flag, p.err)) goto producer_done;
+            mbar_arrive_expect_tx(lr_full, L::LR_A + L::LR_B);
+            const uint32_t dst = sbase + L::OFF_LR;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              tma_load_2d(dst + c * (BM * 16), &tm_z, 32 * j + 8 * c, m0, lr_full);
+              tma_load_2d(dst + L::LR_A + c * (BN * 16), &tm_l2, 32 * j + 8 * c, n0, lr_full);
+            }
+          }
         }
+      producer_done:
+        // every issued copy has landed before the CTA exits
+        for (uint32_t k = (it > NP ? it - NP : 0); k < it; ++k)
+          mbar_wait_bounded(pk_full(k % NP), (k / NP) & 1, LIMIT_NS);
+        if (il > 0) mbar_wait_bounded(lr_full, (il - 1) & 1, LIMIT_NS);
       }
-    producer_done:
-      // drain: every issued load has landed before the CTA exits
-      for (uint32_t k = (it > NP ? it - NP : 0); k < it; ++k)
-        mbar_wait_bounded(pk_full(k % NP), (k / NP) & 1, LIMIT_NS);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t id_i8 = idesc_i8(BM, BN), id_bf = idesc_bf16(BM, BN);
-      uint32_t ite = 0, tb = 0;
-      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-        for (int g = 0; g < G + (p.n_lr > 0 ? 1 : 0); ++g) {
-          const int b = tb & 1;
-          if (!wait_or_abort(tm_empty(b), ((tb >> 1) & 1) ^ 1, abort_flag, p.err)) goto mma_done;
-          const uint32_t d = tmem + b * BN;
-          const int nsub = (g < G) ? 1 : p.n_lr;
-          for (int j = 0; j < nsub; ++j, ++ite) {
-            const int s = ite % NE;
-            if (!wait_or_abort(ex_full(s), (ite / NE) & 1, abort_flag, p.err)) goto mma_done;
-            tc_fence_after();
-            const uint32_t ea = sbase + L::OFF_EX + s * L::EX_STAGE;
-            const uint64_t ad = sdesc_kmajor_noswizzle(ea, 128, 512);
-            const uint64_t bd = sdesc_kmajor_noswizzle(ea + L::EX_A, 128, 512);
+      __syncwarp();
+    } else if (warp == 1) {
+      // ---------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const uint32_t id_i8 = idesc_i8(BM, BN), id_bf = idesc_bf16(BM, BN);
+        uint32_t ite = 0, tb = 0, il = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+          for (int g = 0; g < G + (p.n_lr > 0 ? 1 : 0); ++g) {
+            const int b = tb & 1;
+            if (!wait_or_abort(tm_empty(b), ((tb >> 1) & 1) ^ 1, abort_flag, p.err)) goto mma_done;
+            const uint32_t d = tmem + b * BN;
             if (g < G) {
+              const int s = ite % NE;
+              if (!wait_or_abort(ex_full(s), (ite / NE) & 1, abort_flag, p.err)) goto mma_done;
+              tc_fence_after();
+              const uint32_t ea = sbase + L::OFF_EX + s * L::EX_STAGE;
+              const uint64_t ad = sdesc_kmajor_noswizzle(ea, 128, 512);
+              const uint64_t bd = sdesc_kmajor_noswizzle(ea + L::EX_A, 128, 512);
               mma_i8(d, ad, bd, id_i8, 0u);
               mma_i8(d, ad + 16, bd + 16, id_i8, 1u);
+              mma_commit(ex_empty(s));
+              ++ite;
             } else {
-              mma_bf16(d, ad, bd, id_bf, j > 0 ? 1u : 0u);
-              mma_bf16(d, ad + 16, bd + 16, id_bf, 1u);
-            }
-            mma_commit(ex_empty(s));
-          }
-          mma_commit(tm_full(b));
-          ++tb;
-        }
-      }
-    mma_done:;
-    }
-    __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------------------ expanders
-    const int et = tid - 64;
-    uint32_t itp = 0, ite = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-      const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
-      const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
-      for (int g = 0; g < G + p.n_lr; ++g, ++ite) {
-        const int se = ite % NE;
-        if (!wait_or_abort(ex_empty(se), ((ite / NE) & 1) ^ 1, abort_flag, p.err)) goto exp_done;
-        uint8_t* ea = smem + L::OFF_EX + se * L::EX_STAGE;
-        uint8_t* eb = ea + L::EX_A;
-        if (g < G) {
-          const int sp = itp % NP;
-          if (!wait_or_abort(pk_full(sp), (itp / NP) & 1, abort_flag, p.err)) goto exp_done;
-          const uint8_t* pa = smem + L::OFF_PK + sp * L::PK_STAGE;
-          const uint8_t* pb = pa + L::PK_A;
-#pragma unroll
-          for (int i = et; i < BM * 2; i += N_EXP) expand16(pa + i * 16, ea, i >> 1, i & 1);
-#pragma unroll
-          for (int i = et; i < BN * 2; i += N_EXP) expand16(pb + i * 16, eb, i >> 1, i & 1);
-          mbar_arrive(pk_empty(sp));
-          ++itp;
-        } else {
-          // low-rank slice j: Z[:, 32j:32j+32] and L2T[:, 32j:32j+32] (bf16)
-          const int k0 = (g - G) * 32;
-          for (int i = et; i < BM * 4; i += N_EXP) {
-            const int r = i >> 2, c = i & 3, row = m0 + r, col = k0 + 8 * c;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (row < p.M) {
-              const uint16_t* src = p.Z + (size_t)row * p.rank + col;
-              if ((p.rank & 7) == 0) {
-                if (col < p.rank) v = __ldg(reinterpret_cast<const uint4*>(src));
-              } else {
-                uint16_t e[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) e[q] = (col + q < p.rank) ? src[q] : (uint16_t)0;
-                v.x = e[0] | ((uint32_t)e[1] << 16); v.y = e[2] | ((uint32_t)e[3] << 16);
-                v.z = e[4] | ((uint32_t)e[5] << 16); v.w = e[6] | ((uint32_t)e[7] << 16);
+              for (int j = 0; j < p.n_lr; ++j, ++il) {
+                if (!wait_or_abort(lr_full, il & 1, abort_flag, p.err)) goto mma_done;
+                tc_fence_after();
+                const uint32_t la = sbase + L::OFF_LR;
+                // chunk c of the slice at c * rows * 16 bytes, row r at r * 16
+                const uint64_t ad = sdesc_kmajor_noswizzle(la, BM * 16, 128);
+                const uint64_t bd = sdesc_kmajor_noswizzle(la + L::LR_A, BN * 16, 128);
+                mma_bf16(d, ad, bd, id_bf, j > 0 ? 1u : 0u);
+                mma_bf16(d, ad + ((2 * BM * 16) >> 4), bd + ((2 * BN * 16) >> 4), id_bf, 1u);
+                mma_commit(lr_empty);
               }
             }
-            *reinterpret_cast<uint4*>(ea + (r >> 3) * 512 + c * 128 + (r & 7) * 16) = v;
-          }
-          for (int i = et; i < BN * 4; i += N_EXP) {
-            const int r = i >> 2, c = i & 3;
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-                p.L2T + (size_t)(n0 + r) * p.rank_pad32 + k0 + 8 * c));
-            *reinterpret_cast<uint4*>(eb + (r >> 3) * 512 + c * 128 + (r & 7) * 16) = v;
+            mma_commit(tm_full(b));
+            ++tb;
           }
         }
-        fence_proxy_async_smem();
-        mbar_arrive(ex_full(se));
+      mma_done:;
       }
+      __syncwarp();
+    } else {
+      // ---------------------------------------------------- expanders
+      const int et = tid - EXP_WARP0 * 32;
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+        for (int g = 0; g < G; ++g, ++it) {
+          const int se = it % NE, sp = it % NP;
+          if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err)) goto exp_done;
+          if (!wait_or_abort(pk_full(sp), (it / NP) & 1, abort_flag, p.err)) goto exp_done;
+          uint8_t* ea = smem + L::OFF_EX + se * L::EX_STAGE;
+          const uint8_t* pa = smem + L::OFF_PK + sp * L::PK_STAGE;
+#pragma unroll 2
+          for (int i = et; i < (BM + BN) * 2; i += N_EXP) {
+            if (i < BM * 2) expand16(pa + i * 16, ea, i >> 1, i & 1);
+            else expand16(pa + i * 16, ea + L::EX_A, (i - BM * 2) >> 1, i & 1);
+          }
+          mbar_arrive(pk_empty(sp));
+          fence_proxy_async_smem();
+          mbar_arrive(ex_full(se));
+        }
+      }
+    exp_done:;
     }
-  exp_done:;
   } else {
+    regs_inc<REG_HI>();
     // ------------------------------------------------------ rescale + epilogue
-    const int rw = warp - 4, q = warp & 3, h = rw >> 2;
+    const int rw = warp - RES_WARP0, q = warp & 3, h = rw >> 2;
     float* swb = reinterpret_cast<float*>(smem + L::OFF_SW) + rw * 2 * CW;
     uint8_t* ystage = smem + L::OFF_Y + rw * L::Y_WARP;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
@@ -292,10 +303,9 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
       const int row = m0 + 32 * q + lane;
       const int ncol0 = n0 + h * CW;           // first column of this warp
-      float acc[CW];
+      float2 acc2[CW / 2];
 #pragma unroll
-      for (int j = 0; j < CW; ++j) acc[j] = 0.0f;
-      // scales of group 0
+      for (int j = 0; j < CW / 2; ++j) acc2[j] = make_float2(0.0f, 0.0f);
       constexpr int PER = CW / 32;             // sw values loaded per lane
       float sx_n = (MODE == 0 && row < p.M) ? __ldg(p.s_x + row) : 0.0f;
       float sw_n[PER];
@@ -322,16 +332,32 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         if (!wait_or_abort(tm_full(b), (tb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
+        if (MODE == 0) {
+          const float2 sx2 = make_float2(sx, sx);
+          const uint32_t swa = smem_u32(swg);
 #pragma unroll
-        for (int c = 0; c < CW / 16; ++c) {
-          uint32_t r[16];
-          tmem_ld16(ta + 16 * c, r);
-          tmem_wait_ld();
-          if (MODE == 0) {
+          for (int c = 0; c < CW / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(ta + 32 * c, r);
+            tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              acc[16 * c + j] = fmaf(sx * swg[16 * c + j], (float)(int32_t)r[j], acc[16 * c + j]);
-          } else {
+            for (int j = 0; j < 32; j += 4) {
+              const float4 s4 = lds128(swa + 4u * (32 * c + j));
+              const float2 sc0 = __fmul2_rn(sx2, make_float2(s4.x, s4.y));
+              const float2 sc1 = __fmul2_rn(sx2, make_float2(s4.z, s4.w));
+              const int e = (32 * c + j) >> 1;
+              acc2[e] = __ffma2_rn(sc0, make_float2((float)(int32_t)r[j], (float)(int32_t)r[j + 1]),
+                                   acc2[e]);
+              acc2[e + 1] = __ffma2_rn(
+                  sc1, make_float2((float)(int32_t)r[j + 2], (float)(int32_t)r[j + 3]), acc2[e + 1]);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < CW / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld16(ta + 16 * c, r);
+            tmem_wait_ld();
             const int i = row - p.row0;
             if (i >= 0 && i < p.nrows) {
 #pragma unroll
@@ -354,12 +380,15 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
 #pragma unroll
-        for (int c = 0; c < CW / 16; ++c) {
-          uint32_t r[16];
-          tmem_ld16(ta + 16 * c, r);
+        for (int c = 0; c < CW / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(ta + 32 * c, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) acc[16 * c + j] += __uint_as_float(r[j]);
+          for (int j = 0; j < 32; j += 2) {
+            const int e = (32 * c + j) >> 1;
+            acc2[e] = __fadd2_rn(acc2[e], make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])));
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -384,7 +413,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int j = box * 64 + ch * 8 + e;
-            float y = acc[j] + bb[j];
+            float y = ((j & 1) ? acc2[j >> 1].y : acc2[j >> 1].x) + bb[j];
             if (p.epilogue == SVDQ_EPI_GELU) y = gelu_f(y);
             v[e] = y;
           }
@@ -458,10 +487,15 @@ int num_sms() {
 
 template <int BN, int MODE>
 cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtensorMap& tb,
-                      const CUtensorMap& ty, LinArgs a, int tiles_m, cudaStream_t st) {
+                      const CUtensorMap& ty, const CUtensorMap& tz, const CUtensorMap& tl,
+                      LinArgs a, int tiles_m, cudaStream_t st) {
   using L = Lay<BN>;
   static bool attr = false;
   if (!attr) {
+    cudaFuncAttributes fa;
+    cudaError_t e0 = cudaFuncGetAttributes(&fa, linear_ws_kernel<BN, MODE>);
+    if (e0 != cudaSuccess) return e0;
+    if (fa.numRegs < REG_NEED) return cudaErrorInvalidConfiguration;  // split would not fit
     cudaError_t e = cudaFuncSetAttribute(linear_ws_kernel<BN, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
@@ -469,7 +503,7 @@ cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtens
   }
   a.num_tiles = tiles_m * a.tiles_n;
   const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
-  linear_ws_kernel<BN, MODE><<<grid, THREADS, L::ALLOC, st>>>(ta, tb, ty, a);
+  linear_ws_kernel<BN, MODE><<<grid, THREADS, L::ALLOC, st>>>(ta, tb, ty, tz, tl, a);
   return cudaGetLastError();
 }
 
@@ -485,13 +519,21 @@ cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const
                           const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
                           cudaStream_t st) {
   const int BN = pick_bn(w->N);
-  CUtensorMap ta, tb, ty;
+  CUtensorMap ta, tb, ty, tz, tl;
   if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 32, BM,
                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 32, BN,
                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  tz = ta;
+  tl = ta;
+  if (w->rank > 0 &&
+      (!make_map(&tz, Z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank, M, (uint64_t)w->rank * 2, 8,
+                 BM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+       !make_map(&tl, w->d_L2T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank_pad32, w->N,
+                 (uint64_t)w->rank_pad32 * 2, 8, BN, CU_TENSOR_MAP_SWIZZLE_NONE)))
     return cudaErrorInvalidValue;
   LinArgs a{};
   a.s_x = s_x; a.s_w = w->d_sw; a.Z = Z; a.L2T = w->d_L2T; a.bias = w->d_bias;
@@ -502,8 +544,8 @@ cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const
   a.tile_m0 = 0; a.tile_n0 = 0;
   a.err = w->d_err;
   const int tiles_m = (M + BM - 1) / BM;
-  return BN == 256 ? launch_ws<256, 0>(w, ta, tb, ty, a, tiles_m, st)
-                   : launch_ws<128, 0>(w, ta, tb, ty, a, tiles_m, st);
+  return BN == 256 ? launch_ws<256, 0>(w, ta, tb, ty, tz, tl, a, tiles_m, st)
+                   : launch_ws<128, 0>(w, ta, tb, ty, tz, tl, a, tiles_m, st);
 }
 
 cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int row0,
@@ -523,8 +565,8 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
   const int tm0 = row0 / BM, tm1 = (row0 + nrows - 1) / BM;
   const int tn0 = col0 / BN, tn1 = (col0 + ncols - 1) / BN;
   a.tile_m0 = tm0; a.tile_n0 = tn0; a.tiles_n = tn1 - tn0 + 1;
-  return BN == 256 ? launch_ws<256, 1>(w, ta, tb, ta, a, tm1 - tm0 + 1, st)
-                   : launch_ws<128, 1>(w, ta, tb, ta, a, tm1 - tm0 + 1, st);
+  return BN == 256 ? launch_ws<256, 1>(w, ta, tb, ta, ta, ta, a, tm1 - tm0 + 1, st)
+                   : launch_ws<128, 1>(w, ta, tb, ta, ta, ta, a, tm1 - tm0 + 1, st);
 }
 
 }  // namespace svdq

@@ -167,7 +167,7 @@ static svdq_status pack_impl(int K, int N, int rank, int group, const uint16_t* 
   if (group != SVDQ_GROUP) return SVDQ_ERR_UNSUPPORTED;
   if (K < SVDQ_GROUP || N < 1 || K % SVDQ_GROUP) return SVDQ_ERR_SHAPE;
   if (rank < 0 || lora_rank < 0 || rank > (K < N ? K : N)) return SVDQ_ERR_INVALID_ARG;
-  if (rank + lora_rank > SVDQ_MAX_RANK) return SVDQ_ERR_UNSUPPORTED;
+  if (rank + lora_rank > SVDQ_MAX_RANK || (rank + lora_rank) % 8 != 0) return SVDQ_ERR_UNSUPPORTED;
   if (lora_rank > 0 && (!lora_A || !lora_B)) return SVDQ_ERR_INVALID_ARG;
   if (!(alpha > 0.0 && alpha < 1.0)) return SVDQ_ERR_INVALID_ARG;
   if (!std::isfinite(lora_scale)) return SVDQ_ERR_NUMERIC;
@@ -348,7 +348,7 @@ svdq_status svdq_weights_load(const char* path, cudaStream_t stream, svdq_weight
   }
   const int K = hdr[0], N = hdr[1], r = hdr[2], lr = hdr[3];
   if (hdr[4] != SVDQ_GROUP || K < 64 || K % 64 || N < 1 || r < 0 || lr < 0 ||
-      r + lr > SVDQ_MAX_RANK || K > (1 << 20) || N > (1 << 20)) {
+      r + lr > SVDQ_MAX_RANK || (r + lr) % 8 != 0 || K > (1 << 20) || N > (1 << 20)) {
     std::fclose(f);
     return SVDQ_ERR_IO;
   }
