@@ -2,11 +2,11 @@
 // 6.1, Algorithm 2 steps 4-8; eq. 7), warp-specialised for sm_100a.
 //
 // sm_100a tensor cores have no 4-bit integer kind, so the packed codes are
-// streamed by TMA into shared memory, expanded there to int8 and multiplied
-// with tcgen05.mma.kind::i8 into int32 TMEM accumulators, one per group of
-// 64 K.  Every group's int32 partial P_g is read back with tcgen05.ld and
-// folded into an fp32 register accumulator with the group's scales
-// s_x[g][m] * s_w[g][n].  The low-rank term Z L2 is one more tensor-core
+// streamed by TMA into shared memory, expanded there to int8 (as 16 q, three
+// integer ops per 8 codes) and multiplied with tcgen05.mma.kind::i8 into
+// int32 TMEM accumulators, one per group of 64 K.  Every group's int32
+// partial 256 P_g is read back with tcgen05.ld and folded into an fp32
+// register accumulator with the group's scales 2^-8 s_x[g][m] s_w[g][n].  The low-rank term Z L2 is one more tensor-core
 // stage (kind::f16, bf16 operands, fp32 in TMEM) added unscaled; then the
 // bias (and GELU) are applied and Y is written once, as bf16, by TMA.
 //
@@ -44,7 +44,6 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int NP = 4;            // packed-code stages
-constexpr int NE = 2;            // expanded-operand stages
 constexpr int THREADS = 512;
 constexpr int EXP_WARP0 = 2;     // expanders: warps 2-7
 constexpr int N_EXP = 192;
@@ -77,6 +76,8 @@ struct LinArgs {
 
 template <int BN>
 struct Lay {
+  static constexpr int NB = 512 / BN;                    // TMEM accumulator buffers
+  static constexpr int NE = BN == 256 ? 2 : 4;           // expanded-operand stages
   static constexpr int CW = BN / 2;                      // columns per rescale warp
   static constexpr int Y_BOX = 32 * 64 * 2;              // 32 rows x 64 bf16 (4 KB)
   static constexpr int Y_WARP = (CW / 64) * Y_BOX;
@@ -89,9 +90,9 @@ struct Lay {
   static constexpr int OFF_LR = OFF_EX + NE * EX_STAGE;
   static constexpr int OFF_SW = OFF_LR + LR_A + LR_B;
   static constexpr int OFF_BAR = OFF_SW + N_RES_WARPS * 2 * CW * 4;
-  // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[2],
-  // tm_empty[2], lr_full, lr_empty
-  static constexpr int N_BARS = 2 * NP + 2 * NE + 6;
+  // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[NB],
+  // tm_empty[NB], lr_full, lr_empty
+  static constexpr int N_BARS = 2 * NP + 2 * NE + 2 * NB + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;              // slack for 1024-B alignment
@@ -115,18 +116,22 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
 }
 
 // 16 packed bytes (32 codes of one row) -> two 16-byte core-matrix rows.
+// Each code q becomes the int8 16*q: the high nibble of a byte is already
+// 16*q in place (mask), the low nibble is shifted up by 4 (shift + mask).
+// Products are 256 q_x q_w, so the int32 group sum is 256 P_g (|256 P_g| <=
+// 2^20, exact); the factor 2^-8 is folded into the scale.
 __device__ __forceinline__ void expand16(const uint8_t* src, uint8_t* dst_base, int row,
                                          int half) {
   const uint4 p = *reinterpret_cast<const uint4*>(src);
   uint4 o0, o1;
-  o0.x = sext_nibbles(p.x & 0x0F0F0F0Fu);
-  o0.y = sext_nibbles((p.x >> 4) & 0x0F0F0F0Fu);
-  o0.z = sext_nibbles(p.y & 0x0F0F0F0Fu);
-  o0.w = sext_nibbles((p.y >> 4) & 0x0F0F0F0Fu);
-  o1.x = sext_nibbles(p.z & 0x0F0F0F0Fu);
-  o1.y = sext_nibbles((p.z >> 4) & 0x0F0F0F0Fu);
-  o1.z = sext_nibbles(p.w & 0x0F0F0F0Fu);
-  o1.w = sext_nibbles((p.w >> 4) & 0x0F0F0F0Fu);
+  o0.x = (p.x << 4) & 0xF0F0F0F0u;
+  o0.y = p.x & 0xF0F0F0F0u;
+  o0.z = (p.y << 4) & 0xF0F0F0F0u;
+  o0.w = p.y & 0xF0F0F0F0u;
+  o1.x = (p.z << 4) & 0xF0F0F0F0u;
+  o1.y = p.z & 0xF0F0F0F0u;
+  o1.z = (p.w << 4) & 0xF0F0F0F0u;
+  o1.w = p.w & 0xF0F0F0F0u;
   uint8_t* d = dst_base + (row >> 3) * 512 + (row & 7) * 16 + half * 256;
   *reinterpret_cast<uint4*>(d) = o0;
   *reinterpret_cast<uint4*>(d + 128) = o1;
@@ -153,6 +158,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_l2, const LinArgs p) {
   using L = Lay<BN>;
   constexpr int CW = L::CW;
+  constexpr int NE = L::NE;
+  constexpr int NB = L::NB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -163,9 +170,9 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
   auto ex_full = [&](int s) { return bar0 + 8u * (2 * NP + s); };
   auto ex_empty = [&](int s) { return bar0 + 8u * (2 * NP + NE + s); };
   auto tm_full = [&](int b) { return bar0 + 8u * (2 * NP + 2 * NE + b); };
-  auto tm_empty = [&](int b) { return bar0 + 8u * (2 * NP + 2 * NE + 2 + b); };
-  const uint32_t lr_full = bar0 + 8u * (2 * NP + 2 * NE + 4);
-  const uint32_t lr_empty = bar0 + 8u * (2 * NP + 2 * NE + 5);
+  auto tm_empty = [&](int b) { return bar0 + 8u * (2 * NP + 2 * NE + NB + b); };
+  const uint32_t lr_full = bar0 + 8u * (2 * NP + 2 * NE + 2 * NB);
+  const uint32_t lr_empty = bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -175,14 +182,14 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
   if (tid == 0) {
     for (int s = 0; s < NP; ++s) { mbar_init(pk_full(s), 1); mbar_init(pk_empty(s), N_EXP); }
     for (int s = 0; s < NE; ++s) { mbar_init(ex_full(s), N_EXP); mbar_init(ex_empty(s), 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(tm_full(b), 1); mbar_init(tm_empty(b), N_RES_WARPS); }
+    for (int b = 0; b < NB; ++b) { mbar_init(tm_full(b), 1); mbar_init(tm_empty(b), N_RES_WARPS); }
     mbar_init(lr_full, 1);
     mbar_init(lr_empty, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 2 * BN);
+    tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -232,8 +239,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         uint32_t ite = 0, tb = 0, il = 0;
         for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
           for (int g = 0; g < G + (p.n_lr > 0 ? 1 : 0); ++g) {
-            const int b = tb & 1;
-            if (!wait_or_abort(tm_empty(b), ((tb >> 1) & 1) ^ 1, abort_flag, p.err)) goto mma_done;
+            const int b = tb % NB;
+            if (!wait_or_abort(tm_empty(b), ((tb / NB) & 1) ^ 1, abort_flag, p.err)) goto mma_done;
             const uint32_t d = tmem + b * BN;
             if (g < G) {
               const int s = ite % NE;
@@ -315,7 +322,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         sw_n[e] = (MODE == 0 && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
       }
       for (int g = 0; g < G; ++g, ++tb) {
-        const float sx = sx_n;
+        const float sx = sx_n * 0.00390625f;   // 2^-8 (exact)
         float* swg = swb + (g & 1) * CW;
 #pragma unroll
         for (int e = 0; e < PER; ++e) swg[lane * PER + e] = sw_n[e];
@@ -328,8 +335,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             sw_n[e] = (n < p.N) ? __ldg(p.s_w + (size_t)(g + 1) * p.N + n) : 0.0f;
           }
         }
-        const int b = tb & 1;
-        if (!wait_or_abort(tm_full(b), (tb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        const int b = tb % NB;
+        if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
         if (MODE == 0) {
@@ -364,7 +371,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               for (int j = 0; j < 16; ++j) {
                 const int jj = ncol0 + 16 * c + j - p.col0;
                 if (jj >= 0 && jj < p.ncols)
-                  p.P[((size_t)g * p.nrows + i) * p.ncols + jj] = (int32_t)r[j];
+                  p.P[((size_t)g * p.nrows + i) * p.ncols + jj] = ((int32_t)r[j]) >> 8;
               }
             }
           }
@@ -375,8 +382,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       }
       if (!ok || MODE != 0) continue;
       if (p.n_lr > 0) {
-        const int b = tb & 1;
-        if (!wait_or_abort(tm_full(b), (tb >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        const int b = tb % NB;
+        if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
 #pragma unroll
@@ -442,7 +449,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * BN);
+    tmem_dealloc(tmem, 512);
   }
 }
 
