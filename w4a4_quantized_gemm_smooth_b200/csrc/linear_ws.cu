@@ -98,19 +98,20 @@ struct Lay {
   static constexpr int ALLOC = BYTES + 1024;              // slack for 1024-B alignment
 };
 
+// Bounded wait: the thread sleeps in try_wait (up to 20 us per call) until
+// the phase completes; after LIMIT_NS, or when another thread of the CTA has
+// given up, it returns false.
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
                                               volatile int* abort_flag, int* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 63u) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > LIMIT_NS) {
-        *abort_flag = 1;
-        atomicExch(err, SVDQ_DEVERR_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > LIMIT_NS) {
+      *abort_flag = 1;
+      atomicExch(err, SVDQ_DEVERR_TIMEOUT);
+      return false;
     }
   }
 }
@@ -340,24 +341,29 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
         if (MODE == 0) {
+          // 16-column TMEM loads, double-buffered: the load of chunk c+1 is
+          // in flight while chunk c is rescaled (wait::ld waits for all).
           const float2 sx2 = make_float2(sx, sx);
           const uint32_t swa = smem_u32(swg);
+          uint32_t rb[2][16];
+          tmem_ld16(ta, rb[0]);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < CW / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(ta + 32 * c, r);
-            tmem_wait_ld();
+          for (int c = 0; c < CW / 16; ++c) {
+            if (c + 1 < CW / 16) tmem_ld16(ta + 16 * (c + 1), rb[(c + 1) & 1]);
+            const uint32_t* r = rb[c & 1];
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 s4 = lds128(swa + 4u * (32 * c + j));
+            for (int j = 0; j < 16; j += 4) {
+              const float4 s4 = lds128(swa + 4u * (16 * c + j));
               const float2 sc0 = __fmul2_rn(sx2, make_float2(s4.x, s4.y));
               const float2 sc1 = __fmul2_rn(sx2, make_float2(s4.z, s4.w));
-              const int e = (32 * c + j) >> 1;
+              const int e = (16 * c + j) >> 1;
               acc2[e] = __ffma2_rn(sc0, make_float2((float)(int32_t)r[j], (float)(int32_t)r[j + 1]),
                                    acc2[e]);
               acc2[e + 1] = __ffma2_rn(
                   sc1, make_float2((float)(int32_t)r[j + 2], (float)(int32_t)r[j + 3]), acc2[e + 1]);
             }
+            if (c + 1 < CW / 16) tmem_wait_ld();
           }
         } else {
 #pragma unroll 1
@@ -386,16 +392,19 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
+        uint32_t rb[2][16];
+        tmem_ld16(ta, rb[0]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < CW / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(ta + 32 * c, r);
-          tmem_wait_ld();
+        for (int c = 0; c < CW / 16; ++c) {
+          if (c + 1 < CW / 16) tmem_ld16(ta + 16 * (c + 1), rb[(c + 1) & 1]);
+          const uint32_t* r = rb[c & 1];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int e = (32 * c + j) >> 1;
+          for (int j = 0; j < 16; j += 2) {
+            const int e = (16 * c + j) >> 1;
             acc2[e] = __fadd2_rn(acc2[e], make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])));
           }
+          if (c + 1 < CW / 16) tmem_wait_ld();
         }
         tc_fence_before();
         __syncwarp();

@@ -35,6 +35,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_try_wait, but lets the hardware suspend the thread for up to
+// `hint_ns` while the phase is incomplete instead of returning at once, so a
+// waiting warp does not spin on the issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete, for at most
 // `limit_ns` nanoseconds.  Returns false on timeout (the caller reports it).
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity,
