@@ -4,9 +4,14 @@
 // sm_100a tensor cores have no 4-bit integer kind, so the packed codes are
 // streamed by TMA into shared memory, expanded there to int8 (as 16 q, three
 // integer ops per 8 codes) and multiplied with tcgen05.mma.kind::i8 into
-// int32 TMEM accumulators, one per group of 64 K.  Every group's int32
-// partial 256 P_g is read back with tcgen05.ld and folded into an fp32
-// register accumulator with the group's scales 2^-8 s_x[g][m] s_w[g][n].  The low-rank term Z L2 is one more tensor-core
+// int32 TMEM accumulators, one per group of 64 K.  Each group's accumulator
+// is first set by a bf16 MMA (ones x 786432) to the fp32 value 12582912,
+// whose bit pattern is the int32 0x4B400000; the int8 MMAs then add 256 P_g
+// to those bits, so the word read back is exactly the float
+// 12582912 + 256 P_g (|256 P_g| <= 2^20).  The rescale subtracts the
+// constant (exact) instead of converting int32 -> fp32, and folds the
+// result into an fp32 register accumulator with the scales
+// 2^-8 s_x[g][m] s_w[g][n].  The low-rank term Z L2 is one more tensor-core
 // stage (kind::f16, bf16 operands, fp32 in TMEM) added unscaled; then the
 // bias (and GELU) are applied and Y is written once, as bf16, by TMA.
 //
@@ -50,6 +55,10 @@ constexpr int N_EXP = 192;
 constexpr int RES_WARP0 = 8;     // rescale / epilogue: warps 8-15
 constexpr int N_RES_WARPS = 8;
 constexpr uint64_t LIMIT_NS = 2000000000ull;
+constexpr uint32_t MAGIC_BITS = 0x4B400000u;   // bits of 12582912.0f = 1.5 * 2^23
+constexpr float MAGIC_F = 12582912.0f;
+constexpr uint16_t BF16_ONE = 0x3F80;          // 1.0
+constexpr uint16_t BF16_MAGIC16 = 0x4940;      // 786432 = 1.5 * 2^19; 16 of them make MAGIC_F
 // Register split after launch: the first two warpgroups (producer, MMA,
 // expanders) give registers to the two rescale warpgroups.
 // 256 * REG_LO + 256 * REG_HI
@@ -88,8 +97,19 @@ struct Lay {
   static constexpr int OFF_EX = OFF_PK + NP * PK_STAGE;
   static constexpr int LR_A = BM * 64, LR_B = BN * 64;     // 4 chunks x rows x 16 B
   static constexpr int OFF_LR = OFF_EX + NE * EX_STAGE;
-  static constexpr int OFF_SW = OFF_LR + LR_A + LR_B;
-  static constexpr int OFF_BAR = OFF_SW + N_RES_WARPS * 2 * CW * 4;
+  // per-group scales: ring of NP + NE + NB slots, each s_x[128] then s_w[BN],
+  // filled by the producer warp together with the packed codes.  The producer
+  // may write group j's slot once the expanders released packed stage j - NP,
+  // which (through the MMA and TMEM barriers) implies that the rescale of
+  // group j - NP - NE - NB, the slot's previous owner, has finished.
+  static constexpr int NS = NP + NE + NB;
+  static constexpr int SC_SLOT = (BM + BN) * 4;
+  static constexpr int OFF_SC = OFF_LR + LR_A + LR_B;
+  static constexpr int OFF_BIAS = OFF_SC + NS * SC_SLOT;   // per warp CW floats
+  // constant operands of the accumulator-initialising bf16 MMA (K = 16)
+  static constexpr int INIT_A = BM * 32, INIT_B = BN * 32;
+  static constexpr int OFF_INIT = OFF_BIAS + N_RES_WARPS * CW * 4;
+  static constexpr int OFF_BAR = OFF_INIT + INIT_A + INIT_B;
   // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[NB],
   // tm_empty[NB], lr_full, lr_empty
   static constexpr int N_BARS = 2 * NP + 2 * NE + 2 * NB + 2;
@@ -142,9 +162,10 @@ __device__ __forceinline__ float gelu_f(float y) {
   return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a)) |
-         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
+// Two floats -> packed bf16x2 bits (round to nearest even), x in the low half.
+__device__ __forceinline__ uint32_t bf16x2_bits(float2 v) {
+  const __nv_bfloat162 h = __float22bfloat162_rn(v);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // MODE 0: the layer (rescale, low-rank stage, epilogue, TMA store of Y).
@@ -189,6 +210,13 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     *abort_flag = 0;
     fence_mbarrier_init();
   }
+  {
+    uint32_t* ia = reinterpret_cast<uint32_t*>(smem + L::OFF_INIT);
+    const uint32_t one2 = (uint32_t)BF16_ONE * 0x10001u, mag2 = (uint32_t)BF16_MAGIC16 * 0x10001u;
+    for (int i = tid; i < (L::INIT_A + L::INIT_B) / 4; i += THREADS)
+      ia[i] = (i < L::INIT_A / 4) ? one2 : mag2;
+    fence_proxy_async_smem();
+  }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
@@ -202,21 +230,45 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     regs_dec<REG_LO>();
     if (warp == 0) {
       // ---------------------------------------------------- TMA producer
-      if (lane == 0) {
-        uint32_t it = 0, il = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-          const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
-          const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
-          for (int g = 0; g < G; ++g, ++it) {
-            const int s = it % NP;
-            if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err)) goto producer_done;
+      uint32_t it = 0, il = 0;
+      bool alive = true;
+      for (int t = blockIdx.x; t < p.num_tiles && alive; t += gridDim.x) {
+        const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
+        const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
+        for (int g = 0; g < G; ++g, ++it) {
+          const int s = it % NP;
+          if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
+          if (MODE == 0) {
+            // scales of this group: 4-byte async copies by all lanes, tracked
+            // by the stage's full barrier (raised before lane 0 arrives)
+            const uint32_t slot = sbase + L::OFF_SC + (it % L::NS) * L::SC_SLOT;
+#pragma unroll 4
+            for (int i = lane; i < BM + BN; i += 32) {
+              if (i < BM) {
+                const int row = m0 + i;
+                const bool in = row < p.M;
+                cp_async4(slot + 4 * i, p.s_x + (in ? (size_t)g * p.M + row : 0), in ? 4u : 0u);
+              } else {
+                const int n = n0 + i - BM;
+                const bool in = n < p.N;
+                cp_async4(slot + 4 * i, p.s_w + (in ? (size_t)g * p.N + n : 0), in ? 4u : 0u);
+              }
+            }
+            cp_async_mbar_arrive(pk_full(s));
+            __syncwarp();
+          }
+          if (lane == 0) {
             mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE);
             const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
             tma_load_2d(dst, &tm_a, g * 32, m0, pk_full(s));
             tma_load_2d(dst + L::PK_A, &tm_b, g * 32, n0, pk_full(s));
           }
+          __syncwarp();
+        }
+        if (!alive) break;
+        if (lane == 0) {
           for (int j = 0; j < p.n_lr; ++j, ++il) {
-            if (!wait_or_abort(lr_empty, (il & 1) ^ 1, abort_flag, p.err)) goto producer_done;
+            if (!wait_or_abort(lr_empty, (il & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
             mbar_arrive_expect_tx(lr_full, L::LR_A + L::LR_B);
             const uint32_t dst = sbase + L::OFF_LR;
 #pragma unroll
@@ -226,17 +278,23 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             }
           }
         }
-      producer_done:
-        // every issued copy has landed before the CTA exits
+        alive = __shfl_sync(0xFFFFFFFFu, alive ? 1 : 0, 0) != 0;
+      }
+      // every issued copy has landed before the CTA exits
+      if (lane == 0) {
         for (uint32_t k = (it > NP ? it - NP : 0); k < it; ++k)
           mbar_wait_bounded(pk_full(k % NP), (k / NP) & 1, LIMIT_NS);
         if (il > 0) mbar_wait_bounded(lr_full, (il - 1) & 1, LIMIT_NS);
       }
+      cp_async_wait<0>();
       __syncwarp();
     } else if (warp == 1) {
       // ---------------------------------------------------- MMA issuer
       if (lane == 0) {
         const uint32_t id_i8 = idesc_i8(BM, BN), id_bf = idesc_bf16(BM, BN);
+        // the constant tiles hold one value each, so any layout descriptor works
+        const uint64_t init_ad = sdesc_kmajor_noswizzle(sbase + L::OFF_INIT, 128, 256);
+        const uint64_t init_bd = sdesc_kmajor_noswizzle(sbase + L::OFF_INIT + L::INIT_A, 128, 256);
         uint32_t ite = 0, tb = 0, il = 0;
         for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
           for (int g = 0; g < G + (p.n_lr > 0 ? 1 : 0); ++g) {
@@ -250,7 +308,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               const uint32_t ea = sbase + L::OFF_EX + s * L::EX_STAGE;
               const uint64_t ad = sdesc_kmajor_noswizzle(ea, 128, 512);
               const uint64_t bd = sdesc_kmajor_noswizzle(ea + L::EX_A, 128, 512);
-              mma_i8(d, ad, bd, id_i8, 0u);
+              mma_bf16(d, init_ad, init_bd, id_bf, 0u);   // D = 12582912.0f
+              mma_i8(d, ad, bd, id_i8, 1u);
               mma_i8(d, ad + 16, bd + 16, id_i8, 1u);
               mma_commit(ex_empty(s));
               ++ite;
@@ -301,10 +360,10 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     regs_inc<REG_HI>();
     // ------------------------------------------------------ rescale + epilogue
     const int rw = warp - RES_WARP0, q = warp & 3, h = rw >> 2;
-    float* swb = reinterpret_cast<float*>(smem + L::OFF_SW) + rw * 2 * CW;
+    float* bb = reinterpret_cast<float*>(smem + L::OFF_BIAS) + rw * CW;
     uint8_t* ystage = smem + L::OFF_Y + rw * L::Y_WARP;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    uint32_t tb = 0;
+    uint32_t tb = 0, gs = 0;                   // TMEM use counter, group counter
     bool ok = true;
     for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
       const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
@@ -314,28 +373,15 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       float2 acc2[CW / 2];
 #pragma unroll
       for (int j = 0; j < CW / 2; ++j) acc2[j] = make_float2(0.0f, 0.0f);
-      constexpr int PER = CW / 32;             // sw values loaded per lane
-      float sx_n = (MODE == 0 && row < p.M) ? __ldg(p.s_x + row) : 0.0f;
-      float sw_n[PER];
+      constexpr int PER = CW / 32;             // bias values loaded per lane
+      float bias_n[PER];                       // prefetched for the epilogue
 #pragma unroll
       for (int e = 0; e < PER; ++e) {
         const int n = ncol0 + lane * PER + e;
-        sw_n[e] = (MODE == 0 && n < p.N) ? __ldg(p.s_w + n) : 0.0f;
+        bias_n[e] = (MODE == 0 && n < p.N) ? __uint_as_float((uint32_t)__ldg(p.bias + n) << 16) : 0.0f;
       }
-      for (int g = 0; g < G; ++g, ++tb) {
-        const float sx = sx_n * 0.00390625f;   // 2^-8 (exact)
-        float* swg = swb + (g & 1) * CW;
-#pragma unroll
-        for (int e = 0; e < PER; ++e) swg[lane * PER + e] = sw_n[e];
-        __syncwarp();
-        if (MODE == 0 && g + 1 < G) {
-          sx_n = (row < p.M) ? __ldg(p.s_x + (size_t)(g + 1) * p.M + row) : 0.0f;
-#pragma unroll
-          for (int e = 0; e < PER; ++e) {
-            const int n = ncol0 + lane * PER + e;
-            sw_n[e] = (n < p.N) ? __ldg(p.s_w + (size_t)(g + 1) * p.N + n) : 0.0f;
-          }
-        }
+      for (int g = 0; g < G; ++g, ++tb, ++gs) {
+        const uint32_t slot = sbase + L::OFF_SC + (gs % L::NS) * L::SC_SLOT;
         const int b = tb % NB;
         if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
@@ -343,8 +389,10 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         if (MODE == 0) {
           // 16-column TMEM loads, double-buffered: the load of chunk c+1 is
           // in flight while chunk c is rescaled (wait::ld waits for all).
+          const float sx = lds32(slot + 4u * (32 * q + lane)) * 0.00390625f;   // 2^-8 (exact)
           const float2 sx2 = make_float2(sx, sx);
-          const uint32_t swa = smem_u32(swg);
+          const float2 nmag2 = make_float2(-MAGIC_F, -MAGIC_F);
+          const uint32_t swa = slot + 4u * (BM + h * CW);
           uint32_t rb[2][16];
           tmem_ld16(ta, rb[0]);
           tmem_wait_ld();
@@ -357,11 +405,12 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               const float4 s4 = lds128(swa + 4u * (16 * c + j));
               const float2 sc0 = __fmul2_rn(sx2, make_float2(s4.x, s4.y));
               const float2 sc1 = __fmul2_rn(sx2, make_float2(s4.z, s4.w));
+              // 256 P_g, exactly: the word is the float MAGIC_F + 256 P_g
+              const float2 u0 = __fadd2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), nmag2);
+              const float2 u1 = __fadd2_rn(make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])), nmag2);
               const int e = (16 * c + j) >> 1;
-              acc2[e] = __ffma2_rn(sc0, make_float2((float)(int32_t)r[j], (float)(int32_t)r[j + 1]),
-                                   acc2[e]);
-              acc2[e + 1] = __ffma2_rn(
-                  sc1, make_float2((float)(int32_t)r[j + 2], (float)(int32_t)r[j + 3]), acc2[e + 1]);
+              acc2[e] = __ffma2_rn(sc0, u0, acc2[e]);
+              acc2[e + 1] = __ffma2_rn(sc1, u1, acc2[e + 1]);
             }
             if (c + 1 < CW / 16) tmem_wait_ld();
           }
@@ -377,7 +426,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               for (int j = 0; j < 16; ++j) {
                 const int jj = ncol0 + 16 * c + j - p.col0;
                 if (jj >= 0 && jj < p.ncols)
-                  p.P[((size_t)g * p.nrows + i) * p.ncols + jj] = ((int32_t)r[j]) >> 8;
+                  p.P[((size_t)g * p.nrows + i) * p.ncols + jj] = ((int32_t)(r[j] - MAGIC_BITS)) >> 8;
               }
             }
           }
@@ -412,30 +461,31 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         ++tb;
       }
       // epilogue: bias, GELU, bf16, swizzled staging, TMA store
-      float* bb = swb + (G & 1) * CW;          // not the buffer read last
 #pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        const int n = ncol0 + lane * PER + e;
-        bb[lane * PER + e] = (n < p.N) ? __uint_as_float((uint32_t)__ldg(p.bias + n) << 16) : 0.0f;
-      }
+      for (int e = 0; e < PER; ++e) bb[lane * PER + e] = bias_n[e];
       if (lane == 0) tma_store_wait_read0();
       __syncwarp();
+      const uint32_t bba = smem_u32(bb);
+      const bool gelu = p.epilogue == SVDQ_EPI_GELU;
 #pragma unroll
       for (int box = 0; box < CW / 64; ++box) {
         uint8_t* yb = ystage + box * L::Y_BOX + lane * 128;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-          float v[8];
+          const int j0 = box * 64 + ch * 8;
+          const float4 b0 = lds128(bba + 4u * j0), b1 = lds128(bba + 4u * (j0 + 4));
+          float2 v[4];
+          v[0] = __fadd2_rn(acc2[j0 / 2 + 0], make_float2(b0.x, b0.y));
+          v[1] = __fadd2_rn(acc2[j0 / 2 + 1], make_float2(b0.z, b0.w));
+          v[2] = __fadd2_rn(acc2[j0 / 2 + 2], make_float2(b1.x, b1.y));
+          v[3] = __fadd2_rn(acc2[j0 / 2 + 3], make_float2(b1.z, b1.w));
+          if (gelu) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int j = box * 64 + ch * 8 + e;
-            float y = ((j & 1) ? acc2[j >> 1].y : acc2[j >> 1].x) + bb[j];
-            if (p.epilogue == SVDQ_EPI_GELU) y = gelu_f(y);
-            v[e] = y;
+            for (int e = 0; e < 4; ++e) v[e] = make_float2(gelu_f(v[e].x), gelu_f(v[e].y));
           }
           uint4 o;
-          o.x = pack_bf16x2(v[0], v[1]); o.y = pack_bf16x2(v[2], v[3]);
-          o.z = pack_bf16x2(v[4], v[5]); o.w = pack_bf16x2(v[6], v[7]);
+          o.x = bf16x2_bits(v[0]); o.y = bf16x2_bits(v[1]);
+          o.z = bf16x2_bits(v[2]); o.w = bf16x2_bits(v[3]);
           *reinterpret_cast<uint4*>(yb + ((ch ^ (lane & 7)) * 16)) = o;
         }
       }
