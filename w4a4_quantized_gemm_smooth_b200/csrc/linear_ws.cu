@@ -79,6 +79,7 @@ struct LinArgs {
   int epilogue;
   int tiles_n, num_tiles, tile_m0, tile_n0;
   int* err;
+  int sx_tma;              // 1: s_x rows are 16-byte aligned (M % 4 == 0), copy by TMA
   int32_t* P;              // partial dump (MODE 1)
   int row0, nrows, col0, ncols;
 };
@@ -177,7 +178,9 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_b,
                  const __grid_constant__ CUtensorMap tm_y,
                  const __grid_constant__ CUtensorMap tm_z,
-                 const __grid_constant__ CUtensorMap tm_l2, const LinArgs p) {
+                 const __grid_constant__ CUtensorMap tm_l2,
+                 const __grid_constant__ CUtensorMap tm_sx,
+                 const __grid_constant__ CUtensorMap tm_sw, const LinArgs p) {
   using L = Lay<BN>;
   constexpr int CW = L::CW;
   constexpr int NE = L::NE;
@@ -238,30 +241,30 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         for (int g = 0; g < G; ++g, ++it) {
           const int s = it % NP;
           if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
-          if (MODE == 0) {
-            // scales of this group: 4-byte async copies by all lanes, tracked
-            // by the stage's full barrier (raised before lane 0 arrives)
-            const uint32_t slot = sbase + L::OFF_SC + (it % L::NS) * L::SC_SLOT;
+          const uint32_t slot = sbase + L::OFF_SC + (it % L::NS) * L::SC_SLOT;
+          if (MODE == 0 && !p.sx_tma) {
+            // s_x rows not 16-byte aligned: 4-byte async copies by all lanes,
+            // tracked by the stage's full barrier (raised before lane 0 arrives)
 #pragma unroll 4
-            for (int i = lane; i < BM + BN; i += 32) {
-              if (i < BM) {
-                const int row = m0 + i;
-                const bool in = row < p.M;
-                cp_async4(slot + 4 * i, p.s_x + (in ? (size_t)g * p.M + row : 0), in ? 4u : 0u);
-              } else {
-                const int n = n0 + i - BM;
-                const bool in = n < p.N;
-                cp_async4(slot + 4 * i, p.s_w + (in ? (size_t)g * p.N + n : 0), in ? 4u : 0u);
-              }
+            for (int i = lane; i < BM; i += 32) {
+              const int row = m0 + i;
+              const bool in = row < p.M;
+              cp_async4(slot + 4 * i, p.s_x + (in ? (size_t)g * p.M + row : 0), in ? 4u : 0u);
             }
             cp_async_mbar_arrive(pk_full(s));
             __syncwarp();
           }
           if (lane == 0) {
-            mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE);
+            const uint32_t scale_bytes =
+                MODE == 0 ? (p.sx_tma ? BM * 4 : 0) + BN * 4 : 0;
+            mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE + scale_bytes);
             const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
             tma_load_2d(dst, &tm_a, g * 32, m0, pk_full(s));
             tma_load_2d(dst + L::PK_A, &tm_b, g * 32, n0, pk_full(s));
+            if (MODE == 0) {
+              if (p.sx_tma) tma_load_2d(slot, &tm_sx, m0, g, pk_full(s));
+              tma_load_2d(slot + 4 * BM, &tm_sw, n0, g, pk_full(s));
+            }
           }
           __syncwarp();
         }
@@ -554,7 +557,8 @@ int num_sms() {
 template <int BN, int MODE>
 cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtensorMap& tb,
                       const CUtensorMap& ty, const CUtensorMap& tz, const CUtensorMap& tl,
-                      LinArgs a, int tiles_m, cudaStream_t st) {
+                      const CUtensorMap& tsx, const CUtensorMap& tsw, LinArgs a, int tiles_m,
+                      cudaStream_t st) {
   using L = Lay<BN>;
   static bool attr = false;
   if (!attr) {
@@ -569,7 +573,7 @@ cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtens
   }
   a.num_tiles = tiles_m * a.tiles_n;
   const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
-  linear_ws_kernel<BN, MODE><<<grid, THREADS, L::ALLOC, st>>>(ta, tb, ty, tz, tl, a);
+  linear_ws_kernel<BN, MODE><<<grid, THREADS, L::ALLOC, st>>>(ta, tb, ty, tz, tl, tsx, tsw, a);
   return cudaGetLastError();
 }
 
@@ -595,6 +599,13 @@ cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const
     return cudaErrorInvalidValue;
   tz = ta;
   tl = ta;
+  CUtensorMap tsx = ta, tsw;
+  const bool sx_tma = (M % 4) == 0;
+  if ((sx_tma && !make_map(&tsx, s_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, w->G, (uint64_t)M * 4,
+                           BM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
+      !make_map(&tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N, w->G, (uint64_t)w->N4 * 4,
+                BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
   if (w->rank > 0 &&
       (!make_map(&tz, Z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank, M, (uint64_t)w->rank * 2, 8,
                  BM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
@@ -609,9 +620,10 @@ cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const
   a.tiles_n = (w->N + BN - 1) / BN;
   a.tile_m0 = 0; a.tile_n0 = 0;
   a.err = w->d_err;
+  a.sx_tma = sx_tma ? 1 : 0;
   const int tiles_m = (M + BM - 1) / BM;
-  return BN == 256 ? launch_ws<256, 0>(w, ta, tb, ty, tz, tl, a, tiles_m, st)
-                   : launch_ws<128, 0>(w, ta, tb, ty, tz, tl, a, tiles_m, st);
+  return BN == 256 ? launch_ws<256, 0>(w, ta, tb, ty, tz, tl, tsx, tsw, a, tiles_m, st)
+                   : launch_ws<128, 0>(w, ta, tb, ty, tz, tl, tsx, tsw, a, tiles_m, st);
 }
 
 cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int row0,
@@ -631,8 +643,8 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
   const int tm0 = row0 / BM, tm1 = (row0 + nrows - 1) / BM;
   const int tn0 = col0 / BN, tn1 = (col0 + ncols - 1) / BN;
   a.tile_m0 = tm0; a.tile_n0 = tn0; a.tiles_n = tn1 - tn0 + 1;
-  return BN == 256 ? launch_ws<256, 1>(w, ta, tb, ta, ta, ta, a, tm1 - tm0 + 1, st)
-                   : launch_ws<128, 1>(w, ta, tb, ta, ta, ta, a, tm1 - tm0 + 1, st);
+  return BN == 256 ? launch_ws<256, 1>(w, ta, tb, ta, ta, ta, ta, ta, a, tm1 - tm0 + 1, st)
+                   : launch_ws<128, 1>(w, ta, tb, ta, ta, ta, ta, ta, a, tm1 - tm0 + 1, st);
 }
 
 }  // namespace svdq

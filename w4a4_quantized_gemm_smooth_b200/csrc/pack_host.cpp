@@ -111,7 +111,11 @@ svdq_status upload(svdq_weights* w, cudaStream_t st) {
   svdq_status s;
   if ((s = dev_alloc_copy(&w->d_inv_lambda, w->inv_lambda.data(), (size_t)K, st))) return s;
   if ((s = dev_alloc_copy(&w->d_wq, w->wq.data(), (size_t)N * K / 2, st))) return s;
-  if ((s = dev_alloc_copy(&w->d_sw, w->sw.data(), (size_t)G * N, st))) return s;
+  w->N4 = (N + 3) / 4 * 4;
+  std::vector<float> swp((size_t)G * w->N4, 0.0f);
+  for (int g = 0; g < G; ++g)
+    std::memcpy(&swp[(size_t)g * w->N4], &w->sw[(size_t)g * N], (size_t)N * 4);
+  if ((s = dev_alloc_copy(&w->d_sw, swp.data(), swp.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_L1T, L1T.data(), L1T.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_L2, L2p.data(), L2p.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_L2T, L2T.data(), L2T.size(), st))) return s;

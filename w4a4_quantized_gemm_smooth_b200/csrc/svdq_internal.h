@@ -15,11 +15,12 @@ struct svdq_weights {
   int rank_pad = 0;    // rank rounded up to a multiple of 16 (zero rows)
   int rank_pad32 = 0;  // rank rounded up to a multiple of 32
   int N_pad = 0;       // N rounded up to a multiple of 256
+  int N4 = 0;          // N rounded up to a multiple of 4 (row pitch of d_sw)
   int device = 0;
   // device copies (owned)
   float* d_inv_lambda = nullptr;   // [K]
   uint8_t* d_wq = nullptr;         // [N][K/2] packed residual codes
-  float* d_sw = nullptr;           // [G][N]
+  float* d_sw = nullptr;           // [G][N4] (N4 = N rounded up to 4, zero padded)
   uint16_t* d_L1T = nullptr;       // [rank_pad][K] bf16, transposed L1
   uint16_t* d_L2 = nullptr;        // [rank_pad][N] bf16
   uint16_t* d_L2T = nullptr;       // [N_pad][rank_pad32] bf16, transposed L2
