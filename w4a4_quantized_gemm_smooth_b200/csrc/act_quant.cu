@@ -3,9 +3,9 @@
 // (eq. 1) and, from the same tile, compute the 16-bit down-projection
 // Z = bf16(x~) L1 on the tensor cores (mma.sync bf16, fp32 accumulation).
 //
-// Layout: one CTA of 8 warps owns 32 consecutive tokens and walks K in
-// chunks of 256 channels.  TMA streams 32 x 256 bf16 tiles of X into a
-// 4-stage shared-memory ring (64 KB in flight per SM), so X is read from HBM
+// Layout: one CTA of 8 warps owns 16 consecutive tokens and walks K in
+// chunks of 256 channels (several CTAs per SM).  TMA streams 16 x 256 bf16
+// tiles of X into a 6-stage shared-memory ring, so X is read from HBM
 // exactly once with full-width transactions.  A warp reads one token's 256
 // channels from the ring (16 bytes per lane); the 8 lanes holding one group
 // of 64 find its absmax with three xor-shuffles.  bf16(x~) is staged in
@@ -26,33 +26,41 @@
 namespace svdq {
 namespace {
 
-constexpr int AQ_ROWS = 32;
+constexpr int AQ_ROWS = 16;
 constexpr int AQ_CH = 256;
 constexpr int AQ_THREADS = 256;
-constexpr int AQ_STAGES = 4;
-constexpr int AQ_STAGE_BYTES = AQ_ROWS * AQ_CH * 2;     // 16 KB
+constexpr int AQ_STAGES = 6;
+constexpr int AQ_STAGE_BYTES = AQ_ROWS * AQ_CH * 2;     // 8 KB
 constexpr uint64_t AQ_LIMIT_NS = 2000000000ull;
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+// Two floats -> packed bf16x2 bits (round to nearest even), a in the low half.
+__device__ __forceinline__ uint32_t bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
 
-// Round-half-even of the exact quotient x / s, clamped to [-8, 7]; s > 0.
+constexpr float RN_MAGIC = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer
+
+// Two's-complement nibble of round-half-even(x / s), clamped to [-8, 7]; s > 0.
 // `ss`, `rcp` are s (possibly scaled by 2^64 when s is tiny) and its
 // correctly rounded reciprocal; `scale` is the same power of two for x.
-__device__ __forceinline__ int quant_code(float x, float ss, float rcp, float scale) {
+// Branch-free: q0 = rne(x * rcp) by the magic-number add (|x/s| < 8, far
+// inside its exact range); the exact residual x - q0 s (an fma, exact here)
+// moves q0 by one where the rounded quotient crossed a half, and an exact
+// tie goes to the even neighbour.  The nibble is read from the low bits of
+// the magic-biased float, whose integer bits are 0x4B400000 + q.
+__device__ __forceinline__ uint32_t quant_nibble(float x, float ss, float rcp, float scale) {
   const float xx = __fmul_rn(x, scale);              // exact (power of two)
-  float q = rintf(__fmul_rn(xx, rcp));
+  const float b0 = __fadd_rn(__fmul_rn(xx, rcp), RN_MAGIC);
+  float q = __fsub_rn(b0, RN_MAGIC);                 // rne(xx * rcp)
   const float d2 = 2.0f * __fmaf_rn(-q, ss, xx);     // exact residual, doubled
-  if (d2 > ss) {
-    q += 1.0f;
-  } else if (d2 < -ss) {
-    q -= 1.0f;
-  } else if (fabsf(d2) == ss) {                      // exact tie: go to even
-    const int qi = (int)q;
-    if (qi & 1) q += (d2 > 0.0f) ? 1.0f : -1.0f;
-  }
-  q = fminf(fmaxf(q, -8.0f), 7.0f);
-  return (int)q;
+  const uint32_t odd = __float_as_uint(b0) & 1u;
+  float adj = (d2 > ss) ? 1.0f : ((d2 < -ss) ? -1.0f : 0.0f);
+  adj = (fabsf(d2) == ss && odd) ? copysignf(1.0f, d2) : adj;
+  q = fminf(fmaxf(__fadd_rn(q, adj), -8.0f), 7.0f);
+  return __float_as_uint(__fadd_rn(q, RN_MAGIC)) & 0xFu;
 }
 
 template <int NT>
@@ -80,9 +88,9 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
   const int G = K / 64;
   const int nchunks = (K + AQ_CH - 1) / AQ_CH;
 
-  float zacc[2][NT > 0 ? NT : 1][4];
+  float zacc[1][NT > 0 ? NT : 1][4];
 #pragma unroll
-  for (int a = 0; a < 2; ++a)
+  for (int a = 0; a < 1; ++a)
 #pragma unroll
     for (int b = 0; b < (NT > 0 ? NT : 1); ++b)
 #pragma unroll
@@ -111,10 +119,10 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
     }
     __syncthreads();
     if (abort_sh) break;
-    uint4 cur[4];
+    uint4 cur[2];
     const uint8_t* stage = ring + st * AQ_STAGE_BYTES;
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr)
+    for (int rr = 0; rr < 2; ++rr)
       cur[rr] = (l * 8 < box_cols)
                     ? *reinterpret_cast<const uint4*>(stage + (w + 8 * rr) * box_cols * 2 + l * 16)
                     : make_uint4(0u, 0u, 0u, 0u);
@@ -131,7 +139,7 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
       for (int j = 0; j < 8; ++j) il[j] = 0.0f;
     }
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
+    for (int rr = 0; rr < 2; ++rr) {
       const int lr = w + 8 * rr;
       const int row = row0 + lr;
       const uint32_t u[4] = {cur[rr].x, cur[rr].y, cur[rr].z, cur[rr].w};
@@ -155,28 +163,23 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
         const float ssc = __fmul_rn(s, scale);
         const float rcp = __frcp_rn(ssc);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          packed |= (uint32_t)(quant_code(xh[j], ssc, rcp, scale) & 0xF) << (4 * j);
+        for (int j = 0; j < 8; ++j) packed |= quant_nibble(xh[j], ssc, rcp, scale) << (4 * j);
       }
       if (colok && row < M)
         *reinterpret_cast<uint32_t*>(xq + (size_t)row * (K / 2) + col / 2) = packed;
       if ((l & 7) == 0) ss_tile[l >> 3][lr] = s;
       uint4 hv;
-      hv.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[0])) |
-             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[1])) << 16);
-      hv.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[2])) |
-             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[3])) << 16);
-      hv.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[4])) |
-             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[5])) << 16);
-      hv.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[6])) |
-             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[7])) << 16);
+      hv.x = bf16x2(xh[0], xh[1]);
+      hv.y = bf16x2(xh[2], xh[3]);
+      hv.z = bf16x2(xh[4], xh[5]);
+      hv.w = bf16x2(xh[6], xh[7]);
       *reinterpret_cast<uint4*>(&xs[lr][l * 8]) = hv;
     }
     __syncthreads();
     if (tid < (AQ_CH / 64) * AQ_ROWS) {
-      const int g = c * (AQ_CH / 64) + (tid >> 5);
-      const int row = row0 + (tid & 31);
-      if (g < G && row < M) s_x[(size_t)g * M + row] = ss_tile[tid >> 5][tid & 31];
+      const int g = c * (AQ_CH / 64) + tid / AQ_ROWS;
+      const int row = row0 + tid % AQ_ROWS;
+      if (g < G && row < M) s_x[(size_t)g * M + row] = ss_tile[tid / AQ_ROWS][tid % AQ_ROWS];
     }
     if constexpr (NT > 0) {
 #pragma unroll
@@ -184,17 +187,14 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
         const int kc = (w + 8 * h) * 16;          // k16 step inside the chunk
         const int kglob = c * AQ_CH + kc;
         if (kglob < K) {
-          uint32_t a[2][4];
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
-            ldmatrix_x4(smem_u32(&xs[mt * 16 + (l & 15)][kc + (l >> 4) * 8]), a[mt]);
+          uint32_t a[1][4];
+          ldmatrix_x4(smem_u32(&xs[l & 15][kc + (l >> 4) * 8]), a[0]);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             const uint16_t* bp = L1T + (size_t)(nt * 8 + (l >> 2)) * K + kglob + 2 * (l & 3);
             const uint32_t b0 = __ldg(reinterpret_cast<const uint32_t*>(bp));
             const uint32_t b1 = __ldg(reinterpret_cast<const uint32_t*>(bp + 8));
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) mma_bf16_16816(zacc[mt][nt], a[mt], b0, b1);
+            mma_bf16_16816(zacc[0][nt], a[0], b0, b1);
           }
         }
       }
@@ -218,7 +218,7 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
     constexpr int RP = NT * 8;
     float* rw = red + (size_t)w * AQ_ROWS * RP;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int mt = 0; mt < 1; ++mt)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int r = mt * 16 + (l >> 2);
