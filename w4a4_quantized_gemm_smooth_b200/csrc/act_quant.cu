@@ -63,6 +63,26 @@ __device__ __forceinline__ uint32_t quant_nibble(float x, float ss, float rcp, f
   return __float_as_uint(__fadd_rn(q, RN_MAGIC)) & 0xFu;
 }
 
+// All 8 codes of a lane by the exact path (rare; kept out of line).
+__device__ __noinline__ uint32_t quant8_exact(const float* xh, float ssc, float rcp, float scale) {
+  uint32_t packed = 0u;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) packed |= quant_nibble(xh[j], ssc, rcp, scale) << (4 * j);
+  return packed;
+}
+
+// Fast path of the same rounding for a normal scale s: t = fl(x * fl(1/s))
+// is within |x/s| 2^-23 <= 2^-20 of the exact quotient (|x/s| <= 7 + 2^-21),
+// so unless t lies within 2^-20 of a half-integer, rne(t) = rne(x/s).  Sets
+// `near` when that margin is not met (the caller then takes the exact path).
+__device__ __forceinline__ uint32_t quant_nibble_fast(float x, float rcp, bool& near) {
+  const float t = __fmul_rn(x, rcp);
+  const float b0 = __fadd_rn(t, RN_MAGIC);
+  const float f = __fsub_rn(t, __fsub_rn(b0, RN_MAGIC));     // t - rne(t), exact
+  near |= fabsf(fabsf(f) - 0.5f) <= 0x1p-20f;
+  return __float_as_uint(b0) & 0xFu;                          // |rne(t)| <= 7
+}
+
 template <int NT>
 __global__ void __launch_bounds__(AQ_THREADS)
 act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
@@ -111,8 +131,48 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
     }
   }
 
+  // L1 fragments of the chunk's two k16 steps; for NT <= 8 the next chunk's
+  // are prefetched while this chunk is quantised
+  constexpr bool PF = NT > 0 && NT <= 8;
+  constexpr int NTB = NT > 0 ? NT : 1;
+  uint32_t bfr[2][NTB][2], bnx[2][NTB][2];
+  auto load_frags = [&](int c, uint32_t (&dst)[2][NTB][2]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int kglob = c * AQ_CH + (w + 8 * h) * 16;
+#pragma unroll
+      for (int nt = 0; nt < NTB; ++nt) {
+        if (NT > 0 && kglob < K) {
+          const uint16_t* bp = L1T + (size_t)(nt * 8 + (l >> 2)) * K + kglob + 2 * (l & 3);
+          dst[h][nt][0] = __ldg(reinterpret_cast<const uint32_t*>(bp));
+          dst[h][nt][1] = __ldg(reinterpret_cast<const uint32_t*>(bp + 8));
+        } else {
+          dst[h][nt][0] = dst[h][nt][1] = 0u;
+        }
+      }
+    }
+  };
+  if (PF) load_frags(0, bfr);
+  // smoothing factors of the lane's 8 channels, prefetched one chunk ahead
+  auto load_il = [&](int c, float (&dst)[8]) {
+    const int col = c * AQ_CH + l * 8;
+    if (col < K) {
+      const float4 i0 = __ldg(reinterpret_cast<const float4*>(inv_lambda + col));
+      const float4 i1 = __ldg(reinterpret_cast<const float4*>(inv_lambda + col + 4));
+      dst[0] = i0.x; dst[1] = i0.y; dst[2] = i0.z; dst[3] = i0.w;
+      dst[4] = i1.x; dst[5] = i1.y; dst[6] = i1.z; dst[7] = i1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dst[j] = 0.0f;
+    }
+  };
+  float il[8], il_nx[8];
+  load_il(0, il);
+
   for (int c = 0; c < nchunks; ++c) {
     const int st = c % AQ_STAGES;
+    if (PF && c + 1 < nchunks) load_frags(c + 1, bnx);
+    if (c + 1 < nchunks) load_il(c + 1, il_nx);
     if (!mbar_wait_bounded(smem_u32(&full_bar[st]), (c / AQ_STAGES) & 1, AQ_LIMIT_NS)) {
       atomicExch(err, SVDQ_DEVERR_TIMEOUT);
       abort_sh = 1;
@@ -128,16 +188,6 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
                     : make_uint4(0u, 0u, 0u, 0u);
     const int col = c * AQ_CH + l * 8;
     const bool colok = col < K;
-    float il[8];
-    if (colok) {
-      const float4 i0 = __ldg(reinterpret_cast<const float4*>(inv_lambda + col));
-      const float4 i1 = __ldg(reinterpret_cast<const float4*>(inv_lambda + col + 4));
-      il[0] = i0.x; il[1] = i0.y; il[2] = i0.z; il[3] = i0.w;
-      il[4] = i1.x; il[5] = i1.y; il[6] = i1.z; il[7] = i1.w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) il[j] = 0.0f;
-    }
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int lr = w + 8 * rr;
@@ -158,12 +208,16 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
       const float s = __fdiv_rn(m, 7.0f);
       uint32_t packed = 0u;
       if (s > 0.0f) {
-        const bool tiny = s < 0x1p-64f;
+        const bool tiny = s < 0x1p-64f;         // s subnormal or nearly: exact path
+        bool near = tiny;
         const float scale = tiny ? 0x1p64f : 1.0f;
         const float ssc = __fmul_rn(s, scale);
         const float rcp = __frcp_rn(ssc);
+        if (!tiny) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) packed |= quant_nibble(xh[j], ssc, rcp, scale) << (4 * j);
+          for (int j = 0; j < 8; ++j) packed |= quant_nibble_fast(xh[j], rcp, near) << (4 * j);
+        }
+        if (near) packed = quant8_exact(xh, ssc, rcp, scale);   // rare: exact residual
       }
       if (colok && row < M)
         *reinterpret_cast<uint32_t*>(xq + (size_t)row * (K / 2) + col / 2) = packed;
@@ -191,13 +245,30 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
           ldmatrix_x4(smem_u32(&xs[l & 15][kc + (l >> 4) * 8]), a[0]);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const uint16_t* bp = L1T + (size_t)(nt * 8 + (l >> 2)) * K + kglob + 2 * (l & 3);
-            const uint32_t b0 = __ldg(reinterpret_cast<const uint32_t*>(bp));
-            const uint32_t b1 = __ldg(reinterpret_cast<const uint32_t*>(bp + 8));
+            uint32_t b0, b1;
+            if (PF) {
+              b0 = bfr[h][nt][0];
+              b1 = bfr[h][nt][1];
+            } else {
+              const uint16_t* bp = L1T + (size_t)(nt * 8 + (l >> 2)) * K + kglob + 2 * (l & 3);
+              b0 = __ldg(reinterpret_cast<const uint32_t*>(bp));
+              b1 = __ldg(reinterpret_cast<const uint32_t*>(bp + 8));
+            }
             mma_bf16_16816(zacc[0][nt], a[0], b0, b1);
           }
         }
       }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) il[j] = il_nx[j];
+    if (PF) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int nt = 0; nt < NTB; ++nt) {
+          bfr[h][nt][0] = bnx[h][nt][0];
+          bfr[h][nt][1] = bnx[h][nt][1];
+        }
     }
     __syncthreads();
     if (tid == 0 && c + AQ_STAGES < nchunks) {
