@@ -50,8 +50,7 @@ namespace {
 constexpr int BM = 128;
 constexpr int NP = 4;            // packed-code stages
 constexpr int THREADS = 512;
-constexpr int EXP_WARP0 = 2;     // expanders: warps 2-7
-constexpr int N_EXP = 192;
+constexpr int N_EXP = 192;       // expanders: warps 2-7
 constexpr int RES_WARP0 = 8;     // rescale / epilogue: warps 8-15
 constexpr int N_RES_WARPS = 8;
 constexpr uint64_t LIMIT_NS = 2000000000ull;
@@ -137,27 +136,57 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
   }
 }
 
-// 16 packed bytes (32 codes of one row) -> two 16-byte core-matrix rows.
+// 16 packed bytes (32 codes of one row: the first or second half of the
+// group) -> two 16-byte core-matrix rows at d and d + 128.
 // Each code q becomes the int8 16*q: the high nibble of a byte is already
-// 16*q in place (mask), the low nibble is shifted up by 4 (shift + mask).
+// 16*q in place (mask), the low nibble is moved up by 4 (a funnel rotate,
+// whose wrapped-around bits the mask removes).
 // Products are 256 q_x q_w, so the int32 group sum is 256 P_g (|256 P_g| <=
 // 2^20, exact); the factor 2^-8 is folded into the scale.
-__device__ __forceinline__ void expand16(const uint8_t* src, uint8_t* dst_base, int row,
-                                         int half) {
-  const uint4 p = *reinterpret_cast<const uint4*>(src);
-  uint4 o0, o1;
-  o0.x = (p.x << 4) & 0xF0F0F0F0u;
-  o0.y = p.x & 0xF0F0F0F0u;
-  o0.z = (p.y << 4) & 0xF0F0F0F0u;
-  o0.w = p.y & 0xF0F0F0F0u;
-  o1.x = (p.z << 4) & 0xF0F0F0F0u;
-  o1.y = p.z & 0xF0F0F0F0u;
-  o1.z = (p.w << 4) & 0xF0F0F0F0u;
-  o1.w = p.w & 0xF0F0F0F0u;
-  uint8_t* d = dst_base + (row >> 3) * 512 + (row & 7) * 16 + half * 256;
-  *reinterpret_cast<uint4*>(d) = o0;
-  *reinterpret_cast<uint4*>(d + 128) = o1;
+__device__ __forceinline__ uint32_t rotl4(uint32_t x) {
+  uint32_t y;
+  asm("shf.l.wrap.b32 %0, %1, %1, 4;" : "=r"(y) : "r"(x));
+  return y;
 }
+__device__ __forceinline__ void expand16(uint32_t src, uint32_t d) {
+  const uint4 p = lds128u(src);
+  uint4 o0, o1;
+  o0.x = rotl4(p.x) & 0xF0F0F0F0u;
+  o0.y = p.x & 0xF0F0F0F0u;
+  o0.z = rotl4(p.y) & 0xF0F0F0F0u;
+  o0.w = p.y & 0xF0F0F0F0u;
+  o1.x = rotl4(p.z) & 0xF0F0F0F0u;
+  o1.y = p.z & 0xF0F0F0F0u;
+  o1.z = rotl4(p.w) & 0xF0F0F0F0u;
+  o1.w = p.w & 0xF0F0F0F0u;
+  sts128(d, o0);
+  sts128(d + 128, o1);
+}
+
+// The expanders' share of one group: CNT rounds of 32 consecutive 16-byte
+// units starting at round R0.  Unit j of an operand is half (j >> 3) & 1 of
+// row 8 (j >> 4) + (j & 7), so each quarter-warp reads and writes 128
+// contiguous bytes.  Offsets are fixed per thread and computed once.
+template <int BN, int CNT>
+struct ExpandPlan {
+  uint32_t src[CNT], dst[CNT];
+  __device__ __forceinline__ ExpandPlan(int r0, int lane) {
+    using L = Lay<BN>;
+#pragma unroll
+    for (int k = 0; k < CNT; ++k) {
+      const int u = 32 * (r0 + k) + lane;
+      const bool isa = u < BM * 2;
+      const int j = isa ? u : u - BM * 2;
+      const int hf = (j >> 3) & 1, row = ((j >> 4) << 3) | (j & 7);
+      src[k] = (isa ? 0 : L::PK_A) + hf * (isa ? BM : BN) * 16 + row * 16;
+      dst[k] = (isa ? 0 : L::EX_A) + (row >> 3) * 512 + (row & 7) * 16 + hf * 256;
+    }
+  }
+  __device__ __forceinline__ void run(uint32_t pa, uint32_t ea) const {
+#pragma unroll
+    for (int k = 0; k < CNT; ++k) expand16(pa + src[k], ea + dst[k]);
+  }
+};
 
 __device__ __forceinline__ float gelu_f(float y) {
   return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f));
@@ -259,8 +288,11 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
                 MODE == 0 ? (p.sx_tma ? BM * 4 : 0) + BN * 4 : 0;
             mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE + scale_bytes);
             const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
-            tma_load_2d(dst, &tm_a, g * 32, m0, pk_full(s));
-            tma_load_2d(dst + L::PK_A, &tm_b, g * 32, n0, pk_full(s));
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              tma_load_2d(dst + hh * (BM * 16), &tm_a, g * 32 + 16 * hh, m0, pk_full(s));
+              tma_load_2d(dst + L::PK_A + hh * (BN * 16), &tm_b, g * 32 + 16 * hh, n0, pk_full(s));
+            }
             if (MODE == 0) {
               if (p.sx_tma) tma_load_2d(slot, &tm_sx, m0, g, pk_full(s));
               tma_load_2d(slot + 4 * BM, &tm_sw, n0, g, pk_full(s));
@@ -338,31 +370,44 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       __syncwarp();
     } else {
       // ---------------------------------------------------- expanders
-      const int et = tid - EXP_WARP0 * 32;
-      uint32_t it = 0;
-      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-        for (int g = 0; g < G; ++g, ++it) {
-          const int se = it % NE, sp = it % NP;
-          if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err)) goto exp_done;
-          if (!wait_or_abort(pk_full(sp), (it / NP) & 1, abort_flag, p.err)) goto exp_done;
-          uint8_t* ea = smem + L::OFF_EX + se * L::EX_STAGE;
-          const uint8_t* pa = smem + L::OFF_PK + sp * L::PK_STAGE;
-#pragma unroll 2
-          for (int i = et; i < (BM + BN) * 2; i += N_EXP) {
-            if (i < BM * 2) expand16(pa + i * 16, ea, i >> 1, i & 1);
-            else expand16(pa + i * 16, ea + L::EX_A, (i - BM * 2) >> 1, i & 1);
+      // Warps 4 and 5 sit alone on their SM sub-partitions (with the producer
+      // and the MMA issuer); warps 2+6 and 3+7 share theirs.  Each
+      // sub-partition gets a quarter of the units, so the rescale warps next
+      // to them are slowed alike.
+      constexpr int ROUNDS = (BM + BN) * 2 / 32;
+      static_assert(ROUNDS % 8 == 0, "expander split");
+      auto expand_loop = [&](const auto& plan) {
+        uint32_t it = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+          for (int g = 0; g < G; ++g, ++it) {
+            const int se = it % NE, sp = it % NP;
+            if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err)) return;
+            if (!wait_or_abort(pk_full(sp), (it / NP) & 1, abort_flag, p.err)) return;
+            plan.run(sbase + L::OFF_PK + sp * L::PK_STAGE, sbase + L::OFF_EX + se * L::EX_STAGE);
+            mbar_arrive(pk_empty(sp));
+            fence_proxy_async_smem();
+            mbar_arrive(ex_full(se));
           }
-          mbar_arrive(pk_empty(sp));
-          fence_proxy_async_smem();
-          mbar_arrive(ex_full(se));
         }
+      };
+      if (warp == 4 || warp == 5) {
+        const ExpandPlan<BN, ROUNDS / 4> plan((warp - 4) * (ROUNDS / 4), lane);
+        expand_loop(plan);
+      } else {
+        const int slot_i = (warp & 3) - 2 + 2 * ((warp >> 2) & 1);   // warps 2,3,6,7 -> 0,1,2,3
+        const ExpandPlan<BN, ROUNDS / 8> plan(ROUNDS / 2 + slot_i * (ROUNDS / 8), lane);
+        expand_loop(plan);
       }
-    exp_done:;
     }
   } else {
     regs_inc<REG_HI>();
     // ------------------------------------------------------ rescale + epilogue
+    // TMEM lanes 32q..32q+31 (the warp's quarter), columns h*CW..h*CW+CW-1.
+    // Rescale layout (.16x256b loads): this thread owns rows r0 + 8i (i < 4)
+    // of the quarter and, in each 16-column chunk c, the column pairs
+    // 16c + 8b + 2pq (+1), b < 2.  acc[i][2c + b] holds that pair.
     const int rw = warp - RES_WARP0, q = warp & 3, h = rw >> 2;
+    const int pq = lane & 3, r0 = lane >> 2;
     float* bb = reinterpret_cast<float*>(smem + L::OFF_BIAS) + rw * CW;
     uint8_t* ystage = smem + L::OFF_Y + rw * L::Y_WARP;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
@@ -373,9 +418,11 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
       const int row = m0 + 32 * q + lane;
       const int ncol0 = n0 + h * CW;           // first column of this warp
-      float2 acc2[CW / 2];
+      float2 acc[4][CW / 8];
 #pragma unroll
-      for (int j = 0; j < CW / 2; ++j) acc2[j] = make_float2(0.0f, 0.0f);
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < CW / 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
       constexpr int PER = CW / 32;             // bias values loaded per lane
       float bias_n[PER];                       // prefetched for the epilogue
 #pragma unroll
@@ -390,30 +437,39 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
         if (MODE == 0) {
-          // 16-column TMEM loads, double-buffered: the load of chunk c+1 is
-          // in flight while chunk c is rescaled (wait::ld waits for all).
-          const float sx = lds32(slot + 4u * (32 * q + lane)) * 0.00390625f;   // 2^-8 (exact)
-          const float2 sx2 = make_float2(sx, sx);
+          // 16-column chunks, double-buffered: the loads of chunk c+1 are in
+          // flight while chunk c is rescaled (wait::ld waits for all).
+          float2 sx2[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float v = lds32(slot + 4u * (32 * q + r0 + 8 * i)) * 0.00390625f;  // 2^-8 (exact)
+            sx2[i] = make_float2(v, v);
+          }
           const float2 nmag2 = make_float2(-MAGIC_F, -MAGIC_F);
-          const uint32_t swa = slot + 4u * (BM + h * CW);
+          const uint32_t swa = slot + 4u * (BM + h * CW) + 16u * pq;
           uint32_t rb[2][16];
-          tmem_ld16(ta, rb[0]);
+          tmem_ld16x256b_x2(ta, &rb[0][0]);
+          tmem_ld16x256b_x2(ta + (16u << 16), &rb[0][8]);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < CW / 16; ++c) {
-            if (c + 1 < CW / 16) tmem_ld16(ta + 16 * (c + 1), rb[(c + 1) & 1]);
+            if (c + 1 < CW / 16) {
+              tmem_ld16x256b_x2(ta + 16 * (c + 1), &rb[(c + 1) & 1][0]);
+              tmem_ld16x256b_x2(ta + 16 * (c + 1) + (16u << 16), &rb[(c + 1) & 1][8]);
+            }
             const uint32_t* r = rb[c & 1];
+            const float4 s4 = lds128(swa + 64u * c);   // columns 2pq, 2pq+1, 8+2pq, 9+2pq
 #pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-              const float4 s4 = lds128(swa + 4u * (16 * c + j));
-              const float2 sc0 = __fmul2_rn(sx2, make_float2(s4.x, s4.y));
-              const float2 sc1 = __fmul2_rn(sx2, make_float2(s4.z, s4.w));
-              // 256 P_g, exactly: the word is the float MAGIC_F + 256 P_g
-              const float2 u0 = __fadd2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), nmag2);
-              const float2 u1 = __fadd2_rn(make_float2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])), nmag2);
-              const int e = (16 * c + j) >> 1;
-              acc2[e] = __ffma2_rn(sc0, u0, acc2[e]);
-              acc2[e + 1] = __ffma2_rn(sc1, u1, acc2[e + 1]);
+            for (int bb = 0; bb < 2; ++bb) {
+              const float2 sw2 = bb ? make_float2(s4.z, s4.w) : make_float2(s4.x, s4.y);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                // register of row r0 + 8i: half (i >> 1), row (i & 1) of the 16-lane load
+                const uint32_t* wv = r + 8 * (i >> 1) + 4 * bb + 2 * (i & 1);
+                // 256 P_g, exactly: the word is the float MAGIC_F + 256 P_g
+                const float2 u = __fadd2_rn(make_float2(__uint_as_float(wv[0]), __uint_as_float(wv[1])), nmag2);
+                acc[i][2 * c + bb] = __ffma2_rn(__fmul2_rn(sx2[i], sw2), u, acc[i][2 * c + bb]);
+              }
             }
             if (c + 1 < CW / 16) tmem_wait_ld();
           }
@@ -445,17 +501,24 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
         uint32_t rb[2][16];
-        tmem_ld16(ta, rb[0]);
+        tmem_ld16x256b_x2(ta, &rb[0][0]);
+        tmem_ld16x256b_x2(ta + (16u << 16), &rb[0][8]);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < CW / 16; ++c) {
-          if (c + 1 < CW / 16) tmem_ld16(ta + 16 * (c + 1), rb[(c + 1) & 1]);
+          if (c + 1 < CW / 16) {
+            tmem_ld16x256b_x2(ta + 16 * (c + 1), &rb[(c + 1) & 1][0]);
+            tmem_ld16x256b_x2(ta + 16 * (c + 1) + (16u << 16), &rb[(c + 1) & 1][8]);
+          }
           const uint32_t* r = rb[c & 1];
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const int e = (16 * c + j) >> 1;
-            acc2[e] = __fadd2_rn(acc2[e], make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])));
-          }
+          for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t* wv = r + 8 * (i >> 1) + 4 * bb + 2 * (i & 1);
+              acc[i][2 * c + bb] = __fadd2_rn(acc[i][2 * c + bb],
+                                              make_float2(__uint_as_float(wv[0]), __uint_as_float(wv[1])));
+            }
           if (c + 1 < CW / 16) tmem_wait_ld();
         }
         tc_fence_before();
@@ -468,28 +531,25 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       for (int e = 0; e < PER; ++e) bb[lane * PER + e] = bias_n[e];
       if (lane == 0) tma_store_wait_read0();
       __syncwarp();
-      const uint32_t bba = smem_u32(bb);
+      const float* bb_base = bb;
       const bool gelu = p.epilogue == SVDQ_EPI_GELU;
+      // row r0 + 8i of the warp's 32, column pair 16c + 8b + 2pq: 4 bytes of the
+      // 128-byte row of box c / 4, in 16-byte chunk (2c + b) & 7, swizzled by row
 #pragma unroll
-      for (int box = 0; box < CW / 64; ++box) {
-        uint8_t* yb = ystage + box * L::Y_BOX + lane * 128;
+      for (int c = 0; c < CW / 16; ++c) {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const int j0 = box * 64 + ch * 8;
-          const float4 b0 = lds128(bba + 4u * j0), b1 = lds128(bba + 4u * (j0 + 4));
-          float2 v[4];
-          v[0] = __fadd2_rn(acc2[j0 / 2 + 0], make_float2(b0.x, b0.y));
-          v[1] = __fadd2_rn(acc2[j0 / 2 + 1], make_float2(b0.z, b0.w));
-          v[2] = __fadd2_rn(acc2[j0 / 2 + 2], make_float2(b1.x, b1.y));
-          v[3] = __fadd2_rn(acc2[j0 / 2 + 3], make_float2(b1.z, b1.w));
-          if (gelu) {
+        for (int bb = 0; bb < 2; ++bb) {
+          const int col = 16 * c + 8 * bb + 2 * pq;
+          const float2 bv = *reinterpret_cast<const float2*>(bb_base + col);
+          uint8_t* yb = ystage + (c >> 2) * L::Y_BOX + 4 * pq;
+          const int ch = (2 * c + bb) & 7;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] = make_float2(gelu_f(v[e].x), gelu_f(v[e].y));
+          for (int i = 0; i < 4; ++i) {
+            float2 v = __fadd2_rn(acc[i][2 * c + bb], bv);
+            if (gelu) v = make_float2(gelu_f(v.x), gelu_f(v.y));
+            const int row = r0 + 8 * i;
+            *reinterpret_cast<uint32_t*>(yb + row * 128 + ((ch ^ (row & 7)) * 16)) = bf16x2_bits(v);
           }
-          uint4 o;
-          o.x = bf16x2_bits(v[0]); o.y = bf16x2_bits(v[1]);
-          o.z = bf16x2_bits(v[2]); o.w = bf16x2_bits(v[3]);
-          *reinterpret_cast<uint4*>(yb + ((ch ^ (lane & 7)) * 16)) = o;
         }
       }
       fence_proxy_async_smem();
@@ -590,9 +650,9 @@ cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const
                           cudaStream_t st) {
   const int BN = pick_bn(w->N);
   CUtensorMap ta, tb, ty, tz, tl;
-  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 32, BM,
+  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 16, BM,
                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 32, BN,
+      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 16, BN,
                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
                 CU_TENSOR_MAP_SWIZZLE_128B))
@@ -603,7 +663,7 @@ cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const
   const bool sx_tma = (M % 4) == 0;
   if ((sx_tma && !make_map(&tsx, s_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, w->G, (uint64_t)M * 4,
                            BM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
-      !make_map(&tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N, w->G, (uint64_t)w->N4 * 4,
+      !make_map(&tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N16, w->G, (uint64_t)w->N16 * 4,
                 BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   if (w->rank > 0 &&
@@ -630,9 +690,9 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
                             int nrows, int col0, int ncols, int32_t* P, cudaStream_t st) {
   const int BN = pick_bn(w->N);
   CUtensorMap ta, tb;
-  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 32, BM,
+  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 16, BM,
                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 32, BN,
+      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 16, BN,
                 CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   LinArgs a{};

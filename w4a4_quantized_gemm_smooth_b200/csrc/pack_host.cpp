@@ -111,10 +111,13 @@ svdq_status upload(svdq_weights* w, cudaStream_t st) {
   svdq_status s;
   if ((s = dev_alloc_copy(&w->d_inv_lambda, w->inv_lambda.data(), (size_t)K, st))) return s;
   if ((s = dev_alloc_copy(&w->d_wq, w->wq.data(), (size_t)N * K / 2, st))) return s;
-  w->N4 = (N + 3) / 4 * 4;
-  std::vector<float> swp((size_t)G * w->N4, 0.0f);
+  w->N16 = (N + 15) / 16 * 16;
+  std::vector<float> swp((size_t)G * w->N16, 0.0f);
   for (int g = 0; g < G; ++g)
-    std::memcpy(&swp[(size_t)g * w->N4], &w->sw[(size_t)g * N], (size_t)N * 4);
+    for (int n = 0; n < N; ++n) {
+      const int c = n & 15, pos = (n & ~15) + 4 * ((c & 7) >> 1) + 2 * (c >> 3) + (c & 1);
+      swp[(size_t)g * w->N16 + pos] = w->sw[(size_t)g * N + n];
+    }
   if ((s = dev_alloc_copy(&w->d_sw, swp.data(), swp.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_L1T, L1T.data(), L1T.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_L2, L2p.data(), L2p.size(), st))) return s;

@@ -207,6 +207,16 @@ __device__ __forceinline__ void tma_store_wait0() {
 }
 
 // 32 lanes x 16 consecutive 32-bit TMEM columns.
+// 16 TMEM lanes x 16 columns (.16x256b, two 8-column repeats): thread t gets
+// r[4j + 2i + e] = lane (base + t/4 + 8i), column (8j + 2(t%4) + e).
+__device__ __forceinline__ void tmem_ld16x256b_x2(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "

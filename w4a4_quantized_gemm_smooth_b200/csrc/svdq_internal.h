@@ -15,12 +15,15 @@ struct svdq_weights {
   int rank_pad = 0;    // rank rounded up to a multiple of 16 (zero rows)
   int rank_pad32 = 0;  // rank rounded up to a multiple of 32
   int N_pad = 0;       // N rounded up to a multiple of 256
-  int N4 = 0;          // N rounded up to a multiple of 4 (row pitch of d_sw)
+  int N16 = 0;         // N rounded up to a multiple of 16 (row pitch of d_sw)
   int device = 0;
   // device copies (owned)
   float* d_inv_lambda = nullptr;   // [K]
   uint8_t* d_wq = nullptr;         // [N][K/2] packed residual codes
-  float* d_sw = nullptr;           // [G][N4] (N4 = N rounded up to 4, zero padded)
+  // [G][N16], zero padded; inside each block of 16 columns, column
+  // 8b + 2p + e is stored at 4p + 2b + e, so that the rescale thread that owns
+  // the column pairs 2p, 2p+1 of both 8-column halves reads them as one float4
+  float* d_sw = nullptr;
   uint16_t* d_L1T = nullptr;       // [rank_pad][K] bf16, transposed L1
   uint16_t* d_L2 = nullptr;        // [rank_pad][N] bf16
   uint16_t* d_L2T = nullptr;       // [N_pad][rank_pad32] bf16, transposed L2
