@@ -57,6 +57,29 @@ def _workload(name):
     return specs[name]
 
 
+def _config(spec, ws):
+    """The workload description shared by both arms' JSON lines."""
+    r = spec.rank + spec.lora_rank
+    return {"workload": f"{spec.name} M={spec.M} K={spec.K} N={spec.N} r={r}", "M": spec.M,
+            "K": spec.K, "N": spec.N, "rank": r, "group": 64, "parallelism": f"replicas x{ws}",
+            "l2": "flushed (256 MiB write) before every step"}
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise max of per-rank timings over all ranks (every rank gets
+    the result).  `dist` is torch.distributed when a process group is up."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tops(ops_per_rank, world_size, seconds):
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return world_size * ops_per_rank / seconds / 1e12
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -177,8 +200,7 @@ def run_reference(args, spec):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(ts) / len(ts),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N,
-                   "rank": spec.rank, "sample": st["sample"]},
+        "config": _config(spec, ws),
         "cpu_baseline": {"value": v, "unit": "TOPS", "cores": _blas_threads(),
                          "kind": "oracle", "sample": st["sample"]},
         "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -312,12 +334,10 @@ def run_ours(args, spec):
     (t_e2e,) = _time_steps(e2e, args.steps, flush, stream)
     S.svdq_get_device_error(w0)
 
-    tt = torch.tensor([t_act + t_lin, t_lin, t_act, t_e2e], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    t_step_ms, t_lin_ms, t_act_ms, t_e2e_ms = (float(v) / args.steps for v in tt.tolist())
+    tt = max_over_ranks([t_act + t_lin, t_lin, t_act, t_e2e], dist, "cuda")
+    t_step_ms, t_lin_ms, t_act_ms, t_e2e_ms = (v / args.steps for v in tt)
     ops = 2.0 * M * N * K
-    value = ws * ops / (t_step_ms * 1e-3) / 1e12
+    value = job_tops(ops, ws, t_step_ms * 1e-3)
     bf16_burst, bf16_sust, hbm, which = _peaks()
     int8_peak = 2.0 * bf16_burst          # int8 dense = 2 x bf16 dense (nominal ratio)
     lin_tops = ops / (t_lin_ms * 1e-3) / 1e12
@@ -327,9 +347,7 @@ def run_ours(args, spec):
         "warmup": args.warmup, "ms_per_step": t_step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
-        "config": {"workload": f"{spec.name} M={M} K={K} N={N} r={r}", "M": M, "K": K, "N": N,
-                   "rank": r, "group": 64, "parallelism": f"replicas x{ws}",
-                   "l2": "flushed (256 MiB write) before every step"},
+        "config": _config(spec, ws),
         "roofline": {"bound": "tensor", "achieved": lin_tops, "peak": int8_peak,
                      "unit": "TFLOP/s", "frac": lin_tops / int8_peak, "traffic": None,
                      "kernel": "svdq_linear", "peak_source":
@@ -339,7 +357,7 @@ def run_ours(args, spec):
         "linear_ms": t_lin_ms,
         "lowrank_overhead": {"linear": t_lin_ms / (t_lin0 / args.steps) - 1.0,
                              "layer": t_step_ms / ((t_act0 + t_lin0) / args.steps) - 1.0},
-        "e2e": {"value": ws * ops / (t_e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+        "e2e": {"value": job_tops(ops, ws, t_e2e_ms * 1e-3), "unit": "TOPS",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
