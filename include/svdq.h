@@ -2,7 +2,7 @@
  * svdq.h -- C ABI of the SVDQuant W4A4 linear layer for NVIDIA B200 (sm_100a).
  *
  * The layer (SVDQuant technical review of arXiv:2411.05007v4, section 4.2,
- * eq. 7; section 6.1, Algorithm 2):
+ * eq. 7; section 6.1):
  *
  *     Y = Q(X~) Q(R) + (X~ L1) L2 + b,   X~ = X diag(lambda)^-1,
  *     R = diag(lambda) W - L1 L2                       (section 5, eq. 10)
@@ -80,7 +80,7 @@ svdq_status svdq_calib_absmax(int M, int K, const uint16_t* X, int ldx,
                               float* absmax);
 
 /*
- * Offline transform of one layer (review Algorithm 1, steps 2-5 and 9 with a
+ * Offline transform of one layer (review section 5, the offline procedure with a
  * fixed alpha and no refinement).  Host inputs, device result.
  *   lambda_k = act_absmax[k]^alpha / max_n|W[n][k]|^(1-alpha)   (eq. 4);
  *              lambda_k = 1 if either statistic is 0;
@@ -142,7 +142,7 @@ svdq_status svdq_weights_export(const svdq_weights* w, float* inv_lambda,
                                 uint8_t* wq, float* s_w, uint16_t* L1,
                                 uint16_t* L2, uint16_t* bias, double* sigma);
 
-/* Store / restore a packed layer (Algorithm 1 step 9): versioned header and
+/* Store / restore a packed layer (review section 5): versioned header and
  * raw host arrays.  load uploads to the current device on `stream`. */
 svdq_status svdq_weights_save(const svdq_weights* w, const char* path);
 svdq_status svdq_weights_load(const char* path, cudaStream_t stream,
@@ -150,7 +150,7 @@ svdq_status svdq_weights_load(const char* path, cudaStream_t stream,
 void svdq_weights_free(svdq_weights* w);
 
 /*
- * Fused activation pass (review section 6.1, Algorithm 2 steps 1-3): one
+ * Fused activation pass (review section 6.1, activation side): one
  * kernel reads X once and writes
  *   xq  [M][K/2]   packed INT4 codes of x~ = fl32(x * inv_lambda_k);
  *   s_x [K/64][M]  fp32 scales, fl32(max|x~| / 7) per token and group;
@@ -164,7 +164,7 @@ svdq_status svdq_quantize_act(const svdq_weights* w, int M, const uint16_t* X,
                               cudaStream_t stream);
 
 /*
- * Fused W4A4 product (Algorithm 2 steps 4-8): one kernel computes
+ * Fused W4A4 product (review section 6.1, product side): one kernel computes
  *   P_g = sum_{k in g} q_x q_w       (int32, per group, on the tensor cores)
  *   acc = sum_g s_x[g][m] s_w[g][n] P_g            (fp32)
  *   Y   = bf16(epi(acc + Z L2 + b))                 written once

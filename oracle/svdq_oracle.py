@@ -214,8 +214,8 @@ def leading_svd(Wt, k):
 def pack_weights(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None,
                  lora_A_bits=None, lora_B_bits=None, lora_scale=1.0,
                  smooth=True, svd=None):
-    """Offline transform of one linear layer (review Algorithm 1, steps 2-5
-    and 9, with alpha fixed and no refinement / GPTQ).
+    """Offline transform of one linear layer (the review's offline procedure,
+    section 5, with alpha fixed and no refinement / GPTQ).
 
     W_bits: bf16 bits [N, K] (nn.Linear layout; the math weight W is its
     transpose, K x N, rows = input channels).  act_absmax: [K] calibration
@@ -262,7 +262,7 @@ def pack_weights(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None,
 # runtime: activation quantise + down-projection, then the two-branch product
 # --------------------------------------------------------------------------
 def quantize_act(X_bits, inv_lambda, L1b):
-    """Review Algorithm 2 steps 1-3: x~ = fl32(x * inv_lambda) (eq. 3),
+    """Review section 6.1, activation side: x~ = fl32(x * inv_lambda) (eq. 3),
     eq. 1 per (token, group of 64), and the 16-bit down-projection
     Z = bf16(bf16(x~) L1) with exact accumulation.
     Returns (codes [M, K], s_x [G, M], Z [M, r] float64 bf16 values, xhat)."""
@@ -307,7 +307,7 @@ def gelu(y):
 
 def linear(xcodes, s_x, Z, wcodes, s_w, L2b, bias, apply_gelu=False,
            rows=None, cols=None):
-    """Review Algorithm 2 steps 4-8 / eq. 7:
+    """Review section 6.1, product side / eq. 7:
     Y = sum_g s_x[g, i] s_w[g, n] P_g[i, n] + Z L2 + b (fp64), optional GELU,
     then one bf16 rounding.  Returns (Y float64, Y_bf16 float64 values)."""
     xc = np.asarray(xcodes)

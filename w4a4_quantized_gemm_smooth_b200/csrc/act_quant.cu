@@ -1,4 +1,4 @@
-// Fused activation pass (SVDQuant review section 6.1, Algorithm 2 steps 1-3):
+// Fused activation pass (SVDQuant review section 6.1, activation side):
 // read X once, smooth it (eq. 3), quantise it per token and group of 64
 // (eq. 1) and, from the same tile, compute the 16-bit down-projection
 // Z = bf16(x~) L1 on the tensor cores (mma.sync bf16, fp32 accumulation).

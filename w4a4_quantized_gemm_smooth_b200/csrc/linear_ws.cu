@@ -1,5 +1,5 @@
 // W4A4 product with the 16-bit up-projection fused (SVDQuant review section
-// 6.1, Algorithm 2 steps 4-8; eq. 7), warp-specialised for sm_100a.
+// 6.1, product side; eq. 7), warp-specialised for sm_100a.
 //
 // sm_100a tensor cores have no 4-bit integer kind, so the packed codes are
 // streamed by TMA into shared memory, expanded there to int8 (as 16 q, three

@@ -1,5 +1,5 @@
-// Host side of the C ABI: the offline pack (SVDQuant review Algorithm 1,
-// steps 2-5 and 9), handle management, export, save/load.
+// Host side of the C ABI: the offline pack (SVDQuant review section 5, the
+// offline procedure without refinement), handle management, export, save/load.
 //
 // Exactness contract with the checks: every rounding below is a single IEEE
 // rounding of a value that both sides define the same way, so the codes and
