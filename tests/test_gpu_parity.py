@@ -105,6 +105,7 @@ def test_tiny_layer_gelu_epilogue():
     (1, 64, 128, 8),         # one token, one group
     (333, 1152, 256, 64),    # PixArt width, rank 64
     (128, 256, 128, 0),      # no low-rank branch
+    (130, 8256, 136, 8),     # K too long for the correction operand of 128-column tiles
 ])
 def test_ragged_and_small_shapes(M, K, N, r):
     spec = synth.layer_spec(f"e{M}_{K}_{N}_{r}", M, K, N, r, 100 + M + K + N + r, tiny=True)
