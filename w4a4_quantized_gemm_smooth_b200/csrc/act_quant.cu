@@ -1,21 +1,29 @@
-// Fused activation pass (SVDQuant review section 6.1, activation side):
-// read X once, smooth it (eq. 3), quantise it per token and group of 64
-// (eq. 1) and, from the same tile, compute the 16-bit down-projection
+// Fused activation pass (SVDQuant review section 6.1, activation side): read
+// X once, smooth it (eq. 3), quantise it per token and group of 64 (eq. 1)
+// and, from the same registers, compute the 16-bit down-projection
 // Z = bf16(x~) L1 on the tensor cores (mma.sync bf16, fp32 accumulation).
 //
-// Layout: one CTA of 8 warps owns 16 consecutive tokens and walks K in
-// chunks of 256 channels (several CTAs per SM).  TMA streams 16 x 256 bf16
-// tiles of X into a 6-stage shared-memory ring, so X is read from HBM
-// exactly once with full-width transactions.  A warp reads one token's 256
-// channels from the ring (16 bytes per lane); the 8 lanes holding one group
-// of 64 find its absmax with three xor-shuffles.  bf16(x~) is staged in
-// shared memory for the MMA; the scale tile is staged so that s_x[g][m] is
-// written with contiguous stores.
+// Layout: a CTA owns 32 consecutive tokens and walks K in stages of four
+// groups (256 channels).  A producer warp streams each stage by TMA into a
+// shared-memory ring: the 32 x 64 bf16 tile of X of every group (128-byte
+// swizzled), the matching 64-column slice of L1^T (all branch rows, also
+// swizzled) and the 256 smoothing factors, all on one mbarrier.  Eight
+// compute warps each own one 16-token x 64-channel block of a stage (two
+// token halves x four groups), read it with ldmatrix in the mma.sync A
+// fragment layout and, without any CTA-wide barrier, smooth, quantise,
+// store codes and scales, and multiply the same fragments (as bf16) with
+// L1 fragments read by ldmatrix.  A warp releases the stage with an mbarrier
+// arrive; the producer refills it.  The warps' partial Z (different groups,
+// same tokens) are summed in shared memory at the end.
 //
-// Bit-exact quantiser: x~ = fl32(x * inv_lambda) (one IEEE multiply),
-// s = fl32(m / 7) (IEEE division), and the code is round-half-even of the
-// exact quotient x~/s: a first guess from the correctly rounded reciprocal
-// is corrected with the exact residual x~ - q s computed by an fma.
+// Quantiser: x~ = fl32(x * inv_lambda) (one IEEE multiply), s = fl32(m / 7)
+// (IEEE division) for the group absmax m, and the code is round-half-even of
+// the exact quotient x~/s: a first guess from the correctly rounded
+// reciprocal, with an exact fma-residual path where the guess is within
+// 2^-20 of a half or the scale is tiny.  A lane holds 16 values of each of
+// two tokens; a token's group spans the four lanes of a quad (absmax with
+// two xor-shuffles; codes regrouped into 8-byte stores by a 4 x 4 byte
+// transpose across the quad).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -26,12 +34,32 @@
 namespace svdq {
 namespace {
 
-constexpr int AQ_ROWS = 16;
-constexpr int AQ_CH = 256;
-constexpr int AQ_THREADS = 256;
-constexpr int AQ_STAGES = 6;
-constexpr int AQ_STAGE_BYTES = AQ_ROWS * AQ_CH * 2;     // 8 KB
+constexpr int AQ_ROWS = 32;                 // tokens per CTA
+constexpr int AQ_GPS = 4;                   // groups per stage
+constexpr int AQ_WARPS = 8;                 // compute warps
+constexpr int AQ_THREADS = (AQ_WARPS + 1) * 32;
+constexpr int AQ_XTILE = AQ_ROWS * 128;     // one group of X: 32 rows x 64 bf16
 constexpr uint64_t AQ_LIMIT_NS = 2000000000ull;
+
+// Stage layout: X tiles of the four groups, then their L1^T slices
+// (NT * 8 rows x 128 B each), then the 256 smoothing factors.
+template <int NT>
+struct AqStage {
+  static constexpr int L1_TILE = NT * 8 * 128;
+  static constexpr int OFF_L1 = AQ_GPS * AQ_XTILE;
+  static constexpr int OFF_IL = OFF_L1 + AQ_GPS * L1_TILE;
+  static constexpr int BYTES = OFF_IL + AQ_GPS * 64 * 4;              // multiple of 1024
+  static constexpr int STAGES = (200 * 1024) / BYTES < 4 ? (200 * 1024) / BYTES : 4;
+  static constexpr int RED = AQ_WARPS * 16 * NT * 8 * 4;             // Z partials at the end
+  static_assert(STAGES >= 2, "stage too large");
+  static_assert(RED <= STAGES * BYTES, "reduction buffer aliases the ring");
+};
+
+__device__ __forceinline__ float2 lds64(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
@@ -63,12 +91,30 @@ __device__ __forceinline__ uint32_t quant_nibble(float x, float ss, float rcp, f
   return __float_as_uint(__fadd_rn(q, RN_MAGIC)) & 0xFu;
 }
 
-// All 8 codes of a lane by the exact path (rare; kept out of line).
-__device__ __noinline__ uint32_t quant8_exact(const float* xh, float ssc, float rcp, float scale) {
-  uint32_t packed = 0u;
+// Value j = 4 ks + e of a lane's row (k16 step ks; e: columns 2q, 2q+1,
+// 2q+8, 2q+9) goes to byte ks of word e / 2, low nibble for even e.
+__device__ __forceinline__ void place(uint32_t nib, int j, uint32_t& u0, uint32_t& u1) {
+  const uint32_t v = nib << (8 * (j >> 2) + 4 * (j & 1));
+  if ((j >> 1) & 1) u1 |= v; else u0 |= v;
+}
+
+// All 16 codes of a lane's row by the exact path (rare; kept out of line).
+__device__ __noinline__ void quant16_exact(const float* v, float ssc, float rcp, float scale,
+                                           uint32_t* u) {
+  uint32_t u0 = 0u, u1 = 0u;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) packed |= quant_nibble(xh[j], ssc, rcp, scale) << (4 * j);
-  return packed;
+  for (int j = 0; j < 16; ++j) place(quant_nibble(v[j], ssc, rcp, scale), j, u0, u1);
+  u[0] = u0;
+  u[1] = u1;
+}
+
+// 4 x 4 byte transpose across the lanes of a quad: lane q holds bytes
+// b[q][0..3] (byte j destined for lane j) and returns b[0..3][q].
+__device__ __forceinline__ uint32_t quad_transpose(uint32_t x, int q) {
+  uint32_t p = __shfl_xor_sync(0xFFFFFFFFu, x, 2);
+  const uint32_t y = (q & 2) ? __byte_perm(p, x, 0x7632) : __byte_perm(x, p, 0x5410);
+  p = __shfl_xor_sync(0xFFFFFFFFu, y, 1);
+  return __byte_perm(y, p, (q & 1) ? 0x3715 : 0x6240);
 }
 
 // Fast path of the same rounding for a normal scale s: t = fl(x * fl(1/s))
@@ -84,227 +130,190 @@ __device__ __forceinline__ uint32_t quant_nibble_fast(float x, float rcp, bool& 
 }
 
 template <int NT>
-__global__ void __launch_bounds__(AQ_THREADS)
-act_quant_kernel(const __grid_constant__ CUtensorMap tm_x, int box_cols,
+__global__ void __launch_bounds__(AQ_THREADS, 1)
+act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
+                 const __grid_constant__ CUtensorMap tm_l,   // L1^T [NT*8][K] bf16
                  const float* __restrict__ inv_lambda,
-                 const uint16_t* __restrict__ L1T,   // [NT*8][K] bf16
                  int M, int K, int rank,
                  uint8_t* __restrict__ xq, float* __restrict__ s_x,
                  uint16_t* __restrict__ Z, int* __restrict__ err) {
-  __shared__ __align__(16) uint16_t xs[AQ_ROWS][AQ_CH + 8];
-  __shared__ float ss_tile[AQ_CH / 64][AQ_ROWS];
-  __shared__ __align__(8) uint64_t full_bar[AQ_STAGES];
+  using ST = AqStage<NT>;
+  constexpr int S = ST::STAGES;
+  __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S];
   __shared__ int abort_sh;
-  // dynamic: [AQ_STAGES][32 rows][box_cols] bf16 ring (1024-B aligned),
-  // then [8][AQ_ROWS][NT*8] fp32 reduction buffer when NT > 0
   extern __shared__ uint8_t aq_dyn_raw[];
-  uint8_t* aq_dyn = reinterpret_cast<uint8_t*>(
+  uint8_t* ring_p = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(aq_dyn_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = aq_dyn;
-  float* red = reinterpret_cast<float*>(aq_dyn + AQ_STAGES * AQ_STAGE_BYTES);
+  const uint32_t ring = smem_u32(ring_p);
 
-  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, l = tid & 31;
   const int row0 = blockIdx.x * AQ_ROWS;
   const int G = K / 64;
-  const int nchunks = (K + AQ_CH - 1) / AQ_CH;
+  const int nstages = (G + AQ_GPS - 1) / AQ_GPS;
 
-  float zacc[1][NT > 0 ? NT : 1][4];
-#pragma unroll
-  for (int a = 0; a < 1; ++a)
-#pragma unroll
-    for (int b = 0; b < (NT > 0 ? NT : 1); ++b)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) zacc[a][b][c] = 0.0f;
-
-  const uint32_t stage_bytes = (uint32_t)box_cols * AQ_ROWS * 2;
   if (tid == 0) {
-    for (int s = 0; s < AQ_STAGES; ++s) mbar_init(smem_u32(&full_bar[s]), 1);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), AQ_WARPS);
+    }
     abort_sh = 0;
     fence_mbarrier_init();
   }
   __syncthreads();
-  if (tid == 0) {
-    for (int c = 0; c < AQ_STAGES && c < nchunks; ++c) {
-      mbar_arrive_expect_tx(smem_u32(&full_bar[c]), stage_bytes);
-      tma_load_2d(smem_u32(ring + c * AQ_STAGE_BYTES), &tm_x, c * AQ_CH, row0,
-                  smem_u32(&full_bar[c]));
-    }
-  }
 
-  // L1 fragments of the chunk's two k16 steps; for NT <= 8 the next chunk's
-  // are prefetched while this chunk is quantised
-  constexpr bool PF = NT > 0 && NT <= 8;
-  constexpr int NTB = NT > 0 ? NT : 1;
-  uint32_t bfr[2][NTB][2], bnx[2][NTB][2];
-  auto load_frags = [&](int c, uint32_t (&dst)[2][NTB][2]) {
+  float zacc[NT > 0 ? NT : 1][4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int kglob = c * AQ_CH + (w + 8 * h) * 16;
+  for (int a = 0; a < (NT > 0 ? NT : 1); ++a)
 #pragma unroll
-      for (int nt = 0; nt < NTB; ++nt) {
-        if (NT > 0 && kglob < K) {
-          const uint16_t* bp = L1T + (size_t)(nt * 8 + (l >> 2)) * K + kglob + 2 * (l & 3);
-          dst[h][nt][0] = __ldg(reinterpret_cast<const uint32_t*>(bp));
-          dst[h][nt][1] = __ldg(reinterpret_cast<const uint32_t*>(bp + 8));
-        } else {
-          dst[h][nt][0] = dst[h][nt][1] = 0u;
-        }
-      }
-    }
-  };
-  if (PF) load_frags(0, bfr);
-  // smoothing factors of the lane's 8 channels, prefetched one chunk ahead
-  auto load_il = [&](int c, float (&dst)[8]) {
-    const int col = c * AQ_CH + l * 8;
-    if (col < K) {
-      const float4 i0 = __ldg(reinterpret_cast<const float4*>(inv_lambda + col));
-      const float4 i1 = __ldg(reinterpret_cast<const float4*>(inv_lambda + col + 4));
-      dst[0] = i0.x; dst[1] = i0.y; dst[2] = i0.z; dst[3] = i0.w;
-      dst[4] = i1.x; dst[5] = i1.y; dst[6] = i1.z; dst[7] = i1.w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dst[j] = 0.0f;
-    }
-  };
-  float il[8], il_nx[8];
-  load_il(0, il);
+    for (int b = 0; b < 4; ++b) zacc[a][b] = 0.0f;
 
-  for (int c = 0; c < nchunks; ++c) {
-    const int st = c % AQ_STAGES;
-    if (PF && c + 1 < nchunks) load_frags(c + 1, bnx);
-    if (c + 1 < nchunks) load_il(c + 1, il_nx);
-    if (!mbar_wait_bounded(smem_u32(&full_bar[st]), (c / AQ_STAGES) & 1, AQ_LIMIT_NS)) {
-      atomicExch(err, SVDQ_DEVERR_TIMEOUT);
-      abort_sh = 1;
-    }
-    __syncthreads();
-    if (abort_sh) break;
-    uint4 cur[2];
-    const uint8_t* stage = ring + st * AQ_STAGE_BYTES;
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr)
-      cur[rr] = (l * 8 < box_cols)
-                    ? *reinterpret_cast<const uint4*>(stage + (w + 8 * rr) * box_cols * 2 + l * 16)
-                    : make_uint4(0u, 0u, 0u, 0u);
-    const int col = c * AQ_CH + l * 8;
-    const bool colok = col < K;
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const int lr = w + 8 * rr;
-      const int row = row0 + lr;
-      const uint32_t u[4] = {cur[rr].x, cur[rr].y, cur[rr].z, cur[rr].w};
-      float xh[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        xh[2 * j] = __fmul_rn(bf16lo(u[j]), il[2 * j]);
-        xh[2 * j + 1] = __fmul_rn(bf16hi(u[j]), il[2 * j + 1]);
-      }
-      float m = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(xh[j]));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-      const float s = __fdiv_rn(m, 7.0f);
-      uint32_t packed = 0u;
-      if (s > 0.0f) {
-        const bool tiny = s < 0x1p-64f;         // s subnormal or nearly: exact path
-        bool near = tiny;
-        const float scale = tiny ? 0x1p64f : 1.0f;
-        const float ssc = __fmul_rn(s, scale);
-        const float rcp = __frcp_rn(ssc);
-        if (!tiny) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) packed |= quant_nibble_fast(xh[j], rcp, near) << (4 * j);
+  if (warp == AQ_WARPS) {
+    // ------------------------------------------------------------ producer
+    if (l == 0) {
+      int c = 0;
+      for (; c < nstages; ++c) {
+        const int s = c % S;
+        if (c >= S && !mbar_wait_bounded(smem_u32(&empty_bar[s]), ((c / S) - 1) & 1, AQ_LIMIT_NS)) {
+          atomicExch(err, SVDQ_DEVERR_TIMEOUT);
+          abort_sh = 1;
+          break;
         }
-        if (near) packed = quant8_exact(xh, ssc, rcp, scale);   // rare: exact residual
+        if (*reinterpret_cast<volatile int*>(&abort_sh)) break;
+        const int ng = min(AQ_GPS, G - AQ_GPS * c);
+        const uint32_t fb = smem_u32(&full_bar[s]);
+        mbar_arrive_expect_tx(fb, ng * (AQ_XTILE + ST::L1_TILE + 256));
+        const uint32_t st = ring + s * ST::BYTES;
+        for (int g = 0; g < ng; ++g) {
+          const int col = (AQ_GPS * c + g) * 64;
+          tma_load_2d(st + g * AQ_XTILE, &tm_x, col, row0, fb);
+          if (NT > 0) tma_load_2d(st + ST::OFF_L1 + g * ST::L1_TILE, &tm_l, col, 0, fb);
+        }
+        bulk_load(st + ST::OFF_IL, inv_lambda + AQ_GPS * 64 * c, ng * 256, fb);
       }
-      if (colok && row < M)
-        *reinterpret_cast<uint32_t*>(xq + (size_t)row * (K / 2) + col / 2) = packed;
-      if ((l & 7) == 0) ss_tile[l >> 3][lr] = s;
-      uint4 hv;
-      hv.x = bf16x2(xh[0], xh[1]);
-      hv.y = bf16x2(xh[2], xh[3]);
-      hv.z = bf16x2(xh[4], xh[5]);
-      hv.w = bf16x2(xh[6], xh[7]);
-      *reinterpret_cast<uint4*>(&xs[lr][l * 8]) = hv;
+      // every issued copy lands before the CTA moves on
+      for (int k = (c > S ? c - S : 0); k < c; ++k)
+        mbar_wait_bounded(smem_u32(&full_bar[k % S]), (k / S) & 1, AQ_LIMIT_NS);
     }
-    __syncthreads();
-    if (tid < (AQ_CH / 64) * AQ_ROWS) {
-      const int g = c * (AQ_CH / 64) + tid / AQ_ROWS;
-      const int row = row0 + tid % AQ_ROWS;
-      if (g < G && row < M) s_x[(size_t)g * M + row] = ss_tile[tid / AQ_ROWS][tid % AQ_ROWS];
-    }
-    if constexpr (NT > 0) {
+  } else {
+    // ------------------------------------------------------- compute warps
+    const int rb = warp & 1, gi = warp >> 1, q = l & 3, g8 = l >> 2;
+    for (int c = 0; c < nstages; ++c) {
+      const int s = c % S;
+      if (!mbar_wait_bounded(smem_u32(&full_bar[s]), (c / S) & 1, AQ_LIMIT_NS)) {
+        atomicExch(err, SVDQ_DEVERR_TIMEOUT);
+        abort_sh = 1;
+        break;
+      }
+      if (*reinterpret_cast<volatile int*>(&abort_sh)) break;
+      const int grp = AQ_GPS * c + gi;
+      if (grp < G) {
+        const uint32_t st = ring + s * ST::BYTES;
+        const uint32_t xt = st + gi * AQ_XTILE;
+        // raw X in the A fragment layout: a[ks][0] row g8, cols 16ks+2q (+1);
+        // [1] row g8+8; [2] row g8, cols 16ks+8+2q (+1); [3] row g8+8
+        uint32_t a[4][4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int kc = (w + 8 * h) * 16;          // k16 step inside the chunk
-        const int kglob = c * AQ_CH + kc;
-        if (kglob < K) {
-          uint32_t a[1][4];
-          ldmatrix_x4(smem_u32(&xs[l & 15][kc + (l >> 4) * 8]), a[0]);
+        for (int ks = 0; ks < 4; ++ks) {
+          const int rr = rb * 16 + (l & 15), ch = 2 * ks + (l >> 4);
+          ldmatrix_x4(xt + rr * 128 + ((ch ^ (rr & 7)) << 4), a[ks]);
+        }
+        const uint32_t ilt = st + ST::OFF_IL + gi * 256;
+        float v[2][16];
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            uint32_t b0, b1;
-            if (PF) {
-              b0 = bfr[h][nt][0];
-              b1 = bfr[h][nt][1];
-            } else {
-              const uint16_t* bp = L1T + (size_t)(nt * 8 + (l >> 2)) * K + kglob + 2 * (l & 3);
-              b0 = __ldg(reinterpret_cast<const uint32_t*>(bp));
-              b1 = __ldg(reinterpret_cast<const uint32_t*>(bp + 8));
+        for (int ks = 0; ks < 4; ++ks) {
+          const float2 i0 = lds64(ilt + 4 * (16 * ks + 2 * q));
+          const float2 i1 = lds64(ilt + 4 * (16 * ks + 8 + 2 * q));
+#pragma unroll
+          for (int ri = 0; ri < 2; ++ri) {
+            v[ri][4 * ks + 0] = __fmul_rn(bf16lo(a[ks][ri]), i0.x);
+            v[ri][4 * ks + 1] = __fmul_rn(bf16hi(a[ks][ri]), i0.y);
+            v[ri][4 * ks + 2] = __fmul_rn(bf16lo(a[ks][2 + ri]), i1.x);
+            v[ri][4 * ks + 3] = __fmul_rn(bf16hi(a[ks][2 + ri]), i1.y);
+          }
+        }
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) {
+          float m = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[ri][j]));
+          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+          const float sc = __fdiv_rn(m, 7.0f);
+          uint32_t u[2] = {0u, 0u};
+          if (sc > 0.0f) {
+            const bool tiny = sc < 0x1p-64f;     // s subnormal or nearly: exact path
+            bool near = tiny;
+            const float scale = tiny ? 0x1p64f : 1.0f;
+            const float ssc = __fmul_rn(sc, scale);
+            const float rcp = __frcp_rn(ssc);
+            if (!tiny) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) place(quant_nibble_fast(v[ri][j], rcp, near), j, u[0], u[1]);
             }
-            mma_bf16_16816(zacc[0][nt], a[0], b0, b1);
+            if (near) {                          // rare: exact residual
+              float tmp[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) tmp[j] = v[ri][j];
+              quant16_exact(tmp, ssc, rcp, scale, u);
+            }
+          }
+          const uint32_t w0 = quad_transpose(u[0], q), w1 = quad_transpose(u[1], q);
+          const int row = row0 + rb * 16 + g8 + 8 * ri;
+          if (row < M) {
+            *reinterpret_cast<uint2*>(xq + (size_t)row * (K / 2) + grp * 32 + 8 * q) = make_uint2(w0, w1);
+            if (q == 0) s_x[(size_t)grp * M + row] = sc;
+          }
+        }
+        if constexpr (NT > 0) {
+          const uint32_t lt = st + ST::OFF_L1 + gi * ST::L1_TILE;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            uint32_t af[4];
+            af[0] = bf16x2(v[0][4 * ks + 0], v[0][4 * ks + 1]);
+            af[1] = bf16x2(v[1][4 * ks + 0], v[1][4 * ks + 1]);
+            af[2] = bf16x2(v[0][4 * ks + 2], v[0][4 * ks + 3]);
+            af[3] = bf16x2(v[1][4 * ks + 2], v[1][4 * ks + 3]);
+#pragma unroll
+            for (int j = 0; j < NT / 2; ++j) {
+              // matrices: n-tile 2j (k 0-7, 8-15), n-tile 2j+1 (k 0-7, 8-15)
+              const int mi = l >> 3, n = 16 * j + 8 * (mi >> 1) + (l & 7), ch = 2 * ks + (mi & 1);
+              uint32_t b[4];
+              ldmatrix_x4(lt + n * 128 + ((ch ^ (n & 7)) << 4), b);
+              mma_bf16_16816(zacc[2 * j], af, b[0], b[1]);
+              mma_bf16_16816(zacc[2 * j + 1], af, b[2], b[3]);
+            }
           }
         }
       }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) il[j] = il_nx[j];
-    if (PF) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int nt = 0; nt < NTB; ++nt) {
-          bfr[h][nt][0] = bnx[h][nt][0];
-          bfr[h][nt][1] = bnx[h][nt][1];
-        }
-    }
-    __syncthreads();
-    if (tid == 0 && c + AQ_STAGES < nchunks) {
-      mbar_arrive_expect_tx(smem_u32(&full_bar[st]), stage_bytes);
-      tma_load_2d(smem_u32(ring + st * AQ_STAGE_BYTES), &tm_x, (c + AQ_STAGES) * AQ_CH, row0,
-                  smem_u32(&full_bar[st]));
+      __syncwarp();
+      if (l == 0) mbar_arrive(smem_u32(&empty_bar[s]));
     }
   }
-  if (abort_sh) {
-    // let every issued copy land before the CTA exits
-    if (tid == 0)
-      for (int c = 0; c < AQ_STAGES && c < nchunks; ++c)
-        mbar_wait_bounded(smem_u32(&full_bar[c]), 0, AQ_LIMIT_NS);
-    return;
-  }
+  __syncthreads();
+  if (abort_sh) return;
 
   if constexpr (NT > 0) {
+    // sum the four group-warps of each token half; Z rows in bf16
     constexpr int RP = NT * 8;
-    float* rw = red + (size_t)w * AQ_ROWS * RP;
-#pragma unroll
-    for (int mt = 0; mt < 1; ++mt)
+    float* red = reinterpret_cast<float*>(ring_p);
+    if (warp < AQ_WARPS) {
+      float* rw = red + (size_t)warp * 16 * RP;
+      const int q = l & 3, g8 = l >> 2;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int r = mt * 16 + (l >> 2);
-        const int cc = nt * 8 + 2 * (l & 3);
-        rw[r * RP + cc] = zacc[mt][nt][0];
-        rw[r * RP + cc + 1] = zacc[mt][nt][1];
-        rw[(r + 8) * RP + cc] = zacc[mt][nt][2];
-        rw[(r + 8) * RP + cc + 1] = zacc[mt][nt][3];
+        const int cc = nt * 8 + 2 * q;
+        rw[g8 * RP + cc] = zacc[nt][0];
+        rw[g8 * RP + cc + 1] = zacc[nt][1];
+        rw[(g8 + 8) * RP + cc] = zacc[nt][2];
+        rw[(g8 + 8) * RP + cc + 1] = zacc[nt][3];
       }
+    }
     __syncthreads();
     for (int idx = tid; idx < AQ_ROWS * rank; idx += AQ_THREADS) {
-      const int r = idx / rank, j = idx % rank;
+      const int r = idx / rank, j = idx % rank, hb = r >> 4, r16 = r & 15;
       float sum = 0.0f;
 #pragma unroll
-      for (int ww = 0; ww < 8; ++ww) sum += red[(size_t)ww * AQ_ROWS * RP + r * RP + j];
+      for (int gw = 0; gw < AQ_GPS; ++gw) sum += red[(size_t)(2 * gw + hb) * 16 * RP + r16 * RP + j];
       if (row0 + r < M)
         Z[(size_t)(row0 + r) * rank + j] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
     }
@@ -315,19 +324,33 @@ PFN_cuTensorMapEncodeTiled_v12000 aq_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess && q == cudaDriverEntryPointSuccess)
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) ==
+            cudaSuccess && qr == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
   }
   return fn;
 }
 
+// 2D bf16 map with a 64-column (128-byte), 128-byte-swizzled box.
+bool aq_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch,
+            uint32_t box_rows) {
+  auto fn = aq_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int NT>
 cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
                       uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
-  const size_t red_bytes = NT > 0 ? (size_t)8 * AQ_ROWS * NT * 8 * sizeof(float) : 0;
-  const size_t dyn = (size_t)AQ_STAGES * AQ_STAGE_BYTES + red_bytes + 1024;
+  using ST = AqStage<NT>;
+  const size_t dyn = (size_t)ST::STAGES * ST::BYTES + 1024;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<NT>,
@@ -335,21 +358,15 @@ cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  auto fn = aq_encode_fn();
-  if (!fn) return cudaErrorInvalidValue;
-  const int box_cols = w->K < AQ_CH ? w->K : AQ_CH;
-  CUtensorMap tm;
-  const cuuint64_t dims[2] = {(cuuint64_t)w->K, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)AQ_ROWS};
-  const cuuint32_t estr[2] = {1, 1};
-  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides,
-         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  CUtensorMap tx, tl;
+  if (!aq_map(&tx, X, (uint64_t)w->K, (uint64_t)M, (uint64_t)ldx * 2, AQ_ROWS))
+    return cudaErrorInvalidValue;
+  tl = tx;
+  if (NT > 0 && !aq_map(&tl, w->d_L1T, (uint64_t)w->K, (uint64_t)NT * 8, (uint64_t)w->K * 2, NT * 8))
     return cudaErrorInvalidValue;
   const dim3 grid((M + AQ_ROWS - 1) / AQ_ROWS);
-  act_quant_kernel<NT><<<grid, AQ_THREADS, dyn, st>>>(
-      tm, box_cols, w->d_inv_lambda, w->d_L1T, M, w->K, w->rank, xq, s_x, Z, w->d_err);
+  act_quant_kernel<NT><<<grid, AQ_THREADS, dyn, st>>>(tx, tl, w->d_inv_lambda, M, w->K, w->rank,
+                                                      xq, s_x, Z, w->d_err);
   return cudaGetLastError();
 }
 
