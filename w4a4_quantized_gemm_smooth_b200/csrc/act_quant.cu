@@ -35,22 +35,24 @@ namespace svdq {
 namespace {
 
 constexpr int AQ_ROWS = 32;                 // tokens per CTA
-constexpr int AQ_GPS = 4;                   // groups per stage
-constexpr int AQ_WARPS = 8;                 // compute warps
-constexpr int AQ_THREADS = (AQ_WARPS + 1) * 32;
 constexpr int AQ_XTILE = AQ_ROWS * 128;     // one group of X: 32 rows x 64 bf16
 constexpr uint64_t AQ_LIMIT_NS = 2000000000ull;
 
-// Stage layout: X tiles of the four groups, then their L1^T slices
-// (NT * 8 rows x 128 B each), then the 256 smoothing factors.
+// Stage layout: X tiles of the GPS groups, then their L1^T slices
+// (NT * 8 rows x 128 B each), then the 64 GPS smoothing factors.  Eight
+// groups (16 compute warps) per stage while the L1 slices are small, four
+// (8 warps) for the largest ranks.
 template <int NT>
 struct AqStage {
+  static constexpr int GPS = NT <= 8 ? 8 : 4;
+  static constexpr int WARPS = 2 * GPS;                               // compute warps
+  static constexpr int THREADS = (WARPS + 1) * 32;                    // + the producer warp
   static constexpr int L1_TILE = NT * 8 * 128;
-  static constexpr int OFF_L1 = AQ_GPS * AQ_XTILE;
-  static constexpr int OFF_IL = OFF_L1 + AQ_GPS * L1_TILE;
-  static constexpr int BYTES = OFF_IL + AQ_GPS * 64 * 4;              // multiple of 1024
+  static constexpr int OFF_L1 = GPS * AQ_XTILE;
+  static constexpr int OFF_IL = OFF_L1 + GPS * L1_TILE;
+  static constexpr int BYTES = OFF_IL + GPS * 64 * 4;                 // multiple of 1024
   static constexpr int STAGES = (200 * 1024) / BYTES < 4 ? (200 * 1024) / BYTES : 4;
-  static constexpr int RED = AQ_WARPS * 16 * NT * 8 * 4;             // Z partials at the end
+  static constexpr int RED = WARPS * 16 * NT * 8 * 4;                 // Z partials at the end
   static_assert(STAGES >= 2, "stage too large");
   static_assert(RED <= STAGES * BYTES, "reduction buffer aliases the ring");
 };
@@ -117,20 +119,9 @@ __device__ __forceinline__ uint32_t quad_transpose(uint32_t x, int q) {
   return __byte_perm(y, p, (q & 1) ? 0x3715 : 0x6240);
 }
 
-// Fast path of the same rounding for a normal scale s: t = fl(x * fl(1/s))
-// is within |x/s| 2^-23 <= 2^-20 of the exact quotient (|x/s| <= 7 + 2^-21),
-// so unless t lies within 2^-20 of a half-integer, rne(t) = rne(x/s).  Sets
-// `near` when that margin is not met (the caller then takes the exact path).
-__device__ __forceinline__ uint32_t quant_nibble_fast(float x, float rcp, bool& near) {
-  const float t = __fmul_rn(x, rcp);
-  const float b0 = __fadd_rn(t, RN_MAGIC);
-  const float f = __fsub_rn(t, __fsub_rn(b0, RN_MAGIC));     // t - rne(t), exact
-  near |= fabsf(fabsf(f) - 0.5f) <= 0x1p-20f;
-  return __float_as_uint(b0) & 0xFu;                          // |rne(t)| <= 7
-}
 
 template <int NT>
-__global__ void __launch_bounds__(AQ_THREADS, 1)
+__global__ void __launch_bounds__(AqStage<NT>::THREADS, 1)
 act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_l,   // L1^T [NT*8][K] bf16
                  const float* __restrict__ inv_lambda,
@@ -139,6 +130,7 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
                  uint16_t* __restrict__ Z, int* __restrict__ err) {
   using ST = AqStage<NT>;
   constexpr int S = ST::STAGES;
+  constexpr int AQ_GPS = ST::GPS, AQ_WARPS = ST::WARPS, AQ_THREADS = ST::THREADS;
   __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S];
   __shared__ int abort_sh;
   extern __shared__ uint8_t aq_dyn_raw[];
@@ -225,10 +217,12 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
           const float2 i1 = lds64(ilt + 4 * (16 * ks + 8 + 2 * q));
 #pragma unroll
           for (int ri = 0; ri < 2; ++ri) {
-            v[ri][4 * ks + 0] = __fmul_rn(bf16lo(a[ks][ri]), i0.x);
-            v[ri][4 * ks + 1] = __fmul_rn(bf16hi(a[ks][ri]), i0.y);
-            v[ri][4 * ks + 2] = __fmul_rn(bf16lo(a[ks][2 + ri]), i1.x);
-            v[ri][4 * ks + 3] = __fmul_rn(bf16hi(a[ks][2 + ri]), i1.y);
+            const float2 p0 = __fmul2_rn(make_float2(bf16lo(a[ks][ri]), bf16hi(a[ks][ri])), i0);
+            const float2 p1 = __fmul2_rn(make_float2(bf16lo(a[ks][2 + ri]), bf16hi(a[ks][2 + ri])), i1);
+            v[ri][4 * ks + 0] = p0.x;
+            v[ri][4 * ks + 1] = p0.y;
+            v[ri][4 * ks + 2] = p1.x;
+            v[ri][4 * ks + 3] = p1.y;
           }
         }
 #pragma unroll
@@ -247,8 +241,30 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
             const float ssc = __fmul_rn(sc, scale);
             const float rcp = __frcp_rn(ssc);
             if (!tiny) {
+              // Fast path for a normal scale: t = fl(x * fl(1/s)) is within
+              // |x/s| 2^-23 <= 2^-20 of the exact quotient, so rne(t) = rne(x/s)
+              // unless t lies within 2^-20 of a half-integer.
+              // Pairs (j, j+1) are the two codes of one byte; t = x * fl(1/s),
+              // rne(t) by the magic add, f = t - rne(t) exact; the row is near
+              // a half somewhere iff max |f| >= 1/2 - 2^-20
+              const float2 rc2 = make_float2(rcp, rcp), mg2 = make_float2(RN_MAGIC, RN_MAGIC);
+              const float2 nmg2 = make_float2(-RN_MAGIC, -RN_MAGIC);
+              float fmx = 0.0f;
+              uint32_t by[8];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) place(quant_nibble_fast(v[ri][j], rcp, near), j, u[0], u[1]);
+              for (int j = 0; j < 16; j += 2) {
+                const float2 t = __fmul2_rn(make_float2(v[ri][j], v[ri][j + 1]), rc2);
+                const float2 b = __fadd2_rn(t, mg2);
+                const float2 r = __fadd2_rn(b, nmg2);
+                const float2 f = __fadd2_rn(t, make_float2(-r.x, -r.y));
+                fmx = fmaxf(fmx, fmaxf(fabsf(f.x), fabsf(f.y)));
+                // |rne(t)| <= 7: the low nibble of the biased word is the code
+                by[j >> 1] = (__float_as_uint(b.x) & 0xFu) | ((__float_as_uint(b.y) << 4) & 0xF0u);
+              }
+              near = fmx >= 0.5f - 0x1p-20f;
+              // byte of pair j/2 = 2 ks + h goes to byte ks of word h
+              u[0] = __byte_perm(__byte_perm(by[0], by[2], 0x0040), __byte_perm(by[4], by[6], 0x0040), 0x5410);
+              u[1] = __byte_perm(__byte_perm(by[1], by[3], 0x0040), __byte_perm(by[5], by[7], 0x0040), 0x5410);
             }
             if (near) {                          // rare: exact residual
               float tmp[16];
@@ -365,7 +381,7 @@ cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
   if (NT > 0 && !aq_map(&tl, w->d_L1T, (uint64_t)w->K, (uint64_t)NT * 8, (uint64_t)w->K * 2, NT * 8))
     return cudaErrorInvalidValue;
   const dim3 grid((M + AQ_ROWS - 1) / AQ_ROWS);
-  act_quant_kernel<NT><<<grid, AQ_THREADS, dyn, st>>>(tx, tl, w->d_inv_lambda, M, w->K, w->rank,
+  act_quant_kernel<NT><<<grid, ST::THREADS, dyn, st>>>(tx, tl, w->d_inv_lambda, M, w->K, w->rank,
                                                       xq, s_x, Z, w->d_err);
   return cudaGetLastError();
 }
