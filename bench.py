@@ -38,6 +38,29 @@ import synth  # noqa: E402
 
 METRIC = "svdq_linear effective TOPS (2MNK/s) at FLUX-like shapes; % int8 roofline"
 
+# DRAM bytes (read + write) of one svdq_linear launch on this workload, from
+# the ncu capture summarised in profiles/svdq_linear_flux_qkv.md, valid only
+# for the kernel sources it was taken on (SHA-1 over the files below).
+LINEAR_SOURCES = ("w4a4_quantized_gemm_smooth_b200/csrc/linear_ws.cu",
+                  "w4a4_quantized_gemm_smooth_b200/csrc/ptx.cuh",
+                  "w4a4_quantized_gemm_smooth_b200/csrc/svdq_internal.h")
+LINEAR_TRAFFIC = {"sources_sha1": "2c89f0d9044c284a4d31d69b8ffdd2a897a97169",
+                  "workload": "flux_qkv", "bytes": 24877056 + 32831744}
+
+
+def _linear_traffic(workload):
+    import hashlib
+    h = hashlib.sha1()
+    try:
+        for f in LINEAR_SOURCES:
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    if h.hexdigest() != LINEAR_TRAFFIC["sources_sha1"] or workload != LINEAR_TRAFFIC["workload"]:
+        return None
+    return LINEAR_TRAFFIC["bytes"]
+
 
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -90,7 +113,7 @@ def _dist():
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -105,40 +128,47 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
+    def mark(self, which):
+        """Wall-clock bounds of the timed region (samples outside are dropped)."""
+        setattr(self, which, time.time())
+
     def stop(self):
         if self.proc is None:
             return None
-        time.sleep(0.25)
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.fh.close()
-        sm, mx, reasons = [], [], set()
+        import datetime
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[2]), float(parts[3]),
+                                 {nm for nm, v in zip(names, parts[6:10]) if v.lower() == "active"}))
                 except ValueError:
                     continue
-                for nm, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(nm)
-        if not sm:
+        t0, t1 = getattr(self, "t0", None), getattr(self, "t1", None)
+        inside = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
+        use = inside or rows
+        if not use:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "samples": len(sm), "reasons": sorted(reasons)}
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "samples": len(use), "in_timed_region": bool(inside),
+                "reasons": sorted(set().union(*(r[3] for r in use)))}
 
 
 # --------------------------------------------------------------------------
@@ -321,9 +351,12 @@ def run_ours(args, spec):
     barrier()
     clocks = ClockSampler(local)
     clocks.start()
+    time.sleep(0.2)                      # sampler up before the timed region
     barrier()
+    clocks.mark("t0")
     t_act, t_lin = _time_steps(step, args.steps, flush, stream)
     barrier()
+    clocks.mark("t1")
     clk = clocks.stop()
     S.svdq_get_device_error(w)
 
@@ -349,7 +382,8 @@ def run_ours(args, spec):
         "data": "synthetic",
         "config": _config(spec, ws),
         "roofline": {"bound": "tensor", "achieved": lin_tops, "peak": int8_peak,
-                     "unit": "TFLOP/s", "frac": lin_tops / int8_peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": lin_tops / int8_peak,
+                     "traffic": _linear_traffic(spec.name),
                      "kernel": "svdq_linear", "peak_source":
                      f"{which} bf16 burst {bf16_burst} x 2 (int8/bf16 nominal ratio)"},
         "act_quant": {"ms": t_act_ms, "achieved_gbs": act_gbs, "peak_gbs": hbm,
@@ -375,7 +409,7 @@ def run_ours(args, spec):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="flux_qkv")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
