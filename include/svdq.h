@@ -62,6 +62,7 @@ enum { SVDQ_EPI_NONE = 0, SVDQ_EPI_GELU = 1 };
 
 #define SVDQ_GROUP 64
 #define SVDQ_MAX_RANK 128
+#define SVDQ_MAX_SPLITS 16      /* K splits per output tile in svdq_linear_splitk */
 
 /* Opaque packed layer, immutable after svdq_pack_weights / svdq_weights_load.
  * Holds device copies of every operand plus host copies for export. */
@@ -174,6 +175,36 @@ svdq_status svdq_quantize_act(const svdq_weights* w, int M, const uint16_t* X,
 svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq,
                         const float* s_x, const uint16_t* Z, uint16_t* Y,
                         int ldy, int epilogue, cudaStream_t stream);
+
+/*
+ * Split-K form of svdq_linear for batches too small to fill the GPU with
+ * output tiles (review section 9: PixArt-Sigma layers at a few hundred
+ * tokens).  The K groups of every 128-row output tile are divided into
+ * `splits` consecutive ranges, each handled by its own persistent-CTA work
+ * item; a range's fp32 partial sum of s_x s_w P_g (split 0 also adds Z L2)
+ * goes to the workspace, and the last range of a tile to finish sums the
+ * partials in range order and applies bias, epilogue and the bf16 store.
+ * Same operation as svdq_linear; only the fp32 summation order differs.
+ *
+ * splits: 1 .. min(SVDQ_MAX_SPLITS, K/64), or 0 for the automatic choice
+ *         (one split once the output tiles alone cover half the SMs, else
+ *         about one work item per SM with at least two groups per range).
+ *         One split runs svdq_linear's kernel and gives its exact bits.
+ * workspace: device memory, 256-byte aligned, at least
+ *         svdq_linear_splitk_workspace(w, M, splits) bytes, owned by the
+ *         caller.  Its first part holds arrival counters, which this call
+ *         clears (cudaMemsetAsync on `stream`) before the launch; the rest
+ *         holds the partial tiles.  Calls sharing a workspace must not
+ *         overlap (same stream, or ordered by events).
+ * Errors: as svdq_linear; SVDQ_ERR_INVALID_ARG for a bad split count or a
+ * null workspace, SVDQ_ERR_ALIGNMENT for a misaligned one, SVDQ_ERR_SHAPE
+ * if workspace_bytes is too small.
+ */
+size_t svdq_linear_splitk_workspace(const svdq_weights* w, int M, int splits);
+svdq_status svdq_linear_splitk(const svdq_weights* w, int M, const uint8_t* xq,
+                               const float* s_x, const uint16_t* Z, uint16_t* Y,
+                               int ldy, int epilogue, int splits, void* workspace,
+                               size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the handle's sticky device

@@ -78,6 +78,9 @@ def lib() -> ctypes.CDLL:
         "svdq_linear": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _vp]),
         "svdq_get_device_error": (_i, [_vp, _vp]),
         "svdq_debug_partials": (_i, [_vp, _i, _vp, _i, _i, _i, _i, _vp, _vp]),
+        "svdq_linear_splitk_workspace": (ctypes.c_size_t, [_vp, _i, _i]),
+        "svdq_linear_splitk": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _vp,
+                                    ctypes.c_size_t, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -223,6 +226,23 @@ def svdq_linear(w: Weights, xq, s_x, Z, Y, epilogue=EPI_NONE, stream=None):
     _check(lib().svdq_linear(w.handle, M, _dev_ptr(xq), _dev_ptr(s_x), _dev_ptr(Z),
                              _dev_ptr(Y), Y.stride(0), int(epilogue), _stream_ptr(stream)),
            "svdq_linear")
+
+
+def svdq_linear_splitk_workspace(w: Weights, M: int, splits: int = 0) -> int:
+    """Workspace bytes of svdq_linear_splitk (0 for invalid arguments)."""
+    return int(lib().svdq_linear_splitk_workspace(w.handle, int(M), int(splits)))
+
+
+def svdq_linear_splitk(w: Weights, xq, s_x, Z, Y, workspace, splits=0, epilogue=EPI_NONE,
+                       stream=None):
+    """Split-K svdq_linear.  workspace: cuda tensor of at least
+    svdq_linear_splitk_workspace(w, M, splits) bytes (256-byte aligned)."""
+    M = Y.shape[0]
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().svdq_linear_splitk(w.handle, M, _dev_ptr(xq), _dev_ptr(s_x), _dev_ptr(Z),
+                                    _dev_ptr(Y), Y.stride(0), int(epilogue), int(splits),
+                                    _dev_ptr(workspace), nbytes, _stream_ptr(stream)),
+           "svdq_linear_splitk")
 
 
 def svdq_get_device_error(w: Weights, stream=None):

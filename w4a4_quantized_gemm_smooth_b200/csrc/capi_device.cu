@@ -34,9 +34,11 @@ svdq_status svdq_quantize_act(const svdq_weights* w, int M, const uint16_t* X, i
   return from_launch(svdq::launch_act_quant(w, M, X, ldx, xq, s_x, Z, stream));
 }
 
-svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
-                        const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
-                        cudaStream_t stream) {
+
+namespace {
+// Validation shared by svdq_linear and svdq_linear_splitk.
+svdq_status check_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
+                         const uint16_t* Z, const uint16_t* Y, int ldy, int epilogue) {
   svdq_status s = check_handle(w);
   if (s != SVDQ_OK) return s;
   if (M < 0 || ldy < w->N) return SVDQ_ERR_SHAPE;
@@ -46,7 +48,42 @@ svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq, const f
   if (!aligned16(xq) || !aligned16(s_x) || !aligned16(Y) || (ldy % 8) != 0 ||
       (w->rank > 0 && !aligned16(Z)))
     return SVDQ_ERR_ALIGNMENT;
+  return SVDQ_OK;
+}
+
+int resolve_splits(const svdq_weights* w, int M, int splits) {
+  const int cap = w->G < SVDQ_MAX_SPLITS ? w->G : SVDQ_MAX_SPLITS;
+  if (splits < 0 || splits > cap) return -1;
+  return splits == 0 ? svdq::splitk_auto(w, M) : splits;
+}
+}  // namespace
+
+svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
+                        const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
+                        cudaStream_t stream) {
+  svdq_status s = check_linear(w, M, xq, s_x, Z, Y, ldy, epilogue);
+  if (s != SVDQ_OK || M == 0) return s;
   return from_launch(svdq::launch_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, stream));
+}
+
+size_t svdq_linear_splitk_workspace(const svdq_weights* w, int M, int splits) {
+  if (!w || M <= 0 || !w->d_wq) return 0;
+  const int sp = resolve_splits(w, M, splits);
+  return sp < 1 ? 0 : svdq::splitk_workspace(w, M, sp);
+}
+
+svdq_status svdq_linear_splitk(const svdq_weights* w, int M, const uint8_t* xq,
+                               const float* s_x, const uint16_t* Z, uint16_t* Y, int ldy,
+                               int epilogue, int splits, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+  svdq_status s = check_linear(w, M, xq, s_x, Z, Y, ldy, epilogue);
+  if (s != SVDQ_OK || M == 0) return s;
+  const int sp = resolve_splits(w, M, splits);
+  if (sp < 1 || !workspace) return SVDQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SVDQ_ERR_ALIGNMENT;
+  if (workspace_bytes < svdq::splitk_workspace(w, M, sp)) return SVDQ_ERR_SHAPE;
+  return from_launch(svdq::launch_linear_splitk(w, M, xq, s_x, Z, Y, ldy, epilogue, sp,
+                                                workspace, stream));
 }
 
 svdq_status svdq_debug_partials(const svdq_weights* w, int M, const uint8_t* xq, int row0,

@@ -81,7 +81,26 @@ struct LinArgs {
   int sx_tma;              // 1: s_x rows are 16-byte aligned (M % 4 == 0), copy by TMA
   int32_t* P;              // partial dump (MODE 1)
   int row0, nrows, col0, ncols;
+  int splits;              // K splits per tile (1 except in MODE 3)
+  float* part;             // MODE 3: fp32 partial tiles [tile][split][warp][32 x CW]
+  int* cnt;                // MODE 3: arrivals per (tile, rescale warp), zero between uses
 };
+
+// One unit of work: output tile t, groups [g0, g1) of split sp.  The
+// low-rank stage belongs to split 0.
+struct WorkItem {
+  int t, sp, g0, g1;
+  bool lr;
+};
+__device__ __forceinline__ WorkItem work_item(const LinArgs& p, int wk) {
+  WorkItem w;
+  w.t = wk / p.splits;
+  w.sp = wk - w.t * p.splits;
+  w.g0 = (int)((long long)w.sp * p.G / p.splits);
+  w.g1 = (int)((long long)(w.sp + 1) * p.G / p.splits);
+  w.lr = w.sp == 0;
+  return w;
+}
 
 template <int BN>
 struct Lay {
@@ -201,6 +220,10 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float2 v) {
 // MODE 0: the layer (rescale, low-rank stage, epilogue, TMA store of Y).
 // MODE 1: dump the int32 group partials of the tiles covering the requested
 //         block instead of rescaling them (test hook).
+// MODE 3: the layer with the K groups of each tile split over p.splits work
+//         items; each writes its fp32 partial to p.part, and the last of a
+//         tile's splits (per rescale warp, by an atomic count) sums them in
+//         split order and runs the epilogue.
 template <int BN, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
@@ -211,6 +234,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_sx,
                  const __grid_constant__ CUtensorMap tm_sw, const LinArgs p) {
   using L = Lay<BN>;
+  constexpr bool LAYER = MODE != 1;
+  constexpr bool SPLIT = MODE == 3;
   constexpr int CW = L::CW;
   constexpr int NE = L::NE;
   constexpr int NB = L::NB;
@@ -264,14 +289,16 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       // ---------------------------------------------------- TMA producer
       uint32_t it = 0, il = 0;
       bool alive = true;
-      for (int t = blockIdx.x; t < p.num_tiles && alive; t += gridDim.x) {
+      for (int wk = blockIdx.x; wk < p.num_tiles * p.splits && alive; wk += gridDim.x) {
+        const WorkItem wi = work_item(p, wk);
+        const int t = wi.t;
         const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
         const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
-        for (int g = 0; g < G; ++g, ++it) {
+        for (int g = wi.g0; g < wi.g1; ++g, ++it) {
           const int s = it % NP;
           if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
           const uint32_t slot = sbase + L::OFF_SC + (it % L::NS) * L::SC_SLOT;
-          if (MODE == 0 && !p.sx_tma) {
+          if (LAYER && !p.sx_tma) {
             // s_x rows not 16-byte aligned: 4-byte async copies by all lanes,
             // tracked by the stage's full barrier (raised before lane 0 arrives)
 #pragma unroll 4
@@ -285,7 +312,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
           }
           if (lane == 0) {
             const uint32_t scale_bytes =
-                MODE == 0 ? (p.sx_tma ? BM * 4 : 0) + BN * 4 : 0;
+                LAYER ? (p.sx_tma ? BM * 4 : 0) + BN * 4 : 0;
             mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE + scale_bytes);
             const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
 #pragma unroll
@@ -293,7 +320,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               tma_load_2d(dst + hh * (BM * 16), &tm_a, g * 32 + 16 * hh, m0, pk_full(s));
               tma_load_2d(dst + L::PK_A + hh * (BN * 16), &tm_b, g * 32 + 16 * hh, n0, pk_full(s));
             }
-            if (MODE == 0) {
+            if (LAYER) {
               if (p.sx_tma) tma_load_2d(slot, &tm_sx, m0, g, pk_full(s));
               tma_load_2d(slot + 4 * BM, &tm_sw, n0, g, pk_full(s));
             }
@@ -302,7 +329,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         }
         if (!alive) break;
         if (lane == 0) {
-          for (int j = 0; j < p.n_lr; ++j, ++il) {
+          for (int j = 0; j < (wi.lr ? p.n_lr : 0); ++j, ++il) {
             if (!wait_or_abort(lr_empty, (il & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
             mbar_arrive_expect_tx(lr_full, L::LR_A + L::LR_B);
             const uint32_t dst = sbase + L::OFF_LR;
@@ -331,12 +358,14 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         const uint64_t init_ad = sdesc_kmajor_noswizzle(sbase + L::OFF_INIT, 128, 256);
         const uint64_t init_bd = sdesc_kmajor_noswizzle(sbase + L::OFF_INIT + L::INIT_A, 128, 256);
         uint32_t ite = 0, tb = 0, il = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-          for (int g = 0; g < G + (p.n_lr > 0 ? 1 : 0); ++g) {
+        for (int wk = blockIdx.x; wk < p.num_tiles * p.splits; wk += gridDim.x) {
+          const WorkItem wi = work_item(p, wk);
+          const bool lrs = wi.lr && p.n_lr > 0;
+          for (int g = wi.g0; g < wi.g1 + (lrs ? 1 : 0); ++g) {
             const int b = tb % NB;
             if (!wait_or_abort(tm_empty(b), ((tb / NB) & 1) ^ 1, abort_flag, p.err)) goto mma_done;
             const uint32_t d = tmem + b * BN;
-            if (g < G) {
+            if (g < wi.g1) {
               const int s = ite % NE;
               if (!wait_or_abort(ex_full(s), (ite / NE) & 1, abort_flag, p.err)) goto mma_done;
               tc_fence_after();
@@ -378,8 +407,9 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       static_assert(ROUNDS % 8 == 0, "expander split");
       auto expand_loop = [&](const auto& plan) {
         uint32_t it = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-          for (int g = 0; g < G; ++g, ++it) {
+        for (int wk = blockIdx.x; wk < p.num_tiles * p.splits; wk += gridDim.x) {
+          const WorkItem wi = work_item(p, wk);
+          for (int g = wi.g0; g < wi.g1; ++g, ++it) {
             const int se = it % NE, sp = it % NP;
             if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err)) return;
             if (!wait_or_abort(pk_full(sp), (it / NP) & 1, abort_flag, p.err)) return;
@@ -413,7 +443,9 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     uint32_t tb = 0, gs = 0;                   // TMEM use counter, group counter
     bool ok = true;
-    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+    for (int wk = blockIdx.x; wk < p.num_tiles * p.splits && ok; wk += gridDim.x) {
+      const WorkItem wi = work_item(p, wk);
+      const int t = wi.t;
       const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
       const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
       const int row = m0 + 32 * q + lane;
@@ -428,15 +460,15 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
 #pragma unroll
       for (int e = 0; e < PER; ++e) {
         const int n = ncol0 + lane * PER + e;
-        bias_n[e] = (MODE == 0 && n < p.N) ? __uint_as_float((uint32_t)__ldg(p.bias + n) << 16) : 0.0f;
+        bias_n[e] = (LAYER && n < p.N) ? __uint_as_float((uint32_t)__ldg(p.bias + n) << 16) : 0.0f;
       }
-      for (int g = 0; g < G; ++g, ++tb, ++gs) {
+      for (int g = wi.g0; g < wi.g1; ++g, ++tb, ++gs) {
         const uint32_t slot = sbase + L::OFF_SC + (gs % L::NS) * L::SC_SLOT;
         const int b = tb % NB;
         if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
-        if (MODE == 0) {
+        if (LAYER) {
           // 16-column chunks, double-buffered: the loads of chunk c+1 are in
           // flight while chunk c is rescaled (wait::ld waits for all).
           float2 sx2[4];
@@ -494,8 +526,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         __syncwarp();
         if (lane == 0) mbar_arrive(tm_empty(b));
       }
-      if (!ok || MODE != 0) continue;
-      if (p.n_lr > 0) {
+      if (!ok || !LAYER) continue;
+      if (wi.lr && p.n_lr > 0) {
         const int b = tb % NB;
         if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
@@ -525,6 +557,39 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         __syncwarp();
         if (lane == 0) mbar_arrive(tm_empty(b));
         ++tb;
+      }
+      if (SPLIT) {
+        // write this split's partial (thread-private order, same for every
+        // split), publish it, and let the last arriving split of this warp's
+        // slice sum all of them in split order
+        float2* mine = reinterpret_cast<float2*>(
+            p.part + ((size_t)(t * p.splits + wi.sp) * N_RES_WARPS + rw) * (32 * CW));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int k = 0; k < CW / 8; ++k) mine[(i * (CW / 8) + k) * 32 + lane] = acc[i][k];
+        __threadfence();
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) old = atomicAdd(p.cnt + t * N_RES_WARPS + rw, 1);
+        old = __shfl_sync(0xFFFFFFFFu, old, 0);
+        if (old != p.splits - 1) continue;
+        __threadfence();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int k = 0; k < CW / 8; ++k) acc[i][k] = make_float2(0.0f, 0.0f);
+        for (int sp = 0; sp < p.splits; ++sp) {
+          const float2* src = reinterpret_cast<const float2*>(
+              p.part + ((size_t)(t * p.splits + sp) * N_RES_WARPS + rw) * (32 * CW));
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < CW / 8; ++k)
+              acc[i][k] = __fadd2_rn(acc[i][k], __ldcg(src + (i * (CW / 8) + k) * 32 + lane));
+        }
+        __syncwarp();
+        if (lane == 0) atomicExch(p.cnt + t * N_RES_WARPS + rw, 0);   // ready for the next call
       }
       // epilogue: bias, GELU, bf16, swizzled staging, TMA store
 #pragma unroll
@@ -563,7 +628,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       }
       __syncwarp();
     }
-    if (MODE == 0 && lane == 0) tma_store_wait0();
+    if (LAYER && lane == 0) tma_store_wait0();
     __syncwarp();
   }
 
@@ -632,7 +697,8 @@ cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtens
     attr = true;
   }
   a.num_tiles = tiles_m * a.tiles_n;
-  const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
+  const int work = a.num_tiles * a.splits;
+  const int grid = work < num_sms() ? work : num_sms();
   linear_ws_kernel<BN, MODE><<<grid, THREADS, L::ALLOC, st>>>(ta, tb, ty, tz, tl, tsx, tsw, a);
   return cudaGetLastError();
 }
@@ -643,36 +709,37 @@ int pick_bn(int N) {
   return (r != 0 && r <= 128) ? 128 : 256;
 }
 
-}  // namespace
+struct LinMaps {
+  CUtensorMap ta, tb, ty, tz, tl, tsx, tsw;
+};
 
-cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
-                          const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
-                          cudaStream_t st) {
-  const int BN = pick_bn(w->N);
-  CUtensorMap ta, tb, ty, tz, tl;
-  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 16, BM,
+// Tensor maps and kernel arguments shared by the layer launches.
+bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
+                  const uint16_t* Z, uint16_t* Y, int ldy, int epilogue, int BN, LinMaps& m,
+                  LinArgs& a) {
+  if (!make_map(&m.ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 16, BM,
                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 16, BN,
+      !make_map(&m.tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 16, BN,
                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
+      !make_map(&m.ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
                 CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  tz = ta;
-  tl = ta;
-  CUtensorMap tsx = ta, tsw;
+    return false;
+  m.tz = m.ta;
+  m.tl = m.ta;
+  m.tsx = m.ta;
   const bool sx_tma = (M % 4) == 0;
-  if ((sx_tma && !make_map(&tsx, s_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, w->G, (uint64_t)M * 4,
-                           BM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
-      !make_map(&tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N16, w->G, (uint64_t)w->N16 * 4,
-                BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
+  if ((sx_tma && !make_map(&m.tsx, s_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, w->G,
+                           (uint64_t)M * 4, BM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
+      !make_map(&m.tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N16, w->G,
+                (uint64_t)w->N16 * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
   if (w->rank > 0 &&
-      (!make_map(&tz, Z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank, M, (uint64_t)w->rank * 2, 8,
+      (!make_map(&m.tz, Z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank, M, (uint64_t)w->rank * 2, 8,
                  BM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-       !make_map(&tl, w->d_L2T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank_pad32, w->N,
+       !make_map(&m.tl, w->d_L2T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank_pad32, w->N,
                  (uint64_t)w->rank_pad32 * 2, 8, BN, CU_TENSOR_MAP_SWIZZLE_NONE)))
-    return cudaErrorInvalidValue;
-  LinArgs a{};
+    return false;
+  a = LinArgs{};
   a.s_x = s_x; a.s_w = w->d_sw; a.Z = Z; a.L2T = w->d_L2T; a.bias = w->d_bias;
   a.M = M; a.N = w->N; a.K = w->K; a.G = w->G;
   a.rank = w->rank; a.rank_pad32 = w->rank_pad32; a.n_lr = w->rank_pad32 / 32;
@@ -681,9 +748,66 @@ cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const
   a.tile_m0 = 0; a.tile_n0 = 0;
   a.err = w->d_err;
   a.sx_tma = sx_tma ? 1 : 0;
+  a.splits = 1;
+  return true;
+}
+
+int num_tiles(const svdq_weights* w, int M) {
+  const int BN = pick_bn(w->N);
+  return ((M + BM - 1) / BM) * ((w->N + BN - 1) / BN);
+}
+
+size_t splitk_counter_bytes(const svdq_weights* w, int M) {
+  return ((size_t)num_tiles(w, M) * N_RES_WARPS * sizeof(int) + 255) / 256 * 256;
+}
+
+}  // namespace
+
+cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
+                          const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
+                          cudaStream_t st) {
+  const int BN = pick_bn(w->N);
+  LinMaps m;
+  LinArgs a;
+  if (!build_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, BN, m, a)) return cudaErrorInvalidValue;
   const int tiles_m = (M + BM - 1) / BM;
-  return BN == 256 ? launch_ws<256, 0>(w, ta, tb, ty, tz, tl, tsx, tsw, a, tiles_m, st)
-                   : launch_ws<128, 0>(w, ta, tb, ty, tz, tl, tsx, tsw, a, tiles_m, st);
+  return BN == 256 ? launch_ws<256, 0>(w, m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx, m.tsw, a, tiles_m, st)
+                   : launch_ws<128, 0>(w, m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx, m.tsw, a, tiles_m, st);
+}
+
+int splitk_auto(const svdq_weights* w, int M) {
+  const int tiles = num_tiles(w, M);
+  if (2 * tiles > num_sms()) return 1;          // the tiles alone fill the GPU
+  int s = num_sms() / (tiles > 0 ? tiles : 1);
+  const int cap = w->G / 2 < SVDQ_MAX_SPLITS ? w->G / 2 : SVDQ_MAX_SPLITS;   // >= 2 groups each
+  if (s > cap) s = cap;
+  return s < 1 ? 1 : s;
+}
+
+size_t splitk_workspace(const svdq_weights* w, int M, int splits) {
+  const int BN = pick_bn(w->N);
+  return splitk_counter_bytes(w, M) + (size_t)num_tiles(w, M) * splits * BM * BN * sizeof(float);
+}
+
+cudaError_t launch_linear_splitk(const svdq_weights* w, int M, const uint8_t* xq,
+                                 const float* s_x, const uint16_t* Z, uint16_t* Y, int ldy,
+                                 int epilogue, int splits, void* workspace, cudaStream_t st) {
+  if (splits == 1)      // nothing to split: the plain kernel, same result bits
+    return launch_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, st);
+  const int BN = pick_bn(w->N);
+  LinMaps m;
+  LinArgs a;
+  if (!build_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, BN, m, a)) return cudaErrorInvalidValue;
+  const size_t cb = splitk_counter_bytes(w, M);
+  a.splits = splits;
+  a.cnt = static_cast<int*>(workspace);
+  a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + cb);
+  // the arrival counts must start at zero (the kernel also leaves them at zero)
+  cudaError_t e = cudaMemsetAsync(workspace, 0, cb, st);
+  if (e != cudaSuccess) return e;
+  const int tiles_m = (M + BM - 1) / BM;
+  return BN == 256 ? launch_ws<256, 3>(w, m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx, m.tsw, a, tiles_m, st)
+                   : launch_ws<128, 3>(w, m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx, m.tsw, a, tiles_m, st);
 }
 
 cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int row0,
@@ -698,6 +822,7 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
   LinArgs a{};
   a.M = M; a.N = w->N; a.K = w->K; a.G = w->G;
   a.rank = 0; a.rank_pad32 = 0; a.n_lr = 0; a.epilogue = 0;
+  a.splits = 1;
   a.err = w->d_err;
   a.P = P; a.row0 = row0; a.nrows = nrows; a.col0 = col0; a.ncols = ncols;
   const int tm0 = row0 / BM, tm1 = (row0 + nrows - 1) / BM;

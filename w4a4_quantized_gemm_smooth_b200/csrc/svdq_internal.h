@@ -54,6 +54,14 @@ cudaError_t launch_act_quant(const svdq_weights* w, int M, const uint16_t* X,
 cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq,
                           const float* s_x, const uint16_t* Z, uint16_t* Y,
                           int ldy, int epilogue, cudaStream_t stream);
+// Split-K form of launch_linear (K groups of each tile spread over `splits`
+// work items; workspace = zeroed counters then fp32 partials, sized by
+// splitk_workspace).  splitk_auto picks a split count for M.
+int splitk_auto(const svdq_weights* w, int M);
+size_t splitk_workspace(const svdq_weights* w, int M, int splits);
+cudaError_t launch_linear_splitk(const svdq_weights* w, int M, const uint8_t* xq,
+                                 const float* s_x, const uint16_t* Z, uint16_t* Y, int ldy,
+                                 int epilogue, int splits, void* workspace, cudaStream_t stream);
 cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq,
                             int row0, int nrows, int col0, int ncols,
                             int32_t* P, cudaStream_t stream);
