@@ -207,6 +207,29 @@ svdq_status svdq_linear_splitk(const svdq_weights* w, int M, const uint8_t* xq,
                                size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * svdq_linear_splitk without a workspace argument: the scratch (arrival
+ * counters and fp32 partial tiles) is a fixed 16 MiB device array inside
+ * the library, one per device, so the call allocates nothing (no
+ * cudaMalloc, no allocating library).  The SVDQuant pages have no
+ * counterpart; this exists for allocation-free callers.
+ *
+ * Same arguments and result bits as svdq_linear_splitk with the same
+ * `splits` (0 = automatic).  The call clears the counters before its launch.
+ * Requests whose workspace (svdq_linear_splitk_workspace) exceeds 16 MiB
+ * are rejected with SVDQ_ERR_SHAPE; a single split needs no scratch.
+ * The scratch is shared by every call on the device: calls that overlap
+ * in time (different streams, or handles used concurrently) race and
+ * corrupt each other's results, so order them.  The first call on each
+ * device looks up the array's address (which can load the library's
+ * device code): make it before any stream capture.
+ * Errors: as svdq_linear_splitk; SVDQ_ERR_CUDA if the set-up fails.
+ */
+svdq_status svdq_linear_splitk_noalloc(const svdq_weights* w, int M, const uint8_t* xq,
+                                       const float* s_x, const uint16_t* Z, uint16_t* Y,
+                                       int ldy, int epilogue, int splits,
+                                       cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the handle's sticky device
  * error word: SVDQ_OK, or SVDQ_ERR_DEVICE_TIMEOUT if a bounded wait in a
  * kernel of this handle expired since the last read.

@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
         "svdq_linear_splitk_workspace": (ctypes.c_size_t, [_vp, _i, _i]),
         "svdq_linear_splitk": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _vp,
                                     ctypes.c_size_t, _vp]),
+        "svdq_linear_splitk_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -243,6 +244,16 @@ def svdq_linear_splitk(w: Weights, xq, s_x, Z, Y, workspace, splits=0, epilogue=
                                     _dev_ptr(Y), Y.stride(0), int(epilogue), int(splits),
                                     _dev_ptr(workspace), nbytes, _stream_ptr(stream)),
            "svdq_linear_splitk")
+
+
+def svdq_linear_splitk_noalloc(w: Weights, xq, s_x, Z, Y, splits=0, epilogue=EPI_NONE,
+                               stream=None):
+    """svdq_linear_splitk with the library's fixed device scratch (no allocation)."""
+    M = Y.shape[0]
+    _check(lib().svdq_linear_splitk_noalloc(w.handle, M, _dev_ptr(xq), _dev_ptr(s_x),
+                                            _dev_ptr(Z), _dev_ptr(Y), Y.stride(0),
+                                            int(epilogue), int(splits), _stream_ptr(stream)),
+           "svdq_linear_splitk_noalloc")
 
 
 def svdq_get_device_error(w: Weights, stream=None):

@@ -19,24 +19,8 @@ svdq_status from_launch(cudaError_t e) { return e == cudaSuccess ? SVDQ_OK : SVD
 
 }  // namespace
 
-extern "C" {
-
-svdq_status svdq_quantize_act(const svdq_weights* w, int M, const uint16_t* X, int ldx,
-                              uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t stream) {
-  svdq_status s = check_handle(w);
-  if (s != SVDQ_OK) return s;
-  if (M < 0 || ldx < w->K) return SVDQ_ERR_SHAPE;
-  if (M == 0) return SVDQ_OK;
-  if (!X || !xq || !s_x || (w->rank > 0 && !Z)) return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(X) || !aligned16(xq) || !aligned16(s_x) || (ldx % 8) != 0 ||
-      (w->rank > 0 && !aligned16(Z)))
-    return SVDQ_ERR_ALIGNMENT;
-  return from_launch(svdq::launch_act_quant(w, M, X, ldx, xq, s_x, Z, stream));
-}
-
-
-namespace {
-// Validation shared by svdq_linear and svdq_linear_splitk.
+namespace svdq {
+// Validation shared by the svdq_linear entry points.
 svdq_status check_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
                          const uint16_t* Z, const uint16_t* Y, int ldy, int epilogue) {
   svdq_status s = check_handle(w);
@@ -56,7 +40,27 @@ int resolve_splits(const svdq_weights* w, int M, int splits) {
   if (splits < 0 || splits > cap) return -1;
   return splits == 0 ? svdq::splitk_auto(w, M) : splits;
 }
-}  // namespace
+}  // namespace svdq
+using svdq::check_linear;
+using svdq::resolve_splits;
+
+extern "C" {
+
+svdq_status svdq_quantize_act(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                              uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t stream) {
+  svdq_status s = check_handle(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || ldx < w->K) return SVDQ_ERR_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !xq || !s_x || (w->rank > 0 && !Z)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(xq) || !aligned16(s_x) || (ldx % 8) != 0 ||
+      (w->rank > 0 && !aligned16(Z)))
+    return SVDQ_ERR_ALIGNMENT;
+  return from_launch(svdq::launch_act_quant(w, M, X, ldx, xq, s_x, Z, stream));
+}
+
+
+
 
 svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
                         const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,

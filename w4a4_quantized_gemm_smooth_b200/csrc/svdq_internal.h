@@ -54,6 +54,12 @@ cudaError_t launch_act_quant(const svdq_weights* w, int M, const uint16_t* X,
 cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq,
                           const float* s_x, const uint16_t* Z, uint16_t* Y,
                           int ldy, int epilogue, cudaStream_t stream);
+// Argument checks of the svdq_linear entry points (SVDQ_OK or the error),
+// and the split count a call resolves to (-1: invalid).
+svdq_status check_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
+                         const uint16_t* Z, const uint16_t* Y, int ldy, int epilogue);
+int resolve_splits(const svdq_weights* w, int M, int splits);
+
 // Split-K form of launch_linear (K groups of each tile spread over `splits`
 // work items; workspace = zeroed counters then fp32 partials, sized by
 // splitk_workspace).  splitk_auto picks a split count for M.
