@@ -75,6 +75,7 @@ def _peaks():
 
 def _workload(name):
     specs = dict(synth.WORKLOADS)
+    specs.update({p.name: p for p in synth.pixart_points()})
     if name not in specs:
         raise SystemExit(f"unknown workload {name}; choose from {sorted(specs)}")
     return specs[name]
@@ -431,7 +432,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="flux_qkv")
+    ap.add_argument("--workload", default="flux_qkv",
+                    help="a name of synth.WORKLOADS or of synth.pixart_points()")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
