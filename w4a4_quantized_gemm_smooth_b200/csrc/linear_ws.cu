@@ -74,7 +74,7 @@ struct LinArgs {
   const uint16_t* L2T;     // [N_pad][rank_pad32]
   const uint16_t* bias;
   int M, N, K, G;
-  int rank, rank_pad32, n_lr;
+  int rank, rank_pad32, n_lr;   // n_lr: 16-wide low-rank slices, ceil(rank / 16)
   int epilogue;
   int tiles_n, num_tiles, tile_m0, tile_n0;
   int* err;
@@ -114,7 +114,11 @@ struct Lay {
   static constexpr int OFF_Y = 0;
   static constexpr int OFF_PK = OFF_Y + N_RES_WARPS * Y_WARP;
   static constexpr int OFF_EX = OFF_PK + NP * PK_STAGE;
-  static constexpr int LR_A = BM * 64, LR_B = BN * 64;     // 4 chunks x rows x 16 B
+  // low-rank stage: NLR slots of one 16-wide K slice each (2 chunks x rows x
+  // 16 B of Z and of L2^T), so that slices load while earlier ones multiply
+  // (four slots where shared memory allows: rank 64 in flight at once)
+  static constexpr int NLR = BN == 256 ? 2 : 4;
+  static constexpr int LR_SA = BM * 32, LR_SB = BN * 32, LR_SLOT = LR_SA + LR_SB;
   static constexpr int OFF_LR = OFF_EX + NE * EX_STAGE;
   // per-group scales: ring of NP + NE + NB slots, each s_x[128] then s_w[BN],
   // filled by the producer warp together with the packed codes.  The producer
@@ -123,15 +127,15 @@ struct Lay {
   // group j - NP - NE - NB, the slot's previous owner, has finished.
   static constexpr int NS = NP + NE + NB;
   static constexpr int SC_SLOT = (BM + BN) * 4;
-  static constexpr int OFF_SC = OFF_LR + LR_A + LR_B;
+  static constexpr int OFF_SC = OFF_LR + NLR * LR_SLOT;
   static constexpr int OFF_BIAS = OFF_SC + NS * SC_SLOT;   // per warp CW floats
   // constant operands of the accumulator-initialising bf16 MMA (K = 16)
   static constexpr int INIT_A = BM * 32, INIT_B = BN * 32;
   static constexpr int OFF_INIT = OFF_BIAS + N_RES_WARPS * CW * 4;
   static constexpr int OFF_BAR = OFF_INIT + INIT_A + INIT_B;
   // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[NB],
-  // tm_empty[NB], lr_full, lr_empty
-  static constexpr int N_BARS = 2 * NP + 2 * NE + 2 * NB + 2;
+  // tm_empty[NB], lr_full[NLR], lr_empty[NLR]
+  static constexpr int N_BARS = 2 * NP + 2 * NE + 2 * NB + 2 * NLR;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;              // slack for 1024-B alignment
@@ -250,8 +254,9 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
   auto ex_empty = [&](int s) { return bar0 + 8u * (2 * NP + NE + s); };
   auto tm_full = [&](int b) { return bar0 + 8u * (2 * NP + 2 * NE + b); };
   auto tm_empty = [&](int b) { return bar0 + 8u * (2 * NP + 2 * NE + NB + b); };
-  const uint32_t lr_full = bar0 + 8u * (2 * NP + 2 * NE + 2 * NB);
-  const uint32_t lr_empty = bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + 1);
+  constexpr int NLR = L::NLR;
+  auto lr_full = [&](int s) { return bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + s); };
+  auto lr_empty = [&](int s) { return bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + NLR + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -262,8 +267,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     for (int s = 0; s < NP; ++s) { mbar_init(pk_full(s), 1); mbar_init(pk_empty(s), N_EXP); }
     for (int s = 0; s < NE; ++s) { mbar_init(ex_full(s), N_EXP); mbar_init(ex_empty(s), 1); }
     for (int b = 0; b < NB; ++b) { mbar_init(tm_full(b), 1); mbar_init(tm_empty(b), N_RES_WARPS); }
-    mbar_init(lr_full, 1);
-    mbar_init(lr_empty, 1);
+    for (int s = 0; s < NLR; ++s) { mbar_init(lr_full(s), 1); mbar_init(lr_empty(s), 1); }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -330,13 +334,14 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         if (!alive) break;
         if (lane == 0) {
           for (int j = 0; j < (wi.lr ? p.n_lr : 0); ++j, ++il) {
-            if (!wait_or_abort(lr_empty, (il & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
-            mbar_arrive_expect_tx(lr_full, L::LR_A + L::LR_B);
-            const uint32_t dst = sbase + L::OFF_LR;
+            const int ls = il % NLR;
+            if (!wait_or_abort(lr_empty(ls), ((il / NLR) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
+            mbar_arrive_expect_tx(lr_full(ls), L::LR_SLOT);
+            const uint32_t dst = sbase + L::OFF_LR + ls * L::LR_SLOT;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              tma_load_2d(dst + c * (BM * 16), &tm_z, 32 * j + 8 * c, m0, lr_full);
-              tma_load_2d(dst + L::LR_A + c * (BN * 16), &tm_l2, 32 * j + 8 * c, n0, lr_full);
+            for (int c = 0; c < 2; ++c) {
+              tma_load_2d(dst + c * (BM * 16), &tm_z, 16 * j + 8 * c, m0, lr_full(ls));
+              tma_load_2d(dst + L::LR_SA + c * (BN * 16), &tm_l2, 16 * j + 8 * c, n0, lr_full(ls));
             }
           }
         }
@@ -346,7 +351,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       if (lane == 0) {
         for (uint32_t k = (it > NP ? it - NP : 0); k < it; ++k)
           mbar_wait_bounded(pk_full(k % NP), (k / NP) & 1, LIMIT_NS);
-        if (il > 0) mbar_wait_bounded(lr_full, (il - 1) & 1, LIMIT_NS);
+        for (uint32_t k = (il > NLR ? il - NLR : 0); k < il; ++k)
+          mbar_wait_bounded(lr_full(k % NLR), (k / NLR) & 1, LIMIT_NS);
       }
       cp_async_wait<0>();
       __syncwarp();
@@ -379,15 +385,15 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               ++ite;
             } else {
               for (int j = 0; j < p.n_lr; ++j, ++il) {
-                if (!wait_or_abort(lr_full, il & 1, abort_flag, p.err)) goto mma_done;
+                const int ls = il % NLR;
+                if (!wait_or_abort(lr_full(ls), (il / NLR) & 1, abort_flag, p.err)) goto mma_done;
                 tc_fence_after();
-                const uint32_t la = sbase + L::OFF_LR;
+                const uint32_t la = sbase + L::OFF_LR + ls * L::LR_SLOT;
                 // chunk c of the slice at c * rows * 16 bytes, row r at r * 16
                 const uint64_t ad = sdesc_kmajor_noswizzle(la, BM * 16, 128);
-                const uint64_t bd = sdesc_kmajor_noswizzle(la + L::LR_A, BN * 16, 128);
+                const uint64_t bd = sdesc_kmajor_noswizzle(la + L::LR_SA, BN * 16, 128);
                 mma_bf16(d, ad, bd, id_bf, j > 0 ? 1u : 0u);
-                mma_bf16(d, ad + ((2 * BM * 16) >> 4), bd + ((2 * BN * 16) >> 4), id_bf, 1u);
-                mma_commit(lr_empty);
+                mma_commit(lr_empty(ls));
               }
             }
             mma_commit(tm_full(b));
@@ -742,7 +748,7 @@ bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* 
   a = LinArgs{};
   a.s_x = s_x; a.s_w = w->d_sw; a.Z = Z; a.L2T = w->d_L2T; a.bias = w->d_bias;
   a.M = M; a.N = w->N; a.K = w->K; a.G = w->G;
-  a.rank = w->rank; a.rank_pad32 = w->rank_pad32; a.n_lr = w->rank_pad32 / 32;
+  a.rank = w->rank; a.rank_pad32 = w->rank_pad32; a.n_lr = (w->rank + 15) / 16;
   a.epilogue = epilogue;
   a.tiles_n = (w->N + BN - 1) / BN;
   a.tile_m0 = 0; a.tile_n0 = 0;
