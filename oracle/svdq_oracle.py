@@ -16,6 +16,8 @@ What it computes follows "SVDQuant: How a Small High-Precision Branch Makes
   * two-branch output  Y = (X~ L1) L2 + Q(X~) Q(R)            (section 4.2, eq. 7)
   * LoRA in smoothed coordinates  [L1 | D A] [L2 ; B]          (section 7, eq. 13)
   * MAC and storage ratios                                     (section 6, eqs. 11-12)
+  * calibration refinement: alpha search by the calibrated layer-output
+    error, factors re-fitted to W~ - Q(R)                        (section 5)
 
 Readings taken where the pages leave a step open (each is listed in the
 design notes of the repository):
@@ -46,7 +48,7 @@ __all__ = [
     "calib_absmax", "pack_weights", "quantize_act", "group_partials",
     "linear", "gelu", "layer_forward", "mac_ratio", "storage_ratio",
     "two_branch_unquantized", "dequantize_groups", "residual_quantize",
-    "leading_svd",
+    "leading_svd", "layer_output_error", "refine_factors", "pack_weights_calibrated",
 ]
 
 GROUP = 64
@@ -335,6 +337,78 @@ def layer_forward(X_bits, packed, apply_gelu=False, rows=None, cols=None):
     Y, Yb = linear(xc, s_x, Z, packed["wcodes"], packed["s_w"], packed["L2b"],
                    packed["bias"], apply_gelu, rows, cols)
     return dict(xcodes=xc, s_x=s_x, Z=Z, Y=Y, Ybf16=Yb)
+
+
+# --------------------------------------------------------------------------
+# calibration refinement (review section 5, the offline procedure): search
+# the migration strength alpha by the calibrated layer-output error, with
+# alternating updates of the protected factors from W~ - Q(R)
+# --------------------------------------------------------------------------
+def layer_output_error(X_bits, packed, W_bits):
+    """Relative Frobenius error of the quantised layer (both branches, no
+    bias, before the bf16 output rounding) against X W on the tokens X:
+    ||Y_q - X W||_F / ||X W||_F, all in fp64."""
+    X = bf16_bits_to_f64(X_bits)
+    W = bf16_bits_to_f64(W_bits).T                       # [K, N]
+    ref = X @ W
+    no_bias = dict(packed, bias=np.zeros(W.shape[1]))
+    Yq = layer_forward(X_bits, no_bias)["Y"]
+    return float(np.linalg.norm(Yq - ref) / np.linalg.norm(ref))
+
+
+def _set_factors(p, Wt, L1, L2):
+    """New protected factors for a packed layer: store them as bf16, take R
+    against the stored factors and quantise it again (eqs. 10, 1)."""
+    L1b = round_bf16(L1)
+    L2b = round_bf16(L2)
+    R, codes, s_w = residual_quantize(Wt, L1b, L2b)
+    q = dict(p)
+    q.update(L1=L1, L2=L2, L1b=L1b, L2b=L2b, R=R, wcodes=codes, wq=pack_nibbles(codes), s_w=s_w)
+    return q
+
+
+def refine_factors(p, svd=None):
+    """One alternating step: the rank-r SVD of W~ - deq(Q(R)) gives the new
+    factors, then R is recomputed against W~ and quantised."""
+    Wt = p["Wt"]
+    r = p["L1b"].shape[1]
+    T = Wt - dequantize_groups(p["wcodes"], p["s_w"]).T   # deq(Q(R)) is [N, K]
+    if svd is None:
+        U, S, Vt = np.linalg.svd(T, full_matrices=False)
+    else:
+        U, S, Vt = leading_svd(T, r + 1)
+    return _set_factors(p, Wt, U[:, :r] * S[None, :r], Vt[:r, :])
+
+
+def pack_weights_calibrated(W_bits, X_cal_bits, rank, alphas=(0.3, 0.4, 0.5, 0.6, 0.7),
+                            iters=1, bias_bits=None, lora_A_bits=None, lora_B_bits=None,
+                            lora_scale=1.0, svd=None):
+    """For every candidate alpha: smoothing, SVD, residual quantisation, then
+    `iters` alternating refinements; keep the candidate with the smallest
+    calibrated layer-output error (the first one on ties).  The statistics
+    and the error use the calibration tokens X_cal.  LoRA joins the branch
+    afterwards, as in pack_weights.  Returns (packed, errors per alpha)."""
+    a = calib_absmax(bf16_bits_to_f64(X_cal_bits))
+    best, best_err, errs = None, None, []
+    for alpha in alphas:
+        p = pack_weights(W_bits, a, rank, alpha=alpha, svd=svd)
+        for _ in range(iters):
+            p = refine_factors(p, svd=svd)
+        e = layer_output_error(X_cal_bits, p, W_bits)
+        errs.append(e)
+        if best is None or e < best_err:
+            best, best_err = dict(p, alpha=alpha), e
+    p = best
+    bias = np.zeros(p["N"]) if bias_bits is None else bf16_bits_to_f64(bias_bits)
+    p = dict(p, bias=bias)
+    if lora_A_bits is not None and lora_A_bits.shape[1] > 0:
+        A = bf16_bits_to_f64(lora_A_bits)
+        B = bf16_bits_to_f64(lora_B_bits)
+        DA = (p["lam"][:, None] * A) * float(np.float32(lora_scale))
+        p["L1b"] = np.hstack([p["L1b"], round_bf16(DA)])
+        p["L2b"] = np.vstack([p["L2b"], B])
+        p["rank"] = p["L1b"].shape[1]
+    return p, errs
 
 
 def two_branch_unquantized(X, lam, L1, L2, R, bias):
