@@ -127,6 +127,33 @@ svdq_status svdq_pack_weights_host(int K, int N, int rank, int group,
                                    const uint16_t* lora_B, float lora_scale,
                                    svdq_weights** out);
 
+/*
+ * Offline pack with the calibration refinement of the review's offline
+ * procedure (section 5): for every candidate migration strength alphas[i]
+ * (each in (0, 1)) the layer is smoothed, factored and its residual
+ * quantised as in svdq_pack_weights; then `refine_iters` alternating steps
+ * replace the factors by the rank-r SVD of W~ - deq(Q(R)) and recompute and
+ * quantise R against W~.  Each candidate is scored by the calibrated
+ * layer-output error on the tokens X_cal (host bf16 [M_cal][ldx]):
+ *   err = ||Y_q - X W||_F / ||X W||_F   (fp64, both branches, no bias)
+ * where Y_q is the quantised layer (activation statistics from X_cal).  The
+ * candidate with the smallest error is packed (the first one on ties); LoRA
+ * and bias join as in svdq_pack_weights.  errors (host, n_alpha doubles, may
+ * be NULL) receives every candidate's error.  to_device != 0 uploads to the
+ * current device (stream ordered); 0 gives a host-only handle.
+ * Errors: as svdq_pack_weights; SVDQ_ERR_INVALID_ARG for missing or empty
+ * calibration tokens, an alpha outside (0, 1) or a negative iteration count.
+ */
+svdq_status svdq_pack_weights_calibrated(int K, int N, int rank, int group,
+                                         const uint16_t* W, const uint16_t* X_cal,
+                                         int M_cal, int ldx, int n_alpha,
+                                         const double* alphas, int refine_iters,
+                                         const uint16_t* bias, int lora_rank,
+                                         const uint16_t* lora_A, const uint16_t* lora_B,
+                                         float lora_scale, int to_device,
+                                         cudaStream_t stream, double* errors,
+                                         svdq_weights** out);
+
 /* Sizes of a handle; any output pointer may be NULL.  `rank` is the total
  * branch rank (svd_rank + lora_rank). */
 svdq_status svdq_weights_info(const svdq_weights* w, int* K, int* N, int* rank,

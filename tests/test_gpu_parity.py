@@ -185,3 +185,27 @@ def test_save_load_roundtrip(tmp_path):
     assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
     w.free()
     w2.free()
+
+
+def test_calibrated_pack_layer():
+    """A layer packed with the calibrated alpha search and one refinement
+    runs through the hot path like any other."""
+    spec = synth.layer_spec("calgpu", 192, 640, 320, 24, 55)
+    L = synth.make_layer(spec)
+    w, errs = S.svdq_pack_weights_calibrated(L.W, L.X, 24, refine_iters=1, bias_bits=L.b)
+    p, errs_o = oracle.pack_weights_calibrated(L.W, L.X, 24, iters=1, bias_bits=L.b)
+    assert np.allclose(errs, errs_o, rtol=1e-6, atol=0)
+    X = to_dev(L.X)
+    lin = S.SVDQLinear(w)
+    xq, s_x, Z, Y = lin.buffers(L.X.shape[0])
+    lin.forward(X, out=Y)
+    torch.cuda.synchronize()
+    S.svdq_get_device_error(w)
+    xc, sxo, Zo, xhat = oracle.quantize_act(L.X, p["inv_lambda"], p["L1b"])
+    assert np.array_equal(xq.cpu().numpy(), oracle.pack_nibbles(xc))
+    assert np.array_equal(s_x.cpu().numpy().astype(np.float64), sxo)
+    signs = column_signs(w.export()["L1"], p["L1b"])
+    check_z(to_bits(Z), Zo, xhat, p["L1b"], signs)
+    _, Yo = oracle.linear(xc, sxo, Zo, p["wcodes"], p["s_w"], p["L2b"], p["bias"])
+    assert rel_fro(oracle.bf16_bits_to_f64(to_bits(Y)), Yo) <= Y_REL_FRO
+    w.free()

@@ -1,5 +1,6 @@
-// Host side of the C ABI: the offline pack (SVDQuant review section 5, the
-// offline procedure without refinement), handle management, export, save/load.
+// Host side of the C ABI: the offline pack (SVDQuant review section 5: the
+// offline procedure, with or without the calibrated alpha search and the
+// alternating factor refinement), handle management, export, save/load.
 //
 // Exactness contract with the checks: every rounding below is a single IEEE
 // rounding of a value that both sides define the same way, so the codes and
@@ -131,6 +132,235 @@ svdq_status upload(svdq_weights* w, cudaStream_t st) {
 
 }  // namespace svdq
 
+namespace {
+
+// One candidate of the offline pack: smoothing, protected factors and the
+// quantised residual (math layout: K input channels x N output channels).
+struct Candidate {
+  std::vector<double> lam, Wt;     // lambda [K]; W~ = diag(lambda) W [K][N]
+  std::vector<float> inv_lambda;   // fl32(1 / lambda)
+  std::vector<double> sigma;       // leading singular values [rank + 1]
+  std::vector<uint16_t> L1, L2;    // bf16 factors [K][rank], [rank][N]
+  std::vector<uint8_t> wq;         // packed residual codes [N][K/2]
+  std::vector<float> sw;           // residual scales [G][N]
+};
+
+// eqs. 3-4: lambda from the activation statistic and the weight's per-channel
+// absmax (lambda = 1 where either is 0), then W~.
+svdq_status smooth(int K, int N, const uint16_t* W, const float* act_absmax, double alpha,
+                   Candidate& c) {
+  for (int k = 0; k < K; ++k) {
+    const double a = act_absmax[k];
+    if (!std::isfinite(a) || a < 0) return SVDQ_ERR_NUMERIC;
+  }
+  std::vector<double> wmax(K, 0.0);
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      const double v = bf16_to_f64(W[(size_t)n * K + k]);
+      if (!std::isfinite(v)) return SVDQ_ERR_NUMERIC;
+      wmax[k] = std::fmax(wmax[k], std::fabs(v));
+    }
+  c.lam.assign(K, 1.0);
+  c.inv_lambda.resize(K);
+  for (int k = 0; k < K; ++k) {
+    const double a = act_absmax[k], m = wmax[k];
+    double l = 1.0;
+    if (a > 0.0 && m > 0.0)
+      l = (alpha == 0.5) ? std::sqrt(a) / std::sqrt(m)
+                         : std::pow(a, alpha) / std::pow(m, 1.0 - alpha);
+    c.lam[k] = l;
+    c.inv_lambda[k] = (float)(1.0 / l);
+  }
+  c.Wt.resize((size_t)K * N);
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k)
+      c.Wt[(size_t)k * N + n] = c.lam[k] * bf16_to_f64(W[(size_t)n * K + k]);
+  return SVDQ_OK;
+}
+
+// eq. 10: the rank-r factors of T (stored as bf16) and T's leading singular
+// values.
+svdq_status fit_factors(const double* T, int K, int N, int rank, Candidate& c) {
+  const int nsv = std::min(rank + 1, std::min(K, N));
+  std::vector<double> sig(nsv), L1((size_t)K * (rank > 0 ? rank : 1)),
+      L2((size_t)(rank > 0 ? rank : 1) * N);
+  if (svdq::top_singular(T, K, N, nsv, rank, sig.data(), L1.data(), L2.data()))
+    return SVDQ_ERR_NUMERIC;
+  c.sigma.assign(rank + 1, 0.0);
+  for (int j = 0; j < nsv; ++j) c.sigma[j] = sig[j];
+  c.L1.assign((size_t)K * rank, 0);
+  c.L2.assign((size_t)rank * N, 0);
+  for (int k = 0; k < K; ++k)
+    for (int j = 0; j < rank; ++j) c.L1[(size_t)k * rank + j] = f64_to_bf16(L1[(size_t)k * rank + j]);
+  for (int j = 0; j < rank; ++j)
+    for (int n = 0; n < N; ++n) c.L2[(size_t)j * N + n] = f64_to_bf16(L2[(size_t)j * N + n]);
+  return SVDQ_OK;
+}
+
+// R = W~ - L1b L2b against the stored factors (j ascending, fp64), then eq. 1
+// per (output column, group of 64 input channels).
+void quantize_residual(int K, int N, int rank, Candidate& c) {
+  std::vector<float> R32((size_t)K * N);
+#pragma omp parallel for schedule(static)
+  for (int k = 0; k < K; ++k) {
+    std::vector<double> row(c.Wt.begin() + (size_t)k * N, c.Wt.begin() + (size_t)(k + 1) * N);
+    for (int j = 0; j < rank; ++j) {
+      const double a = bf16_to_f64(c.L1[(size_t)k * rank + j]);
+      const uint16_t* l2 = &c.L2[(size_t)j * N];
+      for (int n = 0; n < N; ++n) row[n] -= a * bf16_to_f64(l2[n]);
+    }
+    for (int n = 0; n < N; ++n) R32[(size_t)k * N + n] = (float)row[n];
+  }
+  const int G = K / SVDQ_GROUP;
+  c.sw.assign((size_t)G * N, 0.0f);
+  c.wq.assign((size_t)N * K / 2, 0);
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; ++n) {
+    int8_t q[64];
+    for (int g = 0; g < G; ++g) {
+      c.sw[(size_t)g * N + n] = quantize_group(&R32[(size_t)g * 64 * N + n], N, q);
+      uint8_t* dst = &c.wq[(size_t)n * (K / 2) + g * 32];
+      for (int b = 0; b < 32; ++b)
+        dst[b] = (uint8_t)((q[2 * b] & 0xF) | ((q[2 * b + 1] & 0xF) << 4));
+    }
+  }
+}
+
+int8_t code_at(const std::vector<uint8_t>& wq, int K, int n, int k) {
+  const uint8_t b = wq[(size_t)n * (K / 2) + k / 2];
+  const int v = (k & 1) ? (b >> 4) : (b & 0xF);
+  return (int8_t)(v >= 8 ? v - 16 : v);
+}
+
+// One alternating refinement: the factors of W~ - deq(Q(R)), then R again.
+svdq_status refine(int K, int N, int rank, Candidate& c) {
+  std::vector<double> T(c.Wt);
+#pragma omp parallel for schedule(static)
+  for (int k = 0; k < K; ++k)
+    for (int n = 0; n < N; ++n)
+      T[(size_t)k * N + n] -= (double)code_at(c.wq, K, n, k) * (double)c.sw[(size_t)(k / 64) * N + n];
+  const svdq_status s = fit_factors(T.data(), K, N, rank, c);
+  if (s != SVDQ_OK) return s;
+  quantize_residual(K, N, rank, c);
+  return SVDQ_OK;
+}
+
+// X W in fp64 on M tokens, [M][N] (the reference of layer_error).
+std::vector<double> dense_reference(int K, int N, const uint16_t* W, const uint16_t* X, int M,
+                                    int ldx) {
+  std::vector<double> ref((size_t)M * N);
+#pragma omp parallel for schedule(dynamic)
+  for (int m = 0; m < M; ++m) {
+    std::vector<double> x(K);
+    for (int k = 0; k < K; ++k) x[k] = bf16_to_f64(X[(size_t)m * ldx + k]);
+    for (int n = 0; n < N; ++n) {
+      const uint16_t* wr = &W[(size_t)n * K];
+      double t = 0.0;
+      for (int k = 0; k < K; ++k) t += x[k] * bf16_to_f64(wr[k]);
+      ref[(size_t)m * N + n] = t;
+    }
+  }
+  return ref;
+}
+
+// Relative Frobenius error, in fp64, of the quantised layer (both branches,
+// no bias, before the bf16 output rounding) against ref = X W on M tokens.
+double layer_error(int K, int N, int rank, const Candidate& c, const std::vector<double>& refm,
+                   const uint16_t* X, int M, int ldx) {
+  const int G = K / SVDQ_GROUP;
+  std::vector<int8_t> wc((size_t)N * K);
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) wc[(size_t)n * K + k] = code_at(c.wq, K, n, k);
+  double num = 0.0, den = 0.0;
+#pragma omp parallel for schedule(dynamic) reduction(+ : num, den)
+  for (int m = 0; m < M; ++m) {
+    std::vector<float> xh(K);
+    std::vector<double> x(K), z(rank > 0 ? rank : 1, 0.0);
+    std::vector<int8_t> xc(K);
+    std::vector<float> sx(G);
+    for (int k = 0; k < K; ++k) {
+      x[k] = bf16_to_f64(X[(size_t)m * ldx + k]);
+      xh[k] = (float)(x[k] * (double)c.inv_lambda[k]);     // one rounding of an exact product
+    }
+    for (int g = 0; g < G; ++g) sx[g] = quantize_group(&xh[(size_t)g * 64], 1, &xc[(size_t)g * 64]);
+    for (int j = 0; j < rank; ++j) {
+      double t = 0.0;
+      for (int k = 0; k < K; ++k)
+        t += bf16_to_f64(f64_to_bf16((double)xh[k])) * bf16_to_f64(c.L1[(size_t)k * rank + j]);
+      z[j] = bf16_to_f64(f64_to_bf16(t));
+    }
+    for (int n = 0; n < N; ++n) {
+      double y = 0.0, ref = 0.0;
+      const int8_t* wn = &wc[(size_t)n * K];
+      for (int g = 0; g < G; ++g) {
+        int p = 0;
+        for (int i = 0; i < 64; ++i) p += (int)xc[g * 64 + i] * (int)wn[g * 64 + i];
+        y += (double)sx[g] * (double)c.sw[(size_t)g * N + n] * (double)p;
+      }
+      for (int j = 0; j < rank; ++j) y += z[j] * bf16_to_f64(c.L2[(size_t)j * N + n]);
+      ref = refm[(size_t)m * N + n];
+      num += (y - ref) * (y - ref);
+      den += ref * ref;
+    }
+  }
+  return den > 0.0 ? std::sqrt(num / den) : 0.0;
+}
+
+svdq_status check_pack_args(int K, int N, int rank, int group, const uint16_t* W, int lora_rank,
+                            const uint16_t* lora_A, const uint16_t* lora_B, float lora_scale,
+                            svdq_weights** out) {
+  if (!out) return SVDQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!W) return SVDQ_ERR_INVALID_ARG;
+  if (group != SVDQ_GROUP) return SVDQ_ERR_UNSUPPORTED;
+  if (K < SVDQ_GROUP || N < 1 || K % SVDQ_GROUP) return SVDQ_ERR_SHAPE;
+  if (rank < 0 || lora_rank < 0 || rank > (K < N ? K : N)) return SVDQ_ERR_INVALID_ARG;
+  if (rank + lora_rank > SVDQ_MAX_RANK || (rank + lora_rank) % 8 != 0) return SVDQ_ERR_UNSUPPORTED;
+  if (lora_rank > 0 && (!lora_A || !lora_B)) return SVDQ_ERR_INVALID_ARG;
+  if (!std::isfinite(lora_scale)) return SVDQ_ERR_NUMERIC;
+  return SVDQ_OK;
+}
+
+// The handle from a finished candidate: eq. 13 (LoRA joins the 16-bit branch
+// in smoothed coordinates), bias, optional upload.
+svdq_status finish(int K, int N, int rank, Candidate& c, const uint16_t* bias, int lora_rank,
+                   const uint16_t* lora_A, const uint16_t* lora_B, float lora_scale,
+                   bool to_device, cudaStream_t stream, svdq_weights** out) {
+  svdq_weights* w = new (std::nothrow) svdq_weights();
+  if (!w) return SVDQ_ERR_OOM;
+  w->K = K; w->N = N; w->G = K / SVDQ_GROUP;
+  w->svd_rank = rank; w->lora_rank = lora_rank; w->rank = rank + lora_rank;
+  w->rank_pad = (w->rank + 15) / 16 * 16;
+  w->inv_lambda = std::move(c.inv_lambda);
+  w->sigma = std::move(c.sigma);
+  w->wq = std::move(c.wq);
+  w->sw = std::move(c.sw);
+  const int rt = w->rank;
+  w->L1.assign((size_t)K * rt, 0);
+  w->L2.assign((size_t)rt * N, 0);
+  for (int k = 0; k < K; ++k)
+    for (int j = 0; j < rank; ++j) w->L1[(size_t)k * rt + j] = c.L1[(size_t)k * rank + j];
+  for (int j = 0; j < rank; ++j)
+    std::memcpy(&w->L2[(size_t)j * N], &c.L2[(size_t)j * N], (size_t)N * 2);
+  for (int k = 0; k < K; ++k)
+    for (int j = 0; j < lora_rank; ++j) {
+      const double a = bf16_to_f64(lora_A[(size_t)k * lora_rank + j]);
+      w->L1[(size_t)k * rt + rank + j] = f64_to_bf16((c.lam[k] * a) * (double)lora_scale);
+    }
+  for (int j = 0; j < lora_rank; ++j)
+    std::memcpy(&w->L2[(size_t)(rank + j) * N], &lora_B[(size_t)j * N], (size_t)N * 2);
+  w->bias.assign(N, 0);
+  if (bias) std::memcpy(w->bias.data(), bias, (size_t)N * 2);
+  if (to_device) {
+    const svdq_status st = svdq::upload(w, stream);
+    if (st != SVDQ_OK) { free_device(w); delete w; return st; }
+  }
+  *out = w;
+  return SVDQ_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* svdq_status_string(int status) {
@@ -163,118 +393,55 @@ svdq_status svdq_calib_absmax(int M, int K, const uint16_t* X, int ldx, float* a
   return SVDQ_OK;
 }
 
+
 static svdq_status pack_impl(int K, int N, int rank, int group, const uint16_t* W,
                              const float* act_absmax, double alpha, const uint16_t* bias,
                              int lora_rank, const uint16_t* lora_A, const uint16_t* lora_B,
                              float lora_scale, bool to_device, cudaStream_t stream,
                              svdq_weights** out) {
-  if (!out) return SVDQ_ERR_INVALID_ARG;
-  *out = nullptr;
-  if (!W || !act_absmax) return SVDQ_ERR_INVALID_ARG;
-  if (group != SVDQ_GROUP) return SVDQ_ERR_UNSUPPORTED;
-  if (K < SVDQ_GROUP || N < 1 || K % SVDQ_GROUP) return SVDQ_ERR_SHAPE;
-  if (rank < 0 || lora_rank < 0 || rank > (K < N ? K : N)) return SVDQ_ERR_INVALID_ARG;
-  if (rank + lora_rank > SVDQ_MAX_RANK || (rank + lora_rank) % 8 != 0) return SVDQ_ERR_UNSUPPORTED;
-  if (lora_rank > 0 && (!lora_A || !lora_B)) return SVDQ_ERR_INVALID_ARG;
-  if (!(alpha > 0.0 && alpha < 1.0)) return SVDQ_ERR_INVALID_ARG;
-  if (!std::isfinite(lora_scale)) return SVDQ_ERR_NUMERIC;
+  svdq_status s = check_pack_args(K, N, rank, group, W, lora_rank, lora_A, lora_B, lora_scale, out);
+  if (s != SVDQ_OK) return s;
+  if (!act_absmax || !(alpha > 0.0 && alpha < 1.0)) return SVDQ_ERR_INVALID_ARG;
+  Candidate c;
+  if ((s = smooth(K, N, W, act_absmax, alpha, c)) != SVDQ_OK) return s;
+  if ((s = fit_factors(c.Wt.data(), K, N, rank, c)) != SVDQ_OK) return s;
+  quantize_residual(K, N, rank, c);
+  return finish(K, N, rank, c, bias, lora_rank, lora_A, lora_B, lora_scale, to_device, stream, out);
+}
 
-  svdq_weights* w = new (std::nothrow) svdq_weights();
-  if (!w) return SVDQ_ERR_OOM;
-  w->K = K; w->N = N; w->G = K / SVDQ_GROUP;
-  w->svd_rank = rank; w->lora_rank = lora_rank; w->rank = rank + lora_rank;
-  w->rank_pad = (w->rank + 15) / 16 * 16;
-
-  // eq. 4 statistics and lambda
-  std::vector<double> lam(K), Wt((size_t)K * N);
-  for (int k = 0; k < K; ++k) {
-    const double a = act_absmax[k];
-    if (!std::isfinite(a) || a < 0) { delete w; return SVDQ_ERR_NUMERIC; }
-  }
-  std::vector<double> wmax(K, 0.0);
-  for (int n = 0; n < N; ++n)
-    for (int k = 0; k < K; ++k) {
-      const double v = bf16_to_f64(W[(size_t)n * K + k]);
-      if (!std::isfinite(v)) { delete w; return SVDQ_ERR_NUMERIC; }
-      wmax[k] = std::fmax(wmax[k], std::fabs(v));
-    }
-  w->inv_lambda.resize(K);
-  for (int k = 0; k < K; ++k) {
-    const double a = act_absmax[k], m = wmax[k];
-    double l = 1.0;
-    if (a > 0.0 && m > 0.0)
-      l = (alpha == 0.5) ? std::sqrt(a) / std::sqrt(m)
-                         : std::pow(a, alpha) / std::pow(m, 1.0 - alpha);
-    lam[k] = l;
-    w->inv_lambda[k] = (float)(1.0 / l);
-  }
-  // eq. 3: W~ = diag(lambda) W in the math layout [K][N]
-  for (int n = 0; n < N; ++n)
-    for (int k = 0; k < K; ++k)
-      Wt[(size_t)k * N + n] = lam[k] * bf16_to_f64(W[(size_t)n * K + k]);
-
-  // eq. 10: leading rank+1 singular triplets (sigma exported for checks)
-  const int nsv = std::min(rank + 1, std::min(K, N));
-  std::vector<double> sig(nsv), L1((size_t)K * (rank > 0 ? rank : 1)),
-      L2((size_t)(rank > 0 ? rank : 1) * N);
-  if (svdq::top_singular(Wt.data(), K, N, nsv, rank, sig.data(), L1.data(), L2.data())) {
-    delete w;
-    return SVDQ_ERR_NUMERIC;
-  }
-  w->sigma.assign(rank + 1, 0.0);
-  for (int j = 0; j < nsv; ++j) w->sigma[j] = sig[j];
-
-  const int rt = w->rank;
-  w->L1.assign((size_t)K * rt, 0);
-  w->L2.assign((size_t)rt * N, 0);
-  for (int k = 0; k < K; ++k)
-    for (int j = 0; j < rank; ++j) w->L1[(size_t)k * rt + j] = f64_to_bf16(L1[(size_t)k * rank + j]);
-  for (int j = 0; j < rank; ++j)
-    for (int n = 0; n < N; ++n) w->L2[(size_t)j * N + n] = f64_to_bf16(L2[(size_t)j * N + n]);
-
-  // residual against the stored factors, then fp32
-  std::vector<float> R32((size_t)K * N);
-#pragma omp parallel for schedule(static)
-  for (int k = 0; k < K; ++k) {
-    double* row = &Wt[(size_t)k * N];
-    for (int j = 0; j < rank; ++j) {
-      const double a = bf16_to_f64(w->L1[(size_t)k * rt + j]);
-      const uint16_t* l2 = &w->L2[(size_t)j * N];
-      for (int n = 0; n < N; ++n) row[n] -= a * bf16_to_f64(l2[n]);
-    }
-    for (int n = 0; n < N; ++n) R32[(size_t)k * N + n] = (float)row[n];
-  }
-  // eq. 1 per (output column, group of 64 input channels)
-  const int G = w->G;
-  w->sw.assign((size_t)G * N, 0.0f);
-  w->wq.assign((size_t)N * K / 2, 0);
-#pragma omp parallel for schedule(static)
-  for (int n = 0; n < N; ++n) {
-    int8_t q[64];
-    for (int g = 0; g < G; ++g) {
-      w->sw[(size_t)g * N + n] = quantize_group(&R32[(size_t)g * 64 * N + n], N, q);
-      uint8_t* dst = &w->wq[(size_t)n * (K / 2) + g * 32];
-      for (int b = 0; b < 32; ++b)
-        dst[b] = (uint8_t)((q[2 * b] & 0xF) | ((q[2 * b + 1] & 0xF) << 4));
+static svdq_status pack_calibrated_impl(int K, int N, int rank, int group, const uint16_t* W,
+                                        const uint16_t* X, int M, int ldx, int n_alpha,
+                                        const double* alphas, int iters, const uint16_t* bias,
+                                        int lora_rank, const uint16_t* lora_A,
+                                        const uint16_t* lora_B, float lora_scale,
+                                        bool to_device, cudaStream_t stream, double* errors,
+                                        svdq_weights** out) {
+  svdq_status s = check_pack_args(K, N, rank, group, W, lora_rank, lora_A, lora_B, lora_scale, out);
+  if (s != SVDQ_OK) return s;
+  if (!X || M < 1 || ldx < K || n_alpha < 1 || !alphas || iters < 0) return SVDQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n_alpha; ++i)
+    if (!(alphas[i] > 0.0 && alphas[i] < 1.0)) return SVDQ_ERR_INVALID_ARG;
+  std::vector<float> a(K, 0.0f);
+  if ((s = svdq_calib_absmax(M, K, X, ldx, a.data())) != SVDQ_OK) return s;
+  const std::vector<double> ref = dense_reference(K, N, W, X, M, ldx);
+  Candidate best;
+  double best_err = 0.0;
+  for (int i = 0; i < n_alpha; ++i) {
+    Candidate c;
+    if ((s = smooth(K, N, W, a.data(), alphas[i], c)) != SVDQ_OK) return s;
+    if ((s = fit_factors(c.Wt.data(), K, N, rank, c)) != SVDQ_OK) return s;
+    quantize_residual(K, N, rank, c);
+    for (int it = 0; it < iters; ++it)
+      if ((s = refine(K, N, rank, c)) != SVDQ_OK) return s;
+    const double e = layer_error(K, N, rank, c, ref, X, M, ldx);
+    if (errors) errors[i] = e;
+    if (i == 0 || e < best_err) {
+      best = std::move(c);
+      best_err = e;
     }
   }
-  // eq. 13: LoRA joins the 16-bit branch in smoothed coordinates
-  for (int k = 0; k < K; ++k)
-    for (int j = 0; j < lora_rank; ++j) {
-      const double a = bf16_to_f64(lora_A[(size_t)k * lora_rank + j]);
-      w->L1[(size_t)k * rt + rank + j] = f64_to_bf16((lam[k] * a) * (double)lora_scale);
-    }
-  for (int j = 0; j < lora_rank; ++j)
-    std::memcpy(&w->L2[(size_t)(rank + j) * N], &lora_B[(size_t)j * N], (size_t)N * 2);
-  w->bias.assign(N, 0);
-  if (bias) std::memcpy(w->bias.data(), bias, (size_t)N * 2);
-
-  if (to_device) {
-    const svdq_status st = svdq::upload(w, stream);
-    if (st != SVDQ_OK) { free_device(w); delete w; return st; }
-  }
-  *out = w;
-  return SVDQ_OK;
+  return finish(K, N, rank, best, bias, lora_rank, lora_A, lora_B, lora_scale, to_device, stream,
+                out);
 }
 
 svdq_status svdq_pack_weights(int K, int N, int rank, int group, const uint16_t* W,
@@ -292,6 +459,18 @@ svdq_status svdq_pack_weights_host(int K, int N, int rank, int group, const uint
                                    float lora_scale, svdq_weights** out) {
   return pack_impl(K, N, rank, group, W, act_absmax, alpha, bias, lora_rank, lora_A,
                    lora_B, lora_scale, false, nullptr, out);
+}
+
+svdq_status svdq_pack_weights_calibrated(int K, int N, int rank, int group, const uint16_t* W,
+                                         const uint16_t* X_cal, int M_cal, int ldx,
+                                         int n_alpha, const double* alphas, int refine_iters,
+                                         const uint16_t* bias, int lora_rank,
+                                         const uint16_t* lora_A, const uint16_t* lora_B,
+                                         float lora_scale, int to_device, cudaStream_t stream,
+                                         double* errors, svdq_weights** out) {
+  return pack_calibrated_impl(K, N, rank, group, W, X_cal, M_cal, ldx, n_alpha, alphas,
+                              refine_iters, bias, lora_rank, lora_A, lora_B, lora_scale,
+                              to_device != 0, stream, errors, out);
 }
 
 svdq_status svdq_weights_info(const svdq_weights* w, int* K, int* N, int* rank,
