@@ -18,6 +18,8 @@ What it computes follows "SVDQuant: How a Small High-Precision Branch Makes
   * MAC and storage ratios                                     (section 6, eqs. 11-12)
   * calibration refinement: alpha search by the calibrated layer-output
     error, factors re-fitted to W~ - Q(R)                        (section 5)
+  * W8A8 comparator: int8 operands, one scale per token / output channel
+    applied once          (section 8, the eight-bit setting; section 9.3, INT8)
 
 Readings taken where the pages leave a step open (each is listed in the
 design notes of the repository):
@@ -49,6 +51,7 @@ __all__ = [
     "linear", "gelu", "layer_forward", "mac_ratio", "storage_ratio",
     "two_branch_unquantized", "dequantize_groups", "residual_quantize",
     "leading_svd", "layer_output_error", "refine_factors", "pack_weights_calibrated",
+    "quantize_rows_int8", "pack_weights_w8a8", "quantize_act_w8a8", "linear_w8a8",
 ]
 
 GROUP = 64
@@ -409,6 +412,78 @@ def pack_weights_calibrated(W_bits, X_cal_bits, rank, alphas=(0.3, 0.4, 0.5, 0.6
         p["L2b"] = np.vstack([p["L2b"], B])
         p["rank"] = p["L1b"].shape[1]
     return p, errs
+
+
+# --------------------------------------------------------------------------
+# W8A8 comparator: the same two-branch layer with 8-bit operands and one
+# scale per token (activations) and per output channel (residual), applied
+# once (review section 8: the eight-bit setting with rank 16, dynamic
+# per-token activation and per-channel weight scales; section 9.3, INT8)
+# --------------------------------------------------------------------------
+def quantize_rows_int8(v):
+    """Symmetric int8 quantisation with one scale per row (last axis):
+    s = fl32(max|v| / 127), q = round-half-even of the exact quotient v/s
+    (exact fp64 comparisons, as in quantize_groups: q*s has at most 31
+    significant bits), clamped to [-128, 127] (|q| <= 127 for a normal s).
+    s = 0 gives codes 0.  Returns (codes int64 like v, scales [...])."""
+    v = np.asarray(v, dtype=np.float64)
+    m = np.max(np.abs(v), axis=-1)
+    s = round_f32(m / 127.0)
+    codes = np.zeros(v.shape, dtype=np.int64)
+    nz = s > 0
+    if np.any(nz):
+        zz = v[nz]
+        ss = np.broadcast_to(s[nz][..., None], zz.shape)
+        q = np.rint(zz / ss)
+        for _ in range(3):
+            two_d = 2.0 * (zz - q * ss)
+            q = np.where(two_d > ss, q + 1, np.where(two_d < -ss, q - 1, q))
+        d = zz - q * ss
+        tie = (2.0 * np.abs(d) == ss) & (np.mod(q, 2) != 0)
+        q = np.where(tie, q + np.sign(d), q)
+        codes[nz] = np.clip(q, -128, 127).astype(np.int64)
+    return codes, s
+
+
+def pack_weights_w8a8(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None, lora_A_bits=None,
+                      lora_B_bits=None, lora_scale=1.0, svd=None):
+    """pack_weights' smoothing, factors and residual R, with R quantised to
+    int8 per output channel (over all K): wcodes8 [N, K], s_w8 [N]."""
+    p = pack_weights(W_bits, act_absmax, rank, alpha=alpha, bias_bits=bias_bits,
+                     lora_A_bits=lora_A_bits, lora_B_bits=lora_B_bits, lora_scale=lora_scale,
+                     svd=svd)
+    codes8, s_w8 = quantize_rows_int8(round_f32(p["R"].T))
+    return dict(p, wcodes8=codes8, s_w8=s_w8)
+
+
+def quantize_act_w8a8(X_bits, inv_lambda, L1b):
+    """x~ = fl32(x * inv_lambda), int8 codes and one scale per token, and
+    the same 16-bit down-projection as quantize_act.
+    Returns (codes [M, K], s_x [M], Z [M, r], xhat)."""
+    X = bf16_bits_to_f64(X_bits)
+    xhat = round_f32(X * np.asarray(inv_lambda, dtype=np.float64)[None, :])
+    codes, s_x = quantize_rows_int8(xhat)
+    r = L1b.shape[1]
+    Z = round_bf16(round_bf16(xhat) @ L1b) if r else np.zeros((X.shape[0], 0))
+    return codes, s_x, Z, xhat
+
+
+def linear_w8a8(xcodes, s_x, Z, wcodes, s_w, L2b, bias, apply_gelu=False, rows=None, cols=None):
+    """Y = s_x[i] s_w[n] sum_k q_x q_w + Z L2 + b (fp64; the integer sum is
+    an fp64 matmul of integers below 2^53 in magnitude, exact), optional
+    GELU, one bf16 rounding.  Returns (Y, Y_bf16)."""
+    xc = np.asarray(xcodes)
+    rows = np.arange(xc.shape[0]) if rows is None else np.asarray(rows)
+    cols = np.arange(np.asarray(wcodes).shape[0]) if cols is None else np.asarray(cols)
+    P = xc[rows].astype(np.float64) @ np.asarray(wcodes)[cols].astype(np.float64).T
+    Y = (np.asarray(s_x, dtype=np.float64)[rows][:, None] *
+         np.asarray(s_w, dtype=np.float64)[cols][None, :]) * P
+    if np.asarray(L2b).shape[0]:
+        Y += np.asarray(Z)[rows] @ np.asarray(L2b)[:, cols]
+    Y += np.asarray(bias, dtype=np.float64)[cols][None, :]
+    if apply_gelu:
+        Y = gelu(Y)
+    return Y, round_bf16(Y)
 
 
 def two_branch_unquantized(X, lam, L1, L2, R, bias):
