@@ -60,6 +60,10 @@ typedef enum {
 
 enum { SVDQ_EPI_NONE = 0, SVDQ_EPI_GELU = 1 };
 
+/* Number format of a packed handle: the W4A4 group format of every call
+ * above, or the W8A8 comparator of svdq_pack_weights_w8a8. */
+enum { SVDQ_FORMAT_W4A4 = 0, SVDQ_FORMAT_W8A8 = 1 };
+
 #define SVDQ_GROUP 64
 #define SVDQ_MAX_RANK 128
 #define SVDQ_MAX_SPLITS 16      /* K splits per output tile in svdq_linear_splitk */
@@ -273,6 +277,66 @@ svdq_status svdq_get_device_error(const svdq_weights* w, cudaStream_t stream);
 svdq_status svdq_debug_partials(const svdq_weights* w, int M, const uint8_t* xq,
                                 int row0, int nrows, int col0, int ncols,
                                 int32_t* P, cudaStream_t stream);
+
+/*
+ * ------------------------------------------------------------------------
+ * W8A8 comparator (review section 8: the eight-bit setting, rank 16 with
+ * dynamic per-token activation and per-channel weight quantisation; its
+ * INT8 rows in section 9.3).  The same two-branch layer with 8-bit
+ * operands and one scale per token / output channel, so the integer
+ * product accumulates over all of K and the scales are applied once:
+ *
+ *     Y = s_x[m] s_w[n] sum_k q_x[m][k] q_w[n][k] + Z L2 + b
+ *
+ * Number format: s = fl32(max|z| / 127) over the whole row (a token of x~,
+ * or an output column of R over all K), code = clamp(round_half_even(z / s),
+ * -128, 127) of the exact quotient (|code| <= 127 for a normal s); s = 0 and
+ * codes 0 for an all-zero row.  Smoothing, the bf16 factors, the residual R
+ * and the bias are those of svdq_pack_weights.
+ * A W8A8 handle is rejected (SVDQ_ERR_INVALID_ARG) by the W4A4 calls, and a
+ * W4A4 handle by the calls below; save/load and LoRA are W4A4 only.
+ * ------------------------------------------------------------------------
+ */
+
+/* Offline pack of the comparator: as svdq_pack_weights (group 64 is not
+ * used; K % 64 == 0 is still required), with R quantised per output channel
+ * over all K.  to_device != 0 uploads to the current device on `stream`
+ * (synchronised); 0 gives a host-only handle for export. */
+svdq_status svdq_pack_weights_w8a8(int K, int N, int rank, const uint16_t* W,
+                                   const float* act_absmax, double alpha,
+                                   const uint16_t* bias, int to_device,
+                                   cudaStream_t stream, svdq_weights** out);
+
+/* Host copies of the comparator's residual: wq8 int8 [N][K], s_w8 fp32 [N]
+ * (either may be NULL).  The other operands come from svdq_weights_export. */
+svdq_status svdq_weights_export_w8a8(const svdq_weights* w, int8_t* wq8, float* s_w8);
+
+/* Format of a handle (SVDQ_FORMAT_*), or -1 for NULL. */
+int svdq_weights_format(const svdq_weights* w);
+
+/*
+ * Activation pass of the comparator: x~ = fl32(x * inv_lambda_k) as in
+ * svdq_quantize_act; then
+ *   xq  [M][K]    int8 codes of x~ with one scale per token;
+ *   s_x [M]       fp32 scales fl32(max_k |x~| / 127);
+ *   Z   [M][rank] bf16 down-projection bf16(bf16(x~) L1), fp32 accumulation.
+ * One kernel: each block of tokens is read once from HBM to take its
+ * absmax and Z, and a second time (from L2) to quantise.
+ */
+svdq_status svdq_quantize_act_w8a8(const svdq_weights* w, int M, const uint16_t* X,
+                                   int ldx, int8_t* xq, float* s_x, uint16_t* Z,
+                                   cudaStream_t stream);
+
+/*
+ * Product of the comparator: one tcgen05 kernel, int8 operands copied by
+ * TMA straight into the tensor-core layout, the int32 sum over all of K in
+ * TMEM, one fp32 scaling s_x[m] s_w[n] per output, then Z L2 (bf16 tensor
+ * cores), bias, optional GELU and the bf16 store of Y [M][ldy], as in
+ * svdq_linear.
+ */
+svdq_status svdq_linear_w8a8(const svdq_weights* w, int M, const int8_t* xq,
+                             const float* s_x, const uint16_t* Z, uint16_t* Y,
+                             int ldy, int epilogue, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -9,8 +9,11 @@ The call names follow include/svdq.h:
     svdq_calib_absmax, svdq_pack_weights, svdq_pack_weights_host,
     svdq_weights_export, svdq_weights_save, svdq_weights_load,
     svdq_quantize_act, svdq_linear, svdq_get_device_error,
-    svdq_debug_partials
-and SVDQLinear bundles one packed layer with its two hot-path calls.
+    svdq_debug_partials, svdq_linear_splitk*, svdq_pack_weights_calibrated,
+    and the W8A8 comparator svdq_pack_weights_w8a8, svdq_quantize_act_w8a8,
+    svdq_linear_w8a8
+and SVDQLinear / W8A8Linear bundle one packed layer with its two hot-path
+calls.
 """
 from __future__ import annotations
 
@@ -24,12 +27,16 @@ __all__ = [
     "svdq_pack_weights", "svdq_pack_weights_host", "svdq_weights_load",
     "svdq_quantize_act", "svdq_linear", "svdq_get_device_error",
     "svdq_debug_partials", "EPI_NONE", "EPI_GELU", "LIB_PATH",
+    "svdq_pack_weights_w8a8", "svdq_quantize_act_w8a8", "svdq_linear_w8a8", "W8A8Linear",
+    "FORMAT_W4A4", "FORMAT_W8A8",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_lib", "libsvdq.so")
 EPI_NONE = 0
 EPI_GELU = 1
+FORMAT_W4A4 = 0
+FORMAT_W8A8 = 1
 
 _STATUS = {
     0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_SHAPE",
@@ -85,6 +92,12 @@ def lib() -> ctypes.CDLL:
         "svdq_linear_splitk": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _vp,
                                     ctypes.c_size_t, _vp]),
         "svdq_linear_splitk_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
+        "svdq_pack_weights_w8a8": (_i, [_i, _i, _i, _vp, _vp, ctypes.c_double, _vp, _i, _vp,
+                                        _vp]),
+        "svdq_weights_export_w8a8": (_i, [_vp, _vp, _vp]),
+        "svdq_weights_format": (_i, [_vp]),
+        "svdq_quantize_act_w8a8": (_i, [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp]),
+        "svdq_linear_w8a8": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -125,6 +138,7 @@ class Weights:
                                        ctypes.byref(lr)), "svdq_weights_info")
         self.K, self.N, self.rank = K.value, N.value, r.value
         self.svd_rank, self.lora_rank = sr.value, lr.value
+        self.format = int(lib().svdq_weights_format(handle))
 
     @property
     def handle(self):
@@ -141,6 +155,11 @@ class Weights:
             self._h, _np_ptr(out["inv_lambda"]), _np_ptr(out["wq"]), _np_ptr(out["s_w"]),
             _np_ptr(out["L1"]), _np_ptr(out["L2"]), _np_ptr(out["bias"]),
             _np_ptr(out["sigma"])), "svdq_weights_export")
+        if self.format == FORMAT_W8A8:
+            out["wq8"] = np.empty((N, K), np.int8)
+            out["s_w8"] = np.empty(N, np.float32)
+            _check(lib().svdq_weights_export_w8a8(self._h, _np_ptr(out["wq8"]),
+                                                  _np_ptr(out["s_w8"])), "svdq_weights_export_w8a8")
         return out
 
     def save(self, path: str):
@@ -280,6 +299,35 @@ def svdq_linear_splitk_noalloc(w: Weights, xq, s_x, Z, Y, splits=0, epilogue=EPI
            "svdq_linear_splitk_noalloc")
 
 
+def svdq_pack_weights_w8a8(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None, to_device=True,
+                           stream=None) -> Weights:
+    """Offline pack of the W8A8 comparator (int8 residual per output channel)."""
+    W_bits, act_absmax, bias_bits, _, _, _ = _pack_args(W_bits, act_absmax, bias_bits, None, None)
+    N, K = W_bits.shape
+    h = _vp()
+    _check(lib().svdq_pack_weights_w8a8(K, N, int(rank), _np_ptr(W_bits), _np_ptr(act_absmax),
+                                        float(alpha), _np_ptr(bias_bits), 1 if to_device else 0,
+                                        _stream_ptr(stream) if to_device else None,
+                                        ctypes.byref(h)), "svdq_pack_weights_w8a8")
+    return Weights(h)
+
+
+def svdq_quantize_act_w8a8(w: Weights, X, xq, s_x, Z=None, stream=None):
+    """X: cuda bf16 [M, K]; xq int8 [M, K]; s_x float32 [M]; Z bf16 [M, rank]."""
+    M = X.shape[0]
+    _check(lib().svdq_quantize_act_w8a8(w.handle, M, _dev_ptr(X), X.stride(0), _dev_ptr(xq),
+                                        _dev_ptr(s_x), _dev_ptr(Z), _stream_ptr(stream)),
+           "svdq_quantize_act_w8a8")
+
+
+def svdq_linear_w8a8(w: Weights, xq, s_x, Z, Y, epilogue=EPI_NONE, stream=None):
+    """Y: cuda bf16 [M, N] (row stride Y.stride(0))."""
+    M = Y.shape[0]
+    _check(lib().svdq_linear_w8a8(w.handle, M, _dev_ptr(xq), _dev_ptr(s_x), _dev_ptr(Z),
+                                  _dev_ptr(Y), Y.stride(0), int(epilogue), _stream_ptr(stream)),
+           "svdq_linear_w8a8")
+
+
 def svdq_get_device_error(w: Weights, stream=None):
     _check(lib().svdq_get_device_error(w.handle, _stream_ptr(stream)), "device")
 
@@ -322,6 +370,32 @@ class SVDQLinear:
             Y = out
         svdq_quantize_act(self.w, X, xq, s_x, Z)
         svdq_linear(self.w, xq, s_x, Z, Y, self.epilogue)
+        return Y
+
+    __call__ = forward
+
+
+class W8A8Linear(SVDQLinear):
+    """The W8A8 comparator layer: svdq_quantize_act_w8a8 then svdq_linear_w8a8."""
+
+    def buffers(self, M: int, device="cuda"):
+        import torch
+        if M != self._M:
+            K, N, r = self.w.K, self.w.N, self.w.rank
+            self.xq = torch.empty((M, K), dtype=torch.int8, device=device)
+            self.s_x = torch.empty((M,), dtype=torch.float32, device=device)
+            self.Z = torch.empty((M, max(r, 1)), dtype=torch.bfloat16, device=device) if r else None
+            self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            self._M = M
+        return self.xq, self.s_x, self.Z, self.Y
+
+    def forward(self, X, out=None):
+        M = X.shape[0]
+        xq, s_x, Z, Y = self.buffers(M, X.device)
+        if out is not None:
+            Y = out
+        svdq_quantize_act_w8a8(self.w, X, xq, s_x, Z)
+        svdq_linear_w8a8(self.w, xq, s_x, Z, Y, self.epilogue)
         return Y
 
     __call__ = forward

@@ -24,6 +24,14 @@
 // two tokens; a token's group spans the four lanes of a quad (absmax with
 // two xor-shuffles; codes regrouped into 8-byte stores by a 4 x 4 byte
 // transpose across the quad).
+//
+// The W8A8 comparator (review section 8, the eight-bit setting) runs the
+// same kernel with one int8 scale per token: the CTA streams its tokens
+// twice.  The first sweep takes each token's absmax of x~ and the
+// down-projection Z; the compute warps then combine their row maxima in
+// shared memory (one named barrier among them) into s = fl32(m / 127); the
+// second sweep (X only, which the first sweep has just brought into L2)
+// quantises and stores 16 contiguous int8 codes per lane and token.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -110,6 +118,50 @@ __device__ __noinline__ void quant16_exact(const float* v, float ssc, float rcp,
   u[1] = u1;
 }
 
+// int8 code of round-half-even(x / s), clamped to [-128, 127]: the exact
+// path of quant_nibble with the comparator's range; |x/s| <= 127.5 keeps the
+// magic-number rounding and the fma residual exact.
+__device__ __forceinline__ uint32_t quant_byte(float x, float ss, float rcp, float scale) {
+  const float xx = __fmul_rn(x, scale);
+  const float b0 = __fadd_rn(__fmul_rn(xx, rcp), RN_MAGIC);
+  float q = __fsub_rn(b0, RN_MAGIC);
+  const float d2 = 2.0f * __fmaf_rn(-q, ss, xx);
+  const uint32_t odd = __float_as_uint(b0) & 1u;
+  float adj = (d2 > ss) ? 1.0f : ((d2 < -ss) ? -1.0f : 0.0f);
+  adj = (fabsf(d2) == ss && odd) ? copysignf(1.0f, d2) : adj;
+  q = fminf(fmaxf(__fadd_rn(q, adj), -128.0f), 127.0f);
+  return __float_as_uint(__fadd_rn(q, RN_MAGIC)) & 0xFFu;
+}
+
+// The 16 int8 codes of one lane's token in a group, as four words: word ks
+// holds columns 16ks + 2q, 2q+1, 2q+8, 2q+9 (bytes 0..3).  Rare exact path.
+__device__ __noinline__ void quant16_byte_exact(const float* v, float ssc, float rcp, float scale,
+                                                uint32_t* wd) {
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    uint32_t x = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x |= quant_byte(v[4 * ks + e], ssc, rcp, scale) << (8 * e);
+    wd[ks] = x;
+  }
+}
+
+// Word transpose across a quad: lane q holds w[0..3] (word ks destined for
+// lane ks) and returns, in o[p], word q of lane p.
+__device__ __forceinline__ void quad_transpose_words(const uint32_t (&w)[4], int q,
+                                                     uint32_t (&o)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) o[k] = (k == q) ? w[k] : 0u;
+#pragma unroll
+  for (int i = 1; i < 4; ++i) {
+    const int p = q ^ i;
+    const uint32_t send = p == 0 ? w[0] : p == 1 ? w[1] : p == 2 ? w[2] : w[3];
+    const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, send, i);   // lane p's word q
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[k] = (k == p) ? got : o[k];
+  }
+}
+
 // 4 x 4 byte transpose across the lanes of a quad: lane q holds bytes
 // b[q][0..3] (byte j destined for lane j) and returns b[0..3][q].
 __device__ __forceinline__ uint32_t quad_transpose(uint32_t x, int q) {
@@ -120,7 +172,7 @@ __device__ __forceinline__ uint32_t quad_transpose(uint32_t x, int q) {
 }
 
 
-template <int NT>
+template <int NT, bool W8>
 __global__ void __launch_bounds__(AqStage<NT>::THREADS, 1)
 act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_l,   // L1^T [NT*8][K] bf16
@@ -133,6 +185,7 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
   constexpr int AQ_GPS = ST::GPS, AQ_WARPS = ST::WARPS, AQ_THREADS = ST::THREADS;
   __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S];
   __shared__ int abort_sh;
+  __shared__ float rowmax_sh[W8 ? AqStage<NT>::GPS : 1][AQ_ROWS];   // W8: per-warp token maxima
   extern __shared__ uint8_t aq_dyn_raw[];
   uint8_t* ring_p = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(aq_dyn_raw) + 1023) & ~uintptr_t(1023));
@@ -142,6 +195,7 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
   const int row0 = blockIdx.x * AQ_ROWS;
   const int G = K / 64;
   const int nstages = (G + AQ_GPS - 1) / AQ_GPS;
+  const int nsweep = W8 ? 2 * nstages : nstages;      // W8: quantising sweep after the first
 
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
@@ -163,7 +217,7 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
     // ------------------------------------------------------------ producer
     if (l == 0) {
       int c = 0;
-      for (; c < nstages; ++c) {
+      for (; c < nsweep; ++c) {
         const int s = c % S;
         if (c >= S && !mbar_wait_bounded(smem_u32(&empty_bar[s]), ((c / S) - 1) & 1, AQ_LIMIT_NS)) {
           atomicExch(err, SVDQ_DEVERR_TIMEOUT);
@@ -171,16 +225,19 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
           break;
         }
         if (*reinterpret_cast<volatile int*>(&abort_sh)) break;
-        const int ng = min(AQ_GPS, G - AQ_GPS * c);
+        const bool second = c >= nstages;              // no L1 slices needed
+        const int cc = second ? c - nstages : c;
+        const int ng = min(AQ_GPS, G - AQ_GPS * cc);
         const uint32_t fb = smem_u32(&full_bar[s]);
-        mbar_arrive_expect_tx(fb, ng * (AQ_XTILE + ST::L1_TILE + 256));
+        const bool with_l1 = NT > 0 && !second;
+        mbar_arrive_expect_tx(fb, ng * (AQ_XTILE + (with_l1 ? ST::L1_TILE : 0) + 256));
         const uint32_t st = ring + s * ST::BYTES;
         for (int g = 0; g < ng; ++g) {
-          const int col = (AQ_GPS * c + g) * 64;
+          const int col = (AQ_GPS * cc + g) * 64;
           tma_load_2d(st + g * AQ_XTILE, &tm_x, col, row0, fb);
-          if (NT > 0) tma_load_2d(st + ST::OFF_L1 + g * ST::L1_TILE, &tm_l, col, 0, fb);
+          if (with_l1) tma_load_2d(st + ST::OFF_L1 + g * ST::L1_TILE, &tm_l, col, 0, fb);
         }
-        bulk_load(st + ST::OFF_IL, inv_lambda + AQ_GPS * 64 * c, ng * 256, fb);
+        bulk_load(st + ST::OFF_IL, inv_lambda + AQ_GPS * 64 * cc, ng * 256, fb);
       }
       // every issued copy lands before the CTA moves on
       for (int k = (c > S ? c - S : 0); k < c; ++k)
@@ -189,15 +246,21 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
   } else {
     // ------------------------------------------------------- compute warps
     const int rb = warp & 1, gi = warp >> 1, q = l & 3, g8 = l >> 2;
-    for (int c = 0; c < nstages; ++c) {
+    float rmax[2] = {0.0f, 0.0f};     // W8: running absmax of the lane's two tokens
+    float wsc[2] = {0.0f, 0.0f}, wss[2] = {0.0f, 0.0f}, wrcp[2] = {0.0f, 0.0f};
+    float wscale[2] = {1.0f, 1.0f};
+    bool wtiny[2] = {false, false};
+    // One stage: the warp's 16 x 64 block of group AQ_GPS * cc + gi.
+    // second: the comparator's quantising sweep (W8 only).
+    auto stage = [&](int c, int cc, bool second) -> bool {
       const int s = c % S;
       if (!mbar_wait_bounded(smem_u32(&full_bar[s]), (c / S) & 1, AQ_LIMIT_NS)) {
         atomicExch(err, SVDQ_DEVERR_TIMEOUT);
         abort_sh = 1;
-        break;
+        return false;
       }
-      if (*reinterpret_cast<volatile int*>(&abort_sh)) break;
-      const int grp = AQ_GPS * c + gi;
+      if (*reinterpret_cast<volatile int*>(&abort_sh)) return false;
+      const int grp = AQ_GPS * cc + gi;
       if (grp < G) {
         const uint32_t st = ring + s * ST::BYTES;
         const uint32_t xt = st + gi * AQ_XTILE;
@@ -225,6 +288,58 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
             v[ri][4 * ks + 3] = p1.y;
           }
         }
+        if constexpr (W8) {
+          if (!second) {
+#pragma unroll
+            for (int ri = 0; ri < 2; ++ri)
+#pragma unroll
+              for (int j = 0; j < 16; ++j) rmax[ri] = fmaxf(rmax[ri], fabsf(v[ri][j]));
+          } else {
+#pragma unroll
+            for (int ri = 0; ri < 2; ++ri) {
+              uint32_t wd[4] = {0u, 0u, 0u, 0u};
+              if (wsc[ri] > 0.0f) {
+                bool near = wtiny[ri];
+                if (!near) {
+                  // t = x * fl(1/s) is within |x/s| 2^-23 < 2^-16 of the exact
+                  // quotient: rne(t) = rne(x/s) unless t is within 2^-15 of a half
+                  const float2 rc2 = make_float2(wrcp[ri], wrcp[ri]);
+                  const float2 mg2 = make_float2(RN_MAGIC, RN_MAGIC);
+                  const float2 nmg2 = make_float2(-RN_MAGIC, -RN_MAGIC);
+                  float fmx = 0.0f;
+#pragma unroll
+                  for (int j = 0; j < 16; j += 2) {
+                    const float2 t = __fmul2_rn(make_float2(v[ri][j], v[ri][j + 1]), rc2);
+                    const float2 b = __fadd2_rn(t, mg2);
+                    const float2 r = __fadd2_rn(b, nmg2);
+                    const float2 f = __fadd2_rn(t, make_float2(-r.x, -r.y));
+                    fmx = fmaxf(fmx, fmaxf(fabsf(f.x), fabsf(f.y)));
+                    // |rne(t)| <= 127: the low byte of the biased word is the code
+                    const uint32_t two = (__float_as_uint(b.x) & 0xFFu) |
+                                         ((__float_as_uint(b.y) & 0xFFu) << 8);
+                    wd[j >> 2] |= two << (16 * ((j >> 1) & 1));
+                  }
+                  near = fmx >= 0.5f - 0x1p-15f;
+                }
+                if (near) {
+                  float tmp[16];
+#pragma unroll
+                  for (int j = 0; j < 16; ++j) tmp[j] = v[ri][j];
+                  quant16_byte_exact(tmp, wss[ri], wrcp[ri], wscale[ri], wd);
+                }
+              }
+              // lane q gets columns 16q .. 16q+15 of the group: from lane p the
+              // bytes of columns 16q + {2p, 2p+1, 2p+8, 2p+9}
+              uint32_t o[4];
+              quad_transpose_words(wd, q, o);
+              const uint4 out = make_uint4(__byte_perm(o[0], o[1], 0x5410), __byte_perm(o[2], o[3], 0x5410),
+                                           __byte_perm(o[0], o[1], 0x7632), __byte_perm(o[2], o[3], 0x7632));
+              const int row = row0 + rb * 16 + g8 + 8 * ri;
+              if (row < M)
+                *reinterpret_cast<uint4*>(xq + (size_t)row * K + grp * 64 + 16 * q) = out;
+            }
+          }
+        } else {
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
           float m = 0.0f;
@@ -280,29 +395,60 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
             if (q == 0) s_x[(size_t)grp * M + row] = sc;
           }
         }
+        }
         if constexpr (NT > 0) {
-          const uint32_t lt = st + ST::OFF_L1 + gi * ST::L1_TILE;
+          if (!second) {
+            const uint32_t lt = st + ST::OFF_L1 + gi * ST::L1_TILE;
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            uint32_t af[4];
-            af[0] = bf16x2(v[0][4 * ks + 0], v[0][4 * ks + 1]);
-            af[1] = bf16x2(v[1][4 * ks + 0], v[1][4 * ks + 1]);
-            af[2] = bf16x2(v[0][4 * ks + 2], v[0][4 * ks + 3]);
-            af[3] = bf16x2(v[1][4 * ks + 2], v[1][4 * ks + 3]);
+            for (int ks = 0; ks < 4; ++ks) {
+              uint32_t af[4];
+              af[0] = bf16x2(v[0][4 * ks + 0], v[0][4 * ks + 1]);
+              af[1] = bf16x2(v[1][4 * ks + 0], v[1][4 * ks + 1]);
+              af[2] = bf16x2(v[0][4 * ks + 2], v[0][4 * ks + 3]);
+              af[3] = bf16x2(v[1][4 * ks + 2], v[1][4 * ks + 3]);
 #pragma unroll
-            for (int j = 0; j < NT / 2; ++j) {
-              // matrices: n-tile 2j (k 0-7, 8-15), n-tile 2j+1 (k 0-7, 8-15)
-              const int mi = l >> 3, n = 16 * j + 8 * (mi >> 1) + (l & 7), ch = 2 * ks + (mi & 1);
-              uint32_t b[4];
-              ldmatrix_x4(lt + n * 128 + ((ch ^ (n & 7)) << 4), b);
-              mma_bf16_16816(zacc[2 * j], af, b[0], b[1]);
-              mma_bf16_16816(zacc[2 * j + 1], af, b[2], b[3]);
+              for (int j = 0; j < NT / 2; ++j) {
+                // matrices: n-tile 2j (k 0-7, 8-15), n-tile 2j+1 (k 0-7, 8-15)
+                const int mi = l >> 3, n = 16 * j + 8 * (mi >> 1) + (l & 7), ch = 2 * ks + (mi & 1);
+                uint32_t b[4];
+                ldmatrix_x4(lt + n * 128 + ((ch ^ (n & 7)) << 4), b);
+                mma_bf16_16816(zacc[2 * j], af, b[0], b[1]);
+                mma_bf16_16816(zacc[2 * j + 1], af, b[2], b[3]);
+              }
             }
           }
         }
       }
       __syncwarp();
       if (l == 0) mbar_arrive(smem_u32(&empty_bar[s]));
+      return true;
+    };
+    bool alive = true;
+    for (int c = 0; c < nstages && alive; ++c) alive = stage(c, c, false);
+    if constexpr (W8) {
+      // per-token scales: quad, then the group-warps of each token half.
+      // Every compute warp reaches this barrier exactly once.
+#pragma unroll
+      for (int ri = 0; ri < 2; ++ri) {
+        rmax[ri] = fmaxf(rmax[ri], __shfl_xor_sync(0xFFFFFFFFu, rmax[ri], 1));
+        rmax[ri] = fmaxf(rmax[ri], __shfl_xor_sync(0xFFFFFFFFu, rmax[ri], 2));
+        if (q == 0) rowmax_sh[gi][rb * 16 + g8 + 8 * ri] = rmax[ri];
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(AQ_WARPS * 32) : "memory");
+#pragma unroll
+      for (int ri = 0; ri < 2; ++ri) {
+        const int rl = rb * 16 + g8 + 8 * ri;
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < AQ_GPS; ++j) m = fmaxf(m, rowmax_sh[j][rl]);
+        wsc[ri] = __fdiv_rn(m, 127.0f);
+        wtiny[ri] = wsc[ri] < 0x1p-64f;
+        wscale[ri] = wtiny[ri] ? 0x1p64f : 1.0f;
+        wss[ri] = __fmul_rn(wsc[ri], wscale[ri]);
+        wrcp[ri] = wsc[ri] > 0.0f ? __frcp_rn(wss[ri]) : 0.0f;
+        if (gi == 0 && q == 0 && row0 + rl < M) s_x[row0 + rl] = wsc[ri];
+      }
+      for (int c = nstages; c < 2 * nstages && alive; ++c) alive = stage(c, c - nstages, true);
     }
   }
   __syncthreads();
@@ -362,14 +508,14 @@ bool aq_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NT>
+template <int NT, bool W8>
 cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
                       uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
   using ST = AqStage<NT>;
   const size_t dyn = (size_t)ST::STAGES * ST::BYTES + 1024;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<NT>,
+    cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<NT, W8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess) return e;
     attr = true;
@@ -381,27 +527,38 @@ cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
   if (NT > 0 && !aq_map(&tl, w->d_L1T, (uint64_t)w->K, (uint64_t)NT * 8, (uint64_t)w->K * 2, NT * 8))
     return cudaErrorInvalidValue;
   const dim3 grid((M + AQ_ROWS - 1) / AQ_ROWS);
-  act_quant_kernel<NT><<<grid, ST::THREADS, dyn, st>>>(tx, tl, w->d_inv_lambda, M, w->K, w->rank,
+  act_quant_kernel<NT, W8><<<grid, ST::THREADS, dyn, st>>>(tx, tl, w->d_inv_lambda, M, w->K, w->rank,
                                                       xq, s_x, Z, w->d_err);
   return cudaGetLastError();
+}
+
+template <bool W8>
+cudaError_t launch_act(const svdq_weights* w, int M, const uint16_t* X, int ldx, uint8_t* xq,
+                       float* s_x, uint16_t* Z, cudaStream_t st) {
+  switch (w->rank_pad / 8) {
+    case 0: return launch_aq<0, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 2: return launch_aq<2, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 4: return launch_aq<4, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 6: return launch_aq<6, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 8: return launch_aq<8, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 10: return launch_aq<10, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 12: return launch_aq<12, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 14: return launch_aq<14, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 16: return launch_aq<16, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_act_quant(const svdq_weights* w, int M, const uint16_t* X, int ldx,
                              uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
-  switch (w->rank_pad / 8) {
-    case 0: return launch_aq<0>(w, M, X, ldx, xq, s_x, Z, st);
-    case 2: return launch_aq<2>(w, M, X, ldx, xq, s_x, Z, st);
-    case 4: return launch_aq<4>(w, M, X, ldx, xq, s_x, Z, st);
-    case 6: return launch_aq<6>(w, M, X, ldx, xq, s_x, Z, st);
-    case 8: return launch_aq<8>(w, M, X, ldx, xq, s_x, Z, st);
-    case 10: return launch_aq<10>(w, M, X, ldx, xq, s_x, Z, st);
-    case 12: return launch_aq<12>(w, M, X, ldx, xq, s_x, Z, st);
-    case 14: return launch_aq<14>(w, M, X, ldx, xq, s_x, Z, st);
-    case 16: return launch_aq<16>(w, M, X, ldx, xq, s_x, Z, st);
-    default: return cudaErrorInvalidValue;
-  }
+  return launch_act<false>(w, M, X, ldx, xq, s_x, Z, st);
+}
+
+cudaError_t launch_act_quant_w8a8(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                                  int8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
+  return launch_act<true>(w, M, X, ldx, reinterpret_cast<uint8_t*>(xq), s_x, Z, st);
 }
 
 }  // namespace svdq

@@ -15,6 +15,15 @@ svdq_status check_handle(const svdq_weights* w) {
   return SVDQ_OK;
 }
 
+// A handle of the W8A8 comparator, uploaded to the current device.
+svdq_status check_handle_w8a8(const svdq_weights* w) {
+  if (!w || w->format != SVDQ_FORMAT_W8A8 || !w->d_wq8 || !w->d_err) return SVDQ_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
+  return SVDQ_OK;
+}
+
 svdq_status from_launch(cudaError_t e) { return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA; }
 
 }  // namespace
@@ -58,10 +67,6 @@ svdq_status svdq_quantize_act(const svdq_weights* w, int M, const uint16_t* X, i
     return SVDQ_ERR_ALIGNMENT;
   return from_launch(svdq::launch_act_quant(w, M, X, ldx, xq, s_x, Z, stream));
 }
-
-
-
-
 svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
                         const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
                         cudaStream_t stream) {
@@ -101,6 +106,34 @@ svdq_status svdq_debug_partials(const svdq_weights* w, int M, const uint8_t* xq,
   if (!xq || !P) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(P)) return SVDQ_ERR_ALIGNMENT;
   return from_launch(svdq::launch_partials(w, M, xq, row0, nrows, col0, ncols, P, stream));
+}
+
+svdq_status svdq_quantize_act_w8a8(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                                   int8_t* xq, float* s_x, uint16_t* Z, cudaStream_t stream) {
+  svdq_status s = check_handle_w8a8(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || ldx < w->K) return SVDQ_ERR_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !xq || !s_x || (w->rank > 0 && !Z)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(xq) || !aligned16(s_x) || (ldx % 8) != 0 ||
+      (w->rank > 0 && !aligned16(Z)))
+    return SVDQ_ERR_ALIGNMENT;
+  return from_launch(svdq::launch_act_quant_w8a8(w, M, X, ldx, xq, s_x, Z, stream));
+}
+
+svdq_status svdq_linear_w8a8(const svdq_weights* w, int M, const int8_t* xq, const float* s_x,
+                             const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
+                             cudaStream_t stream) {
+  svdq_status s = check_handle_w8a8(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || ldy < w->N) return SVDQ_ERR_SHAPE;
+  if (epilogue != SVDQ_EPI_NONE && epilogue != SVDQ_EPI_GELU) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!xq || !s_x || !Y || (w->rank > 0 && !Z)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(s_x) || !aligned16(Y) || (ldy % 8) != 0 ||
+      (w->rank > 0 && !aligned16(Z)))
+    return SVDQ_ERR_ALIGNMENT;
+  return from_launch(svdq::launch_linear_w8a8(w, M, xq, s_x, Z, Y, ldy, epilogue, stream));
 }
 
 }  // extern "C"

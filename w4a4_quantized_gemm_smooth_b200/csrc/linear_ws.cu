@@ -41,6 +41,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include "gemm_common.cuh"
 #include "ptx.cuh"
 #include "svdq_internal.h"
 
@@ -53,7 +54,6 @@ constexpr int THREADS = 512;
 constexpr int N_EXP = 192;       // expanders: warps 2-7
 constexpr int RES_WARP0 = 8;     // rescale / epilogue: warps 8-15
 constexpr int N_RES_WARPS = 8;
-constexpr uint64_t LIMIT_NS = 2000000000ull;
 constexpr uint32_t MAGIC_BITS = 0x4B400000u;   // bits of 12582912.0f = 1.5 * 2^23
 constexpr float MAGIC_F = 12582912.0f;
 constexpr uint16_t BF16_ONE = 0x3F80;          // 1.0
@@ -141,23 +141,6 @@ struct Lay {
   static constexpr int ALLOC = BYTES + 1024;              // slack for 1024-B alignment
 };
 
-// Bounded wait: the thread sleeps in try_wait (up to 20 us per call) until
-// the phase completes; after LIMIT_NS, or when another thread of the CTA has
-// given up, it returns false.
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
-                                              volatile int* abort_flag, int* err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > LIMIT_NS) {
-      *abort_flag = 1;
-      atomicExch(err, SVDQ_DEVERR_TIMEOUT);
-      return false;
-    }
-  }
-}
 
 // 16 packed bytes (32 codes of one row: the first or second half of the
 // group) -> two 16-byte core-matrix rows at d and d + 128.
@@ -211,15 +194,6 @@ struct ExpandPlan {
   }
 };
 
-__device__ __forceinline__ float gelu_f(float y) {
-  return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f));
-}
-
-// Two floats -> packed bf16x2 bits (round to nearest even), x in the low half.
-__device__ __forceinline__ uint32_t bf16x2_bits(float2 v) {
-  const __nv_bfloat162 h = __float22bfloat162_rn(v);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
 
 // MODE 0: the layer (rescale, low-rank stage, epilogue, TMA store of Y).
 // MODE 1: dump the int32 group partials of the tiles covering the requested
@@ -647,43 +621,6 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess && q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// 2D map over a row-major [rows][cols] array with a row pitch in bytes.
-bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols,
-              uint64_t rows, uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows,
-              CUtensorMapSwizzle sw) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {pitch_bytes};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 template <int BN, int MODE>
 cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtensorMap& tb,

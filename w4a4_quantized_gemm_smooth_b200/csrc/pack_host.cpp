@@ -11,6 +11,8 @@
 //   R = W~ - sum_j L1b[k][j] L2b[j][n], j ascending   (fp64; the products of
 //       two bf16 values are exact, each subtraction is rounded once)
 //   s = fl32(max|fl32(R)| / 7), codes = rne of the exact quotient  (eq. 1)
+//   W8A8 comparator: s = fl32(max|fl32(R)| / 127) per output column over
+//   all K, codes rne of the exact quotient clamped to [-128, 127]
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -74,6 +76,33 @@ float quantize_group(const float* z, int stride, int8_t* q) {
   return s;
 }
 
+// The comparator's int8 quantiser: one scale for n fp32 values.
+float quantize_row_int8(const float* z, int n, long stride, int8_t* q) {
+  float m = 0.0f;
+  for (int i = 0; i < n; ++i) m = std::fmax(m, std::fabs(z[(long)i * stride]));
+  const float s = m / 127.0f;  // IEEE fp32 division
+  if (s == 0.0f) {
+    for (int i = 0; i < n; ++i) q[i] = 0;
+    return 0.0f;
+  }
+  const double sd = s;
+  for (int i = 0; i < n; ++i) {
+    const double zd = z[(long)i * stride];
+    double c = std::nearbyint(zd / sd);
+    for (int it = 0; it < 2; ++it) {
+      const double d2 = 2.0 * (zd - c * sd);          // exact (c s has <= 31 bits)
+      if (d2 > sd) c += 1.0;
+      else if (d2 < -sd) c -= 1.0;
+    }
+    const double d2 = 2.0 * (zd - c * sd);
+    if (std::fabs(d2) == sd && std::fmod(c, 2.0) != 0.0) c += (d2 > 0 ? 1.0 : -1.0);
+    if (c > 127.0) c = 127.0;
+    if (c < -128.0) c = -128.0;
+    q[i] = (int8_t)c;
+  }
+  return s;
+}
+
 template <class T>
 svdq_status dev_alloc_copy(T** dst, const T* src, size_t n, cudaStream_t st) {
   if (n == 0) n = 1;
@@ -86,7 +115,9 @@ svdq_status dev_alloc_copy(T** dst, const T* src, size_t n, cudaStream_t st) {
 void free_device(svdq_weights* w) {
   cudaFree(w->d_inv_lambda); cudaFree(w->d_wq); cudaFree(w->d_sw);
   cudaFree(w->d_L1T); cudaFree(w->d_L2); cudaFree(w->d_L2T); cudaFree(w->d_bias);
+  cudaFree(w->d_wq8); cudaFree(w->d_sw8);
   cudaFree(w->d_err);
+  w->d_wq8 = nullptr; w->d_sw8 = nullptr;
   w->d_inv_lambda = nullptr; w->d_wq = nullptr; w->d_sw = nullptr; w->d_L1T = nullptr;
   w->d_L2 = nullptr; w->d_L2T = nullptr; w->d_bias = nullptr; w->d_err = nullptr;
 }
@@ -111,15 +142,22 @@ svdq_status upload(svdq_weights* w, cudaStream_t st) {
     std::memcpy(&L2p[(size_t)j * N], &w->L2[(size_t)j * N], (size_t)N * 2);
   svdq_status s;
   if ((s = dev_alloc_copy(&w->d_inv_lambda, w->inv_lambda.data(), (size_t)K, st))) return s;
-  if ((s = dev_alloc_copy(&w->d_wq, w->wq.data(), (size_t)N * K / 2, st))) return s;
   w->N16 = (N + 15) / 16 * 16;
-  std::vector<float> swp((size_t)G * w->N16, 0.0f);
-  for (int g = 0; g < G; ++g)
-    for (int n = 0; n < N; ++n) {
-      const int c = n & 15, pos = (n & ~15) + 4 * ((c & 7) >> 1) + 2 * (c >> 3) + (c & 1);
-      swp[(size_t)g * w->N16 + pos] = w->sw[(size_t)g * N + n];
-    }
-  if ((s = dev_alloc_copy(&w->d_sw, swp.data(), swp.size(), st))) return s;
+  if (w->format == SVDQ_FORMAT_W8A8) {
+    std::vector<float> sw8p((size_t)w->N_pad, 0.0f);
+    std::memcpy(sw8p.data(), w->sw8.data(), (size_t)N * 4);
+    if ((s = dev_alloc_copy(&w->d_wq8, w->wq8.data(), (size_t)N * K, st))) return s;
+    if ((s = dev_alloc_copy(&w->d_sw8, sw8p.data(), sw8p.size(), st))) return s;
+  } else {
+    if ((s = dev_alloc_copy(&w->d_wq, w->wq.data(), (size_t)N * K / 2, st))) return s;
+    std::vector<float> swp((size_t)G * w->N16, 0.0f);
+    for (int g = 0; g < G; ++g)
+      for (int n = 0; n < N; ++n) {
+        const int c = n & 15, pos = (n & ~15) + 4 * ((c & 7) >> 1) + 2 * (c >> 3) + (c & 1);
+        swp[(size_t)g * w->N16 + pos] = w->sw[(size_t)g * N + n];
+      }
+    if ((s = dev_alloc_copy(&w->d_sw, swp.data(), swp.size(), st))) return s;
+  }
   if ((s = dev_alloc_copy(&w->d_L1T, L1T.data(), L1T.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_L2, L2p.data(), L2p.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_L2T, L2T.data(), L2T.size(), st))) return s;
@@ -143,6 +181,8 @@ struct Candidate {
   std::vector<uint16_t> L1, L2;    // bf16 factors [K][rank], [rank][N]
   std::vector<uint8_t> wq;         // packed residual codes [N][K/2]
   std::vector<float> sw;           // residual scales [G][N]
+  std::vector<int8_t> wq8;         // W8A8 comparator: codes [N][K]
+  std::vector<float> sw8;          //                  scales [N]
 };
 
 // eqs. 3-4: lambda from the activation statistic and the weight's per-channel
@@ -197,9 +237,9 @@ svdq_status fit_factors(const double* T, int K, int N, int rank, Candidate& c) {
   return SVDQ_OK;
 }
 
-// R = W~ - L1b L2b against the stored factors (j ascending, fp64), then eq. 1
-// per (output column, group of 64 input channels).
-void quantize_residual(int K, int N, int rank, Candidate& c) {
+// fl32(R), R = W~ - L1b L2b against the stored factors (j ascending, fp64),
+// [K][N].
+std::vector<float> residual_f32(int K, int N, int rank, const Candidate& c) {
   std::vector<float> R32((size_t)K * N);
 #pragma omp parallel for schedule(static)
   for (int k = 0; k < K; ++k) {
@@ -211,6 +251,12 @@ void quantize_residual(int K, int N, int rank, Candidate& c) {
     }
     for (int n = 0; n < N; ++n) R32[(size_t)k * N + n] = (float)row[n];
   }
+  return R32;
+}
+
+// The residual, then eq. 1 per (output column, group of 64 input channels).
+void quantize_residual(int K, int N, int rank, Candidate& c) {
+  const std::vector<float> R32 = residual_f32(K, N, rank, c);
   const int G = K / SVDQ_GROUP;
   c.sw.assign((size_t)G * N, 0.0f);
   c.wq.assign((size_t)N * K / 2, 0);
@@ -224,6 +270,16 @@ void quantize_residual(int K, int N, int rank, Candidate& c) {
         dst[b] = (uint8_t)((q[2 * b] & 0xF) | ((q[2 * b + 1] & 0xF) << 4));
     }
   }
+}
+
+// The residual, then the comparator's int8 quantiser per output column.
+void quantize_residual_w8(int K, int N, int rank, Candidate& c) {
+  const std::vector<float> R32 = residual_f32(K, N, rank, c);
+  c.sw8.assign(N, 0.0f);
+  c.wq8.assign((size_t)N * K, 0);
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; ++n)
+    c.sw8[n] = quantize_row_int8(&R32[n], K, N, &c.wq8[(size_t)n * K]);
 }
 
 int8_t code_at(const std::vector<uint8_t>& wq, int K, int n, int k) {
@@ -335,6 +391,9 @@ svdq_status finish(int K, int N, int rank, Candidate& c, const uint16_t* bias, i
   w->sigma = std::move(c.sigma);
   w->wq = std::move(c.wq);
   w->sw = std::move(c.sw);
+  w->wq8 = std::move(c.wq8);
+  w->sw8 = std::move(c.sw8);
+  w->format = w->wq8.empty() ? SVDQ_FORMAT_W4A4 : SVDQ_FORMAT_W8A8;
   const int rt = w->rank;
   w->L1.assign((size_t)K * rt, 0);
   w->L2.assign((size_t)rt * N, 0);
@@ -473,6 +532,28 @@ svdq_status svdq_pack_weights_calibrated(int K, int N, int rank, int group, cons
                               to_device != 0, stream, errors, out);
 }
 
+svdq_status svdq_pack_weights_w8a8(int K, int N, int rank, const uint16_t* W,
+                                   const float* act_absmax, double alpha, const uint16_t* bias,
+                                   int to_device, cudaStream_t stream, svdq_weights** out) {
+  svdq_status s = check_pack_args(K, N, rank, SVDQ_GROUP, W, 0, nullptr, nullptr, 1.0f, out);
+  if (s != SVDQ_OK) return s;
+  if (!act_absmax || !(alpha > 0.0 && alpha < 1.0)) return SVDQ_ERR_INVALID_ARG;
+  Candidate c;
+  if ((s = smooth(K, N, W, act_absmax, alpha, c)) != SVDQ_OK) return s;
+  if ((s = fit_factors(c.Wt.data(), K, N, rank, c)) != SVDQ_OK) return s;
+  quantize_residual_w8(K, N, rank, c);
+  return finish(K, N, rank, c, bias, 0, nullptr, nullptr, 1.0f, to_device != 0, stream, out);
+}
+
+svdq_status svdq_weights_export_w8a8(const svdq_weights* w, int8_t* wq8, float* s_w8) {
+  if (!w || w->format != SVDQ_FORMAT_W8A8) return SVDQ_ERR_INVALID_ARG;
+  if (wq8) std::memcpy(wq8, w->wq8.data(), w->wq8.size());
+  if (s_w8) std::memcpy(s_w8, w->sw8.data(), w->sw8.size() * 4);
+  return SVDQ_OK;
+}
+
+int svdq_weights_format(const svdq_weights* w) { return w ? w->format : -1; }
+
 svdq_status svdq_weights_info(const svdq_weights* w, int* K, int* N, int* rank,
                               int* svd_rank, int* lora_rank) {
   if (!w) return SVDQ_ERR_INVALID_ARG;
@@ -502,6 +583,7 @@ static const char kMagic[8] = {'S', 'V', 'D', 'Q', 'W', '0', '0', '1'};
 
 svdq_status svdq_weights_save(const svdq_weights* w, const char* path) {
   if (!w || !path) return SVDQ_ERR_INVALID_ARG;
+  if (w->format != SVDQ_FORMAT_W4A4) return SVDQ_ERR_UNSUPPORTED;
   FILE* f = std::fopen(path, "wb");
   if (!f) return SVDQ_ERR_IO;
   int32_t hdr[6] = {w->K, w->N, w->svd_rank, w->lora_rank, SVDQ_GROUP, 0};

@@ -17,6 +17,7 @@ struct svdq_weights {
   int N_pad = 0;       // N rounded up to a multiple of 256
   int N16 = 0;         // N rounded up to a multiple of 16 (row pitch of d_sw)
   int device = 0;
+  int format = SVDQ_FORMAT_W4A4;   // residual / activation number format
   // device copies (owned)
   float* d_inv_lambda = nullptr;   // [K]
   uint8_t* d_wq = nullptr;         // [N][K/2] packed residual codes
@@ -28,11 +29,15 @@ struct svdq_weights {
   uint16_t* d_L2 = nullptr;        // [rank_pad][N] bf16
   uint16_t* d_L2T = nullptr;       // [N_pad][rank_pad32] bf16, transposed L2
   uint16_t* d_bias = nullptr;      // [N] bf16
+  int8_t* d_wq8 = nullptr;         // W8A8: [N][K] int8 residual codes
+  float* d_sw8 = nullptr;          // W8A8: [N_pad] per-output-channel scales, zero padded
   int* d_err = nullptr;            // sticky device error word
   // host copies (export / save)
   std::vector<float> inv_lambda;
   std::vector<uint8_t> wq;
   std::vector<float> sw;
+  std::vector<int8_t> wq8;         // W8A8 codes [N][K]
+  std::vector<float> sw8;          // W8A8 scales [N]
   std::vector<uint16_t> L1;        // [K][rank]
   std::vector<uint16_t> L2;        // [rank][N]
   std::vector<uint16_t> bias;      // [N]
@@ -68,6 +73,12 @@ size_t splitk_workspace(const svdq_weights* w, int M, int splits);
 cudaError_t launch_linear_splitk(const svdq_weights* w, int M, const uint8_t* xq,
                                  const float* s_x, const uint16_t* Z, uint16_t* Y, int ldy,
                                  int epilogue, int splits, void* workspace, cudaStream_t stream);
+// W8A8 comparator: per-token int8 activation pass and the int8 product.
+cudaError_t launch_act_quant_w8a8(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                                  int8_t* xq, float* s_x, uint16_t* Z, cudaStream_t stream);
+cudaError_t launch_linear_w8a8(const svdq_weights* w, int M, const int8_t* xq, const float* s_x,
+                               const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
+                               cudaStream_t stream);
 cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq,
                             int row0, int nrows, int col0, int ncols,
                             int32_t* P, cudaStream_t stream);
