@@ -42,10 +42,11 @@ METRIC = "svdq_linear effective TOPS (2MNK/s) at FLUX-like shapes; % int8 roofli
 # the ncu capture summarised in profiles/svdq_linear_flux_qkv.md, valid only
 # for the kernel sources it was taken on (SHA-1 over the files below).
 LINEAR_SOURCES = ("w4a4_quantized_gemm_smooth_b200/csrc/linear_ws.cu",
+                  "w4a4_quantized_gemm_smooth_b200/csrc/gemm_common.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/ptx.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/svdq_internal.h")
-LINEAR_TRAFFIC = {"sources_sha1": "2c89f0d9044c284a4d31d69b8ffdd2a897a97169",
-                  "workload": "flux_qkv", "bytes": 24877056 + 32831744}
+LINEAR_TRAFFIC = {"sources_sha1": "58864ad822658f5b949b9ea4be4114ba9c2c4753",
+                  "workload": "flux_qkv", "bytes": 24911104 + 29313792}
 
 
 def _linear_traffic(workload):
@@ -281,6 +282,40 @@ class _Step:
         marks[2].record(stream)
 
 
+class _StepW8(_Step):
+    """The W8A8 comparator: quantize_act_w8a8 then linear_w8a8."""
+
+    def __call__(self, marks, stream):
+        S = self.S
+        marks[0].record(stream)
+        S.svdq_quantize_act_w8a8(self.w, self.X, self.xq, self.s_x, self.Z, stream)
+        marks[1].record(stream)
+        S.svdq_linear_w8a8(self.w, self.xq, self.s_x, self.Z, self.Y, self.epi, stream)
+        marks[2].record(stream)
+
+
+# Rank of the W8A8 comparator: the eight-bit setting's rank (review section 8).
+W8A8_RANK = 16
+
+
+def _time_w8a8(S, spec, L, a, X, flush, stream, steps, int8_peak):
+    """The same workload through the W8A8 comparator (int8 operands, one
+    scale per token / output channel, rank 16): per-kernel times and the
+    GEMM's fraction of the int8 peak."""
+    w8 = S.svdq_pack_weights_w8a8(L.W, a, W8A8_RANK, bias_bits=L.b)
+    lin8 = S.W8A8Linear(w8)
+    step8 = _StepW8(S, w8, X, lin8.buffers(spec.M), S.EPI_NONE)
+    _time_steps(step8, 3, flush, stream)
+    t_act, t_lin = (v / steps for v in _time_steps(step8, steps, flush, stream))
+    S.svdq_get_device_error(w8)
+    w8.free()
+    ops = 2.0 * spec.M * spec.N * spec.K
+    tops = ops / (t_lin * 1e-3) / 1e12
+    return {"rank": W8A8_RANK, "ms_per_step": t_act + t_lin, "act_ms": t_act,
+            "linear_ms": t_lin, "layer_tops": ops / ((t_act + t_lin) * 1e-3) / 1e12,
+            "linear_tops": tops, "linear_frac_int8": tops / int8_peak}
+
+
 def _time_e2e(S, w, Xh, Yh, Xd, bufs, epi, steps):
     """Public API end to end, as a serving loop: every step copies its X from
     pinned host memory to the device, runs svdq_quantize_act and svdq_linear,
@@ -417,6 +452,9 @@ def run_ours(args, spec):
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
+    if not args.no_w8a8:
+        line["w8a8_comparator"] = _time_w8a8(S, spec, L, a, X, flush, stream, args.steps,
+                                             int8_peak)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec)
     if rank == 0:
@@ -436,6 +474,8 @@ def main():
                     help="a name of synth.WORKLOADS or of synth.pixart_points()")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-w8a8", action="store_true",
+                    help="skip the W8A8 comparator's timing")
     args = ap.parse_args()
     spec = _workload(args.workload)
     if args.impl == "reference":

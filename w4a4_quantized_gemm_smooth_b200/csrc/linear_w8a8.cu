@@ -6,7 +6,8 @@
 //
 // With one scale per token and per output channel the integer product needs
 // no per-group rescale: the int8 codes are copied by TMA straight into the
-// tensor-core operand layout (no expansion step) and tcgen05.mma.kind::i8
+// tensor-core operand layout (no expansion step; 64-byte K rows with the
+// 64-byte swizzle, one TMA box per operand and stage) and tcgen05.mma.kind::i8
 // accumulates the whole K range of a 128 x 256 output tile into one int32
 // TMEM accumulator (|sum| <= 127^2 K < 2^31 for K <= 2^17).  The epilogue
 // converts it once (int32 -> fp32, exact below 2^24, one rounding above),
@@ -16,8 +17,8 @@
 //
 // Persistent CTAs (one per SM), static round-robin tiles; 16 warps:
 //   warp 0      TMA producer: 64-K stages of A (128 x 64 B) and B (256 x
-//               64 B) as 16-byte-wide boxes, chunk c at c * rows * 16, row
-//               r at r * 16 (no swizzle); per-tile scales; low-rank slices;
+//               64 B), each one box of 64-byte rows; per-tile scales;
+//               low-rank slices (16-byte-wide boxes, no swizzle);
 //   warp 1      TMEM owner and MMA issuer (one thread);
 //   warps 2-7   idle (they keep the warp-to-TMEM-lane mapping of the
 //               epilogue warps and the register split of the W4A4 kernel);
@@ -42,6 +43,21 @@ __device__ __forceinline__ float2 lds64f(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
   return v;
+}
+
+// Shared-memory descriptor of a K-major operand stored as 64-byte rows with
+// the 64-byte swizzle (8-row atoms of 512 B, as TMA writes them): the stride
+// between 8-row groups is 512 B; the leading offset is unused for this layout
+// (encoded as 1).  Layout type 4 = 64-byte swizzle, version 1.  Advancing the
+// start address by 32 B selects the second K half of the row.
+__device__ __forceinline__ uint64_t sdesc_kmajor_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;
+  return d;
 }
 
 struct W8Args {
@@ -145,11 +161,8 @@ linear_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a,
           if (!wait_or_abort(st_empty(s), ((it / NST) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
           mbar_arrive_expect_tx(st_full(s), L::STAGE);
           const uint32_t dst = sbase + L::OFF_ST + s * L::STAGE;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            tma_load_2d(dst + c * (BM * 16), &tm_a, g * 64 + 16 * c, m0, st_full(s));
-            tma_load_2d(dst + L::ST_A + c * (BN * 16), &tm_b, g * 64 + 16 * c, n0, st_full(s));
-          }
+          tma_load_2d(dst, &tm_a, g * 64, m0, st_full(s));
+          tma_load_2d(dst + L::ST_A, &tm_b, g * 64, n0, st_full(s));
         }
         for (int j = 0; j < p.n_lr && alive; ++j, ++il) {
           const int ls = il % NLR;
@@ -185,9 +198,9 @@ linear_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a,
           tc_fence_after();
           const uint32_t sa = sbase + L::OFF_ST + s * L::STAGE, sb = sa + L::ST_A;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {     // K = 32 each: chunks 2h, 2h+1
-            const uint64_t ad = sdesc_kmajor_noswizzle(sa + h * 2 * (BM * 16), BM * 16, 128);
-            const uint64_t bd = sdesc_kmajor_noswizzle(sb + h * 2 * (BN * 16), BN * 16, 128);
+          for (int h = 0; h < 2; ++h) {     // K = 32 each: bytes 32h .. 32h+31 of the rows
+            const uint64_t ad = sdesc_kmajor_sw64(sa + 32 * h);
+            const uint64_t bd = sdesc_kmajor_sw64(sb + 32 * h);
             mma_i8(d, ad, bd, id_i8, (g > 0 || h > 0) ? 1u : 0u);
           }
           mma_commit(st_empty(s));
@@ -383,10 +396,10 @@ cudaError_t launch_linear_w8a8(const svdq_weights* w, int M, const int8_t* xq, c
   CUtensorMap ta, tb, ty, tz, tl, tsx, tsw;
   const uint64_t sx_pitch = ((uint64_t)M * 4 + 15) / 16 * 16;
   const uint64_t sw_pitch = ((uint64_t)w->N_pad * 4 + 15) / 16 * 16;
-  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K, M, w->K, 16, L::BM,
-                CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&tb, w->d_wq8, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K, w->N, w->K, 16, L::BN,
-                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K, M, w->K, 64, L::BM,
+                CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&tb, w->d_wq8, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K, w->N, w->K, 64, L::BN,
+                CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&tsx, s_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, 1, sx_pitch, L::BM, 1,
