@@ -8,18 +8,22 @@
 // is first set by a bf16 MMA (ones x 786432) to the fp32 value 12582912,
 // whose bit pattern is the int32 0x4B400000; the int8 MMAs then add 256 P_g
 // to those bits, so the word read back is exactly the float
-// 12582912 + 256 P_g (|256 P_g| <= 2^20).  The rescale subtracts the
-// constant (exact) instead of converting int32 -> fp32, and folds the
-// result into an fp32 register accumulator with the scales
-// 2^-8 s_x[g][m] s_w[g][n].  The low-rank term Z L2 is one more tensor-core
+// 12582912 + 256 P_g (|256 P_g| <= 2^20).  The rescale is two fmas per
+// element and no int32 -> fp32 conversion: v = fma(word, s_w, c) with the
+// packed constant c = -fl32(12582912 s_w), i.e. v = 256 P_g s_w rounded once
+// after adding the constant's own rounding residual (at most 0.75 s_w,
+// about 1e-4 of a typical term), then acc = fma(v, 2^-8 s_x, acc).  The low-rank term Z L2 is one more tensor-core
 // stage (kind::f16, bf16 operands, fp32 in TMEM) added unscaled; then the
 // bias (and GELU) are applied and Y is written once, as bf16, by TMA.
 //
 // Persistent CTAs (one per SM, 128 x BN output tiles, static round-robin
 // schedule); 16 warps:
-//   warp 0      TMA producer: packed A (128 rows x 32 B) and B (BN x 32 B)
-//               per group into a 4-stage ring, and the bf16 Z / L2 slices
-//               of the low-rank stage (loaded straight into UMMA layout);
+//   warp 0      TMA producer: packed A (128 rows x 64 B) and B (BN x 64 B)
+//               of two groups per stage, one 64-byte-swizzled box per
+//               operand, into a 2-stage ring (narrow boxes would make the
+//               copy engine's per-row rate the limit), and the bf16 Z / L2
+//               slices of the low-rank stage (loaded straight into UMMA
+//               layout);
 //   warp 1      TMEM owner and MMA issuer (one thread);
 //   warps 2-7   expanders: packed nibbles -> int8 in the UMMA K-major
 //               layout (2-stage ring);
@@ -49,15 +53,14 @@ namespace svdq {
 namespace {
 
 constexpr int BM = 128;
-constexpr int NP = 4;            // packed-code stages
+constexpr int NP = 2;            // packed-code stages (two groups each)
 constexpr int THREADS = 512;
 constexpr int N_EXP = 192;       // expanders: warps 2-7
 constexpr int RES_WARP0 = 8;     // rescale / epilogue: warps 8-15
 constexpr int N_RES_WARPS = 8;
 constexpr uint32_t MAGIC_BITS = 0x4B400000u;   // bits of 12582912.0f = 1.5 * 2^23
-constexpr float MAGIC_F = 12582912.0f;
 constexpr uint16_t BF16_ONE = 0x3F80;          // 1.0
-constexpr uint16_t BF16_MAGIC16 = 0x4940;      // 786432 = 1.5 * 2^19; 16 of them make MAGIC_F
+constexpr uint16_t BF16_MAGIC16 = 0x4940;      // 786432 = 1.5 * 2^19; 16 of them make the bias
 // Register split after launch: the first two warpgroups (producer, MMA,
 // expanders) give registers to the two rescale warpgroups.
 // 256 * REG_LO + 256 * REG_HI
@@ -109,7 +112,10 @@ struct Lay {
   static constexpr int CW = BN / 2;                      // columns per rescale warp
   static constexpr int Y_BOX = 32 * 64 * 2;              // 32 rows x 64 bf16 (4 KB)
   static constexpr int Y_WARP = (CW / 64) * Y_BOX;
-  static constexpr int PK_A = BM * 32, PK_B = BN * 32, PK_STAGE = PK_A + PK_B;
+  // packed stage: 64-byte rows (two groups), 64-byte swizzle: chunk c of
+  // row r at r * 64 + 16 (c ^ ((r >> 1) & 3)); chunk 2 gs + hf is half hf
+  // of group gs of the stage
+  static constexpr int PK_A = BM * 64, PK_B = BN * 64, PK_STAGE = PK_A + PK_B;
   static constexpr int EX_A = BM * 64, EX_B = BN * 64, EX_STAGE = EX_A + EX_B;
   static constexpr int OFF_Y = 0;
   static constexpr int OFF_PK = OFF_Y + N_RES_WARPS * Y_WARP;
@@ -120,13 +126,14 @@ struct Lay {
   static constexpr int NLR = BN == 256 ? 2 : 4;
   static constexpr int LR_SA = BM * 32, LR_SB = BN * 32, LR_SLOT = LR_SA + LR_SB;
   static constexpr int OFF_LR = OFF_EX + NE * EX_STAGE;
-  // per-group scales: ring of NP + NE + NB slots, each s_x[128] then s_w[BN],
-  // filled by the producer warp together with the packed codes.  The producer
-  // may write group j's slot once the expanders released packed stage j - NP,
-  // which (through the MMA and TMEM barriers) implies that the rescale of
-  // group j - NP - NE - NB, the slot's previous owner, has finished.
-  static constexpr int NS = NP + NE + NB;
-  static constexpr int SC_SLOT = (BM + BN) * 4;
+  // per-group scales: ring of 2 NP + NE + NB slots, each s_x[128] then
+  // s_w[BN], filled by the producer warp together with the packed codes.  The
+  // producer writes the slots of groups j, j + 1 (stage k) once the expanders
+  // released stage k - NP, i.e. expanded every group up to j - 2 NP + 1;
+  // through the MMA and TMEM barriers the rescale of group j + 1 - 2 NP - NE
+  // - NB, the previous owner of the last slot written, has then finished.
+  static constexpr int NS = 2 * NP + NE + NB;
+  static constexpr int SC_SLOT = (BM + 2 * BN) * 4;       // s_x, s_w, c
   static constexpr int OFF_SC = OFF_LR + NLR * LR_SLOT;
   static constexpr int OFF_BIAS = OFF_SC + NS * SC_SLOT;   // per warp CW floats
   // constant operands of the accumulator-initialising bf16 MMA (K = 16)
@@ -139,6 +146,7 @@ struct Lay {
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;              // slack for 1024-B alignment
+  static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
 
@@ -171,8 +179,10 @@ __device__ __forceinline__ void expand16(uint32_t src, uint32_t d) {
 
 // The expanders' share of one group: CNT rounds of 32 consecutive 16-byte
 // units starting at round R0.  Unit j of an operand is half (j >> 3) & 1 of
-// row 8 (j >> 4) + (j & 7), so each quarter-warp reads and writes 128
-// contiguous bytes.  Offsets are fixed per thread and computed once.
+// row 8 (j >> 4) + (j & 7), so each quarter-warp reads one half of eight
+// consecutive rows (eight distinct 16-byte bank groups under the 64-byte
+// swizzle) and writes 128 contiguous bytes.  Offsets are fixed per thread
+// and computed once.
 template <int BN, int CNT>
 struct ExpandPlan {
   uint32_t src[CNT], dst[CNT];
@@ -184,13 +194,15 @@ struct ExpandPlan {
       const bool isa = u < BM * 2;
       const int j = isa ? u : u - BM * 2;
       const int hf = (j >> 3) & 1, row = ((j >> 4) << 3) | (j & 7);
-      src[k] = (isa ? 0 : L::PK_A) + hf * (isa ? BM : BN) * 16 + row * 16;
+      // group 0 of the stage; group 1 is chunk + 2, i.e. the offset ^ 32
+      src[k] = (isa ? 0 : L::PK_A) + row * 64 + ((hf ^ ((row >> 1) & 3)) << 4);
       dst[k] = (isa ? 0 : L::EX_A) + (row >> 3) * 512 + (row & 7) * 16 + hf * 256;
     }
   }
-  __device__ __forceinline__ void run(uint32_t pa, uint32_t ea) const {
+  // gsx = 32 * (group within the packed stage)
+  __device__ __forceinline__ void run(uint32_t pa, uint32_t ea, uint32_t gsx) const {
 #pragma unroll
-    for (int k = 0; k < CNT; ++k) expand16(pa + src[k], ea + dst[k]);
+    for (int k = 0; k < CNT; ++k) expand16(pa + (src[k] ^ gsx), ea + dst[k]);
   }
 };
 
@@ -265,44 +277,51 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     regs_dec<REG_LO>();
     if (warp == 0) {
       // ---------------------------------------------------- TMA producer
-      uint32_t it = 0, il = 0;
+      uint32_t it = 0, ig = 0, il = 0;     // packed stages, groups, low-rank slices
       bool alive = true;
       for (int wk = blockIdx.x; wk < p.num_tiles * p.splits && alive; wk += gridDim.x) {
         const WorkItem wi = work_item(p, wk);
         const int t = wi.t;
         const int m0 = (p.tile_m0 + t / p.tiles_n) * BM;
         const int n0 = (p.tile_n0 + t % p.tiles_n) * BN;
-        for (int g = wi.g0; g < wi.g1; ++g, ++it) {
+        for (int g = wi.g0; g < wi.g1; g += 2, ++it) {
+          const int ng = wi.g1 - g < 2 ? 1 : 2;     // groups in this stage
           const int s = it % NP;
           if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
-          const uint32_t slot = sbase + L::OFF_SC + (it % L::NS) * L::SC_SLOT;
           if (LAYER && !p.sx_tma) {
             // s_x rows not 16-byte aligned: 4-byte async copies by all lanes,
             // tracked by the stage's full barrier (raised before lane 0 arrives)
+            for (int k = 0; k < ng; ++k) {
+              const uint32_t slot = sbase + L::OFF_SC + ((ig + k) % L::NS) * L::SC_SLOT;
 #pragma unroll 4
-            for (int i = lane; i < BM; i += 32) {
-              const int row = m0 + i;
-              const bool in = row < p.M;
-              cp_async4(slot + 4 * i, p.s_x + (in ? (size_t)g * p.M + row : 0), in ? 4u : 0u);
+              for (int i = lane; i < BM; i += 32) {
+                const int row = m0 + i;
+                const bool in = row < p.M;
+                cp_async4(slot + 4 * i, p.s_x + (in ? (size_t)(g + k) * p.M + row : 0), in ? 4u : 0u);
+              }
             }
             cp_async_mbar_arrive(pk_full(s));
             __syncwarp();
           }
           if (lane == 0) {
             const uint32_t scale_bytes =
-                LAYER ? (p.sx_tma ? BM * 4 : 0) + BN * 4 : 0;
+                LAYER ? ng * ((p.sx_tma ? BM * 4 : 0) + 2 * BN * 4) : 0;
             mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE + scale_bytes);
             const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              tma_load_2d(dst + hh * (BM * 16), &tm_a, g * 32 + 16 * hh, m0, pk_full(s));
-              tma_load_2d(dst + L::PK_A + hh * (BN * 16), &tm_b, g * 32 + 16 * hh, n0, pk_full(s));
-            }
+            // one box per operand: packed bytes [32 g, 32 g + 64); a group
+            // past the end of K reads as zeros and is not used
+            tma_load_2d(dst, &tm_a, g * 32, m0, pk_full(s));
+            tma_load_2d(dst + L::PK_A, &tm_b, g * 32, n0, pk_full(s));
             if (LAYER) {
-              if (p.sx_tma) tma_load_2d(slot, &tm_sx, m0, g, pk_full(s));
-              tma_load_2d(slot + 4 * BM, &tm_sw, n0, g, pk_full(s));
+              for (int k = 0; k < ng; ++k) {
+                const uint32_t slot = sbase + L::OFF_SC + ((ig + k) % L::NS) * L::SC_SLOT;
+                if (p.sx_tma) tma_load_2d(slot, &tm_sx, m0, g + k, pk_full(s));
+                tma_load_2d(slot + 4 * BM, &tm_sw, n0, 2 * (g + k), pk_full(s));
+                tma_load_2d(slot + 4 * (BM + BN), &tm_sw, n0, 2 * (g + k) + 1, pk_full(s));
+              }
             }
           }
+          ig += ng;
           __syncwarp();
         }
         if (!alive) break;
@@ -386,17 +405,22 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       constexpr int ROUNDS = (BM + BN) * 2 / 32;
       static_assert(ROUNDS % 8 == 0, "expander split");
       auto expand_loop = [&](const auto& plan) {
-        uint32_t it = 0;
+        uint32_t ist = 0, it = 0;            // packed stages, groups
         for (int wk = blockIdx.x; wk < p.num_tiles * p.splits; wk += gridDim.x) {
           const WorkItem wi = work_item(p, wk);
-          for (int g = wi.g0; g < wi.g1; ++g, ++it) {
-            const int se = it % NE, sp = it % NP;
-            if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err)) return;
-            if (!wait_or_abort(pk_full(sp), (it / NP) & 1, abort_flag, p.err)) return;
-            plan.run(sbase + L::OFF_PK + sp * L::PK_STAGE, sbase + L::OFF_EX + se * L::EX_STAGE);
+          for (int g = wi.g0; g < wi.g1; g += 2, ++ist) {
+            const int ng = wi.g1 - g < 2 ? 1 : 2;
+            const int sp = ist % NP;
+            if (!wait_or_abort(pk_full(sp), (ist / NP) & 1, abort_flag, p.err)) return;
+            for (int k = 0; k < ng; ++k, ++it) {
+              const int se = it % NE;
+              if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err)) return;
+              plan.run(sbase + L::OFF_PK + sp * L::PK_STAGE, sbase + L::OFF_EX + se * L::EX_STAGE,
+                       32u * k);
+              fence_proxy_async_smem();
+              mbar_arrive(ex_full(se));
+            }
             mbar_arrive(pk_empty(sp));
-            fence_proxy_async_smem();
-            mbar_arrive(ex_full(se));
           }
         }
       };
@@ -457,7 +481,6 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             const float v = lds32(slot + 4u * (32 * q + r0 + 8 * i)) * 0.00390625f;  // 2^-8 (exact)
             sx2[i] = make_float2(v, v);
           }
-          const float2 nmag2 = make_float2(-MAGIC_F, -MAGIC_F);
           const uint32_t swa = slot + 4u * (BM + h * CW) + 16u * pq;
           uint32_t rb[2][16];
           tmem_ld16x256b_x2(ta, &rb[0][0]);
@@ -471,16 +494,19 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             }
             const uint32_t* r = rb[c & 1];
             const float4 s4 = lds128(swa + 64u * c);   // columns 2pq, 2pq+1, 8+2pq, 9+2pq
+            const float4 c4 = lds128(swa + 4u * BN + 64u * c);   // their constants
 #pragma unroll
             for (int bb = 0; bb < 2; ++bb) {
               const float2 sw2 = bb ? make_float2(s4.z, s4.w) : make_float2(s4.x, s4.y);
+              const float2 cc2 = bb ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 // register of row r0 + 8i: half (i >> 1), row (i & 1) of the 16-lane load
                 const uint32_t* wv = r + 8 * (i >> 1) + 4 * bb + 2 * (i & 1);
-                // 256 P_g, exactly: the word is the float MAGIC_F + 256 P_g
-                const float2 u = __fadd2_rn(make_float2(__uint_as_float(wv[0]), __uint_as_float(wv[1])), nmag2);
-                acc[i][2 * c + bb] = __ffma2_rn(__fmul2_rn(sx2[i], sw2), u, acc[i][2 * c + bb]);
+                // the word is the float SVDQ_ACC_BIAS + 256 P_g: v ~ 256 P_g s_w
+                const float2 v = __ffma2_rn(make_float2(__uint_as_float(wv[0]), __uint_as_float(wv[1])),
+                                            sw2, cc2);
+                acc[i][2 * c + bb] = __ffma2_rn(v, sx2[i], acc[i][2 * c + bb]);
               }
             }
             if (c + 1 < CW / 16) tmem_wait_ld();
@@ -660,10 +686,10 @@ struct LinMaps {
 bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
                   const uint16_t* Z, uint16_t* Y, int ldy, int epilogue, int BN, LinMaps& m,
                   LinArgs& a) {
-  if (!make_map(&m.ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 16, BM,
-                CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&m.tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 16, BN,
-                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  if (!make_map(&m.ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 64, BM,
+                CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&m.tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 64, BN,
+                CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map(&m.ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return false;
@@ -673,7 +699,7 @@ bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* 
   const bool sx_tma = (M % 4) == 0;
   if ((sx_tma && !make_map(&m.tsx, s_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, w->G,
                            (uint64_t)M * 4, BM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
-      !make_map(&m.tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N16, w->G,
+      !make_map(&m.tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N16, 2 * w->G,
                 (uint64_t)w->N16 * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
   if (w->rank > 0 &&
@@ -757,10 +783,10 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
                             int nrows, int col0, int ncols, int32_t* P, cudaStream_t st) {
   const int BN = pick_bn(w->N);
   CUtensorMap ta, tb;
-  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 16, BM,
-                CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 16, BN,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 64, BM,
+                CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 64, BN,
+                CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   LinArgs a{};
   a.M = M; a.N = w->N; a.K = w->K; a.G = w->G;
