@@ -68,6 +68,7 @@ constexpr uint16_t BF16_MAGIC16 = 0x4940;      // 786432 = 1.5 * 2^19; 16 of the
 // count); the launcher checks the compiled count before every launch.
 constexpr int REG_LO = 56;
 constexpr int REG_HI = 200;
+constexpr int RCH = 2;           // 16-column TMEM chunks per rescale load batch
 constexpr int REG_NEED = (256 * REG_LO + 256 * REG_HI + THREADS - 1) / THREADS;
 
 struct LinArgs {
@@ -482,34 +483,45 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             sx2[i] = make_float2(v, v);
           }
           const uint32_t swa = slot + 4u * (BM + h * CW) + 16u * pq;
-          uint32_t rb[2][16];
-          tmem_ld16x256b_x2(ta, &rb[0][0]);
-          tmem_ld16x256b_x2(ta + (16u << 16), &rb[0][8]);
+          // batches of RCH 16-column chunks, double-buffered: the loads of
+          // batch cb+1 are in flight while batch cb is rescaled (wait::ld
+          // waits for all of them)
+          uint32_t rb[2][16 * RCH];
+          auto load_batch = [&](int cb, uint32_t* dst) {
+#pragma unroll
+            for (int u = 0; u < RCH; ++u) {
+              tmem_ld16x256b_x2(ta + 16 * (cb * RCH + u), dst + 16 * u);
+              tmem_ld16x256b_x2(ta + 16 * (cb * RCH + u) + (16u << 16), dst + 16 * u + 8);
+            }
+          };
+          constexpr int NBATCH = CW / (16 * RCH);
+          load_batch(0, rb[0]);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < CW / 16; ++c) {
-            if (c + 1 < CW / 16) {
-              tmem_ld16x256b_x2(ta + 16 * (c + 1), &rb[(c + 1) & 1][0]);
-              tmem_ld16x256b_x2(ta + 16 * (c + 1) + (16u << 16), &rb[(c + 1) & 1][8]);
-            }
-            const uint32_t* r = rb[c & 1];
-            const float4 s4 = lds128(swa + 64u * c);   // columns 2pq, 2pq+1, 8+2pq, 9+2pq
-            const float4 c4 = lds128(swa + 4u * BN + 64u * c);   // their constants
+          for (int cb = 0; cb < NBATCH; ++cb) {
+            if (cb + 1 < NBATCH) load_batch(cb + 1, rb[(cb + 1) & 1]);
 #pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-              const float2 sw2 = bb ? make_float2(s4.z, s4.w) : make_float2(s4.x, s4.y);
-              const float2 cc2 = bb ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+            for (int u = 0; u < RCH; ++u) {
+              const int c = cb * RCH + u;
+              const uint32_t* r = rb[cb & 1] + 16 * u;
+              const float4 s4 = lds128(swa + 64u * c);   // columns 2pq, 2pq+1, 8+2pq, 9+2pq
+              const float4 c4 = lds128(swa + 4u * BN + 64u * c);   // their constants
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                // register of row r0 + 8i: half (i >> 1), row (i & 1) of the 16-lane load
-                const uint32_t* wv = r + 8 * (i >> 1) + 4 * bb + 2 * (i & 1);
-                // the word is the float SVDQ_ACC_BIAS + 256 P_g: v ~ 256 P_g s_w
-                const float2 v = __ffma2_rn(make_float2(__uint_as_float(wv[0]), __uint_as_float(wv[1])),
-                                            sw2, cc2);
-                acc[i][2 * c + bb] = __ffma2_rn(v, sx2[i], acc[i][2 * c + bb]);
+              for (int bb = 0; bb < 2; ++bb) {
+                const float2 sw2 = bb ? make_float2(s4.z, s4.w) : make_float2(s4.x, s4.y);
+                const float2 cc2 = bb ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  // register of row r0 + 8i: half (i >> 1), row (i & 1) of the 16-lane load
+                  const uint32_t* wv = r + 8 * (i >> 1) + 4 * bb + 2 * (i & 1);
+                  // the word is the float SVDQ_ACC_BIAS + 256 P_g: v ~ 256 P_g s_w
+                  const float2 v = __ffma2_rn(make_float2(__uint_as_float(wv[0]), __uint_as_float(wv[1])),
+                                              sw2, cc2);
+                  acc[i][2 * c + bb] = __ffma2_rn(v, sx2[i], acc[i][2 * c + bb]);
+                }
               }
             }
-            if (c + 1 < CW / 16) tmem_wait_ld();
+            if (cb + 1 < NBATCH) tmem_wait_ld();
           }
         } else {
 #pragma unroll 1
