@@ -9,10 +9,14 @@
 // whose bit pattern is the int32 0x4B400000; the int8 MMAs then add 256 P_g
 // to those bits, so the word read back is exactly the float
 // 12582912 + 256 P_g (|256 P_g| <= 2^20).  The rescale is two fmas per
-// element and no int32 -> fp32 conversion: v = fma(word, s_w, c) with the
-// packed constant c = -fl32(12582912 s_w), i.e. v = 256 P_g s_w rounded once
-// after adding the constant's own rounding residual (at most 0.75 s_w,
-// about 1e-4 of a typical term), then acc = fma(v, 2^-8 s_x, acc).  The low-rank term Z L2 is one more tensor-core
+// element and no int32 -> fp32 conversion: v = fma(word, s_w, c) with
+// c = -fl32(12582912 s_w) (one multiply per column pair, shared by the
+// thread's four rows), i.e. v = 256 P_g s_w rounded once after adding the
+// constant's own rounding residual (at most 0.75 s_w, about 1e-4 of a
+// typical term), then acc = fma(v, 2^-8 s_x, acc).  Only s_w is read from
+// shared memory: a broadcast 128-bit load costs four wavefronts whatever
+// the number of distinct addresses, so scale loads are the rescale's
+// largest shared-memory cost.  The low-rank term Z L2 is one more tensor-core
 // stage (kind::f16, bf16 operands, fp32 in TMEM) added unscaled; then the
 // bias (and GELU) are applied and Y is written once, as bf16, by TMA.
 //
@@ -134,7 +138,7 @@ struct Lay {
   // through the MMA and TMEM barriers the rescale of group j + 1 - 2 NP - NE
   // - NB, the previous owner of the last slot written, has then finished.
   static constexpr int NS = 2 * NP + NE + NB;
-  static constexpr int SC_SLOT = (BM + 2 * BN) * 4;       // s_x, s_w, c
+  static constexpr int SC_SLOT = (BM + BN) * 4;
   static constexpr int OFF_SC = OFF_LR + NLR * LR_SLOT;
   static constexpr int OFF_BIAS = OFF_SC + NS * SC_SLOT;   // per warp CW floats
   // constant operands of the accumulator-initialising bf16 MMA (K = 16)
@@ -306,7 +310,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
           }
           if (lane == 0) {
             const uint32_t scale_bytes =
-                LAYER ? ng * ((p.sx_tma ? BM * 4 : 0) + 2 * BN * 4) : 0;
+                LAYER ? ng * ((p.sx_tma ? BM * 4 : 0) + BN * 4) : 0;
             mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE + scale_bytes);
             const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
             // one box per operand: packed bytes [32 g, 32 g + 64); a group
@@ -317,8 +321,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               for (int k = 0; k < ng; ++k) {
                 const uint32_t slot = sbase + L::OFF_SC + ((ig + k) % L::NS) * L::SC_SLOT;
                 if (p.sx_tma) tma_load_2d(slot, &tm_sx, m0, g + k, pk_full(s));
-                tma_load_2d(slot + 4 * BM, &tm_sw, n0, 2 * (g + k), pk_full(s));
-                tma_load_2d(slot + 4 * (BM + BN), &tm_sw, n0, 2 * (g + k) + 1, pk_full(s));
+                tma_load_2d(slot + 4 * BM, &tm_sw, n0, g + k, pk_full(s));
               }
             }
           }
@@ -505,11 +508,10 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               const int c = cb * RCH + u;
               const uint32_t* r = rb[cb & 1] + 16 * u;
               const float4 s4 = lds128(swa + 64u * c);   // columns 2pq, 2pq+1, 8+2pq, 9+2pq
-              const float4 c4 = lds128(swa + 4u * BN + 64u * c);   // their constants
 #pragma unroll
               for (int bb = 0; bb < 2; ++bb) {
                 const float2 sw2 = bb ? make_float2(s4.z, s4.w) : make_float2(s4.x, s4.y);
-                const float2 cc2 = bb ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+                const float2 cc2 = __fmul2_rn(sw2, make_float2(-SVDQ_ACC_BIAS, -SVDQ_ACC_BIAS));
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                   // register of row r0 + 8i: half (i >> 1), row (i & 1) of the 16-lane load
@@ -711,7 +713,7 @@ bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* 
   const bool sx_tma = (M % 4) == 0;
   if ((sx_tma && !make_map(&m.tsx, s_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, w->G,
                            (uint64_t)M * 4, BM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
-      !make_map(&m.tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N16, 2 * w->G,
+      !make_map(&m.tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N16, w->G,
                 (uint64_t)w->N16 * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
   if (w->rank > 0 &&

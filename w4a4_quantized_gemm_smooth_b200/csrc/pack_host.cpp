@@ -150,14 +150,11 @@ svdq_status upload(svdq_weights* w, cudaStream_t st) {
     if ((s = dev_alloc_copy(&w->d_sw8, sw8p.data(), sw8p.size(), st))) return s;
   } else {
     if ((s = dev_alloc_copy(&w->d_wq, w->wq.data(), (size_t)N * K / 2, st))) return s;
-    std::vector<float> swp((size_t)2 * G * w->N16, 0.0f);
+    std::vector<float> swp((size_t)G * w->N16, 0.0f);
     for (int g = 0; g < G; ++g)
       for (int n = 0; n < N; ++n) {
         const int c = n & 15, pos = (n & ~15) + 4 * ((c & 7) >> 1) + 2 * (c >> 3) + (c & 1);
-        const float sw = w->sw[(size_t)g * N + n];
-        swp[(size_t)(2 * g) * w->N16 + pos] = sw;
-        // -fl32(bias * s_w): the product is exact in fp64, one rounding to fp32
-        swp[(size_t)(2 * g + 1) * w->N16 + pos] = (float)(-(double)SVDQ_ACC_BIAS * (double)sw);
+        swp[(size_t)g * w->N16 + pos] = w->sw[(size_t)g * N + n];
       }
     if ((s = dev_alloc_copy(&w->d_sw, swp.data(), swp.size(), st))) return s;
   }

@@ -21,11 +21,9 @@ struct svdq_weights {
   // device copies (owned)
   float* d_inv_lambda = nullptr;   // [K]
   uint8_t* d_wq = nullptr;         // [N][K/2] packed residual codes
-  // [2G][N16], zero padded: row 2g holds s_w of group g, row 2g + 1 the
-  // rescale constant c = -fl32(SVDQ_ACC_BIAS * s_w) of the same columns.
-  // Inside each block of 16 columns, column 8b + 2p + e is stored at
-  // 4p + 2b + e, so that the rescale thread that owns the column pairs 2p,
-  // 2p+1 of both 8-column halves reads them as one float4
+  // [G][N16], zero padded; inside each block of 16 columns, column
+  // 8b + 2p + e is stored at 4p + 2b + e, so that the rescale thread that owns
+  // the column pairs 2p, 2p+1 of both 8-column halves reads them as one float4
   float* d_sw = nullptr;
   uint16_t* d_L1T = nullptr;       // [rank_pad][K] bf16, transposed L1
   uint16_t* d_L2 = nullptr;        // [rank_pad][N] bf16
@@ -48,7 +46,7 @@ struct svdq_weights {
 
 // The GEMM's int32 group accumulators start from the float 1.5 * 2^23 (bit
 // pattern 0x4B400000), so the word read back is the float SVDQ_ACC_BIAS +
-// 256 P_g; the rescale removes the bias with the constant c of d_sw.
+// 256 P_g; the rescale removes the bias with c = -fl32(SVDQ_ACC_BIAS s_w).
 constexpr float SVDQ_ACC_BIAS = 12582912.0f;
 
 // Device error word values.
