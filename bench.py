@@ -45,8 +45,8 @@ LINEAR_SOURCES = ("w4a4_quantized_gemm_smooth_b200/csrc/linear_ws.cu",
                   "w4a4_quantized_gemm_smooth_b200/csrc/gemm_common.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/ptx.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/svdq_internal.h")
-LINEAR_TRAFFIC = {"sources_sha1": "58864ad822658f5b949b9ea4be4114ba9c2c4753",
-                  "workload": "flux_qkv", "bytes": 24911104 + 29313792}
+LINEAR_TRAFFIC = {"sources_sha1": "4c18e40cd87dfbec7e35922f21fbf97dfcc7d13b",
+                  "workload": "flux_qkv", "bytes": 24867840 + 28838912}
 
 
 def _linear_traffic(workload):
