@@ -20,6 +20,8 @@ What it computes follows "SVDQuant: How a Small High-Precision Branch Makes
     error, factors re-fitted to W~ - Q(R)                        (section 5)
   * W8A8 comparator: int8 operands, one scale per token / output channel
     applied once          (section 8, the eight-bit setting; section 9.3, INT8)
+  * NVFP4 variant: E2M1 codes in groups of 16 with E4M3 group scales and
+    an fp32 scale per row                         (section 8; section 9.1)
 
 Readings taken where the pages leave a step open (each is listed in the
 design notes of the repository):
@@ -52,6 +54,9 @@ __all__ = [
     "two_branch_unquantized", "dequantize_groups", "residual_quantize",
     "leading_svd", "layer_output_error", "refine_factors", "pack_weights_calibrated",
     "quantize_rows_int8", "pack_weights_w8a8", "quantize_act_w8a8", "linear_w8a8",
+    "NVFP4_GROUP", "E2M1_VALUES", "round_e4m3", "e4m3_bits", "e2m1_codes", "e2m1_values",
+    "quantize_nvfp4_rows", "dequantize_nvfp4", "pack_weights_nvfp4", "quantize_act_nvfp4",
+    "linear_nvfp4",
 ]
 
 GROUP = 64
@@ -478,6 +483,144 @@ def linear_w8a8(xcodes, s_x, Z, wcodes, s_w, L2b, bias, apply_gelu=False, rows=N
     P = xc[rows].astype(np.float64) @ np.asarray(wcodes)[cols].astype(np.float64).T
     Y = (np.asarray(s_x, dtype=np.float64)[rows][:, None] *
          np.asarray(s_w, dtype=np.float64)[cols][None, :]) * P
+    if np.asarray(L2b).shape[0]:
+        Y += np.asarray(Z)[rows] @ np.asarray(L2b)[:, cols]
+    Y += np.asarray(bias, dtype=np.float64)[cols][None, :]
+    if apply_gelu:
+        Y = gelu(Y)
+    return Y, round_bf16(Y)
+
+
+# --------------------------------------------------------------------------
+# NVFP4 variant: FP4 (E2M1) codes in groups of 16 along K with FP8 (E4M3)
+# group scales (review section 8: "NVFP4 uses group size 16 with FP8
+# scales"; section 9.1 on the nonuniform FP4 grid).  Reading: each row (a
+# token of x~, or an output column of R, over all K) also has an fp32 scale
+# s = fl32(max|row| / (6 * 448)), so that the group scales use E4M3's range:
+#     b = e4m3(fl32(max|group| / fl32(6 s))),  q = e2m1(z / (b s)),
+# both rounded to nearest, ties to even, saturating at 448 and 6.
+# --------------------------------------------------------------------------
+NVFP4_GROUP = 16
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+_E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+E4M3_MAX = 448.0
+
+
+def round_e4m3(t):
+    """Round non-negative float64 values to FP8 E4M3 (4 significant bits,
+    exponent bias 7, subnormal quantum 2^-9, largest finite 448), nearest
+    with ties to even, saturating at 448.  Returns float64 values."""
+    t = np.asarray(t, dtype=np.float64)
+    out = np.zeros_like(t)
+    pos = t > 0
+    if np.any(pos):
+        tp = t[pos]
+        _, e = np.frexp(tp)                        # tp = m 2^e, 0.5 <= m < 1
+        qexp = np.maximum(e - 4, -9)               # quantum exponent: 3 fraction bits, min 2^-9
+        v = np.ldexp(np.rint(np.ldexp(tp, -qexp)), qexp)
+        out[pos] = np.minimum(v, E4M3_MAX)
+    return out
+
+
+def e4m3_bits(v):
+    """Bit patterns (uint8) of non-negative E4M3 values (as from round_e4m3)."""
+    v = np.asarray(v, dtype=np.float64)
+    bits = np.zeros(v.shape, dtype=np.uint8)
+    nz = v > 0
+    if np.any(nz):
+        m, e = np.frexp(v[nz])                     # v = m 2^e
+        ebias = e - 1 + 7                          # exponent field of a normal
+        sub = ebias <= 0
+        man = np.where(sub, np.rint(v[nz] * 2.0 ** 9), np.rint((m * 2 - 1) * 8))
+        field = np.where(sub, 0, ebias)
+        bits[nz] = ((field << 3) | man.astype(np.int64)).astype(np.uint8)
+    return bits
+
+
+def e2m1_codes(z, d):
+    """FP4 E2M1 codes (bit 3 = sign, bits 0-2 = index into E2M1_VALUES) of the
+    exact quotients z / d, d > 0 (float64, z / d decided by exact fp64
+    comparisons of |z| with the grid midpoints times d), nearest with ties
+    to the even index, saturating at 6.  A zero magnitude has no sign."""
+    z = np.asarray(z, dtype=np.float64)
+    d = np.broadcast_to(np.asarray(d, dtype=np.float64), z.shape)
+    a = np.abs(z)
+    mids = _E2M1_MIDS[None, :] * d.reshape(-1)[:, None]      # exact: <= 31 bits
+    af = a.reshape(-1)
+    idx = np.sum(mids < af[:, None], axis=1)
+    tie = np.zeros_like(af, dtype=bool)
+    ok = idx < 7
+    tie[ok] = af[ok] == mids[ok, idx[ok]]
+    idx = np.where(tie & (idx % 2 == 1), idx + 1, idx).reshape(z.shape)
+    sign = (z < 0) & (idx > 0)
+    return (idx | (sign.astype(np.int64) << 3)).astype(np.int64)
+
+
+def e2m1_values(codes):
+    c = np.asarray(codes, dtype=np.int64)
+    v = E2M1_VALUES[c & 7]
+    return np.where(c & 8, -v, v)
+
+
+def quantize_nvfp4_rows(v):
+    """v float64 [rows, K] of fp32 values (K % 16 == 0) -> (codes [rows, K],
+    group scales b [rows, K/16] as E4M3 values, row scales s [rows])."""
+    v = np.asarray(v, dtype=np.float64)
+    rows, K = v.shape
+    if K % NVFP4_GROUP:
+        raise ValueError("K must be a multiple of 16")
+    s = round_f32(np.max(np.abs(v), axis=1) / (6.0 * E4M3_MAX))
+    d6 = round_f32(6.0 * s)
+    g = v.reshape(rows, K // NVFP4_GROUP, NVFP4_GROUP)
+    mg = np.max(np.abs(g), axis=2)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.where(d6[:, None] > 0, round_f32(mg / d6[:, None]), 0.0)
+    b = round_e4m3(t)
+    d = b * s[:, None]                             # exact: 4 x 24 bits
+    codes = np.zeros(g.shape, dtype=np.int64)
+    live = d > 0
+    if np.any(live):
+        codes[live] = e2m1_codes(g[live], d[live][:, None])
+    return codes.reshape(rows, K), b, s
+
+
+def dequantize_nvfp4(codes, b, s):
+    rows, K = np.asarray(codes).shape
+    v = e2m1_values(codes).reshape(rows, K // NVFP4_GROUP, NVFP4_GROUP)
+    return (v * (np.asarray(b)[:, :, None] * np.asarray(s)[:, None, None])).reshape(rows, K)
+
+
+def pack_weights_nvfp4(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None, svd=None):
+    """pack_weights' smoothing, factors and residual R, with R quantised by
+    the NVFP4 rule per output column: wcodes4 [N, K], wb4 [N, K/16], ws4 [N]."""
+    p = pack_weights(W_bits, act_absmax, rank, alpha=alpha, bias_bits=bias_bits, svd=svd)
+    codes, b, s = quantize_nvfp4_rows(round_f32(p["R"].T))
+    return dict(p, wcodes4=codes, wb4=b, ws4=s)
+
+
+def quantize_act_nvfp4(X_bits, inv_lambda, L1b):
+    """x~ = fl32(x * inv_lambda), its NVFP4 codes, group and row scales, and
+    the 16-bit down-projection of quantize_act.
+    Returns (codes [M, K], b [M, K/16], s [M], Z [M, r], xhat)."""
+    X = bf16_bits_to_f64(X_bits)
+    xhat = round_f32(X * np.asarray(inv_lambda, dtype=np.float64)[None, :])
+    codes, b, s = quantize_nvfp4_rows(xhat)
+    r = L1b.shape[1]
+    Z = round_bf16(round_bf16(xhat) @ L1b) if r else np.zeros((X.shape[0], 0))
+    return codes, b, s, Z, xhat
+
+
+def linear_nvfp4(xcodes, xb, xs, Z, wcodes, wb, ws, L2b, bias, apply_gelu=False, rows=None,
+                 cols=None):
+    """Y = deq(X) deq(W)^T + Z L2 + b with deq = code value x group scale x
+    row scale (every dequantised value is exact in fp64), fp64 sums,
+    optional GELU, one bf16 rounding.  Returns (Y, Y_bf16)."""
+    xc = np.asarray(xcodes)
+    rows = np.arange(xc.shape[0]) if rows is None else np.asarray(rows)
+    cols = np.arange(np.asarray(wcodes).shape[0]) if cols is None else np.asarray(cols)
+    Xq = dequantize_nvfp4(xc[rows], np.asarray(xb)[rows], np.asarray(xs)[rows])
+    Wq = dequantize_nvfp4(np.asarray(wcodes)[cols], np.asarray(wb)[cols], np.asarray(ws)[cols])
+    Y = Xq @ Wq.T
     if np.asarray(L2b).shape[0]:
         Y += np.asarray(Z)[rows] @ np.asarray(L2b)[:, cols]
     Y += np.asarray(bias, dtype=np.float64)[cols][None, :]
