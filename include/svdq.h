@@ -62,7 +62,7 @@ enum { SVDQ_EPI_NONE = 0, SVDQ_EPI_GELU = 1 };
 
 /* Number format of a packed handle: the W4A4 group format of every call
  * above, or the W8A8 comparator of svdq_pack_weights_w8a8. */
-enum { SVDQ_FORMAT_W4A4 = 0, SVDQ_FORMAT_W8A8 = 1 };
+enum { SVDQ_FORMAT_W4A4 = 0, SVDQ_FORMAT_W8A8 = 1, SVDQ_FORMAT_NVFP4 = 2 };
 
 #define SVDQ_GROUP 64
 #define SVDQ_MAX_RANK 128
@@ -337,6 +337,70 @@ svdq_status svdq_quantize_act_w8a8(const svdq_weights* w, int M, const uint16_t*
 svdq_status svdq_linear_w8a8(const svdq_weights* w, int M, const int8_t* xq,
                              const float* s_x, const uint16_t* Z, uint16_t* Y,
                              int ldy, int epilogue, cudaStream_t stream);
+
+/*
+ * ------------------------------------------------------------------------
+ * NVFP4 variant (review section 8: NVFP4 uses groups of 16 with FP8
+ * scales; section 9.1 on the nonuniform FP4 grid).  The same two-branch
+ * layer with FP4 E2M1 operands whose groups of 16 along K carry an FP8 E4M3
+ * scale, applied by the tensor cores (block-scaled MMA), and an fp32 scale
+ * per row (token of x~, output column of R):
+ *
+ *   s = fl32(max|row| / 2688)                      (2688 = 6 * 448)
+ *   b = e4m3(fl32(max|group| / fl32(6 s)))         nearest-even, <= 448
+ *   q = e2m1(z / (b s))                            nearest-even on
+ *                                                  {0, .5, 1, 1.5, 2, 3, 4, 6}
+ *   Y = s_x[m] s_w[n] sum_k (q_x b_x)(q_w b_w) + Z L2 + b
+ *
+ * Codes: two per byte, even k in the low nibble, bit 3 = sign.  Group
+ * scales cross this ABI in the tensor-core atom layout: for rows
+ * [128 a, 128 a + 128) and K block kb of 64, a 512-byte atom at
+ * (a * K/64 + kb) * 512 holds row r's four scales at 16 (r % 32) + 4 (r / 32);
+ * svdq_nvfp4_sf_bytes(rows, K) gives the size (rows padded to 128).
+ * K % 64 == 0; save/load and LoRA are W4A4 only; the W4A4 and W8A8 calls
+ * reject an NVFP4 handle and these calls reject the others.
+ * ------------------------------------------------------------------------
+ */
+
+/* Offline pack (as svdq_pack_weights_w8a8, with R quantised by the NVFP4
+ * rule per output column). */
+svdq_status svdq_pack_weights_nvfp4(int K, int N, int rank, const uint16_t* W,
+                                    const float* act_absmax, double alpha,
+                                    const uint16_t* bias, int to_device,
+                                    cudaStream_t stream, svdq_weights** out);
+
+/* Host copies of the NVFP4 residual: codes [N][K/2], E4M3 group-scale bits
+ * sf [N][K/16] (row-major, not the atom layout), row scales s_w [N]. */
+svdq_status svdq_weights_export_nvfp4(const svdq_weights* w, uint8_t* codes, uint8_t* sf,
+                                      float* s_w);
+
+/* Bytes of a group-scale array in the atom layout (0 for invalid sizes). */
+size_t svdq_nvfp4_sf_bytes(int rows, int K);
+
+/*
+ * Activation pass: x~ = fl32(x * inv_lambda_k); then
+ *   xq  [M][K/2]  packed E2M1 codes;
+ *   sfa           E4M3 group scales, atom layout, svdq_nvfp4_sf_bytes(M, K)
+ *                 bytes (the rows past M are written as 0);
+ *   s_x [M]       fp32 row scales;
+ *   Z   [M][rank] bf16 down-projection bf16(bf16(x~) L1), fp32 accumulation.
+ * One kernel, two sweeps of each token block as svdq_quantize_act_w8a8.
+ */
+svdq_status svdq_quantize_act_nvfp4(const svdq_weights* w, int M, const uint16_t* X,
+                                    int ldx, uint8_t* xq, uint8_t* sfa, float* s_x,
+                                    uint16_t* Z, cudaStream_t stream);
+
+/*
+ * Product: one tcgen05 kernel (kind::mxf4nvf4 block-scaled MMA, scales
+ * staged into TMEM by tcgen05.cp) accumulating sum_k (q_x b_x)(q_w b_w)
+ * in fp32, and the low-rank product Z L2 (bf16 tensor cores) in a second
+ * TMEM buffer; the epilogue forms s_x s_w acc + Z L2 + b (optional GELU)
+ * and stores bf16 Y [M][ldy].  Inputs as produced by
+ * svdq_quantize_act_nvfp4.
+ */
+svdq_status svdq_linear_nvfp4(const svdq_weights* w, int M, const uint8_t* xq,
+                              const uint8_t* sfa, const float* s_x, const uint16_t* Z,
+                              uint16_t* Y, int ldy, int epilogue, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

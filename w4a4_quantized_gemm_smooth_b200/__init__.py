@@ -10,10 +10,11 @@ The call names follow include/svdq.h:
     svdq_weights_export, svdq_weights_save, svdq_weights_load,
     svdq_quantize_act, svdq_linear, svdq_get_device_error,
     svdq_debug_partials, svdq_linear_splitk*, svdq_pack_weights_calibrated,
-    and the W8A8 comparator svdq_pack_weights_w8a8, svdq_quantize_act_w8a8,
-    svdq_linear_w8a8
-and SVDQLinear / W8A8Linear bundle one packed layer with its two hot-path
-calls.
+    the W8A8 comparator svdq_pack_weights_w8a8, svdq_quantize_act_w8a8,
+    svdq_linear_w8a8, and the NVFP4 variant svdq_pack_weights_nvfp4,
+    svdq_quantize_act_nvfp4, svdq_linear_nvfp4
+and SVDQLinear / W8A8Linear / NVFP4Linear bundle one packed layer with its
+two hot-path calls.
 """
 from __future__ import annotations
 
@@ -28,7 +29,8 @@ __all__ = [
     "svdq_quantize_act", "svdq_linear", "svdq_get_device_error",
     "svdq_debug_partials", "EPI_NONE", "EPI_GELU", "LIB_PATH",
     "svdq_pack_weights_w8a8", "svdq_quantize_act_w8a8", "svdq_linear_w8a8", "W8A8Linear",
-    "FORMAT_W4A4", "FORMAT_W8A8",
+    "FORMAT_W4A4", "FORMAT_W8A8", "FORMAT_NVFP4", "svdq_pack_weights_nvfp4",
+    "svdq_quantize_act_nvfp4", "svdq_linear_nvfp4", "svdq_nvfp4_sf_bytes", "NVFP4Linear",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -37,6 +39,7 @@ EPI_NONE = 0
 EPI_GELU = 1
 FORMAT_W4A4 = 0
 FORMAT_W8A8 = 1
+FORMAT_NVFP4 = 2
 
 _STATUS = {
     0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_SHAPE",
@@ -98,6 +101,12 @@ def lib() -> ctypes.CDLL:
         "svdq_weights_format": (_i, [_vp]),
         "svdq_quantize_act_w8a8": (_i, [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp]),
         "svdq_linear_w8a8": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _vp]),
+        "svdq_pack_weights_nvfp4": (_i, [_i, _i, _i, _vp, _vp, ctypes.c_double, _vp, _i, _vp,
+                                         _vp]),
+        "svdq_weights_export_nvfp4": (_i, [_vp, _vp, _vp, _vp]),
+        "svdq_nvfp4_sf_bytes": (ctypes.c_size_t, [_i, _i]),
+        "svdq_quantize_act_nvfp4": (_i, [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
+        "svdq_linear_nvfp4": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -160,6 +169,12 @@ class Weights:
             out["s_w8"] = np.empty(N, np.float32)
             _check(lib().svdq_weights_export_w8a8(self._h, _np_ptr(out["wq8"]),
                                                   _np_ptr(out["s_w8"])), "svdq_weights_export_w8a8")
+        if self.format == FORMAT_NVFP4:
+            out["wq4"] = np.empty((N, K // 2), np.uint8)
+            out["sf4"] = np.empty((N, K // 16), np.uint8)
+            out["s_w4"] = np.empty(N, np.float32)
+            _check(lib().svdq_weights_export_nvfp4(self._h, _np_ptr(out["wq4"]), _np_ptr(out["sf4"]),
+                                                   _np_ptr(out["s_w4"])), "svdq_weights_export_nvfp4")
         return out
 
     def save(self, path: str):
@@ -328,6 +343,40 @@ def svdq_linear_w8a8(w: Weights, xq, s_x, Z, Y, epilogue=EPI_NONE, stream=None):
            "svdq_linear_w8a8")
 
 
+def svdq_pack_weights_nvfp4(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None, to_device=True,
+                            stream=None) -> Weights:
+    """Offline pack of the NVFP4 variant (E2M1 residual, E4M3 group scales)."""
+    W_bits, act_absmax, bias_bits, _, _, _ = _pack_args(W_bits, act_absmax, bias_bits, None, None)
+    N, K = W_bits.shape
+    h = _vp()
+    _check(lib().svdq_pack_weights_nvfp4(K, N, int(rank), _np_ptr(W_bits), _np_ptr(act_absmax),
+                                         float(alpha), _np_ptr(bias_bits), 1 if to_device else 0,
+                                         _stream_ptr(stream) if to_device else None,
+                                         ctypes.byref(h)), "svdq_pack_weights_nvfp4")
+    return Weights(h)
+
+
+def svdq_nvfp4_sf_bytes(rows: int, K: int) -> int:
+    return int(lib().svdq_nvfp4_sf_bytes(int(rows), int(K)))
+
+
+def svdq_quantize_act_nvfp4(w: Weights, X, xq, sfa, s_x, Z=None, stream=None):
+    """X: cuda bf16 [M, K]; xq uint8 [M, K/2]; sfa uint8 [svdq_nvfp4_sf_bytes(M, K)];
+    s_x float32 [M]; Z bf16 [M, rank] (stored divided by s_x)."""
+    M = X.shape[0]
+    _check(lib().svdq_quantize_act_nvfp4(w.handle, M, _dev_ptr(X), X.stride(0), _dev_ptr(xq),
+                                         _dev_ptr(sfa), _dev_ptr(s_x), _dev_ptr(Z),
+                                         _stream_ptr(stream)), "svdq_quantize_act_nvfp4")
+
+
+def svdq_linear_nvfp4(w: Weights, xq, sfa, s_x, Z, Y, epilogue=EPI_NONE, stream=None):
+    """Y: cuda bf16 [M, N] (row stride Y.stride(0))."""
+    M = Y.shape[0]
+    _check(lib().svdq_linear_nvfp4(w.handle, M, _dev_ptr(xq), _dev_ptr(sfa), _dev_ptr(s_x),
+                                   _dev_ptr(Z), _dev_ptr(Y), Y.stride(0), int(epilogue),
+                                   _stream_ptr(stream)), "svdq_linear_nvfp4")
+
+
 def svdq_get_device_error(w: Weights, stream=None):
     _check(lib().svdq_get_device_error(w.handle, _stream_ptr(stream)), "device")
 
@@ -396,6 +445,33 @@ class W8A8Linear(SVDQLinear):
             Y = out
         svdq_quantize_act_w8a8(self.w, X, xq, s_x, Z)
         svdq_linear_w8a8(self.w, xq, s_x, Z, Y, self.epilogue)
+        return Y
+
+    __call__ = forward
+
+
+class NVFP4Linear(SVDQLinear):
+    """The NVFP4 layer: svdq_quantize_act_nvfp4 then svdq_linear_nvfp4."""
+
+    def buffers(self, M: int, device="cuda"):
+        import torch
+        if M != self._M:
+            K, N, r = self.w.K, self.w.N, self.w.rank
+            self.xq = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+            self.sfa = torch.empty((svdq_nvfp4_sf_bytes(M, K),), dtype=torch.uint8, device=device)
+            self.s_x = torch.empty((M,), dtype=torch.float32, device=device)
+            self.Z = torch.empty((M, max(r, 1)), dtype=torch.bfloat16, device=device) if r else None
+            self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            self._M = M
+        return self.xq, self.sfa, self.s_x, self.Z, self.Y
+
+    def forward(self, X, out=None):
+        M = X.shape[0]
+        xq, sfa, s_x, Z, Y = self.buffers(M, X.device)
+        if out is not None:
+            Y = out
+        svdq_quantize_act_nvfp4(self.w, X, xq, sfa, s_x, Z)
+        svdq_linear_nvfp4(self.w, xq, sfa, s_x, Z, Y, self.epilogue)
         return Y
 
     __call__ = forward

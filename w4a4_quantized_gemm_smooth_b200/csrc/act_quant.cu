@@ -32,6 +32,15 @@
 // shared memory (one named barrier among them) into s = fl32(m / 127); the
 // second sweep (X only, which the first sweep has just brought into L2)
 // quantises and stores 16 contiguous int8 codes per lane and token.
+//
+// The NVFP4 variant (review section 8: groups of 16 with FP8 scales) takes
+// the same two sweeps with s = fl32(m / 2688) per token; in the second, each
+// 16-column block's absmax (the four lanes of a quad, four values each) gives
+// the E4M3 group scale b, and each E2M1 code is decided by seven exact
+// comparisons |x| <> mid_j b s (one fma each, exact sign), ties to the even
+// code.  Codes are packed as the INT4 codes are; the four group scales of a
+// token and 64-column group form one 32-bit word of the tensor-core scale
+// atom.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -162,6 +171,40 @@ __device__ __forceinline__ void quad_transpose_words(const uint32_t (&w)[4], int
   }
 }
 
+// FP8 E4M3 value of a non-negative fp32 t (nearest, ties to even, saturating
+// at 448) and its bit pattern.
+__device__ __forceinline__ float e4m3_round(float t) {
+  if (!(t > 0.0f)) return 0.0f;
+  if (t >= 448.0f) return 448.0f;
+  const int ex = (int)((__float_as_uint(t) >> 23) & 0xFF) - 127;   // floor(log2 t) for a normal t
+  const int qexp = ex - 3 > -9 ? ex - 3 : -9;
+  const float v = ldexpf(rintf(ldexpf(t, -qexp)), qexp);            // power-of-two scalings: exact
+  return v < 448.0f ? v : 448.0f;
+}
+__device__ __forceinline__ uint32_t e4m3_byte(float v) {
+  if (!(v > 0.0f)) return 0u;
+  if (v < 0x1p-6f) return (uint32_t)rintf(v * 512.0f);
+  const uint32_t u = __float_as_uint(v);
+  return ((((u >> 23) & 0xFF) - 120u) << 3) | ((u >> 20) & 7u);
+}
+
+// E2M1 code of the exact quotient x / (b s): bd_j = mid_j b (exact in fp32),
+// the sign of fma(bd_j, s, -|x|) is that of mid_j b s - |x| (exact).
+__device__ __forceinline__ uint32_t e2m1_code(float x, float b, float s) {
+  const float a = fabsf(x);
+  const float mids[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+  int idx = 0;
+  bool tie = false;
+#pragma unroll
+  for (int j = 0; j < 7; ++j) {
+    const float c = __fmaf_rn(mids[j] * b, s, -a);
+    idx += c < 0.0f ? 1 : 0;
+    tie = (c == 0.0f && idx == j) ? true : tie;
+  }
+  if (tie && (idx & 1)) ++idx;
+  return (uint32_t)idx | ((x < 0.0f && idx > 0) ? 8u : 0u);
+}
+
 // 4 x 4 byte transpose across the lanes of a quad: lane q holds bytes
 // b[q][0..3] (byte j destined for lane j) and returns b[0..3][q].
 __device__ __forceinline__ uint32_t quad_transpose(uint32_t x, int q) {
@@ -172,14 +215,17 @@ __device__ __forceinline__ uint32_t quad_transpose(uint32_t x, int q) {
 }
 
 
-template <int NT, bool W8>
+// FMT: 0 W4A4 groups of 64; 1 W8A8 comparator; 2 NVFP4 variant.
+template <int NT, int FMT>
 __global__ void __launch_bounds__(AqStage<NT>::THREADS, 1)
 act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_l,   // L1^T [NT*8][K] bf16
                  const float* __restrict__ inv_lambda,
                  int M, int K, int rank,
                  uint8_t* __restrict__ xq, float* __restrict__ s_x,
-                 uint16_t* __restrict__ Z, int* __restrict__ err) {
+                 uint16_t* __restrict__ Z, uint8_t* __restrict__ sfa,
+                 int* __restrict__ err) {
+  constexpr bool W8 = FMT != 0;                // two sweeps, one scale per token
   using ST = AqStage<NT>;
   constexpr int S = ST::STAGES;
   constexpr int AQ_GPS = ST::GPS, AQ_WARPS = ST::WARPS, AQ_THREADS = ST::THREADS;
@@ -294,6 +340,41 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
             for (int ri = 0; ri < 2; ++ri)
 #pragma unroll
               for (int j = 0; j < 16; ++j) rmax[ri] = fmaxf(rmax[ri], fabsf(v[ri][j]));
+          } else if constexpr (FMT == 2) {
+#pragma unroll
+            for (int ri = 0; ri < 2; ++ri) {
+              // group scales of the four 16-column blocks (same in all four lanes)
+              float bs[4];
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                float mg = fmaxf(fmaxf(fabsf(v[ri][4 * ks]), fabsf(v[ri][4 * ks + 1])),
+                                 fmaxf(fabsf(v[ri][4 * ks + 2]), fabsf(v[ri][4 * ks + 3])));
+                mg = fmaxf(mg, __shfl_xor_sync(0xFFFFFFFFu, mg, 1));
+                mg = fmaxf(mg, __shfl_xor_sync(0xFFFFFFFFu, mg, 2));
+                bs[ks] = wss[ri] > 0.0f ? e4m3_round(__fdiv_rn(mg, wss[ri])) : 0.0f;
+              }
+              uint32_t by[8];
+#pragma unroll
+              for (int j = 0; j < 16; j += 2) {
+                const float bb = bs[j >> 2];
+                const uint32_t c0 = bb > 0.0f ? e2m1_code(v[ri][j] * wscale[ri], bb, wsc[ri]) : 0u;
+                const uint32_t c1 = bb > 0.0f ? e2m1_code(v[ri][j + 1] * wscale[ri], bb, wsc[ri]) : 0u;
+                by[j >> 1] = c0 | (c1 << 4);
+              }
+              uint32_t u[2];
+              u[0] = __byte_perm(__byte_perm(by[0], by[2], 0x0040), __byte_perm(by[4], by[6], 0x0040), 0x5410);
+              u[1] = __byte_perm(__byte_perm(by[1], by[3], 0x0040), __byte_perm(by[5], by[7], 0x0040), 0x5410);
+              const uint32_t w0 = quad_transpose(u[0], q), w1 = quad_transpose(u[1], q);
+              const int rl = rb * 16 + g8 + 8 * ri, row = row0 + rl;
+              if (row < M)
+                *reinterpret_cast<uint2*>(xq + (size_t)row * (K / 2) + grp * 32 + 8 * q) = make_uint2(w0, w1);
+              if (q == 0) {
+                const uint32_t word = e4m3_byte(bs[0]) | (e4m3_byte(bs[1]) << 8) |
+                                      (e4m3_byte(bs[2]) << 16) | (e4m3_byte(bs[3]) << 24);
+                const int a = row >> 7, r = row & 127;
+                *reinterpret_cast<uint32_t*>(sfa + ((size_t)a * G + grp) * 512 + 16 * (r & 31) + 4 * (r >> 5)) = word;
+              }
+            }
           } else {
 #pragma unroll
             for (int ri = 0; ri < 2; ++ri) {
@@ -441,12 +522,23 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
         float m = 0.0f;
 #pragma unroll
         for (int j = 0; j < AQ_GPS; ++j) m = fmaxf(m, rowmax_sh[j][rl]);
-        wsc[ri] = __fdiv_rn(m, 127.0f);
-        wtiny[ri] = wsc[ri] < 0x1p-64f;
-        wscale[ri] = wtiny[ri] ? 0x1p64f : 1.0f;
-        wss[ri] = __fmul_rn(wsc[ri], wscale[ri]);
-        wrcp[ri] = wsc[ri] > 0.0f ? __frcp_rn(wss[ri]) : 0.0f;
-        if (gi == 0 && q == 0 && row0 + rl < M) s_x[row0 + rl] = wsc[ri];
+        if constexpr (FMT == 2) {
+          // s = fl32(m / 2688); wss = fl32(6 s); the codes are decided on
+          // x 2^64 against s 2^64 when s is tiny (exact power-of-two scaling)
+          const float sr = __fdiv_rn(m, 2688.0f);
+          wss[ri] = __fmul_rn(6.0f, sr);
+          wtiny[ri] = sr < 0x1p-64f;
+          wscale[ri] = wtiny[ri] ? 0x1p64f : 1.0f;
+          wsc[ri] = __fmul_rn(sr, wscale[ri]);
+          if (gi == 0 && q == 0 && row0 + rl < M) s_x[row0 + rl] = sr;
+        } else {
+          wsc[ri] = __fdiv_rn(m, 127.0f);
+          wtiny[ri] = wsc[ri] < 0x1p-64f;
+          wscale[ri] = wtiny[ri] ? 0x1p64f : 1.0f;
+          wss[ri] = __fmul_rn(wsc[ri], wscale[ri]);
+          wrcp[ri] = wsc[ri] > 0.0f ? __frcp_rn(wss[ri]) : 0.0f;
+          if (gi == 0 && q == 0 && row0 + rl < M) s_x[row0 + rl] = wsc[ri];
+        }
       }
       for (int c = nstages; c < 2 * nstages && alive; ++c) alive = stage(c, c - nstages, true);
     }
@@ -508,14 +600,14 @@ bool aq_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NT, bool W8>
+template <int NT, int FMT>
 cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
-                      uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
+                      uint8_t* xq, float* s_x, uint16_t* Z, uint8_t* sfa, cudaStream_t st) {
   using ST = AqStage<NT>;
   const size_t dyn = (size_t)ST::STAGES * ST::BYTES + 1024;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<NT, W8>,
+    cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<NT, FMT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess) return e;
     attr = true;
@@ -526,25 +618,27 @@ cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
   tl = tx;
   if (NT > 0 && !aq_map(&tl, w->d_L1T, (uint64_t)w->K, (uint64_t)NT * 8, (uint64_t)w->K * 2, NT * 8))
     return cudaErrorInvalidValue;
-  const dim3 grid((M + AQ_ROWS - 1) / AQ_ROWS);
-  act_quant_kernel<NT, W8><<<grid, ST::THREADS, dyn, st>>>(tx, tl, w->d_inv_lambda, M, w->K, w->rank,
-                                                      xq, s_x, Z, w->d_err);
+  // NVFP4: cover whole 128-row blocks, so that every scale-atom row is written
+  const int rows = FMT == 2 ? (M + 127) / 128 * 128 : M;
+  const dim3 grid((rows + AQ_ROWS - 1) / AQ_ROWS);
+  act_quant_kernel<NT, FMT><<<grid, ST::THREADS, dyn, st>>>(tx, tl, w->d_inv_lambda, M, w->K,
+                                                           w->rank, xq, s_x, Z, sfa, w->d_err);
   return cudaGetLastError();
 }
 
-template <bool W8>
+template <int FMT>
 cudaError_t launch_act(const svdq_weights* w, int M, const uint16_t* X, int ldx, uint8_t* xq,
-                       float* s_x, uint16_t* Z, cudaStream_t st) {
+                       float* s_x, uint16_t* Z, uint8_t* sfa, cudaStream_t st) {
   switch (w->rank_pad / 8) {
-    case 0: return launch_aq<0, W8>(w, M, X, ldx, xq, s_x, Z, st);
-    case 2: return launch_aq<2, W8>(w, M, X, ldx, xq, s_x, Z, st);
-    case 4: return launch_aq<4, W8>(w, M, X, ldx, xq, s_x, Z, st);
-    case 6: return launch_aq<6, W8>(w, M, X, ldx, xq, s_x, Z, st);
-    case 8: return launch_aq<8, W8>(w, M, X, ldx, xq, s_x, Z, st);
-    case 10: return launch_aq<10, W8>(w, M, X, ldx, xq, s_x, Z, st);
-    case 12: return launch_aq<12, W8>(w, M, X, ldx, xq, s_x, Z, st);
-    case 14: return launch_aq<14, W8>(w, M, X, ldx, xq, s_x, Z, st);
-    case 16: return launch_aq<16, W8>(w, M, X, ldx, xq, s_x, Z, st);
+    case 0: return launch_aq<0, FMT>(w, M, X, ldx, xq, s_x, Z, sfa, st);
+    case 2: return launch_aq<2, FMT>(w, M, X, ldx, xq, s_x, Z, sfa, st);
+    case 4: return launch_aq<4, FMT>(w, M, X, ldx, xq, s_x, Z, sfa, st);
+    case 6: return launch_aq<6, FMT>(w, M, X, ldx, xq, s_x, Z, sfa, st);
+    case 8: return launch_aq<8, FMT>(w, M, X, ldx, xq, s_x, Z, sfa, st);
+    case 10: return launch_aq<10, FMT>(w, M, X, ldx, xq, s_x, Z, sfa, st);
+    case 12: return launch_aq<12, FMT>(w, M, X, ldx, xq, s_x, Z, sfa, st);
+    case 14: return launch_aq<14, FMT>(w, M, X, ldx, xq, s_x, Z, sfa, st);
+    case 16: return launch_aq<16, FMT>(w, M, X, ldx, xq, s_x, Z, sfa, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -553,12 +647,18 @@ cudaError_t launch_act(const svdq_weights* w, int M, const uint16_t* X, int ldx,
 
 cudaError_t launch_act_quant(const svdq_weights* w, int M, const uint16_t* X, int ldx,
                              uint8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
-  return launch_act<false>(w, M, X, ldx, xq, s_x, Z, st);
+  return launch_act<0>(w, M, X, ldx, xq, s_x, Z, nullptr, st);
 }
 
 cudaError_t launch_act_quant_w8a8(const svdq_weights* w, int M, const uint16_t* X, int ldx,
                                   int8_t* xq, float* s_x, uint16_t* Z, cudaStream_t st) {
-  return launch_act<true>(w, M, X, ldx, reinterpret_cast<uint8_t*>(xq), s_x, Z, st);
+  return launch_act<1>(w, M, X, ldx, reinterpret_cast<uint8_t*>(xq), s_x, Z, nullptr, st);
+}
+
+cudaError_t launch_act_quant_nvfp4(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                                   uint8_t* xq, uint8_t* sfa, float* s_x, uint16_t* Z,
+                                   cudaStream_t st) {
+  return launch_act<2>(w, M, X, ldx, xq, s_x, Z, sfa, st);
 }
 
 }  // namespace svdq

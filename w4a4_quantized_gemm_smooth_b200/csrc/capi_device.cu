@@ -24,6 +24,15 @@ svdq_status check_handle_w8a8(const svdq_weights* w) {
   return SVDQ_OK;
 }
 
+// A handle of the NVFP4 variant, uploaded to the current device.
+svdq_status check_handle_nvfp4(const svdq_weights* w) {
+  if (!w || w->format != SVDQ_FORMAT_NVFP4 || !w->d_wq4 || !w->d_err) return SVDQ_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
+  return SVDQ_OK;
+}
+
 svdq_status from_launch(cudaError_t e) { return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA; }
 
 }  // namespace
@@ -134,6 +143,35 @@ svdq_status svdq_linear_w8a8(const svdq_weights* w, int M, const int8_t* xq, con
       (w->rank > 0 && !aligned16(Z)))
     return SVDQ_ERR_ALIGNMENT;
   return from_launch(svdq::launch_linear_w8a8(w, M, xq, s_x, Z, Y, ldy, epilogue, stream));
+}
+
+svdq_status svdq_quantize_act_nvfp4(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                                    uint8_t* xq, uint8_t* sfa, float* s_x, uint16_t* Z,
+                                    cudaStream_t stream) {
+  svdq_status s = check_handle_nvfp4(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || ldx < w->K) return SVDQ_ERR_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !xq || !sfa || !s_x || (w->rank > 0 && !Z)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(xq) || !aligned16(sfa) || !aligned16(s_x) || (ldx % 8) != 0 ||
+      (w->rank > 0 && !aligned16(Z)))
+    return SVDQ_ERR_ALIGNMENT;
+  return from_launch(svdq::launch_act_quant_nvfp4(w, M, X, ldx, xq, sfa, s_x, Z, stream));
+}
+
+svdq_status svdq_linear_nvfp4(const svdq_weights* w, int M, const uint8_t* xq, const uint8_t* sfa,
+                              const float* s_x, const uint16_t* Z, uint16_t* Y, int ldy,
+                              int epilogue, cudaStream_t stream) {
+  svdq_status s = check_handle_nvfp4(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || ldy < w->N) return SVDQ_ERR_SHAPE;
+  if (epilogue != SVDQ_EPI_NONE && epilogue != SVDQ_EPI_GELU) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!xq || !sfa || !s_x || !Y || (w->rank > 0 && !Z)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(sfa) || !aligned16(s_x) || !aligned16(Y) || (ldy % 8) != 0 ||
+      (w->rank > 0 && !aligned16(Z)))
+    return SVDQ_ERR_ALIGNMENT;
+  return from_launch(svdq::launch_linear_nvfp4(w, M, xq, sfa, s_x, Z, Y, ldy, epilogue, stream));
 }
 
 }  // extern "C"

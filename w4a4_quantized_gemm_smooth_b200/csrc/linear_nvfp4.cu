@@ -1,0 +1,361 @@
+// NVFP4 product (SVDQuant review section 8: NVFP4 uses groups of 16 with
+// FP8 scales; section 9.1), warp-specialised for sm_100a:
+//
+//   Y = bf16(epi(s_x[m] s_w[n] sum_k (q_x b_x)(q_w b_w) + Z L2 + b))
+//
+// The tensor cores apply the E4M3 group scales themselves
+// (tcgen05.mma.kind::mxf4nvf4.block_scale, 16-element blocks): the packed
+// E2M1 codes go from TMA straight into the operand tiles, the group scales
+// are copied from shared memory into TMEM with tcgen05.cp, and the fp32 sum
+// over all of K stays in one TMEM accumulator.  The low-rank product Z L2
+// runs on the tensor cores (kind::f16, bf16 operands) into a separate TMEM
+// buffer; the epilogue computes s_x s_w acc + Z L2 + b (and GELU) per output
+// and stores Y by TMA.
+//
+// Persistent CTAs (one per SM), 128 x 128 tiles, static round-robin; 8 warps:
+//   warp 0    TMA producer: 128-K stages of A and B (one 64-byte-swizzled
+//             box each: 128 rows x 64 B) and the two 512-byte group-scale
+//             atoms of A and of B (bulk copies); low-rank slices at tile end;
+//   warp 1    TMEM owner and MMA issuer: per stage two tcgen05.cp of each
+//             operand's atoms into TMEM and two block-scaled MMAs (K = 64);
+//   warps 2-3 idle;
+//   warps 4-7 epilogue: warp w owns TMEM lanes 32 (w % 4)..; two 128-column
+//             accumulator buffers let tile t+1 accumulate while tile t is
+//             drained (the low-rank buffer is single: its stage comes at the
+//             end of a tile, after the previous tile's epilogue has read it).
+// TMEM: accumulators [0, 256), low-rank [256, 384), A scales [384, 392),
+// B scales [392, 400).
+// Every wait is bounded (the handle's error word is raised on expiry).
+#include "gemm_common.cuh"
+
+namespace svdq {
+namespace {
+
+constexpr int F4_BM = 128, F4_BN = 128;
+constexpr int F4_THREADS = 256;
+constexpr int F4_EPI0 = 4;         // epilogue warps 4-7
+
+struct F4Args {
+  const float* s_x;
+  const float* s_w;
+  const uint16_t* bias;
+  const uint8_t* sfa;      // activation group scales, atom layout
+  const uint8_t* sfb;      // weight group scales, atom layout
+  int M, N, K;
+  int nkb;                 // K blocks of 64
+  int n_lr;                // 16-wide low-rank slices
+  int epilogue;
+  int tiles_n, num_tiles;
+  int* err;
+};
+
+struct F4Lay {
+  static constexpr int BM = F4_BM, BN = F4_BN;
+  static constexpr int ST_A = BM * 64, ST_B = BN * 64;       // 128 K of packed FP4
+  static constexpr int ST_SFA = 1024, ST_SFB = 1024;          // two 512-byte atoms each
+  static constexpr int STAGE = ST_A + ST_B + ST_SFA + ST_SFB;
+  static constexpr int NST = 8;
+  static constexpr int NLR = 2;
+  static constexpr int LR_SA = BM * 32, LR_SB = BN * 32, LR_SLOT = LR_SA + LR_SB;
+  static constexpr int Y_BOX = 32 * 64 * 2;                   // 32 rows x 64 bf16
+  static constexpr int Y_WARP = 2 * Y_BOX;                    // 128 columns
+  static constexpr int OFF_ST = 0;
+  static constexpr int OFF_LR = OFF_ST + NST * STAGE;
+  static constexpr int OFF_Y = OFF_LR + NLR * LR_SLOT;
+  static constexpr int OFF_BAR = OFF_Y + 4 * Y_WARP;
+  // st_full[NST], st_empty[NST], tm_full[2], tm_empty[2], lr_full[NLR], lr_empty[NLR],
+  // lrb_empty (low-rank TMEM buffer read by the epilogue)
+  static constexpr int N_BARS = 2 * NST + 4 + 2 * NLR + 1;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+  static_assert(ALLOC <= 227 * 1024, "shared memory");
+  static_assert(STAGE % 1024 == 0 && OFF_Y % 1024 == 0, "alignment");
+};
+
+constexpr uint32_t TM_LR = 256;                    // low-rank accumulator
+constexpr uint32_t TM_SFA = 384, TM_SFB = 392;     // TMEM columns of the group scales
+
+// Instruction descriptor of the block-scaled FP4 MMA: E2M1 A and B (K-major),
+// UE4M3 scales, fp32 D, M = 128, N = 128, K = 64, scale ids 0.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10)                 // A, B: E2M1
+         | ((uint32_t)(N >> 3) << 17)           // N / 8
+         | (0u << 23)                           // scale format UE4M3
+         | ((uint32_t)(M >> 4) << 24);          // M / 16
+}
+
+// K-major operand as 64-byte rows with the 64-byte swizzle (see linear_w8a8).
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;
+  return d;
+}
+
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+      "}\n" ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+      "r"(sfb_tmem));
+}
+
+// 32 rows x 128 bits from shared memory (a 512-byte scale atom, 16 bytes per
+// row) into TMEM, replicated to the four lane quarters.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint32_t satom) {
+  const uint64_t d = sdesc_kmajor_noswizzle(satom, 128, 128);
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d));
+}
+
+__global__ void __launch_bounds__(F4_THREADS, 1)
+linear_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ CUtensorMap tm_y,
+                    const __grid_constant__ CUtensorMap tm_z,
+                    const __grid_constant__ CUtensorMap tm_l2, const F4Args p) {
+  using L = F4Lay;
+  constexpr int BM = L::BM, BN = L::BN, NST = L::NST, NLR = L::NLR;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::OFF_BAR;
+  auto st_full = [&](int s) { return bar0 + 8u * s; };
+  auto st_empty = [&](int s) { return bar0 + 8u * (NST + s); };
+  auto tm_full = [&](int b) { return bar0 + 8u * (2 * NST + b); };
+  auto tm_empty = [&](int b) { return bar0 + 8u * (2 * NST + 2 + b); };
+  auto lr_full = [&](int s) { return bar0 + 8u * (2 * NST + 4 + s); };
+  auto lr_empty = [&](int s) { return bar0 + 8u * (2 * NST + 4 + NLR + s); };
+  const uint32_t lrb_empty = bar0 + 8u * (2 * NST + 4 + 2 * NLR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nst = (p.nkb + 1) / 2;            // 128-K stages per tile
+
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) { mbar_init(st_full(s), 1); mbar_init(st_empty(s), 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(tm_full(b), 1); mbar_init(tm_empty(b), 4); }
+    for (int s = 0; s < NLR; ++s) { mbar_init(lr_full(s), 1); mbar_init(lr_empty(s), 1); }
+    mbar_init(lrb_empty, 4);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      uint32_t it = 0, il = 0;
+      bool alive = true;
+      for (int t = blockIdx.x; t < p.num_tiles && alive; t += gridDim.x) {
+        const int mb = t / p.tiles_n, nb = t % p.tiles_n;
+        const int m0 = mb * BM, n0 = nb * BN;
+        for (int s = 0; s < nst; ++s, ++it) {
+          const int st = it % NST;
+          if (!wait_or_abort(st_empty(st), ((it / NST) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
+          const int kb0 = 2 * s, nk = p.nkb - kb0 < 2 ? 1 : 2;
+          mbar_arrive_expect_tx(st_full(st), L::ST_A + L::ST_B + nk * 1024);
+          const uint32_t dst = sbase + L::OFF_ST + st * L::STAGE;
+          tma_load_2d(dst, &tm_a, s * 64, m0, st_full(st));
+          tma_load_2d(dst + L::ST_A, &tm_b, s * 64, n0, st_full(st));
+          bulk_load(dst + L::ST_A + L::ST_B, p.sfa + ((size_t)mb * p.nkb + kb0) * 512, nk * 512,
+                    st_full(st));
+          bulk_load(dst + L::ST_A + L::ST_B + L::ST_SFA, p.sfb + ((size_t)(n0 / 128) * p.nkb + kb0) * 512,
+                    nk * 512, st_full(st));
+        }
+        for (int j = 0; j < p.n_lr && alive; ++j, ++il) {
+          const int ls = il % NLR;
+          if (!wait_or_abort(lr_empty(ls), ((il / NLR) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
+          mbar_arrive_expect_tx(lr_full(ls), L::LR_SLOT);
+          const uint32_t dst = sbase + L::OFF_LR + ls * L::LR_SLOT;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            tma_load_2d(dst + c * (BM * 16), &tm_z, 16 * j + 8 * c, m0, lr_full(ls));
+            tma_load_2d(dst + L::LR_SA + c * (BN * 16), &tm_l2, 16 * j + 8 * c, n0, lr_full(ls));
+          }
+        }
+      }
+      for (uint32_t k = (it > NST ? it - NST : 0); k < it; ++k)
+        mbar_wait_bounded(st_full(k % NST), (k / NST) & 1, LIMIT_NS);
+      for (uint32_t k = (il > NLR ? il - NLR : 0); k < il; ++k)
+        mbar_wait_bounded(lr_full(k % NLR), (k / NLR) & 1, LIMIT_NS);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------- MMA issuer
+      const uint32_t id_f4 = idesc_nvf4(BM, BN), id_bf = idesc_bf16(BM, BN);
+      uint32_t it = 0, tb = 0, il = 0;
+      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tb) {
+        const int b = tb & 1;
+        if (!wait_or_abort(tm_empty(b), ((tb >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+        const uint32_t d = tmem + b * BN;
+        bool ok = true;
+        for (int s = 0; s < nst; ++s, ++it) {
+          const int st = it % NST;
+          if (!wait_or_abort(st_full(st), (it / NST) & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = sbase + L::OFF_ST + st * L::STAGE;
+          const uint32_t sb = sa + L::ST_A, ssfa = sb + L::ST_B, ssfb = ssfa + L::ST_SFA;
+          const int nk = p.nkb - 2 * s < 2 ? 1 : 2;
+          for (int h = 0; h < nk; ++h) {
+            // this K block's scales: 4 TMEM columns per operand
+            tmem_cp_sf(tmem + TM_SFA + 4 * h, ssfa + 512 * h);
+            tmem_cp_sf(tmem + TM_SFB + 4 * h, ssfb + 512 * h);
+          }
+          for (int h = 0; h < nk; ++h)
+            mma_nvf4(d, sdesc_sw64(sa + 32 * h), sdesc_sw64(sb + 32 * h), id_f4,
+                     tmem + TM_SFA + 4 * h, tmem + TM_SFB + 4 * h, (s > 0 || h > 0) ? 1u : 0u);
+          mma_commit(st_empty(st));
+        }
+        if (!ok) break;
+        // the low-rank buffer: free once the previous tile's epilogue read it
+        if (p.n_lr > 0 && !wait_or_abort(lrb_empty, (tb & 1) ^ 1, abort_flag, p.err)) break;
+        for (int j = 0; j < p.n_lr; ++j, ++il) {
+          const int ls = il % NLR;
+          if (!wait_or_abort(lr_full(ls), (il / NLR) & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t la = sbase + L::OFF_LR + ls * L::LR_SLOT;
+          mma_bf16(tmem + TM_LR, sdesc_kmajor_noswizzle(la, BM * 16, 128),
+                   sdesc_kmajor_noswizzle(la + L::LR_SA, BN * 16, 128), id_bf, j > 0 ? 1u : 0u);
+          mma_commit(lr_empty(ls));
+        }
+        if (!ok) break;
+        mma_commit(tm_full(b));
+      }
+    }
+    __syncwarp();
+  } else if (warp >= F4_EPI0) {
+    // ------------------------------------------------------ epilogue
+    // thread = one row of the warp's quarter; 32-column TMEM loads
+    const int q = warp & 3;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    uint8_t* ystage = smem + L::OFF_Y + q * L::Y_WARP;
+    const bool gelu = p.epilogue == SVDQ_EPI_GELU;
+    uint32_t tb = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tb) {
+      const int m0 = (t / p.tiles_n) * BM, n0 = (t % p.tiles_n) * BN;
+      const int row = m0 + 32 * q + lane;
+      const float sx = row < p.M ? __ldg(p.s_x + row) : 0.0f;
+      const int b = tb & 1;
+      if (!wait_or_abort(tm_full(b), (tb >> 1) & 1, abort_flag, p.err)) break;
+      tc_fence_after();
+      if (lane == 0) tma_store_wait_read0();
+      __syncwarp();
+      const bool lr = p.n_lr > 0;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32], z[32];
+        tmem_ld32(tmem + b * BN + 32 * c + lane_off, r);
+        if (lr) tmem_ld32(tmem + TM_LR + 32 * c + lane_off, z);
+        tmem_wait_ld();
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const int n = n0 + 32 * c + j;
+          const float w0 = n < p.N ? __ldg(p.s_w + n) : 0.0f;
+          const float w1 = n + 1 < p.N ? __ldg(p.s_w + n + 1) : 0.0f;
+          float b0 = n < p.N ? __uint_as_float((uint32_t)__ldg(p.bias + n) << 16) : 0.0f;
+          float b1 = n + 1 < p.N ? __uint_as_float((uint32_t)__ldg(p.bias + n + 1) << 16) : 0.0f;
+          if (lr) {
+            b0 = __fadd_rn(__uint_as_float(z[j]), b0);
+            b1 = __fadd_rn(__uint_as_float(z[j + 1]), b1);
+          }
+          float2 v = make_float2(__fmaf_rn(__fmul_rn(sx, w0), __uint_as_float(r[j]), b0),
+                                 __fmaf_rn(__fmul_rn(sx, w1), __uint_as_float(r[j + 1]), b1));
+          if (gelu) v = make_float2(gelu_f(v.x), gelu_f(v.y));
+          packed[j >> 1] = bf16x2_bits(v);
+        }
+        // row `lane` of box c / 2: 64 bytes at 16-byte chunk (4 (c & 1) + u) ^ (lane & 7)
+        uint8_t* yb = ystage + (c >> 1) * L::Y_BOX + lane * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(yb + ((((c & 1) * 4 + u) ^ (lane & 7)) << 4)) =
+              make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(tm_empty(b));
+        if (lr) mbar_arrive(lrb_empty);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int box = 0; box < 2; ++box)
+          tma_store_2d(&tm_y, n0 + 64 * box, m0 + 32 * q, smem_u32(ystage + box * L::Y_BOX));
+        tma_store_commit();
+      }
+      __syncwarp();
+    }
+    if (lane == 0) tma_store_wait0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_linear_nvfp4(const svdq_weights* w, int M, const uint8_t* xq,
+                                const uint8_t* sfa, const float* s_x, const uint16_t* Z,
+                                uint16_t* Y, int ldy, int epilogue, cudaStream_t st) {
+  using L = F4Lay;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(linear_nvfp4_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap ta, tb, ty, tz, tl;
+  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 64, L::BM,
+                CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&tb, w->d_wq4, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 64, L::BN,
+                CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  tz = ta;
+  tl = ta;
+  if (w->rank > 0 &&
+      (!make_map(&tz, Z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank, M, (uint64_t)w->rank * 2, 8,
+                 L::BM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+       !make_map(&tl, w->d_L2T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank_pad32, w->N,
+                 (uint64_t)w->rank_pad32 * 2, 8, L::BN, CU_TENSOR_MAP_SWIZZLE_NONE)))
+    return cudaErrorInvalidValue;
+  F4Args a{};
+  a.s_x = s_x; a.s_w = w->d_sw4; a.bias = w->d_bias; a.sfa = sfa; a.sfb = w->d_sfb4;
+  a.M = M; a.N = w->N; a.K = w->K; a.nkb = w->K / 64;
+  a.n_lr = (w->rank + 15) / 16;
+  a.epilogue = epilogue;
+  a.tiles_n = (w->N + L::BN - 1) / L::BN;
+  a.num_tiles = ((M + L::BM - 1) / L::BM) * a.tiles_n;
+  a.err = w->d_err;
+  const int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
+  linear_nvfp4_kernel<<<grid, F4_THREADS, L::ALLOC, st>>>(ta, tb, ty, tz, tl, a);
+  return cudaGetLastError();
+}
+
+}  // namespace svdq

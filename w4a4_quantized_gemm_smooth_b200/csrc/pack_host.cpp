@@ -13,6 +13,9 @@
 //   s = fl32(max|fl32(R)| / 7), codes = rne of the exact quotient  (eq. 1)
 //   W8A8 comparator: s = fl32(max|fl32(R)| / 127) per output column over
 //   all K, codes rne of the exact quotient clamped to [-128, 127]
+//   NVFP4 variant: s = fl32(max|fl32(R)| / 2688) per output column,
+//   b = e4m3(fl32(max|group of 16| / fl32(6 s))), codes e2m1 of the exact
+//   quotient z / (b s), nearest with ties to even
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -103,6 +106,62 @@ float quantize_row_int8(const float* z, int n, long stride, int8_t* q) {
   return s;
 }
 
+// FP8 E4M3 rounding of a non-negative value: 4 significant bits, exponent
+// bias 7, subnormal quantum 2^-9, nearest with ties to even, saturating at
+// 448 (the largest finite value).
+double round_e4m3(double t) {
+  if (!(t > 0.0)) return 0.0;
+  int e = 0;
+  std::frexp(t, &e);                                  // t = f 2^e, 0.5 <= f < 1
+  const int qexp = e - 4 > -9 ? e - 4 : -9;
+  const double v = std::ldexp(std::nearbyint(std::ldexp(t, -qexp)), qexp);
+  return v < 448.0 ? v : 448.0;
+}
+
+uint8_t e4m3_bits(double v) {
+  if (!(v > 0.0)) return 0;
+  if (v < 0x1p-6) return (uint8_t)std::nearbyint(v * 512.0);   // subnormal: m 2^-9
+  int e = 0;
+  const double f = std::frexp(v, &e);
+  return (uint8_t)(((e - 1 + 7) << 3) | (int)std::nearbyint((2.0 * f - 1.0) * 8.0));
+}
+
+// FP4 E2M1 code of the exact quotient z / d (d > 0): index into
+// {0, .5, 1, 1.5, 2, 3, 4, 6} by exact comparisons with the midpoints times
+// d (each product has at most 31 significant bits), ties to the even index,
+// saturating at 6; bit 3 is the sign of a nonzero magnitude.
+uint8_t e2m1_code(double z, double d) {
+  static const double mids[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+  const double a = std::fabs(z);
+  int idx = 0;
+  while (idx < 7 && mids[idx] * d < a) ++idx;
+  if (idx < 7 && mids[idx] * d == a && (idx & 1)) ++idx;
+  return (uint8_t)(idx | ((z < 0.0 && idx > 0) ? 8 : 0));
+}
+
+// The NVFP4 rule on one row of K fp32 values (stride between elements):
+// packed codes (K/2 bytes, even k in the low nibble), E4M3 group scale bits
+// (K/16 bytes), and the row scale.
+float quantize_row_nvfp4(const float* z, int K, long stride, uint8_t* codes, uint8_t* sf) {
+  float m = 0.0f;
+  for (int i = 0; i < K; ++i) m = std::fmax(m, std::fabs(z[(long)i * stride]));
+  const float srow = m / 2688.0f;                      // IEEE fp32 division
+  const float d6 = 6.0f * srow;                        // IEEE fp32 product
+  for (int g = 0; g < K / 16; ++g) {
+    float mg = 0.0f;
+    for (int i = 0; i < 16; ++i) mg = std::fmax(mg, std::fabs(z[(long)(16 * g + i) * stride]));
+    const double b = d6 > 0.0f ? round_e4m3((double)(mg / d6)) : 0.0;
+    sf[g] = e4m3_bits(b);
+    const double d = b * (double)srow;                 // exact
+    for (int i = 0; i < 16; i += 2) {
+      const uint8_t c0 = d > 0.0 ? e2m1_code(z[(long)(16 * g + i) * stride], d) : 0;
+      const uint8_t c1 = d > 0.0 ? e2m1_code(z[(long)(16 * g + i + 1) * stride], d) : 0;
+      codes[8 * g + i / 2] = (uint8_t)(c0 | (c1 << 4));
+    }
+  }
+  return srow;
+}
+
 template <class T>
 svdq_status dev_alloc_copy(T** dst, const T* src, size_t n, cudaStream_t st) {
   if (n == 0) n = 1;
@@ -116,8 +175,10 @@ void free_device(svdq_weights* w) {
   cudaFree(w->d_inv_lambda); cudaFree(w->d_wq); cudaFree(w->d_sw);
   cudaFree(w->d_L1T); cudaFree(w->d_L2); cudaFree(w->d_L2T); cudaFree(w->d_bias);
   cudaFree(w->d_wq8); cudaFree(w->d_sw8);
+  cudaFree(w->d_wq4); cudaFree(w->d_sfb4); cudaFree(w->d_sw4);
   cudaFree(w->d_err);
   w->d_wq8 = nullptr; w->d_sw8 = nullptr;
+  w->d_wq4 = nullptr; w->d_sfb4 = nullptr; w->d_sw4 = nullptr;
   w->d_inv_lambda = nullptr; w->d_wq = nullptr; w->d_sw = nullptr; w->d_L1T = nullptr;
   w->d_L2 = nullptr; w->d_L2T = nullptr; w->d_bias = nullptr; w->d_err = nullptr;
 }
@@ -143,7 +204,17 @@ svdq_status upload(svdq_weights* w, cudaStream_t st) {
   svdq_status s;
   if ((s = dev_alloc_copy(&w->d_inv_lambda, w->inv_lambda.data(), (size_t)K, st))) return s;
   w->N16 = (N + 15) / 16 * 16;
-  if (w->format == SVDQ_FORMAT_W8A8) {
+  if (w->format == SVDQ_FORMAT_NVFP4) {
+    std::vector<float> swp((size_t)w->N_pad, 0.0f);
+    std::memcpy(swp.data(), w->sw4.data(), (size_t)N * 4);
+    std::vector<uint8_t> sfb(svdq::nvfp4_sf_bytes(N, K), 0);
+    for (int n = 0; n < N; ++n)
+      for (int g = 0; g < K / 16; ++g)
+        sfb[svdq::nvfp4_sf_offset(n, g, K)] = w->sf4[(size_t)n * (K / 16) + g];
+    if ((s = dev_alloc_copy(&w->d_wq4, w->wq4.data(), (size_t)N * K / 2, st))) return s;
+    if ((s = dev_alloc_copy(&w->d_sfb4, sfb.data(), sfb.size(), st))) return s;
+    if ((s = dev_alloc_copy(&w->d_sw4, swp.data(), swp.size(), st))) return s;
+  } else if (w->format == SVDQ_FORMAT_W8A8) {
     std::vector<float> sw8p((size_t)w->N_pad, 0.0f);
     std::memcpy(sw8p.data(), w->sw8.data(), (size_t)N * 4);
     if ((s = dev_alloc_copy(&w->d_wq8, w->wq8.data(), (size_t)N * K, st))) return s;
@@ -183,6 +254,9 @@ struct Candidate {
   std::vector<float> sw;           // residual scales [G][N]
   std::vector<int8_t> wq8;         // W8A8 comparator: codes [N][K]
   std::vector<float> sw8;          //                  scales [N]
+  std::vector<uint8_t> wq4;        // NVFP4: packed codes [N][K/2]
+  std::vector<uint8_t> sf4;        //        E4M3 group scales [N][K/16]
+  std::vector<float> sw4;          //        row scales [N]
 };
 
 // eqs. 3-4: lambda from the activation statistic and the weight's per-channel
@@ -280,6 +354,17 @@ void quantize_residual_w8(int K, int N, int rank, Candidate& c) {
 #pragma omp parallel for schedule(static)
   for (int n = 0; n < N; ++n)
     c.sw8[n] = quantize_row_int8(&R32[n], K, N, &c.wq8[(size_t)n * K]);
+}
+
+// The residual, then the NVFP4 rule per output column.
+void quantize_residual_nvfp4(int K, int N, int rank, Candidate& c) {
+  const std::vector<float> R32 = residual_f32(K, N, rank, c);
+  c.sw4.assign(N, 0.0f);
+  c.wq4.assign((size_t)N * K / 2, 0);
+  c.sf4.assign((size_t)N * K / 16, 0);
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; ++n)
+    c.sw4[n] = quantize_row_nvfp4(&R32[n], K, N, &c.wq4[(size_t)n * K / 2], &c.sf4[(size_t)n * K / 16]);
 }
 
 int8_t code_at(const std::vector<uint8_t>& wq, int K, int n, int k) {
@@ -393,7 +478,11 @@ svdq_status finish(int K, int N, int rank, Candidate& c, const uint16_t* bias, i
   w->sw = std::move(c.sw);
   w->wq8 = std::move(c.wq8);
   w->sw8 = std::move(c.sw8);
-  w->format = w->wq8.empty() ? SVDQ_FORMAT_W4A4 : SVDQ_FORMAT_W8A8;
+  w->wq4 = std::move(c.wq4);
+  w->sf4 = std::move(c.sf4);
+  w->sw4 = std::move(c.sw4);
+  w->format = !w->wq8.empty() ? SVDQ_FORMAT_W8A8
+                              : !w->wq4.empty() ? SVDQ_FORMAT_NVFP4 : SVDQ_FORMAT_W4A4;
   const int rt = w->rank;
   w->L1.assign((size_t)K * rt, 0);
   w->L2.assign((size_t)rt * N, 0);
@@ -553,6 +642,32 @@ svdq_status svdq_weights_export_w8a8(const svdq_weights* w, int8_t* wq8, float* 
 }
 
 int svdq_weights_format(const svdq_weights* w) { return w ? w->format : -1; }
+
+svdq_status svdq_pack_weights_nvfp4(int K, int N, int rank, const uint16_t* W,
+                                    const float* act_absmax, double alpha, const uint16_t* bias,
+                                    int to_device, cudaStream_t stream, svdq_weights** out) {
+  svdq_status s = check_pack_args(K, N, rank, SVDQ_GROUP, W, 0, nullptr, nullptr, 1.0f, out);
+  if (s != SVDQ_OK) return s;
+  if (!act_absmax || !(alpha > 0.0 && alpha < 1.0)) return SVDQ_ERR_INVALID_ARG;
+  Candidate c;
+  if ((s = smooth(K, N, W, act_absmax, alpha, c)) != SVDQ_OK) return s;
+  if ((s = fit_factors(c.Wt.data(), K, N, rank, c)) != SVDQ_OK) return s;
+  quantize_residual_nvfp4(K, N, rank, c);
+  return finish(K, N, rank, c, bias, 0, nullptr, nullptr, 1.0f, to_device != 0, stream, out);
+}
+
+svdq_status svdq_weights_export_nvfp4(const svdq_weights* w, uint8_t* codes, uint8_t* sf,
+                                      float* s_w) {
+  if (!w || w->format != SVDQ_FORMAT_NVFP4) return SVDQ_ERR_INVALID_ARG;
+  if (codes) std::memcpy(codes, w->wq4.data(), w->wq4.size());
+  if (sf) std::memcpy(sf, w->sf4.data(), w->sf4.size());
+  if (s_w) std::memcpy(s_w, w->sw4.data(), w->sw4.size() * 4);
+  return SVDQ_OK;
+}
+
+size_t svdq_nvfp4_sf_bytes(int rows, int K) {
+  return rows > 0 && K > 0 && K % 64 == 0 ? svdq::nvfp4_sf_bytes(rows, K) : 0;
+}
 
 svdq_status svdq_weights_info(const svdq_weights* w, int* K, int* N, int* rank,
                               int* svd_rank, int* lora_rank) {

@@ -31,6 +31,10 @@ struct svdq_weights {
   uint16_t* d_bias = nullptr;      // [N] bf16
   int8_t* d_wq8 = nullptr;         // W8A8: [N][K] int8 residual codes
   float* d_sw8 = nullptr;          // W8A8: [N_pad] per-output-channel scales, zero padded
+  uint8_t* d_wq4 = nullptr;        // NVFP4: [N][K/2] packed E2M1 codes
+  uint8_t* d_sfb4 = nullptr;       // NVFP4: group scales in the tensor-core atom layout
+                                   //   [N_pad/128][K/64][512 B] (svdq::nvfp4_sf_offset)
+  float* d_sw4 = nullptr;          // NVFP4: [N_pad] row scales, zero padded
   int* d_err = nullptr;            // sticky device error word
   // host copies (export / save)
   std::vector<float> inv_lambda;
@@ -38,6 +42,9 @@ struct svdq_weights {
   std::vector<float> sw;
   std::vector<int8_t> wq8;         // W8A8 codes [N][K]
   std::vector<float> sw8;          // W8A8 scales [N]
+  std::vector<uint8_t> wq4;        // NVFP4 codes [N][K/2]
+  std::vector<uint8_t> sf4;        // NVFP4 E4M3 group scales [N][K/16]
+  std::vector<float> sw4;          // NVFP4 row scales [N]
   std::vector<uint16_t> L1;        // [K][rank]
   std::vector<uint16_t> L2;        // [rank][N]
   std::vector<uint16_t> bias;      // [N]
@@ -53,6 +60,18 @@ constexpr float SVDQ_ACC_BIAS = 12582912.0f;
 enum { SVDQ_DEVERR_NONE = 0, SVDQ_DEVERR_TIMEOUT = 1 };
 
 namespace svdq {
+
+// NVFP4 group-scale atom layout shared by the pack, the activation pass and
+// the GEMM: the scales of rows [128 a, 128 a + 128) and K block kb (64
+// elements, four groups of 16) form a 512-byte atom; row r (within the
+// block) sits at byte 16 (r % 32) + 4 (r / 32), group j (within the K
+// block) at + j.  This is the layout tcgen05.cp 32x128b.warpx4 turns into
+// the tensor-core scale-factor layout in TMEM.
+inline size_t nvfp4_sf_offset(int row, int k16, int K) {
+  const int a = row >> 7, r = row & 127, kb = k16 >> 2;
+  return ((size_t)a * (K / 64) + kb) * 512 + 16 * (r & 31) + 4 * (r >> 5) + (k16 & 3);
+}
+inline size_t nvfp4_sf_bytes(int rows, int K) { return (size_t)((rows + 127) / 128) * (K / 64) * 512; }
 
 // Upload the host copies of `w` to the current device (allocates).
 svdq_status upload(svdq_weights* w, cudaStream_t stream);
@@ -84,6 +103,13 @@ cudaError_t launch_act_quant_w8a8(const svdq_weights* w, int M, const uint16_t* 
 cudaError_t launch_linear_w8a8(const svdq_weights* w, int M, const int8_t* xq, const float* s_x,
                                const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
                                cudaStream_t stream);
+// NVFP4 variant: activation pass and block-scaled product.
+cudaError_t launch_act_quant_nvfp4(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                                   uint8_t* xq, uint8_t* sfa, float* s_x, uint16_t* Z,
+                                   cudaStream_t stream);
+cudaError_t launch_linear_nvfp4(const svdq_weights* w, int M, const uint8_t* xq,
+                                const uint8_t* sfa, const float* s_x, const uint16_t* Z,
+                                uint16_t* Y, int ldy, int epilogue, cudaStream_t stream);
 cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq,
                             int row0, int nrows, int col0, int ncols,
                             int32_t* P, cudaStream_t stream);
