@@ -316,6 +316,40 @@ def _time_w8a8(S, spec, L, a, X, flush, stream, steps, int8_peak):
             "linear_tops": tops, "linear_frac_int8": tops / int8_peak}
 
 
+class _StepF4(_Step):
+    """The NVFP4 variant: quantize_act_nvfp4 then linear_nvfp4."""
+
+    def __init__(self, S, w, X, bufs, epi):
+        self.S, self.w, self.X, self.epi = S, w, X, epi
+        self.xq, self.sfa, self.s_x, self.Z, self.Y = bufs
+
+    def __call__(self, marks, stream):
+        S = self.S
+        marks[0].record(stream)
+        S.svdq_quantize_act_nvfp4(self.w, self.X, self.xq, self.sfa, self.s_x, self.Z, stream)
+        marks[1].record(stream)
+        S.svdq_linear_nvfp4(self.w, self.xq, self.sfa, self.s_x, self.Z, self.Y, self.epi, stream)
+        marks[2].record(stream)
+
+
+def _time_nvfp4(S, spec, L, a, X, flush, stream, steps, fp4_peak):
+    """The same workload through the NVFP4 variant (same rank): per-kernel
+    times and the GEMM's fraction of the FP4 peak."""
+    w4 = S.svdq_pack_weights_nvfp4(L.W, a, spec.rank, bias_bits=L.b)
+    lin = S.NVFP4Linear(w4)
+    step = _StepF4(S, w4, X, lin.buffers(spec.M), S.EPI_NONE)
+    _time_steps(step, 3, flush, stream)
+    t_act, t_lin = (v / steps for v in _time_steps(step, steps, flush, stream))
+    S.svdq_get_device_error(w4)
+    w4.free()
+    ops = 2.0 * spec.M * spec.N * spec.K
+    tops = ops / (t_lin * 1e-3) / 1e12
+    return {"rank": spec.rank, "ms_per_step": t_act + t_lin, "act_ms": t_act, "linear_ms": t_lin,
+            "layer_tops": ops / ((t_act + t_lin) * 1e-3) / 1e12, "linear_tflops": tops,
+            "linear_frac_fp4": tops / fp4_peak,
+            "peak_source": "measured bf16 burst x 4 (fp4/bf16 nominal ratio)"}
+
+
 def _time_e2e(S, w, Xh, Yh, Xd, bufs, epi, steps):
     """Public API end to end, as a serving loop: every step copies its X from
     pinned host memory to the device, runs svdq_quantize_act and svdq_linear,
@@ -455,6 +489,9 @@ def run_ours(args, spec):
     if not args.no_w8a8:
         line["w8a8_comparator"] = _time_w8a8(S, spec, L, a, X, flush, stream, args.steps,
                                              int8_peak)
+    if not args.no_nvfp4:
+        line["nvfp4_variant"] = _time_nvfp4(S, spec, L, a, X, flush, stream, args.steps,
+                                            4.0 * bf16_burst)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec)
     if rank == 0:
@@ -476,6 +513,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-w8a8", action="store_true",
                     help="skip the W8A8 comparator's timing")
+    ap.add_argument("--no-nvfp4", action="store_true",
+                    help="skip the NVFP4 variant's timing")
     args = ap.parse_args()
     spec = _workload(args.workload)
     if args.impl == "reference":

@@ -23,8 +23,11 @@
 //             accumulator buffers let tile t+1 accumulate while tile t is
 //             drained (the low-rank buffer is single: its stage comes at the
 //             end of a tile, after the previous tile's epilogue has read it).
-// TMEM: accumulators [0, 256), low-rank [256, 384), A scales [384, 392),
-// B scales [392, 400).
+// TMEM: accumulators [0, 256), low-rank [256, 384), and one 16-column slot
+// of group scales per shared-memory stage [384, 512) (A: 4 columns per K
+// block, B: 4 columns per K block), so the scale copies of a stage never wait
+// for the MMAs of an earlier one: a slot is refilled only after its stage's
+// MMAs have completed (the stage's empty barrier).
 // Every wait is bounded (the handle's error word is raised on expiry).
 #include "gemm_common.cuh"
 
@@ -54,7 +57,7 @@ struct F4Lay {
   static constexpr int ST_A = BM * 64, ST_B = BN * 64;       // 128 K of packed FP4
   static constexpr int ST_SFA = 1024, ST_SFB = 1024;          // two 512-byte atoms each
   static constexpr int STAGE = ST_A + ST_B + ST_SFA + ST_SFB;
-  static constexpr int NST = 8;
+  static constexpr int NST = 8;          // also the TMEM scale slots (8 x 16 columns)
   static constexpr int NLR = 2;
   static constexpr int LR_SA = BM * 32, LR_SB = BN * 32, LR_SLOT = LR_SA + LR_SB;
   static constexpr int Y_BOX = 32 * 64 * 2;                   // 32 rows x 64 bf16
@@ -73,8 +76,20 @@ struct F4Lay {
   static_assert(STAGE % 1024 == 0 && OFF_Y % 1024 == 0, "alignment");
 };
 
+// True in one lane of the (converged) calling warp: the issuing lane of
+// single-thread tcgen05 instructions in warp-uniform code.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 constexpr uint32_t TM_LR = 256;                    // low-rank accumulator
-constexpr uint32_t TM_SFA = 384, TM_SFB = 392;     // TMEM columns of the group scales
+constexpr uint32_t TM_SF = 384;                    // group-scale slots, 16 columns per stage
 
 // Instruction descriptor of the block-scaled FP4 MMA: E2M1 A and B (K-major),
 // UE4M3 scales, fp32 D, M = 128, N = 128, K = 64, scale ids 0.
@@ -197,49 +212,64 @@ linear_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------- MMA issuer
-      const uint32_t id_f4 = idesc_nvf4(BM, BN), id_bf = idesc_bf16(BM, BN);
-      uint32_t it = 0, tb = 0, il = 0;
-      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tb) {
-        const int b = tb & 1;
-        if (!wait_or_abort(tm_empty(b), ((tb >> 1) & 1) ^ 1, abort_flag, p.err)) break;
-        const uint32_t d = tmem + b * BN;
-        bool ok = true;
-        for (int s = 0; s < nst; ++s, ++it) {
-          const int st = it % NST;
-          if (!wait_or_abort(st_full(st), (it / NST) & 1, abort_flag, p.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sa = sbase + L::OFF_ST + st * L::STAGE;
-          const uint32_t sb = sa + L::ST_A, ssfa = sb + L::ST_B, ssfb = ssfa + L::ST_SFA;
-          const int nk = p.nkb - 2 * s < 2 ? 1 : 2;
+    // ------------------------------------------------------ MMA issuer
+    // The whole warp walks the loop with warp-uniform operands (lane 0
+    // waits, the result is broadcast); one elected lane issues the tcgen05
+    // instructions.  Issuing from a lane-0-only branch cost ~100 cycles per
+    // tcgen05 instruction, more than the MMAs themselves.
+    const uint32_t id_f4 = idesc_nvf4(BM, BN), id_bf = idesc_bf16(BM, BN);
+    const uint32_t tm = __shfl_sync(0xFFFFFFFFu, tmem, 0);
+    auto wait_warp = [&](uint32_t bar, uint32_t parity) -> bool {
+      int ok = 1;
+      if (lane == 0) ok = wait_or_abort(bar, parity, abort_flag, p.err) ? 1 : 0;
+      return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+    };
+    uint32_t it = 0, tb = 0, il = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tb) {
+      const int b = tb & 1;
+      if (!wait_warp(tm_empty(b), ((tb >> 1) & 1) ^ 1)) break;
+      const uint32_t d = tm + b * BN;
+      bool ok = true;
+      for (int s = 0; s < nst; ++s, ++it) {
+        const int st = it % NST;
+        if (!wait_warp(st_full(st), (it / NST) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = sbase + L::OFF_ST + st * L::STAGE;
+        const uint32_t sb = sa + L::ST_A, ssfa = sb + L::ST_B, ssfb = ssfa + L::ST_SFA;
+        const int nk = p.nkb - 2 * s < 2 ? 1 : 2;
+        const uint32_t sf = tm + TM_SF + 16 * st;   // A: +4h, B: +8+4h
+        if (elect_one()) {
           for (int h = 0; h < nk; ++h) {
             // this K block's scales: 4 TMEM columns per operand
-            tmem_cp_sf(tmem + TM_SFA + 4 * h, ssfa + 512 * h);
-            tmem_cp_sf(tmem + TM_SFB + 4 * h, ssfb + 512 * h);
+            tmem_cp_sf(sf + 4 * h, ssfa + 512 * h);
+            tmem_cp_sf(sf + 8 + 4 * h, ssfb + 512 * h);
           }
           for (int h = 0; h < nk; ++h)
             mma_nvf4(d, sdesc_sw64(sa + 32 * h), sdesc_sw64(sb + 32 * h), id_f4,
-                     tmem + TM_SFA + 4 * h, tmem + TM_SFB + 4 * h, (s > 0 || h > 0) ? 1u : 0u);
+                     sf + 4 * h, sf + 8 + 4 * h, (s > 0 || h > 0) ? 1u : 0u);
           mma_commit(st_empty(st));
         }
-        if (!ok) break;
-        // the low-rank buffer: free once the previous tile's epilogue read it
-        if (p.n_lr > 0 && !wait_or_abort(lrb_empty, (tb & 1) ^ 1, abort_flag, p.err)) break;
-        for (int j = 0; j < p.n_lr; ++j, ++il) {
-          const int ls = il % NLR;
-          if (!wait_or_abort(lr_full(ls), (il / NLR) & 1, abort_flag, p.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t la = sbase + L::OFF_LR + ls * L::LR_SLOT;
-          mma_bf16(tmem + TM_LR, sdesc_kmajor_noswizzle(la, BM * 16, 128),
+        __syncwarp();
+      }
+      if (!ok) break;
+      // the low-rank buffer: free once the previous tile's epilogue read it
+      if (p.n_lr > 0 && !wait_warp(lrb_empty, (tb & 1) ^ 1)) break;
+      for (int j = 0; j < p.n_lr; ++j, ++il) {
+        const int ls = il % NLR;
+        if (!wait_warp(lr_full(ls), (il / NLR) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t la = sbase + L::OFF_LR + ls * L::LR_SLOT;
+        if (elect_one()) {
+          mma_bf16(tm + TM_LR, sdesc_kmajor_noswizzle(la, BM * 16, 128),
                    sdesc_kmajor_noswizzle(la + L::LR_SA, BN * 16, 128), id_bf, j > 0 ? 1u : 0u);
           mma_commit(lr_empty(ls));
         }
-        if (!ok) break;
-        mma_commit(tm_full(b));
+        __syncwarp();
       }
+      if (!ok) break;
+      if (elect_one()) mma_commit(tm_full(b));
+      __syncwarp();
     }
-    __syncwarp();
   } else if (warp >= F4_EPI0) {
     // ------------------------------------------------------ epilogue
     // thread = one row of the warp's quarter; 32-column TMEM loads
