@@ -177,8 +177,11 @@ __device__ __forceinline__ float e4m3_round(float t) {
   if (!(t > 0.0f)) return 0.0f;
   if (t >= 448.0f) return 448.0f;
   const int ex = (int)((__float_as_uint(t) >> 23) & 0xFF) - 127;   // floor(log2 t) for a normal t
-  const int qexp = ex - 3 > -9 ? ex - 3 : -9;
-  const float v = ldexpf(rintf(ldexpf(t, -qexp)), qexp);            // power-of-two scalings: exact
+  const int qexp = ex - 3 > -9 ? ex - 3 : -9;                      // in [-9, 5]
+  // 2^-qexp and 2^qexp as floats (normal exponents): exact scalings
+  const float up = __uint_as_float((uint32_t)(127 - qexp) << 23);
+  const float dn = __uint_as_float((uint32_t)(127 + qexp) << 23);
+  const float v = rintf(t * up) * dn;
   return v < 448.0f ? v : 448.0f;
 }
 __device__ __forceinline__ uint32_t e4m3_byte(float v) {
@@ -203,6 +206,39 @@ __device__ __forceinline__ uint32_t e2m1_code(float x, float b, float s) {
   }
   if (tie && (idx & 1)) ++idx;
   return (uint32_t)idx | ((x < 0.0f && idx > 0) ? 8u : 0u);
+}
+
+// E2M1 code from u = |x| fl(1/fl(b s)), within 2^-22 (relative) of the exact
+// quotient: the grid is spaced 0.5 below 2, 1 below 4, then {4, 6}; `near`
+// is raised when u lies within 2^-18 of a midpoint (the exact path decides).
+__device__ __forceinline__ uint32_t e2m1_fast(float x, float r, bool& near) {
+  const float u = fabsf(x) * r;
+  uint32_t k;
+  if (u < 2.0f) {
+    const float t = 2.0f * u, rt = rintf(t);
+    k = (uint32_t)rt;
+    near |= fabsf(t - rt) > 0.5f - 0x1p-18f;
+  } else if (u < 4.0f) {
+    const float t = u - 2.0f, rt = rintf(t);
+    k = 4u + (uint32_t)rt;
+    near |= fabsf(t - rt) > 0.5f - 0x1p-18f;
+  } else {
+    k = u <= 5.0f ? 6u : 7u;
+    near |= fabsf(u - 5.0f) < 0x1p-17f;
+  }
+  return k | ((x < 0.0f && k > 0u) ? 8u : 0u);
+}
+
+// All 16 codes of a lane's token by the exact comparisons (rare).
+__device__ __noinline__ void e2m1_exact16(const float* v, const float* bs, float scale, float s,
+                                          uint32_t* by) {
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    const float bb = bs[j >> 2];
+    const uint32_t c0 = bb > 0.0f ? e2m1_code(v[j] * scale, bb, s) : 0u;
+    const uint32_t c1 = bb > 0.0f ? e2m1_code(v[j + 1] * scale, bb, s) : 0u;
+    by[j >> 1] = c0 | (c1 << 4);
+  }
 }
 
 // 4 x 4 byte transpose across the lanes of a quad: lane q holds bytes
@@ -354,12 +390,22 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
                 bs[ks] = wss[ri] > 0.0f ? e4m3_round(__fdiv_rn(mg, wss[ri])) : 0.0f;
               }
               uint32_t by[8];
+              bool near = wtiny[ri];           // tiny row scale: exact path only
+              if (!near) {
+                float rb[4];
 #pragma unroll
-              for (int j = 0; j < 16; j += 2) {
-                const float bb = bs[j >> 2];
-                const uint32_t c0 = bb > 0.0f ? e2m1_code(v[ri][j] * wscale[ri], bb, wsc[ri]) : 0u;
-                const uint32_t c1 = bb > 0.0f ? e2m1_code(v[ri][j + 1] * wscale[ri], bb, wsc[ri]) : 0u;
-                by[j >> 1] = c0 | (c1 << 4);
+                for (int ks = 0; ks < 4; ++ks)
+                  rb[ks] = bs[ks] > 0.0f ? __frcp_rn(__fmul_rn(bs[ks], wsc[ri])) : 0.0f;
+#pragma unroll
+                for (int j = 0; j < 16; j += 2)
+                  by[j >> 1] = e2m1_fast(v[ri][j], rb[j >> 2], near) |
+                               (e2m1_fast(v[ri][j + 1], rb[j >> 2], near) << 4);
+              }
+              if (near) {
+                float tmp[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) tmp[j] = v[ri][j];
+                e2m1_exact16(tmp, bs, wscale[ri], wsc[ri], by);
               }
               uint32_t u[2];
               u[0] = __byte_perm(__byte_perm(by[0], by[2], 0x0040), __byte_perm(by[4], by[6], 0x0040), 0x5410);
