@@ -45,8 +45,8 @@ LINEAR_SOURCES = ("w4a4_quantized_gemm_smooth_b200/csrc/linear_ws.cu",
                   "w4a4_quantized_gemm_smooth_b200/csrc/gemm_common.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/ptx.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/svdq_internal.h")
-LINEAR_TRAFFIC = {"sources_sha1": "4c18e40cd87dfbec7e35922f21fbf97dfcc7d13b",
-                  "workload": "flux_qkv", "bytes": 24867840 + 28838912}
+LINEAR_TRAFFIC = {"sources_sha1": "48a8524739dac299cf113651cbe1c1819047cab9",
+                  "workload": "flux_qkv", "bytes": 24867328 + 28369920}
 
 
 def _linear_traffic(workload):
