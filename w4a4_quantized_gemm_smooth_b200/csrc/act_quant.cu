@@ -34,13 +34,13 @@
 // quantises and stores 16 contiguous int8 codes per lane and token.
 //
 // The NVFP4 variant (review section 8: groups of 16 with FP8 scales) takes
-// the same two sweeps with s = fl32(m / 2688) per token; in the second, each
-// 16-column block's absmax (the four lanes of a quad, four values each) gives
-// the E4M3 group scale b, and each E2M1 code is decided by seven exact
-// comparisons |x| <> mid_j b s (one fma each, exact sign), ties to the even
-// code.  Codes are packed as the INT4 codes are; the four group scales of a
-// token and 64-column group form one 32-bit word of the tensor-core scale
-// atom.
+// the same two sweeps with s = fl32(m / 2688) per token.  The second sweep
+// needs no Z, so it leaves the fragment layout: each lane reads 32
+// contiguous columns of one token from the swizzled tile, takes the two
+// 16-column group maxima in-thread (E4M3 group scale b), decides each E2M1
+// code from one reciprocal per group (exact comparisons |x| <> mid_j b s,
+// one fma each, only near a midpoint), and writes its 32 codes with one
+// 16-byte store and its two group scales into the tensor-core scale atom.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -229,16 +229,61 @@ __device__ __forceinline__ uint32_t e2m1_fast(float x, float r, bool& near) {
   return k | ((x < 0.0f && k > 0u) ? 8u : 0u);
 }
 
-// All 16 codes of a lane's token by the exact comparisons (rare).
-__device__ __noinline__ void e2m1_exact16(const float* v, const float* bs, float scale, float s,
-                                          uint32_t* by) {
+// NVFP4 second sweep, one lane = 32 contiguous columns (two groups of 16) of
+// one token, read straight from the 128-byte-swizzled X tile: group maxima
+// in-thread, codes packed in column order (one 16-byte store), the two group
+// scales as one 16-bit store into the scale atom.
+// rs: token scale (x 2^64 when tiny); d6 = fl32(6 s); sc = 2^64 or 1.
+__device__ __forceinline__ void nvfp4_row32(uint32_t xrow, int rl, int hh, uint32_t ilt, float rs,
+                                            float d6, float sc, bool tiny, uint8_t* xq_dst,
+                                            uint8_t* sf_dst) {
+  float v[32];
 #pragma unroll
-  for (int j = 0; j < 16; j += 2) {
-    const float bb = bs[j >> 2];
-    const uint32_t c0 = bb > 0.0f ? e2m1_code(v[j] * scale, bb, s) : 0u;
-    const uint32_t c1 = bb > 0.0f ? e2m1_code(v[j + 1] * scale, bb, s) : 0u;
-    by[j >> 1] = c0 | (c1 << 4);
+  for (int i = 0; i < 4; ++i) {
+    const uint4 raw = lds128u(xrow + (((4 * hh + i) ^ (rl & 7)) << 4));
+    const float4 i0 = lds128(ilt + 4 * (32 * hh + 8 * i));
+    const float4 i1 = lds128(ilt + 4 * (32 * hh + 8 * i + 4));
+    const float2 p0 = __fmul2_rn(make_float2(bf16lo(raw.x), bf16hi(raw.x)), make_float2(i0.x, i0.y));
+    const float2 p1 = __fmul2_rn(make_float2(bf16lo(raw.y), bf16hi(raw.y)), make_float2(i0.z, i0.w));
+    const float2 p2 = __fmul2_rn(make_float2(bf16lo(raw.z), bf16hi(raw.z)), make_float2(i1.x, i1.y));
+    const float2 p3 = __fmul2_rn(make_float2(bf16lo(raw.w), bf16hi(raw.w)), make_float2(i1.z, i1.w));
+    v[8 * i + 0] = p0.x; v[8 * i + 1] = p0.y; v[8 * i + 2] = p1.x; v[8 * i + 3] = p1.y;
+    v[8 * i + 4] = p2.x; v[8 * i + 5] = p2.y; v[8 * i + 6] = p3.x; v[8 * i + 7] = p3.y;
   }
+  float bs[2];
+#pragma unroll
+  for (int bk = 0; bk < 2; ++bk) {
+    float mg = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) mg = fmaxf(mg, fabsf(v[16 * bk + j]));
+    bs[bk] = d6 > 0.0f ? e4m3_round(__fdiv_rn(mg, d6)) : 0.0f;
+  }
+  uint32_t w[4];
+  bool near = tiny;
+  if (!near) {
+    const float r0 = bs[0] > 0.0f ? __frcp_rn(__fmul_rn(bs[0], rs)) : 0.0f;
+    const float r1 = bs[1] > 0.0f ? __frcp_rn(__fmul_rn(bs[1], rs)) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t x = 0u;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x |= e2m1_fast(v[8 * i + e], i < 2 ? r0 : r1, near) << (4 * e);
+      w[i] = x;
+    }
+  }
+  if (near) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t x = 0u;
+      const float bb = bs[i >> 1];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        x |= (bb > 0.0f ? e2m1_code(v[8 * i + e] * sc, bb, rs) : 0u) << (4 * e);
+      w[i] = x;
+    }
+  }
+  if (xq_dst) *reinterpret_cast<uint4*>(xq_dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint16_t*>(sf_dst) = (uint16_t)(e4m3_byte(bs[0]) | (e4m3_byte(bs[1]) << 8));
 }
 
 // 4 x 4 byte transpose across the lanes of a quad: lane q holds bytes
@@ -330,6 +375,10 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int rb = warp & 1, gi = warp >> 1, q = l & 3, g8 = l >> 2;
     float rmax[2] = {0.0f, 0.0f};     // W8: running absmax of the lane's two tokens
     float wsc[2] = {0.0f, 0.0f}, wss[2] = {0.0f, 0.0f}, wrcp[2] = {0.0f, 0.0f};
+    // NVFP4 second sweep: this lane's token rl4 = 16 rb + l / 2 and its scales
+    const int rl4 = rb * 16 + (l >> 1), hh4 = l & 1;
+    float f4s = 0.0f, f4d6 = 0.0f, f4sc = 1.0f;
+    bool f4tiny = false;
     float wscale[2] = {1.0f, 1.0f};
     bool wtiny[2] = {false, false};
     // One stage: the warp's 16 x 64 block of group AQ_GPS * cc + gi.
@@ -343,7 +392,13 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
       }
       if (*reinterpret_cast<volatile int*>(&abort_sh)) return false;
       const int grp = AQ_GPS * cc + gi;
-      if (grp < G) {
+      if (FMT == 2 && second && grp < G) {
+        const uint32_t st = ring + s * ST::BYTES;
+        const int row = row0 + rl4, a = row >> 7, r = row & 127;
+        nvfp4_row32(st + gi * AQ_XTILE + rl4 * 128, rl4, hh4, st + ST::OFF_IL + gi * 256, f4s, f4d6,
+                    f4sc, f4tiny, row < M ? xq + (size_t)row * (K / 2) + grp * 32 + 16 * hh4 : nullptr,
+                    sfa + ((size_t)a * G + grp) * 512 + 16 * (r & 31) + 4 * (r >> 5) + 2 * hh4);
+      } else if (grp < G) {
         const uint32_t st = ring + s * ST::BYTES;
         const uint32_t xt = st + gi * AQ_XTILE;
         // raw X in the A fragment layout: a[ks][0] row g8, cols 16ks+2q (+1);
@@ -376,51 +431,6 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
             for (int ri = 0; ri < 2; ++ri)
 #pragma unroll
               for (int j = 0; j < 16; ++j) rmax[ri] = fmaxf(rmax[ri], fabsf(v[ri][j]));
-          } else if constexpr (FMT == 2) {
-#pragma unroll
-            for (int ri = 0; ri < 2; ++ri) {
-              // group scales of the four 16-column blocks (same in all four lanes)
-              float bs[4];
-#pragma unroll
-              for (int ks = 0; ks < 4; ++ks) {
-                float mg = fmaxf(fmaxf(fabsf(v[ri][4 * ks]), fabsf(v[ri][4 * ks + 1])),
-                                 fmaxf(fabsf(v[ri][4 * ks + 2]), fabsf(v[ri][4 * ks + 3])));
-                mg = fmaxf(mg, __shfl_xor_sync(0xFFFFFFFFu, mg, 1));
-                mg = fmaxf(mg, __shfl_xor_sync(0xFFFFFFFFu, mg, 2));
-                bs[ks] = wss[ri] > 0.0f ? e4m3_round(__fdiv_rn(mg, wss[ri])) : 0.0f;
-              }
-              uint32_t by[8];
-              bool near = wtiny[ri];           // tiny row scale: exact path only
-              if (!near) {
-                float rb[4];
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                  rb[ks] = bs[ks] > 0.0f ? __frcp_rn(__fmul_rn(bs[ks], wsc[ri])) : 0.0f;
-#pragma unroll
-                for (int j = 0; j < 16; j += 2)
-                  by[j >> 1] = e2m1_fast(v[ri][j], rb[j >> 2], near) |
-                               (e2m1_fast(v[ri][j + 1], rb[j >> 2], near) << 4);
-              }
-              if (near) {
-                float tmp[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) tmp[j] = v[ri][j];
-                e2m1_exact16(tmp, bs, wscale[ri], wsc[ri], by);
-              }
-              uint32_t u[2];
-              u[0] = __byte_perm(__byte_perm(by[0], by[2], 0x0040), __byte_perm(by[4], by[6], 0x0040), 0x5410);
-              u[1] = __byte_perm(__byte_perm(by[1], by[3], 0x0040), __byte_perm(by[5], by[7], 0x0040), 0x5410);
-              const uint32_t w0 = quad_transpose(u[0], q), w1 = quad_transpose(u[1], q);
-              const int rl = rb * 16 + g8 + 8 * ri, row = row0 + rl;
-              if (row < M)
-                *reinterpret_cast<uint2*>(xq + (size_t)row * (K / 2) + grp * 32 + 8 * q) = make_uint2(w0, w1);
-              if (q == 0) {
-                const uint32_t word = e4m3_byte(bs[0]) | (e4m3_byte(bs[1]) << 8) |
-                                      (e4m3_byte(bs[2]) << 16) | (e4m3_byte(bs[3]) << 24);
-                const int a = row >> 7, r = row & 127;
-                *reinterpret_cast<uint32_t*>(sfa + ((size_t)a * G + grp) * 512 + 16 * (r & 31) + 4 * (r >> 5)) = word;
-              }
-            }
           } else {
 #pragma unroll
             for (int ri = 0; ri < 2; ++ri) {
@@ -577,6 +587,16 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
           wscale[ri] = wtiny[ri] ? 0x1p64f : 1.0f;
           wsc[ri] = __fmul_rn(sr, wscale[ri]);
           if (gi == 0 && q == 0 && row0 + rl < M) s_x[row0 + rl] = sr;
+          if (ri == 0) {                       // the row-contiguous sweep's token
+            float m4 = 0.0f;
+#pragma unroll
+            for (int j = 0; j < AQ_GPS; ++j) m4 = fmaxf(m4, rowmax_sh[j][rl4]);
+            const float s4 = __fdiv_rn(m4, 2688.0f);
+            f4d6 = __fmul_rn(6.0f, s4);
+            f4tiny = s4 < 0x1p-64f;
+            f4sc = f4tiny ? 0x1p64f : 1.0f;
+            f4s = __fmul_rn(s4, f4sc);
+          }
         } else {
           wsc[ri] = __fdiv_rn(m, 127.0f);
           wtiny[ri] = wsc[ri] < 0x1p-64f;
