@@ -3,13 +3,14 @@
 // and, from the same registers, compute the 16-bit down-projection
 // Z = bf16(x~) L1 on the tensor cores (mma.sync bf16, fp32 accumulation).
 //
-// Layout: a CTA owns 32 consecutive tokens and walks K in stages of four
-// groups (256 channels).  A producer warp streams each stage by TMA into a
-// shared-memory ring: the 32 x 64 bf16 tile of X of every group (128-byte
-// swizzled), the matching 64-column slice of L1^T (all branch rows, also
-// swizzled) and the 256 smoothing factors, all on one mbarrier.  Eight
-// compute warps each own one 16-token x 64-channel block of a stage (two
-// token halves x four groups), read it with ldmatrix in the mma.sync A
+// Layout: a CTA owns 32 consecutive tokens and walks K in stages of eight
+// groups (512 channels; four for branch ranks above 64).  A producer warp
+// streams each stage by TMA into a shared-memory ring: the 32 x 64 bf16 tile
+// of X of every group (128-byte swizzled), the matching 64-column slice of
+// L1^T (all branch rows, also swizzled) and the stage's smoothing factors,
+// all on one mbarrier.  Sixteen compute warps (eight for the largest ranks)
+// each own one 16-token x 64-channel block of a stage (two token halves x
+// the stage's groups), read it with ldmatrix in the mma.sync A
 // fragment layout and, without any CTA-wide barrier, smooth, quantise,
 // store codes and scales, and multiply the same fragments (as bf16) with
 // L1 fragments read by ldmatrix.  A warp releases the stage with an mbarrier
@@ -671,12 +672,14 @@ cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
                       uint8_t* xq, float* s_x, uint16_t* Z, uint8_t* sfa, cudaStream_t st) {
   using ST = AqStage<NT>;
   const size_t dyn = (size_t)ST::STAGES * ST::BYTES + 1024;
-  static bool attr = false;
-  if (!attr) {
+  static bool attr[64] = {};          // per device: the shared-memory limit is per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr[dev]) {
     cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<NT, FMT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr[dev] = true;
   }
   CUtensorMap tx, tl;
   if (!aq_map(&tx, X, (uint64_t)w->K, (uint64_t)M, (uint64_t)ldx * 2, AQ_ROWS))

@@ -71,6 +71,15 @@ inline bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The current device, for the per-device "attributes set" flags of the
+// launchers (a kernel's dynamic shared-memory limit is a per-device setting).
+constexpr int kMaxDevices = 64;
+inline int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
 inline int num_sms() {
   static int n = 0;
   if (!n) {

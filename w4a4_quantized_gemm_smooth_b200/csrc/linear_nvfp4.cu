@@ -352,12 +352,14 @@ cudaError_t launch_linear_nvfp4(const svdq_weights* w, int M, const uint8_t* xq,
                                 const uint8_t* sfa, const float* s_x, const uint16_t* Z,
                                 uint16_t* Y, int ldy, int epilogue, cudaStream_t st) {
   using L = F4Lay;
-  static bool attr = false;
-  if (!attr) {
+  static bool attr[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (!attr[dev]) {
     cudaError_t e = cudaFuncSetAttribute(linear_nvfp4_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr[dev] = true;
   }
   CUtensorMap ta, tb, ty, tz, tl;
   if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 64, L::BM,

@@ -382,8 +382,10 @@ cudaError_t launch_linear_w8a8(const svdq_weights* w, int M, const int8_t* xq, c
                                const uint16_t* Z, uint16_t* Y, int ldy, int epilogue,
                                cudaStream_t st) {
   using L = W8Lay;
-  static bool attr = false;
-  if (!attr) {
+  static bool attr[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (!attr[dev]) {
     cudaFuncAttributes fa;
     cudaError_t e0 = cudaFuncGetAttributes(&fa, linear_w8a8_kernel);
     if (e0 != cudaSuccess) return e0;
@@ -391,7 +393,7 @@ cudaError_t launch_linear_w8a8(const svdq_weights* w, int M, const int8_t* xq, c
     cudaError_t e = cudaFuncSetAttribute(linear_w8a8_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr[dev] = true;
   }
   CUtensorMap ta, tb, ty, tz, tl, tsx, tsw;
   const uint64_t sx_pitch = ((uint64_t)M * 4 + 15) / 16 * 16;

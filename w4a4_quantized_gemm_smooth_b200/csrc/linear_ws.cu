@@ -668,8 +668,10 @@ cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtens
                       const CUtensorMap& tsx, const CUtensorMap& tsw, LinArgs a, int tiles_m,
                       cudaStream_t st) {
   using L = Lay<BN>;
-  static bool attr = false;
-  if (!attr) {
+  static bool attr[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (!attr[dev]) {
     cudaFuncAttributes fa;
     cudaError_t e0 = cudaFuncGetAttributes(&fa, linear_ws_kernel<BN, MODE>);
     if (e0 != cudaSuccess) return e0;
@@ -677,7 +679,7 @@ cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtens
     cudaError_t e = cudaFuncSetAttribute(linear_ws_kernel<BN, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr[dev] = true;
   }
   a.num_tiles = tiles_m * a.tiles_n;
   const int work = a.num_tiles * a.splits;
