@@ -115,6 +115,24 @@ def test_nvfp4_matches_oracle(M, K, N, r, epi):
     check_nvfp4(spec, epi)
 
 
+def test_nvfp4_row_pitch():
+    """Y written into a wider buffer (ldy > N): the columns past N stay untouched."""
+    spec = synth.layer_spec("f4_ldy", 200, 512, 264, 16, 84, tiny=True)
+    L = synth.make_layer(spec)
+    a = S.svdq_calib_absmax(L.X)
+    w = S.svdq_pack_weights_nvfp4(L.W, a, 16, bias_bits=L.b)
+    lin = S.NVFP4Linear(w)
+    xq, sfa, s_x, Z, Y = lin.buffers(200)
+    full = torch.full((200, 320), -7.0, dtype=torch.bfloat16, device="cuda")
+    lin.forward(_to_dev(L.X), out=full[:, :264])
+    lin.forward(_to_dev(L.X), out=Y)
+    torch.cuda.synchronize()
+    S.svdq_get_device_error(w)
+    assert np.array_equal(_bits(full[:, :264]), _bits(Y))
+    assert torch.all(full[:, 264:] == -7.0)
+    w.free()
+
+
 def test_nvfp4_zero_and_single_outlier_tokens():
     spec = synth.layer_spec("f4_edge", 96, 256, 264, 8, 81, tiny=True)
     L = synth.make_layer(spec)
