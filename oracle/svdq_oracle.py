@@ -18,6 +18,7 @@ What it computes follows "SVDQuant: How a Small High-Precision Branch Makes
   * MAC and storage ratios                                     (section 6, eqs. 11-12)
   * calibration refinement: alpha search by the calibrated layer-output
     error, factors re-fitted to W~ - Q(R)                        (section 5)
+  * GPTQ rounding of the residual on the calibration Hessian   (section 8)
   * W8A8 comparator: int8 operands, one scale per token / output channel
     applied once          (section 8, the eight-bit setting; section 9.3, INT8)
   * NVFP4 variant: E2M1 codes in groups of 16 with E4M3 group scales and
@@ -54,6 +55,7 @@ __all__ = [
     "two_branch_unquantized", "dequantize_groups", "residual_quantize",
     "leading_svd", "layer_output_error", "refine_factors", "pack_weights_calibrated",
     "quantize_rows_int8", "pack_weights_w8a8", "quantize_act_w8a8", "linear_w8a8",
+    "gptq_hessian", "gptq_quantize_residual",
     "NVFP4_GROUP", "E2M1_VALUES", "round_e4m3", "e4m3_bits", "e2m1_codes", "e2m1_values",
     "quantize_nvfp4_rows", "dequantize_nvfp4", "pack_weights_nvfp4", "quantize_act_nvfp4",
     "linear_nvfp4",
@@ -364,6 +366,66 @@ def layer_output_error(X_bits, packed, W_bits):
     return float(np.linalg.norm(Yq - ref) / np.linalg.norm(ref))
 
 
+def gptq_hessian(X_bits, inv_lambda):
+    """H = X~^T X~ (fp64) on the calibration tokens, X~ = fl32(x * inv_lambda):
+    the second moment of the smoothed activations the residual multiplies."""
+    X = bf16_bits_to_f64(X_bits)
+    Xh = round_f32(X * np.asarray(inv_lambda, dtype=np.float64)[None, :])
+    return Xh.T @ Xh
+
+
+def gptq_quantize_residual(R, H, damp=0.01):
+    """GPTQ rounding of the residual R [K, N] (the review's offline procedure,
+    section 8: "residual weights use GPTQ"; the published algorithm of
+    Frantar et al.).  H is dampened by damp * mean(diag H) (a channel the
+    calibration never activates gets H_kk = 1); U is the upper Cholesky
+    factor of H^-1.  Input channels are taken in order; on entering a group
+    of 64 the eq. 1 scale of every output column is taken from the current
+    (updated) group; then each channel k is quantised (eq. 1 on fl32 of the
+    updated value) and its error err = (w - q s) / U_kk is pushed onto the
+    later channels: R[j] -= U_kj err.  Returns (codes [N, K], s_w [G, N])."""
+    R = np.array(R, dtype=np.float64, copy=True)
+    K, N = R.shape
+    Hd = np.array(H, dtype=np.float64, copy=True)
+    dead = np.diag(Hd) == 0
+    Hd[dead, dead] = 1.0
+    Hd += damp * np.mean(np.diag(Hd)) * np.eye(K)
+    U = np.linalg.cholesky(np.linalg.inv(Hd)).T            # upper, H^-1 = U^T U
+    G = K // GROUP
+    codes = np.zeros((N, K), dtype=np.int64)
+    s_w = np.zeros((G, N))
+    for k in range(K):
+        g = k // GROUP
+        if k % GROUP == 0:
+            _, s_w[g] = quantize_groups(round_f32(R[k:k + GROUP].T))
+        s = s_w[g]
+        w32 = round_f32(R[k])
+        q = np.zeros(N, dtype=np.int64)
+        nz = s > 0
+        if np.any(nz):
+            c, _ = _round_with_scale(w32[nz], s[nz])
+            q[nz] = c
+        codes[:, k] = q
+        err = (R[k] - q * s) / U[k, k]
+        R[k + 1:] -= np.outer(U[k, k + 1:], err)
+    return codes, s_w
+
+
+def _round_with_scale(z, s):
+    """Codes of eq. 1 for values z with given scales s (exact round-half-even
+    of z / s by fp64 comparisons, clamped to [-8, 7])."""
+    z = np.asarray(z, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)
+    q = np.rint(z / s)
+    for _ in range(3):
+        two_d = 2.0 * (z - q * s)
+        q = np.where(two_d > s, q + 1, np.where(two_d < -s, q - 1, q))
+    d = z - q * s
+    tie = (2.0 * np.abs(d) == s) & (np.mod(q, 2) != 0)
+    q = np.where(tie, q + np.sign(d), q)
+    return np.clip(q, -8, 7).astype(np.int64), s
+
+
 def _set_factors(p, Wt, L1, L2):
     """New protected factors for a packed layer: store them as bf16, take R
     against the stored factors and quantise it again (eqs. 10, 1)."""
@@ -388,20 +450,33 @@ def refine_factors(p, svd=None):
     return _set_factors(p, Wt, U[:, :r] * S[None, :r], Vt[:r, :])
 
 
+def _with_gptq(p, H):
+    """The packed layer with its residual R quantised by GPTQ instead."""
+    codes, s_w = gptq_quantize_residual(p["R"], H)
+    return dict(p, wcodes=codes, wq=pack_nibbles(codes), s_w=s_w)
+
+
 def pack_weights_calibrated(W_bits, X_cal_bits, rank, alphas=(0.3, 0.4, 0.5, 0.6, 0.7),
                             iters=1, bias_bits=None, lora_A_bits=None, lora_B_bits=None,
-                            lora_scale=1.0, svd=None):
+                            lora_scale=1.0, svd=None, gptq=False):
     """For every candidate alpha: smoothing, SVD, residual quantisation, then
     `iters` alternating refinements; keep the candidate with the smallest
     calibrated layer-output error (the first one on ties).  The statistics
-    and the error use the calibration tokens X_cal.  LoRA joins the branch
-    afterwards, as in pack_weights.  Returns (packed, errors per alpha)."""
+    and the error use the calibration tokens X_cal.  gptq=True quantises
+    every residual (the first and each refined one) with GPTQ on the
+    calibration Hessian of the candidate's smoothed activations.  LoRA joins
+    the branch afterwards, as in pack_weights.  Returns (packed, errors)."""
     a = calib_absmax(bf16_bits_to_f64(X_cal_bits))
     best, best_err, errs = None, None, []
     for alpha in alphas:
         p = pack_weights(W_bits, a, rank, alpha=alpha, svd=svd)
+        H = gptq_hessian(X_cal_bits, p["inv_lambda"]) if gptq else None
+        if gptq:
+            p = _with_gptq(p, H)
         for _ in range(iters):
             p = refine_factors(p, svd=svd)
+            if gptq:
+                p = _with_gptq(p, H)
         e = layer_output_error(X_cal_bits, p, W_bits)
         errs.append(e)
         if best is None or e < best_err:
