@@ -145,13 +145,24 @@ svdq_status svdq_pack_weights_host(int K, int N, int rank, int group,
  * and bias join as in svdq_pack_weights.  errors (host, n_alpha doubles, may
  * be NULL) receives every candidate's error.  to_device != 0 uploads to the
  * current device (stream ordered); 0 gives a host-only handle.
+ * gptq != 0 rounds every residual (the first and each refined one) with
+ * GPTQ (review section 8: "residual weights use GPTQ"; the published
+ * algorithm of Frantar et al.) instead of to nearest:
+ *   H = X~^T X~ on the calibration tokens (x~ = fl32(x * inv_lambda)),
+ *   dampened by 1 % of its mean diagonal (an unused channel gets H_kk = 1);
+ *   U = upper Cholesky factor of H^-1; input channels in order: on entering
+ *   a group of 64 each output column's scale comes from the updated group
+ *   (eq. 1), then channel k is rounded (eq. 1 on fl32 of the updated value)
+ *   and its error (w - q s) / U_kk is subtracted from every later channel j
+ *   times U_kj.  The cost is O(K^3 + N K^2) host work per candidate.
  * Errors: as svdq_pack_weights; SVDQ_ERR_INVALID_ARG for missing or empty
- * calibration tokens, an alpha outside (0, 1) or a negative iteration count.
+ * calibration tokens, an alpha outside (0, 1) or a negative iteration count;
+ * SVDQ_ERR_NUMERIC if the dampened Hessian is not positive definite.
  */
 svdq_status svdq_pack_weights_calibrated(int K, int N, int rank, int group,
                                          const uint16_t* W, const uint16_t* X_cal,
                                          int M_cal, int ldx, int n_alpha,
-                                         const double* alphas, int refine_iters,
+                                         const double* alphas, int refine_iters, int gptq,
                                          const uint16_t* bias, int lora_rank,
                                          const uint16_t* lora_A, const uint16_t* lora_B,
                                          float lora_scale, int to_device,

@@ -39,6 +39,33 @@ def test_calibrated_pack_matches_oracle(case):
     w.free()
 
 
+@pytest.mark.parametrize("case", ["tiny", "tall"])
+def test_gptq_pack_matches_oracle(case):
+    """GPTQ rounding of the residual (with one refinement step, which rounds
+    the refined residual by GPTQ again): the library's host Cholesky and the
+    oracle's LAPACK one give the same codes and scales."""
+    if case == "tiny":
+        spec = synth.WORKLOADS["tiny"]
+    else:
+        spec = synth.layer_spec("gq_tall", 96, 640, 192, 24, 43)
+    L = synth.make_layer(spec)
+    alphas = (0.4, 0.6)
+    w, errs = S.svdq_pack_weights_calibrated(L.W, L.X, spec.rank, alphas=alphas, refine_iters=1,
+                                             bias_bits=L.b, to_device=False, gptq=True)
+    p, errs_o = oracle.pack_weights_calibrated(L.W, L.X, spec.rank, alphas=alphas, iters=1,
+                                               bias_bits=L.b, gptq=True)
+    assert np.allclose(errs, errs_o, rtol=1e-6, atol=0)
+    assert alphas[int(np.argmin(errs))] == p["alpha"]
+    e = w.export()
+    assert np.array_equal(e["wq"], p["wq"])
+    assert np.array_equal(e["s_w"].astype(np.float64), p["s_w"])
+    # and GPTQ beats rounding to nearest on the calibrated error
+    _, errs_rtn = S.svdq_pack_weights_calibrated(L.W, L.X, spec.rank, alphas=alphas, refine_iters=1,
+                                                 to_device=False)
+    assert min(errs) < min(errs_rtn)
+    w.free()
+
+
 def test_one_alpha_without_refinement_is_the_plain_pack():
     L = synth.make_layer(synth.WORKLOADS["tiny"])
     w, errs = S.svdq_pack_weights_calibrated(L.W, L.X, 16, alphas=(0.5,), refine_iters=0,

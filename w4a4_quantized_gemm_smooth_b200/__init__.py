@@ -81,7 +81,7 @@ def lib() -> ctypes.CDLL:
                                         _i, _vp, _vp, ctypes.c_float, _vp]),
         "svdq_weights_info": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
         "svdq_pack_weights_calibrated": (_i, [_i, _i, _i, _i, _vp, _vp, _i, _i, _i, _vp, _i,
-                                              _vp, _i, _vp, _vp, ctypes.c_float, _i, _vp,
+                                              _i, _vp, _i, _vp, _vp, ctypes.c_float, _i, _vp,
                                               _vp, _vp]),
         "svdq_weights_export": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
         "svdq_weights_save": (_i, [_vp, ctypes.c_char_p]),
@@ -244,9 +244,11 @@ def svdq_pack_weights_host(W_bits, act_absmax, rank, alpha=0.5, bias_bits=None,
 
 def svdq_pack_weights_calibrated(W_bits, X_cal_bits, rank, alphas=(0.3, 0.4, 0.5, 0.6, 0.7),
                                  refine_iters=1, bias_bits=None, lora_A_bits=None,
-                                 lora_B_bits=None, lora_scale=1.0, to_device=True, stream=None):
-    """Pack with the calibrated alpha search and the alternating factor
-    refinement.  X_cal_bits: host bf16 bits [M_cal, K] (calibration tokens).
+                                 lora_B_bits=None, lora_scale=1.0, to_device=True, stream=None,
+                                 gptq=False):
+    """Pack with the calibrated alpha search, the alternating factor
+    refinement and, with gptq=True, GPTQ rounding of the residual.
+    X_cal_bits: host bf16 bits [M_cal, K] (calibration tokens).
     Returns (Weights, errors per alpha)."""
     X_cal_bits = np.ascontiguousarray(X_cal_bits, dtype=np.uint16)
     W_bits, _, bias_bits, A, B, lr = _pack_args(
@@ -257,7 +259,8 @@ def svdq_pack_weights_calibrated(W_bits, X_cal_bits, rank, alphas=(0.3, 0.4, 0.5
     h = _vp()
     _check(lib().svdq_pack_weights_calibrated(
         K, N, int(rank), 64, _np_ptr(W_bits), _np_ptr(X_cal_bits), X_cal_bits.shape[0], K,
-        len(al), _np_ptr(al), int(refine_iters), _np_ptr(bias_bits), lr, _np_ptr(A), _np_ptr(B),
+        len(al), _np_ptr(al), int(refine_iters), 1 if gptq else 0, _np_ptr(bias_bits), lr,
+        _np_ptr(A), _np_ptr(B),
         float(lora_scale), 1 if to_device else 0, _stream_ptr(stream) if to_device else None,
         _np_ptr(errs), ctypes.byref(h)), "svdq_pack_weights_calibrated")
     return Weights(h), errs

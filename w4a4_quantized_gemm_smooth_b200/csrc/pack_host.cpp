@@ -373,8 +373,138 @@ int8_t code_at(const std::vector<uint8_t>& wq, int K, int n, int k) {
   return (int8_t)(v >= 8 ? v - 16 : v);
 }
 
+// ---------------------------------------------------------------- GPTQ
+// The residual rounded by GPTQ (the review's offline procedure: "residual
+// weights use GPTQ"; the published algorithm of Frantar et al.) on the
+// Hessian H = X~^T X~ of the calibration tokens in smoothed coordinates.
+
+// Exact round-half-even of zd / sd (sd > 0), clamped to [-8, 7].
+int code_of(double zd, double sd) {
+  double c = std::nearbyint(zd / sd);
+  for (int it = 0; it < 2; ++it) {
+    const double d2 = 2.0 * (zd - c * sd);          // exact
+    if (d2 > sd) c += 1.0;
+    else if (d2 < -sd) c -= 1.0;
+  }
+  const double d2 = 2.0 * (zd - c * sd);
+  if (std::fabs(d2) == sd && std::fmod(c, 2.0) != 0.0) c += (d2 > 0 ? 1.0 : -1.0);
+  return (int)std::fmax(-8.0, std::fmin(7.0, c));
+}
+
+// In-place lower Cholesky factor of the symmetric positive definite n x n
+// row-major A (only the lower triangle is read and written).
+bool cholesky_lower(std::vector<double>& A, int n) {
+  for (int j = 0; j < n; ++j) {
+    double d = A[(size_t)j * n + j];
+    for (int k = 0; k < j; ++k) d -= A[(size_t)j * n + k] * A[(size_t)j * n + k];
+    if (!(d > 0.0)) return false;
+    d = std::sqrt(d);
+    A[(size_t)j * n + j] = d;
+#pragma omp parallel for schedule(static)
+    for (int i = j + 1; i < n; ++i) {
+      double v = A[(size_t)i * n + j];
+      for (int k = 0; k < j; ++k) v -= A[(size_t)i * n + k] * A[(size_t)j * n + k];
+      A[(size_t)i * n + j] = v / d;
+    }
+  }
+  return true;
+}
+
+// U (upper, row-major) with H^-1 = U^T U for the dampened Hessian: H + damp
+// mean(diag H) I, a channel the calibration never activates given H_kk = 1.
+svdq_status gptq_factor(std::vector<double> H, int K, std::vector<double>& U) {
+  double mean = 0.0;
+  for (int k = 0; k < K; ++k) {
+    if (H[(size_t)k * K + k] == 0.0) H[(size_t)k * K + k] = 1.0;
+    mean += H[(size_t)k * K + k];
+  }
+  mean /= K;
+  for (int k = 0; k < K; ++k) H[(size_t)k * K + k] += 0.01 * mean;
+  if (!cholesky_lower(H, K)) return SVDQ_ERR_NUMERIC;         // H = L L^T
+  // Linv = L^-1 (lower), column by column by forward substitution
+  std::vector<double> Linv((size_t)K * K, 0.0);
+#pragma omp parallel for schedule(dynamic)
+  for (int c = 0; c < K; ++c) {
+    for (int i = c; i < K; ++i) {
+      double v = (i == c) ? 1.0 : 0.0;
+      for (int k = c; k < i; ++k) v -= H[(size_t)i * K + k] * Linv[(size_t)k * K + c];
+      Linv[(size_t)i * K + c] = v / H[(size_t)i * K + i];
+    }
+  }
+  // Hinv = Linv^T Linv (symmetric; lower triangle suffices for the next factor)
+  std::vector<double> Hinv((size_t)K * K, 0.0);
+#pragma omp parallel for schedule(dynamic)
+  for (int i = 0; i < K; ++i)
+    for (int j = 0; j <= i; ++j) {
+      double v = 0.0;
+      for (int k = i; k < K; ++k) v += Linv[(size_t)k * K + i] * Linv[(size_t)k * K + j];
+      Hinv[(size_t)i * K + j] = v;
+    }
+  if (!cholesky_lower(Hinv, K)) return SVDQ_ERR_NUMERIC;       // Hinv = L2 L2^T
+  U.assign((size_t)K * K, 0.0);
+  for (int i = 0; i < K; ++i)
+    for (int j = 0; j <= i; ++j) U[(size_t)j * K + i] = Hinv[(size_t)i * K + j];   // U = L2^T
+  return SVDQ_OK;
+}
+
+// H = X~^T X~ in fp64 over the calibration tokens, X~ = fl32(x inv_lambda).
+std::vector<double> gptq_hessian(int K, const uint16_t* X, int M, int ldx,
+                                 const std::vector<float>& inv_lambda) {
+  std::vector<double> XT((size_t)K * M);
+  for (int m = 0; m < M; ++m)
+    for (int k = 0; k < K; ++k)
+      XT[(size_t)k * M + m] = (double)(float)(bf16_to_f64(X[(size_t)m * ldx + k]) * (double)inv_lambda[k]);
+  std::vector<double> H((size_t)K * K);
+#pragma omp parallel for schedule(dynamic)
+  for (int i = 0; i < K; ++i)
+    for (int j = 0; j <= i; ++j) {
+      double v = 0.0;
+      for (int m = 0; m < M; ++m) v += XT[(size_t)i * M + m] * XT[(size_t)j * M + m];
+      H[(size_t)i * K + j] = v;
+      H[(size_t)j * K + i] = v;
+    }
+  return H;
+}
+
+// The residual R = W~ - L1b L2b, then GPTQ per output column (the columns
+// are independent): on entering a group of 64 the eq. 1 scale comes from the
+// updated group; channel k's error (w - q s) / U_kk moves the later channels
+// by U_kj.
+void gptq_residual(int K, int N, int rank, const std::vector<double>& U, Candidate& c) {
+  const int G = K / SVDQ_GROUP;
+  c.sw.assign((size_t)G * N, 0.0f);
+  c.wq.assign((size_t)N * K / 2, 0);
+#pragma omp parallel for schedule(dynamic)
+  for (int n = 0; n < N; ++n) {
+    std::vector<double> r(K);
+    for (int k = 0; k < K; ++k) {
+      double v = c.Wt[(size_t)k * N + n];
+      for (int j = 0; j < rank; ++j)
+        v -= bf16_to_f64(c.L1[(size_t)k * rank + j]) * bf16_to_f64(c.L2[(size_t)j * N + n]);
+      r[k] = v;
+    }
+    std::vector<int8_t> q(K);
+    float s = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      if (k % SVDQ_GROUP == 0) {
+        float m = 0.0f;
+        for (int i = 0; i < SVDQ_GROUP; ++i) m = std::fmax(m, std::fabs((float)r[k + i]));
+        s = m / 7.0f;
+        c.sw[(size_t)(k / SVDQ_GROUP) * N + n] = s;
+      }
+      const int qk = s > 0.0f ? code_of((double)(float)r[k], (double)s) : 0;
+      q[k] = (int8_t)qk;
+      const double err = (r[k] - (double)qk * (double)s) / U[(size_t)k * K + k];
+      const double* urow = &U[(size_t)k * K];
+      for (int j = k + 1; j < K; ++j) r[j] -= urow[j] * err;
+    }
+    uint8_t* dst = &c.wq[(size_t)n * (K / 2)];
+    for (int b = 0; b < K / 2; ++b) dst[b] = (uint8_t)((q[2 * b] & 0xF) | ((q[2 * b + 1] & 0xF) << 4));
+  }
+}
+
 // One alternating refinement: the factors of W~ - deq(Q(R)), then R again.
-svdq_status refine(int K, int N, int rank, Candidate& c) {
+svdq_status refine(int K, int N, int rank, Candidate& c, const std::vector<double>* U) {
   std::vector<double> T(c.Wt);
 #pragma omp parallel for schedule(static)
   for (int k = 0; k < K; ++k)
@@ -382,7 +512,8 @@ svdq_status refine(int K, int N, int rank, Candidate& c) {
       T[(size_t)k * N + n] -= (double)code_at(c.wq, K, n, k) * (double)c.sw[(size_t)(k / 64) * N + n];
   const svdq_status s = fit_factors(T.data(), K, N, rank, c);
   if (s != SVDQ_OK) return s;
-  quantize_residual(K, N, rank, c);
+  if (U) gptq_residual(K, N, rank, *U, c);
+  else quantize_residual(K, N, rank, c);
   return SVDQ_OK;
 }
 
@@ -559,7 +690,8 @@ static svdq_status pack_impl(int K, int N, int rank, int group, const uint16_t* 
 
 static svdq_status pack_calibrated_impl(int K, int N, int rank, int group, const uint16_t* W,
                                         const uint16_t* X, int M, int ldx, int n_alpha,
-                                        const double* alphas, int iters, const uint16_t* bias,
+                                        const double* alphas, int iters, int gptq,
+                                        const uint16_t* bias,
                                         int lora_rank, const uint16_t* lora_A,
                                         const uint16_t* lora_B, float lora_scale,
                                         bool to_device, cudaStream_t stream, double* errors,
@@ -578,9 +710,13 @@ static svdq_status pack_calibrated_impl(int K, int N, int rank, int group, const
     Candidate c;
     if ((s = smooth(K, N, W, a.data(), alphas[i], c)) != SVDQ_OK) return s;
     if ((s = fit_factors(c.Wt.data(), K, N, rank, c)) != SVDQ_OK) return s;
-    quantize_residual(K, N, rank, c);
+    std::vector<double> U;
+    if (gptq && (s = gptq_factor(gptq_hessian(K, X, M, ldx, c.inv_lambda), K, U)) != SVDQ_OK)
+      return s;
+    if (gptq) gptq_residual(K, N, rank, U, c);
+    else quantize_residual(K, N, rank, c);
     for (int it = 0; it < iters; ++it)
-      if ((s = refine(K, N, rank, c)) != SVDQ_OK) return s;
+      if ((s = refine(K, N, rank, c, gptq ? &U : nullptr)) != SVDQ_OK) return s;
     const double e = layer_error(K, N, rank, c, ref, X, M, ldx);
     if (errors) errors[i] = e;
     if (i == 0 || e < best_err) {
@@ -612,12 +748,12 @@ svdq_status svdq_pack_weights_host(int K, int N, int rank, int group, const uint
 svdq_status svdq_pack_weights_calibrated(int K, int N, int rank, int group, const uint16_t* W,
                                          const uint16_t* X_cal, int M_cal, int ldx,
                                          int n_alpha, const double* alphas, int refine_iters,
-                                         const uint16_t* bias, int lora_rank,
+                                         int gptq, const uint16_t* bias, int lora_rank,
                                          const uint16_t* lora_A, const uint16_t* lora_B,
                                          float lora_scale, int to_device, cudaStream_t stream,
                                          double* errors, svdq_weights** out) {
   return pack_calibrated_impl(K, N, rank, group, W, X_cal, M_cal, ldx, n_alpha, alphas,
-                              refine_iters, bias, lora_rank, lora_A, lora_B, lora_scale,
+                              refine_iters, gptq, bias, lora_rank, lora_A, lora_B, lora_scale,
                               to_device != 0, stream, errors, out);
 }
 
