@@ -187,13 +187,16 @@ def test_save_load_roundtrip(tmp_path):
     w2.free()
 
 
-def test_calibrated_pack_layer():
+@pytest.mark.parametrize("gptq", [False, True])
+def test_calibrated_pack_layer(gptq):
     """A layer packed with the calibrated alpha search and one refinement
-    runs through the hot path like any other."""
+    (and GPTQ rounding of the residual) runs through the hot path like any
+    other."""
     spec = synth.layer_spec("calgpu", 192, 640, 320, 24, 55)
     L = synth.make_layer(spec)
-    w, errs = S.svdq_pack_weights_calibrated(L.W, L.X, 24, refine_iters=1, bias_bits=L.b)
-    p, errs_o = oracle.pack_weights_calibrated(L.W, L.X, 24, iters=1, bias_bits=L.b)
+    w, errs = S.svdq_pack_weights_calibrated(L.W, L.X, 24, refine_iters=1, bias_bits=L.b,
+                                             gptq=gptq)
+    p, errs_o = oracle.pack_weights_calibrated(L.W, L.X, 24, iters=1, bias_bits=L.b, gptq=gptq)
     assert np.allclose(errs, errs_o, rtol=1e-6, atol=0)
     X = to_dev(L.X)
     lin = S.SVDQLinear(w)
