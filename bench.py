@@ -350,6 +350,70 @@ def _time_nvfp4(S, spec, L, a, X, flush, stream, steps, fp4_peak):
             "peak_source": "measured bf16 burst x 4 (fp4/bf16 nominal ratio)"}
 
 
+class _StepPair:
+    """The feed-forward pair fc2(GELU(fc1(X))): fused (fc1's epilogue emits
+    fc2's activation side) or unfused (fc1 stores H, fc2's activation pass
+    reads it), with an event between the kernels."""
+
+    def __init__(self, S, mlp, X, fused):
+        self.S, self.mlp, self.X, self.fused = S, mlp, X, fused
+        self.n_phases = 3 if fused else 4
+
+    def __call__(self, marks, stream):
+        S, m = self.S, self.mlp
+        a, b = m.fc1, m.fc2
+        marks[0].record(stream)
+        S.svdq_quantize_act(a.w, self.X, a.xq, a.s_x, a.Z, stream)
+        marks[1].record(stream)
+        if self.fused:
+            S.svdq_linear_quantize_next(a.w, b.w, a.xq, a.s_x, a.Z, b.xq, b.s_x, b.Z, m.ws,
+                                        S.EPI_GELU, stream)
+        else:
+            S.svdq_linear(a.w, a.xq, a.s_x, a.Z, m.H, S.EPI_GELU, stream)
+            marks[2].record(stream)
+            S.svdq_quantize_act(b.w, m.H, b.xq, b.s_x, b.Z, stream)
+        marks[-2].record(stream)
+        S.svdq_linear(b.w, b.xq, b.s_x, b.Z, b.Y, S.EPI_NONE, stream)
+        marks[-1].record(stream)
+
+
+def _time_mlp_pair(S, flush, stream, steps):
+    """The FLUX feed-forward pair (fc1 3072 -> 12288, GELU, fc2 12288 -> 3072,
+    rank 32, 4608 tokens) with and without the cross-layer fusion.  fc2 is
+    calibrated on fc1's output."""
+    import torch
+    s1, s2 = synth.WORKLOADS["flux_mlp_fc1"], synth.WORKLOADS["flux_mlp_fc2"]
+    L1, L2 = synth.make_layer(s1), synth.make_layer(s2)
+    w1 = S.svdq_pack_weights(L1.W, S.svdq_calib_absmax(L1.X), s1.rank, bias_bits=L1.b)
+    X = _to_dev(L1.X)
+    H = S.SVDQLinear(w1, S.EPI_GELU)(X)
+    torch.cuda.synchronize()
+    Hb = H.cpu().view(torch.int16).numpy().view(np.uint16)
+    w2 = S.svdq_pack_weights(L2.W, S.svdq_calib_absmax(Hb), s2.rank, bias_bits=L2.b)
+    mlp = S.SVDQMLP(w1, w2)
+    mlp.buffers(s1.M)
+    out = {"workload": "flux_mlp_fc1 -> GELU -> flux_mlp_fc2", "M": s1.M,
+           "dims": [s1.K, s1.N, s2.N], "rank": [s1.rank, s2.rank]}
+    for fused in (False, True):
+        st = _StepPair(S, mlp, X, fused)
+        _time_steps(st, 3, flush, stream)
+        ph = [v / steps for v in _time_steps(st, steps, flush, stream)]
+        key = "fused" if fused else "unfused"
+        out[key + "_ms"] = sum(ph)
+        out[key + "_phases_ms"] = ph
+    S.svdq_get_device_error(w1)
+    S.svdq_get_device_error(w2)
+    ops = 2.0 * s1.M * (s1.K * s1.N + s2.K * s2.N)
+    out["phases"] = {"unfused": ["act fc1", "fc1 -> H", "act fc2", "fc2"],
+                     "fused": ["act fc1", "fc1 -> fc2 codes, scales, Z", "fc2"]}
+    out["pair_tops_unfused"] = ops / (out["unfused_ms"] * 1e-3) / 1e12
+    out["pair_tops_fused"] = ops / (out["fused_ms"] * 1e-3) / 1e12
+    out["saving"] = 1.0 - out["fused_ms"] / out["unfused_ms"]
+    w1.free()
+    w2.free()
+    return out
+
+
 def _time_e2e(S, w, Xh, Yh, Xd, bufs, epi, steps):
     """Public API end to end, as a serving loop: every step copies its X from
     pinned host memory to the device, runs svdq_quantize_act and svdq_linear,
@@ -492,6 +556,8 @@ def run_ours(args, spec):
     if not args.no_nvfp4:
         line["nvfp4_variant"] = _time_nvfp4(S, spec, L, a, X, flush, stream, args.steps,
                                             4.0 * bf16_burst)
+    if args.mlp_pair:
+        line["cross_layer_fusion"] = _time_mlp_pair(S, flush, stream, args.steps)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec)
     if rank == 0:
@@ -515,6 +581,9 @@ def main():
                     help="skip the W8A8 comparator's timing")
     ap.add_argument("--no-nvfp4", action="store_true",
                     help="skip the NVFP4 variant's timing")
+    ap.add_argument("--mlp-pair", action="store_true",
+                    help="also time the FLUX feed-forward pair with and without the "
+                         "cross-layer fusion")
     args = ap.parse_args()
     spec = _workload(args.workload)
     if args.impl == "reference":

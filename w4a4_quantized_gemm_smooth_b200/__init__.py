@@ -12,9 +12,11 @@ The call names follow include/svdq.h:
     svdq_debug_partials, svdq_linear_splitk*, svdq_pack_weights_calibrated,
     the W8A8 comparator svdq_pack_weights_w8a8, svdq_quantize_act_w8a8,
     svdq_linear_w8a8, and the NVFP4 variant svdq_pack_weights_nvfp4,
-    svdq_quantize_act_nvfp4, svdq_linear_nvfp4
+    svdq_quantize_act_nvfp4, svdq_linear_nvfp4, and the cross-layer fusion
+    svdq_linear_quantize_next
 and SVDQLinear / W8A8Linear / NVFP4Linear bundle one packed layer with its
-two hot-path calls.
+two hot-path calls; SVDQMLP chains two layers (fc1, GELU, fc2) with or
+without the fusion.
 """
 from __future__ import annotations
 
@@ -31,6 +33,7 @@ __all__ = [
     "svdq_pack_weights_w8a8", "svdq_quantize_act_w8a8", "svdq_linear_w8a8", "W8A8Linear",
     "FORMAT_W4A4", "FORMAT_W8A8", "FORMAT_NVFP4", "svdq_pack_weights_nvfp4",
     "svdq_quantize_act_nvfp4", "svdq_linear_nvfp4", "svdq_nvfp4_sf_bytes", "NVFP4Linear",
+    "svdq_linear_quantize_next", "svdq_linear_quantize_next_workspace", "SVDQMLP",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -107,6 +110,9 @@ def lib() -> ctypes.CDLL:
         "svdq_nvfp4_sf_bytes": (ctypes.c_size_t, [_i, _i]),
         "svdq_quantize_act_nvfp4": (_i, [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
         "svdq_linear_nvfp4": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp]),
+        "svdq_linear_quantize_next_workspace": (ctypes.c_size_t, [_vp, _i]),
+        "svdq_linear_quantize_next": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+                                           _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -288,6 +294,26 @@ def svdq_linear(w: Weights, xq, s_x, Z, Y, epilogue=EPI_NONE, stream=None):
     _check(lib().svdq_linear(w.handle, M, _dev_ptr(xq), _dev_ptr(s_x), _dev_ptr(Z),
                              _dev_ptr(Y), Y.stride(0), int(epilogue), _stream_ptr(stream)),
            "svdq_linear")
+
+
+def svdq_linear_quantize_next_workspace(w_next: Weights, M: int) -> int:
+    """Workspace bytes of svdq_linear_quantize_next (fp32 [M, rank_next])."""
+    return int(lib().svdq_linear_quantize_next_workspace(w_next.handle, int(M)))
+
+
+def svdq_linear_quantize_next(w: Weights, w_next: Weights, xq, s_x, Z, xq_next, s_x_next,
+                              Z_next, workspace, epilogue=EPI_NONE, stream=None):
+    """The layer of w with the next layer's activation pass in its epilogue:
+    writes xq_next uint8 [M, N/2], s_x_next float32 [N/64, M] and Z_next bf16
+    [M, rank_next] (None when rank_next == 0) instead of Y.  workspace: cuda
+    float32 tensor of M * rank_next elements (None when rank_next == 0)."""
+    M = xq.shape[0]
+    _check(lib().svdq_linear_quantize_next(w.handle, w_next.handle, M, _dev_ptr(xq),
+                                           _dev_ptr(s_x), _dev_ptr(Z), int(epilogue),
+                                           _dev_ptr(xq_next), _dev_ptr(s_x_next),
+                                           _dev_ptr(Z_next), _dev_ptr(workspace),
+                                           _stream_ptr(stream)),
+           "svdq_linear_quantize_next")
 
 
 def svdq_linear_splitk_workspace(w: Weights, M: int, splits: int = 0) -> int:
@@ -475,6 +501,53 @@ class NVFP4Linear(SVDQLinear):
             Y = out
         svdq_quantize_act_nvfp4(self.w, X, xq, sfa, s_x, Z)
         svdq_linear_nvfp4(self.w, xq, sfa, s_x, Z, Y, self.epilogue)
+        return Y
+
+    __call__ = forward
+
+
+class SVDQMLP:
+    """Two packed layers applied in sequence, fc2(GELU(fc1(X))), as in a
+    transformer block's feed-forward part.
+
+    forward(X, fused=True) runs svdq_quantize_act(fc1), then
+    svdq_linear_quantize_next (fc1 with GELU, emitting fc2's codes, scales
+    and Z), then svdq_linear(fc2): the hidden activation never reaches device
+    memory.  fused=False runs the four plain calls, storing the bf16 hidden
+    activation H in between.  Buffers are reallocated only when M changes.
+    """
+
+    def __init__(self, fc1: Weights, fc2: Weights):
+        if fc2.K != fc1.N:
+            raise ValueError("fc2's K must equal fc1's N")
+        self.fc1 = SVDQLinear(fc1, EPI_GELU)
+        self.fc2 = SVDQLinear(fc2)
+        self._M = -1
+        self.H = self.ws = None
+
+    def buffers(self, M: int, device="cuda"):
+        import torch
+        self.fc1.buffers(M, device)
+        self.fc2.buffers(M, device)
+        if M != self._M:
+            self.H = torch.empty((M, self.fc1.w.N), dtype=torch.bfloat16, device=device)
+            n = self.fc2.w.rank * M
+            self.ws = torch.empty((max(n, 1),), dtype=torch.float32, device=device) if n else None
+            self._M = M
+        return self.H, self.ws
+
+    def forward(self, X, fused: bool = True, out=None):
+        M = X.shape[0]
+        H, ws = self.buffers(M, X.device)
+        a, b = self.fc1, self.fc2
+        Y = b.Y if out is None else out
+        svdq_quantize_act(a.w, X, a.xq, a.s_x, a.Z)
+        if fused:
+            svdq_linear_quantize_next(a.w, b.w, a.xq, a.s_x, a.Z, b.xq, b.s_x, b.Z, ws, EPI_GELU)
+        else:
+            svdq_linear(a.w, a.xq, a.s_x, a.Z, H, EPI_GELU)
+            svdq_quantize_act(b.w, H, b.xq, b.s_x, b.Z)
+        svdq_linear(b.w, b.xq, b.s_x, b.Z, Y)
         return Y
 
     __call__ = forward

@@ -84,6 +84,35 @@ svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq, const f
   return from_launch(svdq::launch_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, stream));
 }
 
+size_t svdq_linear_quantize_next_workspace(const svdq_weights* w_next, int M) {
+  if (!w_next || M <= 0 || !w_next->d_wq) return 0;
+  return (size_t)M * w_next->rank * sizeof(float);
+}
+
+svdq_status svdq_linear_quantize_next(const svdq_weights* w, const svdq_weights* w_next,
+                                      int M, const uint8_t* xq, const float* s_x,
+                                      const uint16_t* Z, int epilogue, uint8_t* xq_next,
+                                      float* s_x_next, uint16_t* Z_next, float* workspace,
+                                      cudaStream_t stream) {
+  svdq_status s = check_handle(w);
+  if (s != SVDQ_OK) return s;
+  s = check_handle(w_next);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || w_next->K != w->N || w_next->rank > 32) return SVDQ_ERR_SHAPE;
+  if (epilogue != SVDQ_EPI_NONE && epilogue != SVDQ_EPI_GELU) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  const bool z2 = w_next->rank > 0;
+  if (!xq || !s_x || (w->rank > 0 && !Z) || !xq_next || !s_x_next ||
+      (z2 && (!Z_next || !workspace)))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(s_x) || (w->rank > 0 && !aligned16(Z)) ||
+      !aligned16(xq_next) || !aligned16(s_x_next) ||
+      (z2 && (!aligned16(Z_next) || !aligned16(workspace))))
+    return SVDQ_ERR_ALIGNMENT;
+  return from_launch(svdq::launch_linear_next(w, w_next, M, xq, s_x, Z, epilogue, xq_next,
+                                              s_x_next, Z_next, workspace, stream));
+}
+
 size_t svdq_linear_splitk_workspace(const svdq_weights* w, int M, int splits) {
   if (!w || M <= 0 || !w->d_wq) return 0;
   const int sp = resolve_splits(w, M, splits);

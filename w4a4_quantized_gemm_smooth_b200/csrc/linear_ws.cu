@@ -51,6 +51,7 @@
 
 #include "gemm_common.cuh"
 #include "ptx.cuh"
+#include "quant_common.cuh"
 #include "svdq_internal.h"
 
 namespace svdq {
@@ -92,6 +93,13 @@ struct LinArgs {
   int splits;              // K splits per tile (1 except in MODE 3)
   float* part;             // MODE 3: fp32 partial tiles [tile][split][warp][32 x CW]
   int* cnt;                // MODE 3: arrivals per (tile, rescale warp), zero between uses
+  // MODE 4: the next layer's activation side from this layer's output
+  const float* inv_lambda2;  // [N]: the next layer's smoothing factors (its K = this N)
+  uint8_t* xq2;              // [M][N / 2] packed codes
+  float* s_x2;               // [N / 64][M] group scales
+  float* zacc;               // [M][rank2] fp32 down-projection, accumulated over the tiles
+  int rank2, rank2_pad;      // the next layer's rank, and rounded up to 16
+  int n_l1;                  // 128-column L1^T parts per tile (0 without a low-rank branch)
 };
 
 // One unit of work: output tile t, groups [g0, g1) of split sp.  The
@@ -141,19 +149,25 @@ struct Lay {
   static constexpr int SC_SLOT = (BM + BN) * 4;
   static constexpr int OFF_SC = OFF_LR + NLR * LR_SLOT;
   static constexpr int OFF_BIAS = OFF_SC + NS * SC_SLOT;   // per warp CW floats
+  // MODE 4: the next layer's smoothing factors of the warp's columns
+  static constexpr int OFF_ILAM = OFF_BIAS + N_RES_WARPS * CW * 4;
   // constant operands of the accumulator-initialising bf16 MMA (K = 16)
   static constexpr int INIT_A = BM * 32, INIT_B = BN * 32;
-  static constexpr int OFF_INIT = OFF_BIAS + N_RES_WARPS * CW * 4;
+  static constexpr int OFF_INIT = OFF_ILAM + N_RES_WARPS * CW * 4;
   static constexpr int OFF_BAR = OFF_INIT + INIT_A + INIT_B;
   // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[NB],
-  // tm_empty[NB], lr_full[NLR], lr_empty[NLR]
-  static constexpr int N_BARS = 2 * NP + 2 * NE + 2 * NB + 2 * NLR;
+  // tm_empty[NB], lr_full[NLR], lr_empty[NLR], xh_full
+  static constexpr int N_BARS = 2 * NP + 2 * NE + 2 * NB + 2 * NLR + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;              // slack for 1024-B alignment
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
+
+__device__ __forceinline__ void sts32u(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 // 16 packed bytes (32 codes of one row: the first or second half of the
 // group) -> two 16-byte core-matrix rows at d and d + 128.
@@ -219,6 +233,13 @@ struct ExpandPlan {
 //         items; each writes its fp32 partial to p.part, and the last of a
 //         tile's splits (per rescale warp, by an atomic count) sums them in
 //         split order and runs the epilogue.
+// MODE 4: the layer, followed in the epilogue by the next layer's activation
+//         side instead of the store of Y: the bf16 output tile is smoothed
+//         with the next layer's factors, quantised per token and group of 64
+//         (a tile holds whole groups) into packed codes and scales, and
+//         multiplied on the tensor cores, as bf16, with the matching rows of
+//         the next layer's L1; the fp32 partial down-projections of a row's
+//         tiles are summed in p.zacc by atomic adds.
 template <int BN, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
@@ -227,10 +248,12 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_z,
                  const __grid_constant__ CUtensorMap tm_l2,
                  const __grid_constant__ CUtensorMap tm_sx,
-                 const __grid_constant__ CUtensorMap tm_sw, const LinArgs p) {
+                 const __grid_constant__ CUtensorMap tm_sw,
+                 const __grid_constant__ CUtensorMap tm_l1, const LinArgs p) {
   using L = Lay<BN>;
   constexpr bool LAYER = MODE != 1;
   constexpr bool SPLIT = MODE == 3;
+  constexpr bool FUSE = MODE == 4;
   constexpr int CW = L::CW;
   constexpr int NE = L::NE;
   constexpr int NB = L::NB;
@@ -248,17 +271,18 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
   constexpr int NLR = L::NLR;
   auto lr_full = [&](int s) { return bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + s); };
   auto lr_empty = [&](int s) { return bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + NLR + s); };
+  const uint32_t xh_full = bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + 2 * NLR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = p.G;
 
   if (tid == 0) {
     for (int s = 0; s < NP; ++s) { mbar_init(pk_full(s), 1); mbar_init(pk_empty(s), N_EXP); }
     for (int s = 0; s < NE; ++s) { mbar_init(ex_full(s), N_EXP); mbar_init(ex_empty(s), 1); }
     for (int b = 0; b < NB; ++b) { mbar_init(tm_full(b), 1); mbar_init(tm_empty(b), N_RES_WARPS); }
     for (int s = 0; s < NLR; ++s) { mbar_init(lr_full(s), 1); mbar_init(lr_empty(s), 1); }
+    mbar_init(xh_full, N_RES_WARPS);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -341,6 +365,18 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               tma_load_2d(dst + L::LR_SA + c * (BN * 16), &tm_l2, 16 * j + 8 * c, n0, lr_full(ls));
             }
           }
+          // MODE 4: the next layer's L1^T rows of this tile's columns, in
+          // 128-column parts through the same slots (rank2_pad rows x 256 B
+          // each, chunk c of 8 columns at c * rank2_pad * 16, row r at r * 16)
+          for (int u = 0; FUSE && alive && u < p.n_l1; ++u, ++il) {
+            const int ls = il % NLR;
+            if (!wait_or_abort(lr_empty(ls), ((il / NLR) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
+            mbar_arrive_expect_tx(lr_full(ls), (uint32_t)p.rank2_pad * 256u);
+            const uint32_t dst = sbase + L::OFF_LR + ls * L::LR_SLOT;
+#pragma unroll 4
+            for (int c = 0; c < 16; ++c)
+              tma_load_2d(dst + c * (p.rank2_pad * 16), &tm_l1, n0 + 128 * u + 8 * c, 0, lr_full(ls));
+          }
         }
         alive = __shfl_sync(0xFFFFFFFFu, alive ? 1 : 0, 0) != 0;
       }
@@ -360,7 +396,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         // the constant tiles hold one value each, so any layout descriptor works
         const uint64_t init_ad = sdesc_kmajor_noswizzle(sbase + L::OFF_INIT, 128, 256);
         const uint64_t init_bd = sdesc_kmajor_noswizzle(sbase + L::OFF_INIT + L::INIT_A, 128, 256);
-        uint32_t ite = 0, tb = 0, il = 0;
+        uint32_t ite = 0, tb = 0, il = 0, ixh = 0;
         for (int wk = blockIdx.x; wk < p.num_tiles * p.splits; wk += gridDim.x) {
           const WorkItem wi = work_item(p, wk);
           const bool lrs = wi.lr && p.n_lr > 0;
@@ -395,6 +431,34 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             }
             mma_commit(tm_full(b));
             ++tb;
+          }
+          if (FUSE && p.n_l1 > 0) {
+            // the next layer's down-projection of this tile: x~ (bf16, written
+            // by the epilogue) times its L1 rows, into the next TMEM buffer
+            const int b = tb % NB;
+            if (!wait_or_abort(tm_empty(b), ((tb / NB) & 1) ^ 1, abort_flag, p.err)) goto mma_done;
+            if (!wait_or_abort(xh_full, ixh & 1, abort_flag, p.err)) goto mma_done;
+            tc_fence_after();
+            const uint32_t d = tmem + b * BN;
+            const uint32_t id_z = idesc_bf16(BM, p.rank2_pad);
+            for (int u = 0; u < p.n_l1; ++u, ++il) {
+              const int ls = il % NLR;
+              if (!wait_or_abort(lr_full(ls), (il / NLR) & 1, abort_flag, p.err)) goto mma_done;
+              tc_fence_after();
+              const uint32_t la = sbase + L::OFF_LR + ls * L::LR_SLOT;
+              for (int j = 0; j < 8; ++j) {
+                // A: chunk kc of x~ at kc * BM * 16 bytes, row r at r * 16
+                const uint64_t ad = sdesc_kmajor_noswizzle(
+                    sbase + L::OFF_Y + (16 * u + 2 * j) * (BM * 16), BM * 16, 128);
+                const uint64_t bd = sdesc_kmajor_noswizzle(la + 2 * j * (p.rank2_pad * 16),
+                                                           p.rank2_pad * 16, 128);
+                mma_bf16(d, ad, bd, id_z, (u > 0 || j > 0) ? 1u : 0u);
+              }
+              mma_commit(lr_empty(ls));
+            }
+            mma_commit(tm_full(b));
+            ++tb;
+            ++ixh;
           }
         }
       mma_done:;
@@ -465,10 +529,12 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         for (int j = 0; j < CW / 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
       constexpr int PER = CW / 32;             // bias values loaded per lane
       float bias_n[PER];                       // prefetched for the epilogue
+      float ilam_n[PER];                       // MODE 4: the next layer's smoothing factors
 #pragma unroll
       for (int e = 0; e < PER; ++e) {
         const int n = ncol0 + lane * PER + e;
         bias_n[e] = (LAYER && n < p.N) ? __uint_as_float((uint32_t)__ldg(p.bias + n) << 16) : 0.0f;
+        ilam_n[e] = (FUSE && n < p.N) ? __ldg(p.inv_lambda2 + n) : 0.0f;
       }
       for (int g = wi.g0; g < wi.g1; ++g, ++tb, ++gs) {
         const uint32_t slot = sbase + L::OFF_SC + (gs % L::NS) * L::SC_SLOT;
@@ -611,6 +677,87 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         __syncwarp();
         if (lane == 0) atomicExch(p.cnt + t * N_RES_WARPS + rw, 0);   // ready for the next call
       }
+      if constexpr (FUSE) {
+        // epilogue of MODE 4: h = bf16(bias (+ GELU)) exactly as the stored Y
+        // would be, x~ = fl32(h inv_lambda2), the codes and scale of each of
+        // the warp's 64-column groups per row, and bf16(x~) into the
+        // down-projection's A operand (the Y staging area, unused here)
+        float* lb = reinterpret_cast<float*>(smem + L::OFF_ILAM) + rw * CW;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+          bb[lane * PER + e] = bias_n[e];
+          lb[lane * PER + e] = ilam_n[e];
+        }
+        __syncwarp();
+        const bool gelu = p.epilogue == SVDQ_EPI_GELU;
+        const bool zlr = p.n_l1 > 0;
+        const uint32_t xa = sbase + L::OFF_Y;
+#pragma unroll
+        for (int j = 0; j < CW / 64; ++j) {
+          const int gcol = ncol0 + 64 * j;       // first column of the group
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int rl = 32 * q + r0 + 8 * i;  // row within the tile
+            float v[16];                         // value 4 cc + 2 b2 + e: column 16 cc + 8 b2 + 2 pq + e
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+              for (int b2 = 0; b2 < 2; ++b2) {
+                const int c = 4 * j + cc;
+                const int col = 16 * c + 8 * b2 + 2 * pq;
+                const float2 bv = *reinterpret_cast<const float2*>(bb + col);
+                const float2 lv = *reinterpret_cast<const float2*>(lb + col);
+                float2 y = __fadd2_rn(acc[i][2 * c + b2], bv);
+                if (gelu) y = make_float2(gelu_f(y.x), gelu_f(y.y));
+                const uint32_t hb = bf16x2_bits(y);
+                const float2 xh = __fmul2_rn(
+                    make_float2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xFFFF0000u)), lv);
+                v[4 * cc + 2 * b2] = xh.x;
+                v[4 * cc + 2 * b2 + 1] = xh.y;
+                if (zlr) {
+                  // chunk kc = column / 8 of the tile at kc * BM * 16, row at 16 each
+                  const uint32_t kc = (uint32_t)(h * CW + 16 * c + 8 * b2) >> 3;
+                  sts32u(xa + kc * (BM * 16) + rl * 16 + 4 * pq, bf16x2_bits(xh));
+                }
+              }
+            }
+            uint32_t u[2];
+            const float sc = quant_group16(v, u);
+            const uint32_t w0 = quad_transpose(u[0], pq), w1 = quad_transpose(u[1], pq);
+            const int row = m0 + rl;
+            if (row < p.M && gcol < p.N) {
+              *reinterpret_cast<uint2*>(p.xq2 + (size_t)row * (p.N / 2) + gcol / 2 + 8 * pq) =
+                  make_uint2(w0, w1);
+              if (pq == 0) p.s_x2[(size_t)(gcol / 64) * p.M + row] = sc;
+            }
+          }
+        }
+        if (zlr) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xh_full);
+          // the tile's partial down-projection: 32x32b load, lane = row
+          const int b = tb % NB;
+          if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          if (16 * h < p.rank2_pad) {
+            uint32_t r[16];
+            tmem_ld16(tmem + b * BN + 16 * h + lane_off, r);
+            tmem_wait_ld();
+            const int row = m0 + 32 * q + lane;
+            if (row < p.M) {
+              float* zr = p.zacc + (size_t)row * p.rank2 + 16 * h;
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj)
+                if (16 * h + jj < p.rank2) atomicAdd(zr + jj, __uint_as_float(r[jj]));
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tm_empty(b));
+          ++tb;
+        }
+      } else {
       // epilogue: bias, GELU, bf16, swizzled staging, TMA store
 #pragma unroll
       for (int e = 0; e < PER; ++e) bb[lane * PER + e] = bias_n[e];
@@ -647,6 +794,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         tma_store_commit();
       }
       __syncwarp();
+      }
     }
     if (LAYER && lane == 0) tma_store_wait0();
     __syncwarp();
@@ -662,11 +810,12 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
 
 // ------------------------------------------------------------------ host side
 
+struct LinMaps {
+  CUtensorMap ta, tb, ty, tz, tl, tsx, tsw, tl1;
+};
+
 template <int BN, int MODE>
-cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtensorMap& tb,
-                      const CUtensorMap& ty, const CUtensorMap& tz, const CUtensorMap& tl,
-                      const CUtensorMap& tsx, const CUtensorMap& tsw, LinArgs a, int tiles_m,
-                      cudaStream_t st) {
+cudaError_t launch_ws(const LinMaps& m, LinArgs a, int tiles_m, cudaStream_t st) {
   using L = Lay<BN>;
   static bool attr[kMaxDevices] = {};
   const int dev = current_device();
@@ -684,7 +833,8 @@ cudaError_t launch_ws(const svdq_weights* w, const CUtensorMap& ta, const CUtens
   a.num_tiles = tiles_m * a.tiles_n;
   const int work = a.num_tiles * a.splits;
   const int grid = work < num_sms() ? work : num_sms();
-  linear_ws_kernel<BN, MODE><<<grid, THREADS, L::ALLOC, st>>>(ta, tb, ty, tz, tl, tsx, tsw, a);
+  linear_ws_kernel<BN, MODE><<<grid, THREADS, L::ALLOC, st>>>(m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx,
+                                                              m.tsw, m.tl1, a);
   return cudaGetLastError();
 }
 
@@ -694,10 +844,6 @@ int pick_bn(int N) {
   return (r != 0 && r <= 128) ? 128 : 256;
 }
 
-struct LinMaps {
-  CUtensorMap ta, tb, ty, tz, tl, tsx, tsw;
-};
-
 // Tensor maps and kernel arguments shared by the layer launches.
 bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* s_x,
                   const uint16_t* Z, uint16_t* Y, int ldy, int epilogue, int BN, LinMaps& m,
@@ -705,11 +851,14 @@ bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* 
   if (!make_map(&m.ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 64, BM,
                 CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map(&m.tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 64, BN,
-                CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map(&m.ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
-                CU_TENSOR_MAP_SWIZZLE_128B))
+                CU_TENSOR_MAP_SWIZZLE_64B))
+    return false;
+  m.ty = m.ta;   // no Y in MODE 4
+  if (Y && !make_map(&m.ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
     return false;
   m.tz = m.ta;
+  m.tl1 = m.ta;
   m.tl = m.ta;
   m.tsx = m.ta;
   const bool sx_tma = (M % 4) == 0;
@@ -756,8 +905,7 @@ cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const
   LinArgs a;
   if (!build_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, BN, m, a)) return cudaErrorInvalidValue;
   const int tiles_m = (M + BM - 1) / BM;
-  return BN == 256 ? launch_ws<256, 0>(w, m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx, m.tsw, a, tiles_m, st)
-                   : launch_ws<128, 0>(w, m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx, m.tsw, a, tiles_m, st);
+  return BN == 256 ? launch_ws<256, 0>(m, a, tiles_m, st) : launch_ws<128, 0>(m, a, tiles_m, st);
 }
 
 int splitk_auto(const svdq_weights* w, int M) {
@@ -791,19 +939,19 @@ cudaError_t launch_linear_splitk(const svdq_weights* w, int M, const uint8_t* xq
   cudaError_t e = cudaMemsetAsync(workspace, 0, cb, st);
   if (e != cudaSuccess) return e;
   const int tiles_m = (M + BM - 1) / BM;
-  return BN == 256 ? launch_ws<256, 3>(w, m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx, m.tsw, a, tiles_m, st)
-                   : launch_ws<128, 3>(w, m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx, m.tsw, a, tiles_m, st);
+  return BN == 256 ? launch_ws<256, 3>(m, a, tiles_m, st) : launch_ws<128, 3>(m, a, tiles_m, st);
 }
 
 cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int row0,
                             int nrows, int col0, int ncols, int32_t* P, cudaStream_t st) {
   const int BN = pick_bn(w->N);
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 64, BM,
+  LinMaps m;
+  if (!make_map(&m.ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 64, BM,
                 CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map(&tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 64, BN,
+      !make_map(&m.tb, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 64, BN,
                 CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
+  m.ty = m.tz = m.tl = m.tsx = m.tsw = m.tl1 = m.ta;
   LinArgs a{};
   a.M = M; a.N = w->N; a.K = w->K; a.G = w->G;
   a.rank = 0; a.rank_pad32 = 0; a.n_lr = 0; a.epilogue = 0;
@@ -813,8 +961,50 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
   const int tm0 = row0 / BM, tm1 = (row0 + nrows - 1) / BM;
   const int tn0 = col0 / BN, tn1 = (col0 + ncols - 1) / BN;
   a.tile_m0 = tm0; a.tile_n0 = tn0; a.tiles_n = tn1 - tn0 + 1;
-  return BN == 256 ? launch_ws<256, 1>(w, ta, tb, ta, ta, ta, ta, ta, a, tm1 - tm0 + 1, st)
-                   : launch_ws<128, 1>(w, ta, tb, ta, ta, ta, ta, ta, a, tm1 - tm0 + 1, st);
+  return BN == 256 ? launch_ws<256, 1>(m, a, tm1 - tm0 + 1, st)
+                   : launch_ws<128, 1>(m, a, tm1 - tm0 + 1, st);
+}
+
+namespace {
+// Z = bf16(zacc), element by element (the next layer's Z of MODE 4).
+__global__ void zacc_to_bf16_kernel(const float* __restrict__ zacc, uint16_t* __restrict__ Z,
+                                    long long n) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    Z[i] = __bfloat16_as_ushort(__float2bfloat16_rn(zacc[i]));
+}
+}  // namespace
+
+cudaError_t launch_linear_next(const svdq_weights* w, const svdq_weights* w2, int M,
+                               const uint8_t* xq, const float* s_x, const uint16_t* Z,
+                               int epilogue, uint8_t* xq2, float* s_x2, uint16_t* Z2,
+                               float* zacc, cudaStream_t st) {
+  const int BN = pick_bn(w->N);
+  LinMaps m;
+  LinArgs a;
+  if (!build_linear(w, M, xq, s_x, Z, nullptr, w->N, epilogue, BN, m, a)) return cudaErrorInvalidValue;
+  a.inv_lambda2 = w2->d_inv_lambda;
+  a.xq2 = xq2;
+  a.s_x2 = s_x2;
+  a.zacc = zacc;
+  a.rank2 = w2->rank;
+  a.rank2_pad = w2->rank_pad;
+  a.n_l1 = w2->rank > 0 ? BN / 128 : 0;
+  const long long nz = (long long)M * w2->rank;
+  if (w2->rank > 0) {
+    if (!make_map(&m.tl1, w2->d_L1T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w2->K, w2->rank_pad,
+                  (uint64_t)w2->K * 2, 8, w2->rank_pad, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(zacc, 0, (size_t)nz * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+  }
+  const int tiles_m = (M + BM - 1) / BM;
+  cudaError_t e = BN == 256 ? launch_ws<256, 4>(m, a, tiles_m, st) : launch_ws<128, 4>(m, a, tiles_m, st);
+  if (e != cudaSuccess || nz == 0) return e;
+  long long blocks = (nz + 255) / 256;
+  if (blocks > 8LL * num_sms()) blocks = 8LL * num_sms();
+  zacc_to_bf16_kernel<<<(int)blocks, 256, 0, st>>>(zacc, Z2, nz);
+  return cudaGetLastError();
 }
 
 }  // namespace svdq
