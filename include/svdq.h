@@ -282,10 +282,11 @@ svdq_status svdq_linear_splitk_noalloc(const svdq_weights* w, int M, const uint8
  *   xq_next, s_x_next: the codes and scales svdq_quantize_act(w_next, h)
  *                      would write (bit-exact: same quantiser);
  *   Z_next [M][rank_next] bf16(bf16(x~) L1_next) with x~ = fl32(h inv_lambda_next),
- *          fp32 accumulation whose order differs from svdq_quantize_act's
- *          (the column tiles' partial products are added atomically), so
- *          Z_next agrees with it to within fp32 summation error before the
- *          bf16 rounding (a one-ulp bf16 difference is possible).
+ *          fp32 accumulation in an order that differs from svdq_quantize_act's
+ *          (each output column tile's partial product, then their sum in
+ *          column-tile order), so Z_next agrees with it to within fp32
+ *          summation error before the bf16 rounding (a one-ulp bf16
+ *          difference is possible).  The result is deterministic.
  * A 128 x 128 or 128 x 256 output tile holds whole 64-column groups of the
  * next layer's K, so its codes and scales are complete in the epilogue;
  * only Z_next needs the cross-tile sum.
@@ -293,22 +294,26 @@ svdq_status svdq_linear_splitk_noalloc(const svdq_weights* w, int M, const uint8
  * w_next: a W4A4 handle on the same device with K == w's N and rank <= 32.
  * xq_next [M][N/2] uint8, s_x_next [N/64][M] fp32, Z_next [M][rank_next]
  * bf16 (may be NULL when rank_next == 0), device, 16-byte aligned.
- * workspace: device fp32 [M][rank_next], 16-byte aligned, owned by the
- * caller (svdq_linear_quantize_next_workspace gives its size in bytes; NULL
- * when rank_next == 0); the call clears it (cudaMemsetAsync on `stream`),
- * accumulates Z_next in it and converts it.  Calls sharing a workspace must
- * not overlap.  Launches: the clear, the layer kernel, and one small
- * conversion kernel.  A device timeout is reported on w's error word.
+ * workspace: device memory owned by the caller, 16-byte aligned, of at
+ * least svdq_linear_quantize_next_workspace(w, w_next, M) bytes (fp32
+ * [column tiles of w][M][rank_next], the tiles' partial Z_next; 0 bytes and
+ * NULL allowed when rank_next == 0).  Every byte the call reads it has
+ * written first, so the workspace needs no initialisation; calls sharing
+ * one must not overlap.  Launches: the layer kernel and one small kernel
+ * that sums the partials and rounds them to bf16.  A device timeout is
+ * reported on w's error word.
  * Errors: as svdq_linear; SVDQ_ERR_SHAPE when w_next's K differs from w's
- * N or its rank exceeds 32; SVDQ_ERR_INVALID_ARG for a handle of another
- * format or device, or a missing output.
+ * N, its rank exceeds 32, or workspace_bytes is too small;
+ * SVDQ_ERR_INVALID_ARG for a handle of another format or device, or a
+ * missing output.
  */
-size_t svdq_linear_quantize_next_workspace(const svdq_weights* w_next, int M);
+size_t svdq_linear_quantize_next_workspace(const svdq_weights* w, const svdq_weights* w_next,
+                                           int M);
 svdq_status svdq_linear_quantize_next(const svdq_weights* w, const svdq_weights* w_next,
                                       int M, const uint8_t* xq, const float* s_x,
                                       const uint16_t* Z, int epilogue, uint8_t* xq_next,
-                                      float* s_x_next, uint16_t* Z_next, float* workspace,
-                                      cudaStream_t stream);
+                                      float* s_x_next, uint16_t* Z_next, void* workspace,
+                                      size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the handle's sticky device

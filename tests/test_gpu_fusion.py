@@ -57,9 +57,10 @@ def _fused(w1, w2, lin1, epi):
     xq2 = torch.full((M, N // 2), 0xAB, dtype=torch.uint8, device="cuda")
     s_x2 = torch.full((N // 64, M), -1.0, dtype=torch.float32, device="cuda")
     Z2 = torch.empty((M, r2), dtype=torch.bfloat16, device="cuda") if r2 else None
-    nws = S.svdq_linear_quantize_next_workspace(w2, M)
-    assert nws == 4 * M * r2
-    ws = torch.full((max(M * r2, 1),), 3.0, dtype=torch.float32, device="cuda") if r2 else None
+    nws = S.svdq_linear_quantize_next_workspace(w1, w2, M)
+    tiles_n = -(-N // (128 if N <= 128 or 0 < N % 256 <= 128 else 256))
+    assert nws == 4 * tiles_n * M * r2
+    ws = torch.full((max(nws // 4, 1),), 3.0, dtype=torch.float32, device="cuda") if r2 else None
     S.svdq_linear_quantize_next(w1, w2, lin1.xq, lin1.s_x, lin1.Z, xq2, s_x2, Z2, ws, epi)
     torch.cuda.synchronize()
     S.svdq_get_device_error(w1)
@@ -153,12 +154,16 @@ def test_fused_next_rejects_mismatched_layers():
     xq2 = torch.empty((64, 160), dtype=torch.uint8, device="cuda")
     s_x2 = torch.empty((5, 64), dtype=torch.float32, device="cuda")
     Z2 = torch.empty((64, 16), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty((64 * 16,), dtype=torch.float32, device="cuda")
+    ws = torch.empty((S.svdq_linear_quantize_next_workspace(w1, w2, 64) // 4,),
+                     dtype=torch.float32, device="cuda")
     with pytest.raises(S.SVDQError) as e:
         S.svdq_linear_quantize_next(w1, w_bad, lin1.xq, lin1.s_x, lin1.Z, xq2, s_x2, Z2, ws)
     assert e.value.status == 2              # SVDQ_ERR_SHAPE
     with pytest.raises(S.SVDQError) as e:
         S.svdq_linear_quantize_next(w1, w2, lin1.xq, lin1.s_x, lin1.Z, xq2, s_x2, Z2, None)
     assert e.value.status == 1              # SVDQ_ERR_INVALID_ARG: no workspace
+    with pytest.raises(S.SVDQError) as e:
+        S.svdq_linear_quantize_next(w1, w2, lin1.xq, lin1.s_x, lin1.Z, xq2, s_x2, Z2, ws[:-4])
+    assert e.value.status == 2              # SVDQ_ERR_SHAPE: workspace too small
     for w in (w1, w2, w_bad):
         w.free()

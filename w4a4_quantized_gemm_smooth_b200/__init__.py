@@ -110,9 +110,9 @@ def lib() -> ctypes.CDLL:
         "svdq_nvfp4_sf_bytes": (ctypes.c_size_t, [_i, _i]),
         "svdq_quantize_act_nvfp4": (_i, [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
         "svdq_linear_nvfp4": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp]),
-        "svdq_linear_quantize_next_workspace": (ctypes.c_size_t, [_vp, _i]),
+        "svdq_linear_quantize_next_workspace": (ctypes.c_size_t, [_vp, _vp, _i]),
         "svdq_linear_quantize_next": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
-                                           _vp]),
+                                           ctypes.c_size_t, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -296,9 +296,10 @@ def svdq_linear(w: Weights, xq, s_x, Z, Y, epilogue=EPI_NONE, stream=None):
            "svdq_linear")
 
 
-def svdq_linear_quantize_next_workspace(w_next: Weights, M: int) -> int:
-    """Workspace bytes of svdq_linear_quantize_next (fp32 [M, rank_next])."""
-    return int(lib().svdq_linear_quantize_next_workspace(w_next.handle, int(M)))
+def svdq_linear_quantize_next_workspace(w: Weights, w_next: Weights, M: int) -> int:
+    """Workspace bytes of svdq_linear_quantize_next (the column tiles'
+    partial Z_next, fp32; 0 when rank_next == 0 or for invalid arguments)."""
+    return int(lib().svdq_linear_quantize_next_workspace(w.handle, w_next.handle, int(M)))
 
 
 def svdq_linear_quantize_next(w: Weights, w_next: Weights, xq, s_x, Z, xq_next, s_x_next,
@@ -306,12 +307,14 @@ def svdq_linear_quantize_next(w: Weights, w_next: Weights, xq, s_x, Z, xq_next, 
     """The layer of w with the next layer's activation pass in its epilogue:
     writes xq_next uint8 [M, N/2], s_x_next float32 [N/64, M] and Z_next bf16
     [M, rank_next] (None when rank_next == 0) instead of Y.  workspace: cuda
-    float32 tensor of M * rank_next elements (None when rank_next == 0)."""
+    tensor of at least svdq_linear_quantize_next_workspace(w, w_next, M)
+    bytes (None when rank_next == 0)."""
     M = xq.shape[0]
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().svdq_linear_quantize_next(w.handle, w_next.handle, M, _dev_ptr(xq),
                                            _dev_ptr(s_x), _dev_ptr(Z), int(epilogue),
                                            _dev_ptr(xq_next), _dev_ptr(s_x_next),
-                                           _dev_ptr(Z_next), _dev_ptr(workspace),
+                                           _dev_ptr(Z_next), _dev_ptr(workspace), nbytes,
                                            _stream_ptr(stream)),
            "svdq_linear_quantize_next")
 
@@ -531,8 +534,8 @@ class SVDQMLP:
         self.fc2.buffers(M, device)
         if M != self._M:
             self.H = torch.empty((M, self.fc1.w.N), dtype=torch.bfloat16, device=device)
-            n = self.fc2.w.rank * M
-            self.ws = torch.empty((max(n, 1),), dtype=torch.float32, device=device) if n else None
+            n = svdq_linear_quantize_next_workspace(self.fc1.w, self.fc2.w, M)
+            self.ws = torch.empty((n,), dtype=torch.uint8, device=device) if n else None
             self._M = M
         return self.H, self.ws
 

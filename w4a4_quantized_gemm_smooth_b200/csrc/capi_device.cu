@@ -84,16 +84,17 @@ svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq, const f
   return from_launch(svdq::launch_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, stream));
 }
 
-size_t svdq_linear_quantize_next_workspace(const svdq_weights* w_next, int M) {
-  if (!w_next || M <= 0 || !w_next->d_wq) return 0;
-  return (size_t)M * w_next->rank * sizeof(float);
+size_t svdq_linear_quantize_next_workspace(const svdq_weights* w, const svdq_weights* w_next,
+                                           int M) {
+  if (!w || !w_next || M <= 0 || !w->d_wq || !w_next->d_wq || w_next->K != w->N) return 0;
+  return svdq::linear_next_workspace(w, w_next, M);
 }
 
 svdq_status svdq_linear_quantize_next(const svdq_weights* w, const svdq_weights* w_next,
                                       int M, const uint8_t* xq, const float* s_x,
                                       const uint16_t* Z, int epilogue, uint8_t* xq_next,
-                                      float* s_x_next, uint16_t* Z_next, float* workspace,
-                                      cudaStream_t stream) {
+                                      float* s_x_next, uint16_t* Z_next, void* workspace,
+                                      size_t workspace_bytes, cudaStream_t stream) {
   svdq_status s = check_handle(w);
   if (s != SVDQ_OK) return s;
   s = check_handle(w_next);
@@ -109,8 +110,10 @@ svdq_status svdq_linear_quantize_next(const svdq_weights* w, const svdq_weights*
       !aligned16(xq_next) || !aligned16(s_x_next) ||
       (z2 && (!aligned16(Z_next) || !aligned16(workspace))))
     return SVDQ_ERR_ALIGNMENT;
+  if (z2 && workspace_bytes < svdq::linear_next_workspace(w, w_next, M)) return SVDQ_ERR_SHAPE;
   return from_launch(svdq::launch_linear_next(w, w_next, M, xq, s_x, Z, epilogue, xq_next,
-                                              s_x_next, Z_next, workspace, stream));
+                                              s_x_next, Z_next, static_cast<float*>(workspace),
+                                              stream));
 }
 
 size_t svdq_linear_splitk_workspace(const svdq_weights* w, int M, int splits) {

@@ -97,7 +97,7 @@ struct LinArgs {
   const float* inv_lambda2;  // [N]: the next layer's smoothing factors (its K = this N)
   uint8_t* xq2;              // [M][N / 2] packed codes
   float* s_x2;               // [N / 64][M] group scales
-  float* zacc;               // [M][rank2] fp32 down-projection, accumulated over the tiles
+  float* zpart;              // [tiles_n][M][rank2] fp32 down-projection of each column tile
   int rank2, rank2_pad;      // the next layer's rank, and rounded up to 16
   int n_l1;                  // 128-column L1^T parts per tile (0 without a low-rank branch)
 };
@@ -238,8 +238,9 @@ struct ExpandPlan {
 //         with the next layer's factors, quantised per token and group of 64
 //         (a tile holds whole groups) into packed codes and scales, and
 //         multiplied on the tensor cores, as bf16, with the matching rows of
-//         the next layer's L1; the fp32 partial down-projections of a row's
-//         tiles are summed in p.zacc by atomic adds.
+//         the next layer's L1; each tile stores its fp32 partial
+//         down-projection in p.zpart, summed in column-tile order by a
+//         second kernel.
 template <int BN, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
@@ -746,10 +747,14 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             tmem_wait_ld();
             const int row = m0 + 32 * q + lane;
             if (row < p.M) {
-              float* zr = p.zacc + (size_t)row * p.rank2 + 16 * h;
+              // rank2 is a multiple of 8: whole 16-byte stores
+              float4* zr = reinterpret_cast<float4*>(
+                  p.zpart + ((size_t)(t % p.tiles_n) * p.M + row) * p.rank2 + 16 * h);
 #pragma unroll
-              for (int jj = 0; jj < 16; ++jj)
-                if (16 * h + jj < p.rank2) atomicAdd(zr + jj, __uint_as_float(r[jj]));
+              for (int jj = 0; jj < 4; ++jj)
+                if (16 * h + 4 * jj < p.rank2)
+                  zr[jj] = make_float4(__uint_as_float(r[4 * jj]), __uint_as_float(r[4 * jj + 1]),
+                                       __uint_as_float(r[4 * jj + 2]), __uint_as_float(r[4 * jj + 3]));
             }
           }
           tc_fence_before();
@@ -966,19 +971,28 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
 }
 
 namespace {
-// Z = bf16(zacc), element by element (the next layer's Z of MODE 4).
-__global__ void zacc_to_bf16_kernel(const float* __restrict__ zacc, uint16_t* __restrict__ Z,
-                                    long long n) {
+// Z = bf16(sum over the column tiles t, in order, of part[t]) element by
+// element: the next layer's Z of MODE 4.
+__global__ void zpart_sum_kernel(const float* __restrict__ part, uint16_t* __restrict__ Z,
+                                 long long n, int tiles) {
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (long long)gridDim.x * blockDim.x)
-    Z[i] = __bfloat16_as_ushort(__float2bfloat16_rn(zacc[i]));
+       i += (long long)gridDim.x * blockDim.x) {
+    float s = 0.0f;
+    for (int t = 0; t < tiles; ++t) s = __fadd_rn(s, __ldcs(part + (size_t)t * n + i));
+    Z[i] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+  }
 }
 }  // namespace
+
+size_t linear_next_workspace(const svdq_weights* w, const svdq_weights* w2, int M) {
+  const int BN = pick_bn(w->N);
+  return (size_t)((w->N + BN - 1) / BN) * M * w2->rank * sizeof(float);
+}
 
 cudaError_t launch_linear_next(const svdq_weights* w, const svdq_weights* w2, int M,
                                const uint8_t* xq, const float* s_x, const uint16_t* Z,
                                int epilogue, uint8_t* xq2, float* s_x2, uint16_t* Z2,
-                               float* zacc, cudaStream_t st) {
+                               float* zpart, cudaStream_t st) {
   const int BN = pick_bn(w->N);
   LinMaps m;
   LinArgs a;
@@ -986,7 +1000,7 @@ cudaError_t launch_linear_next(const svdq_weights* w, const svdq_weights* w2, in
   a.inv_lambda2 = w2->d_inv_lambda;
   a.xq2 = xq2;
   a.s_x2 = s_x2;
-  a.zacc = zacc;
+  a.zpart = zpart;
   a.rank2 = w2->rank;
   a.rank2_pad = w2->rank_pad;
   a.n_l1 = w2->rank > 0 ? BN / 128 : 0;
@@ -995,15 +1009,13 @@ cudaError_t launch_linear_next(const svdq_weights* w, const svdq_weights* w2, in
     if (!make_map(&m.tl1, w2->d_L1T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w2->K, w2->rank_pad,
                   (uint64_t)w2->K * 2, 8, w2->rank_pad, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
-    cudaError_t e = cudaMemsetAsync(zacc, 0, (size_t)nz * sizeof(float), st);
-    if (e != cudaSuccess) return e;
   }
   const int tiles_m = (M + BM - 1) / BM;
   cudaError_t e = BN == 256 ? launch_ws<256, 4>(m, a, tiles_m, st) : launch_ws<128, 4>(m, a, tiles_m, st);
   if (e != cudaSuccess || nz == 0) return e;
   long long blocks = (nz + 255) / 256;
   if (blocks > 8LL * num_sms()) blocks = 8LL * num_sms();
-  zacc_to_bf16_kernel<<<(int)blocks, 256, 0, st>>>(zacc, Z2, nz);
+  zpart_sum_kernel<<<(int)blocks, 256, 0, st>>>(zpart, Z2, nz, a.tiles_n);
   return cudaGetLastError();
 }
 

@@ -111,11 +111,13 @@ cudaError_t launch_linear_nvfp4(const svdq_weights* w, int M, const uint8_t* xq,
                                 const uint8_t* sfa, const float* s_x, const uint16_t* Z,
                                 uint16_t* Y, int ldy, int epilogue, cudaStream_t stream);
 // launch_linear whose epilogue emits the next layer's activation side (codes,
-// scales, Z through the fp32 accumulator zacc of M x rank2 floats) instead of Y.
+// scales, and Z through per-column-tile fp32 partials in zpart, sized by
+// linear_next_workspace) instead of Y.
+size_t linear_next_workspace(const svdq_weights* w, const svdq_weights* w2, int M);
 cudaError_t launch_linear_next(const svdq_weights* w, const svdq_weights* w2, int M,
                                const uint8_t* xq, const float* s_x, const uint16_t* Z,
                                int epilogue, uint8_t* xq2, float* s_x2, uint16_t* Z2,
-                               float* zacc, cudaStream_t stream);
+                               float* zpart, cudaStream_t stream);
 cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq,
                             int row0, int nrows, int col0, int ncols,
                             int32_t* P, cudaStream_t stream);
