@@ -715,69 +715,53 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         const bool gelu = p.epilogue == SVDQ_EPI_GELU;
         const bool zlr = p.n_l1 > 0;
         const uint32_t xa = sbase + L::OFF_Y;
-        // pass 1: h = bf16(epi(acc + b)), kept packed, and bf16(x~) into the
-        // down-projection's A operand (chunk kc = column / 8 of the tile at
-        // kc * BM * 16 bytes, row at 16 bytes each), released to the MMA
-        // warp before the quantiser runs
-        uint32_t hb[4][CW / 8];
+        // one row and 64-column group per iteration: h = bf16(epi(acc + b)),
+        // x~ = fl32(h inv_lambda2), bf16(x~) into the down-projection's A
+        // operand (chunk kc = column / 8 of the tile at kc * BM * 16 bytes,
+        // row at 16 bytes each), then the group's codes and scale
+#pragma unroll 1
+        for (int ji = 0; ji < 4 * (CW / 64); ++ji) {
+          const int j = ji >> 2;
+          float2 a8[8];                          // acc[i][8 j + k], i = ji % 4
+          row_group(acc, ji, a8);
+          const int gcol = ncol0 + 64 * j;       // first column of the group
+          const int rl = 32 * q + r0 + 8 * (ji & 3);   // row within the tile
+          float v[16];                           // value 4 cc + 2 b2 + e: column 16 cc + 8 b2 + 2 pq + e
 #pragma unroll
-        for (int c = 0; c < CW / 16; ++c) {
+          for (int cc = 0; cc < 4; ++cc) {
 #pragma unroll
-          for (int b2 = 0; b2 < 2; ++b2) {
-            const int col = 16 * c + 8 * b2 + 2 * pq;
-            const float2 bv = *reinterpret_cast<const float2*>(bb + col);
-            const float2 lv = *reinterpret_cast<const float2*>(lb + col);
-            const uint32_t kc = (uint32_t)(h * CW + 16 * c + 8 * b2) >> 3;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              float2 y = __fadd2_rn(acc[i][2 * c + b2], bv);
+            for (int b2 = 0; b2 < 2; ++b2) {
+              const int c = 4 * j + cc;
+              const int col = 16 * c + 8 * b2 + 2 * pq;
+              const float2 bv = *reinterpret_cast<const float2*>(bb + col);
+              const float2 lv = *reinterpret_cast<const float2*>(lb + col);
+              float2 y = __fadd2_rn(a8[2 * cc + b2], bv);
               if (gelu) y = make_float2(gelu_f(y.x), gelu_f(y.y));
-              const uint32_t h2 = bf16x2_bits(y);
-              hb[i][2 * c + b2] = h2;
+              const uint32_t hb = bf16x2_bits(y);
+              const float2 xh = __fmul2_rn(
+                  make_float2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xFFFF0000u)), lv);
+              v[4 * cc + 2 * b2] = xh.x;
+              v[4 * cc + 2 * b2 + 1] = xh.y;
               if (zlr) {
-                const float2 xh = __fmul2_rn(
-                    make_float2(__uint_as_float(h2 << 16), __uint_as_float(h2 & 0xFFFF0000u)), lv);
-                sts32u(xa + kc * (BM * 16) + (32 * q + r0 + 8 * i) * 16 + 4 * pq, bf16x2_bits(xh));
+                const uint32_t kc = (uint32_t)(h * CW + 16 * c + 8 * b2) >> 3;
+                sts32u(xa + kc * (BM * 16) + rl * 16 + 4 * pq, bf16x2_bits(xh));
               }
             }
+          }
+          uint32_t u[2];
+          const float sc = quant_group16(v, u);
+          const uint32_t w0 = quad_transpose(u[0], pq), w1 = quad_transpose(u[1], pq);
+          const int row = m0 + rl;
+          if (row < p.M && gcol < p.N) {
+            *reinterpret_cast<uint2*>(p.xq2 + (size_t)row * (p.N / 2) + gcol / 2 + 8 * pq) =
+                make_uint2(w0, w1);
+            if (pq == 0) p.s_x2[(size_t)(gcol / 64) * p.M + row] = sc;
           }
         }
         if (zlr) {
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(xh_full);
-        }
-        // pass 2: x~ = fl32(h inv_lambda2) again (one exact-per-element
-        // multiply) and the codes and scale of one row and group per iteration
-#pragma unroll 1
-        for (int ji = 0; ji < 4 * (CW / 64); ++ji) {
-          const int j = ji >> 2;
-          uint32_t h8[8];                        // hb[i][8 j + k]
-          row_group(hb, ji, h8);
-          const int gcol = ncol0 + 64 * j;       // first column of the group
-          float v[16];                           // value 4 cc + 2 b2 + e: column 16 cc + 8 b2 + 2 pq + e
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-#pragma unroll
-            for (int b2 = 0; b2 < 2; ++b2) {
-              const int col = 16 * (4 * j + cc) + 8 * b2 + 2 * pq;
-              const float2 lv = *reinterpret_cast<const float2*>(lb + col);
-              const uint32_t h2 = h8[2 * cc + b2];
-              const float2 xh = __fmul2_rn(
-                  make_float2(__uint_as_float(h2 << 16), __uint_as_float(h2 & 0xFFFF0000u)), lv);
-              v[4 * cc + 2 * b2] = xh.x;
-              v[4 * cc + 2 * b2 + 1] = xh.y;
-            }
-          }
-          uint32_t u[2];
-          const float sc = quant_group16(v, u);
-          const uint32_t w0 = quad_transpose(u[0], pq), w1 = quad_transpose(u[1], pq);
-          const int row = m0 + 32 * q + r0 + 8 * (ji & 3);
-          if (row < p.M && gcol < p.N) {
-            *reinterpret_cast<uint2*>(p.xq2 + (size_t)row * (p.N / 2) + gcol / 2 + 8 * pq) =
-                make_uint2(w0, w1);
-            if (pq == 0) p.s_x2[(size_t)(gcol / 64) * p.M + row] = sc;
-          }
         }
         if (zlr) {
           // the tile's partial down-projection: 32x32b load, lane = row
