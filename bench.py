@@ -45,8 +45,8 @@ LINEAR_SOURCES = ("w4a4_quantized_gemm_smooth_b200/csrc/linear_ws.cu",
                   "w4a4_quantized_gemm_smooth_b200/csrc/gemm_common.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/ptx.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/svdq_internal.h")
-LINEAR_TRAFFIC = {"sources_sha1": "ff402fa1268b135b420a06fee3858d3f34ccbe25",
-                  "workload": "flux_qkv", "bytes": 24890880 + 29434112}
+LINEAR_TRAFFIC = {"sources_sha1": "2f7b14133f67c66d30b0b346e308367e43fb5d32",
+                  "workload": "flux_qkv", "bytes": 24905216 + 28370176}
 
 
 def _linear_traffic(workload):
