@@ -20,6 +20,12 @@
 // stage (kind::f16, bf16 operands, fp32 in TMEM) added unscaled; then the
 // bias (and GELU) are applied and Y is written once, as bf16, by TMA.
 //
+// The same kernel can instead hand its output to the next layer (MODE 4,
+// the cross-layer fusion): the epilogue quantises the bf16 tile with the
+// next layer's smoothing factors into that layer's codes and scales, and
+// one more tensor-core stage multiplies it with the next layer's L1 rows
+// for a per-tile partial of that layer's down-projection.
+//
 // Persistent CTAs (one per SM, 128 x BN output tiles, static round-robin
 // schedule); 16 warps:
 //   warp 0      TMA producer: packed A (128 rows x 64 B) and B (BN x 64 B)
