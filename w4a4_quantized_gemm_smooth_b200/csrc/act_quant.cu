@@ -172,23 +172,17 @@ __device__ __forceinline__ uint32_t e2m1_code(float x, float b, float s) {
 }
 
 // E2M1 code from u = |x| fl(1/fl(b s)), within 2^-22 (relative) of the exact
-// quotient: the grid is spaced 0.5 below 2, 1 below 4, then {4, 6}; `near`
-// is raised when u lies within 2^-18 of a midpoint (the exact path decides).
+// quotient, without branches: the grid {0, .5, 1, 1.5, 2, 3, 4, 6} maps onto
+// the integers 0..7 under the concave piecewise-linear c(u) = min(2u, u + 2,
+// u/2 + 4), so the code is rne(c) (its ties are the grid's midpoints, and
+// rne's even choice is the even code), capped at 7.  `near` is raised when
+// c lies within 2^-18 of a half below 7 (the exact path decides).
 __device__ __forceinline__ uint32_t e2m1_fast(float x, float r, bool& near) {
   const float u = fabsf(x) * r;
-  uint32_t k;
-  if (u < 2.0f) {
-    const float t = 2.0f * u, rt = rintf(t);
-    k = (uint32_t)rt;
-    near |= fabsf(t - rt) > 0.5f - 0x1p-18f;
-  } else if (u < 4.0f) {
-    const float t = u - 2.0f, rt = rintf(t);
-    k = 4u + (uint32_t)rt;
-    near |= fabsf(t - rt) > 0.5f - 0x1p-18f;
-  } else {
-    k = u <= 5.0f ? 6u : 7u;
-    near |= fabsf(u - 5.0f) < 0x1p-17f;
-  }
+  const float c = fminf(2.0f * u, fminf(u + 2.0f, __fmaf_rn(0.5f, u, 4.0f)));
+  const float rc = rintf(c);
+  near |= (fabsf(c - rc) > 0.5f - 0x1p-18f) && (c < 7.25f);
+  const uint32_t k = (uint32_t)fminf(rc, 7.0f);
   return k | ((x < 0.0f && k > 0u) ? 8u : 0u);
 }
 
