@@ -513,11 +513,12 @@ class SVDQMLP:
     """Two packed layers applied in sequence, fc2(GELU(fc1(X))), as in a
     transformer block's feed-forward part.
 
-    forward(X, fused=True) runs svdq_quantize_act(fc1), then
-    svdq_linear_quantize_next (fc1 with GELU, emitting fc2's codes, scales
-    and Z), then svdq_linear(fc2): the hidden activation never reaches device
-    memory.  fused=False runs the four plain calls, storing the bf16 hidden
-    activation H in between.  Buffers are reallocated only when M changes.
+    forward(X) runs the four plain calls, storing the bf16 hidden activation
+    H in between (the faster chain on B200).  forward(X, fused=True) runs
+    svdq_quantize_act(fc1), then svdq_linear_quantize_next (fc1 with GELU,
+    emitting fc2's codes, scales and Z), then svdq_linear(fc2): H never
+    reaches device memory, and fc2's codes and scales are the same bits.
+    Buffers are reallocated only when M changes.
     """
 
     def __init__(self, fc1: Weights, fc2: Weights):
@@ -539,7 +540,7 @@ class SVDQMLP:
             self._M = M
         return self.H, self.ws
 
-    def forward(self, X, fused: bool = True, out=None):
+    def forward(self, X, fused: bool = False, out=None):
         M = X.shape[0]
         H, ws = self.buffers(M, X.device)
         a, b = self.fc1, self.fc2
