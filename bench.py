@@ -122,7 +122,10 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # raw samples: $SVDQ_CLOCKS_DIR if set, else the system temp directory
+        import tempfile
+        d = os.environ.get("SVDQ_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(d, f"svdq_clocks_gpu{gpu_index}.csv")
 
     def start(self):
         try:
