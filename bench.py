@@ -584,10 +584,12 @@ def main():
                     help="skip the W8A8 comparator's timing")
     ap.add_argument("--no-nvfp4", action="store_true",
                     help="skip the NVFP4 variant's timing")
-    ap.add_argument("--mlp-pair", action="store_true",
-                    help="also time the FLUX feed-forward pair with and without the "
-                         "cross-layer fusion")
+    ap.add_argument("--no-mlp-pair", action="store_true",
+                    help="skip the FLUX feed-forward pair (with and without the cross-layer "
+                         "fusion)")
+    ap.add_argument("--mlp-pair", action="store_true", help=argparse.SUPPRESS)   # the default
     args = ap.parse_args()
+    args.mlp_pair = not args.no_mlp_pair
     spec = _workload(args.workload)
     if args.impl == "reference":
         run_reference(args, spec)
