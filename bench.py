@@ -45,7 +45,7 @@ LINEAR_SOURCES = ("w4a4_quantized_gemm_smooth_b200/csrc/linear_ws.cu",
                   "w4a4_quantized_gemm_smooth_b200/csrc/gemm_common.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/ptx.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/svdq_internal.h")
-LINEAR_TRAFFIC = {"sources_sha1": "f40bb0263b3f75b9f2f9ab84e37b41baec136f35",
+LINEAR_TRAFFIC = {"sources_sha1": "86e314bfcfca76a8097ed75e947da04cee8198bd",
                   "workload": "flux_qkv", "bytes": 24905216 + 28370176}
 
 

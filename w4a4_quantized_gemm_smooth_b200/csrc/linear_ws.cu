@@ -707,7 +707,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         if (lane == 0) atomicExch(p.cnt + t * N_RES_WARPS + rw, 0);   // ready for the next call
       }
       if constexpr (FUSE) {
-        // epilogue of MODE 4: h = bf16(bias (+ GELU)) exactly as the stored Y
+        // epilogue of MODE 4: h = bf16(epi(acc + bias)) exactly as the stored Y
         // would be, x~ = fl32(h inv_lambda2), the codes and scale of each of
         // the warp's 64-column groups per row, and bf16(x~) into the
         // down-projection's A operand (the Y staging area, unused here)
@@ -768,8 +768,6 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(xh_full);
-        }
-        if (zlr) {
           // the tile's partial down-projection: 32x32b load, lane = row
           const int b = tb % NB;
           if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
