@@ -1,0 +1,45 @@
+"""The library's host pack against the oracle on seeded random shapes, by
+the two-level rule for factors that any SVD may return up to sign and
+rounding: the singular values agree to 1e-10, and, given the library's own
+exported bf16 factors, the oracle's residual quantisation (eq. 10, then
+eq. 1 per group) reproduces the library's weight codes and scales bit for
+bit."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+import w4a4_quantized_gemm_smooth_b200 as S
+
+
+def _cases(n=8, seed=2024):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        K = 64 * int(rng.integers(1, 13))
+        N = 8 * int(rng.integers(2, 51))
+        rmax = min(32, (min(K, N) - 1) // 8 * 8)
+        r = 8 * int(rng.integers(0, rmax // 8 + 1))
+        alpha = float(rng.choice([0.5, 0.4, 0.6]))
+        out.append((K, N, r, alpha, 5000 + i))
+    return out
+
+
+@pytest.mark.parametrize("K,N,r,alpha,seed", _cases())
+def test_host_pack_two_level_parity(K, N, r, alpha, seed):
+    L = synth.make_layer(synth.layer_spec(f"rp{seed}", 32, K, N, r, seed, tiny=(K <= 512)))
+    a = S.svdq_calib_absmax(L.X)
+    w = S.svdq_pack_weights_host(L.W, a, r, alpha=alpha, bias_bits=L.b)
+    e = w.export()
+    W = oracle.bf16_bits_to_f64(L.W).T                              # [K, N]
+    lam = oracle.smoothing_lambda(a.astype(np.float64), np.max(np.abs(W), axis=1), alpha)
+    assert np.array_equal(e["inv_lambda"].astype(np.float64), oracle.round_f32(1.0 / lam))
+    Wt = lam[:, None] * W
+    sv = np.linalg.svd(Wt, compute_uv=False)
+    assert np.max(np.abs(e["sigma"] - sv[:r + 1]) / sv[:r + 1]) < 1e-10
+    L1b = oracle.bf16_bits_to_f64(e["L1"])[:, :r]
+    L2b = oracle.bf16_bits_to_f64(e["L2"])[:r]
+    _, codes, s_w = oracle.residual_quantize(Wt, L1b, L2b)
+    assert np.array_equal(e["wq"], oracle.pack_nibbles(codes))
+    assert np.array_equal(e["s_w"].astype(np.float64), s_w)
+    w.free()
