@@ -43,3 +43,38 @@ def test_host_pack_two_level_parity(K, N, r, alpha, seed):
     assert np.array_equal(e["wq"], oracle.pack_nibbles(codes))
     assert np.array_equal(e["s_w"].astype(np.float64), s_w)
     w.free()
+
+
+def _residual_from_library(L, a, e, r, alpha):
+    W = oracle.bf16_bits_to_f64(L.W).T
+    lam = oracle.smoothing_lambda(a.astype(np.float64), np.max(np.abs(W), axis=1), alpha)
+    assert np.array_equal(e["inv_lambda"].astype(np.float64), oracle.round_f32(1.0 / lam))
+    L1b = oracle.bf16_bits_to_f64(e["L1"])[:, :r]
+    L2b = oracle.bf16_bits_to_f64(e["L2"])[:r]
+    R, _, _ = oracle.residual_quantize(lam[:, None] * W, L1b, L2b)
+    return oracle.round_f32(R.T)
+
+
+@pytest.mark.parametrize("K,N,r,alpha,seed", _cases(6, seed=77))
+def test_w8a8_host_pack_two_level_parity(K, N, r, alpha, seed):
+    L = synth.make_layer(synth.layer_spec(f"r8{seed}", 32, K, N, r, seed, tiny=(K <= 512)))
+    a = S.svdq_calib_absmax(L.X)
+    w = S.svdq_pack_weights_w8a8(L.W, a, r, alpha=alpha, bias_bits=L.b, to_device=False)
+    e = w.export()
+    codes8, s_w8 = oracle.quantize_rows_int8(_residual_from_library(L, a, e, r, alpha))
+    assert np.array_equal(e["wq8"].astype(np.int64), codes8)
+    assert np.array_equal(e["s_w8"].astype(np.float64), s_w8)
+    w.free()
+
+
+@pytest.mark.parametrize("K,N,r,alpha,seed", _cases(6, seed=78))
+def test_nvfp4_host_pack_two_level_parity(K, N, r, alpha, seed):
+    L = synth.make_layer(synth.layer_spec(f"r4{seed}", 32, K, N, r, seed, tiny=(K <= 512)))
+    a = S.svdq_calib_absmax(L.X)
+    w = S.svdq_pack_weights_nvfp4(L.W, a, r, alpha=alpha, bias_bits=L.b, to_device=False)
+    e = w.export()
+    codes, b, s = oracle.quantize_nvfp4_rows(_residual_from_library(L, a, e, r, alpha))
+    assert np.array_equal(e["wq4"], oracle.pack_nibbles(codes))
+    assert np.array_equal(e["sf4"], oracle.e4m3_bits(b))
+    assert np.array_equal(e["s_w4"].astype(np.float64), s)
+    w.free()
