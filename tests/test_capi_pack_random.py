@@ -78,3 +78,36 @@ def test_nvfp4_host_pack_two_level_parity(K, N, r, alpha, seed):
     assert np.array_equal(e["sf4"], oracle.e4m3_bits(b))
     assert np.array_equal(e["s_w4"].astype(np.float64), s)
     w.free()
+
+
+def _gptq_cases(n=4, seed=99):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        K = 64 * int(rng.integers(1, 9))
+        N = 8 * int(rng.integers(2, 30))
+        r = 8 * int(rng.integers(0, min(4, (min(K, N) - 1) // 8) + 1))
+        out.append((K, N, r, 600 + i))
+    return out
+
+
+@pytest.mark.parametrize("K,N,r,seed", _gptq_cases())
+def test_gptq_host_pack_two_level_parity(K, N, r, seed):
+    """The calibrated pack with GPTQ rounding (one alpha, no refinement):
+    given the library's factors and the calibration Hessian, the oracle's
+    GPTQ gives the library's codes and scales bit for bit."""
+    L = synth.make_layer(synth.layer_spec(f"gq{seed}", 96, K, N, r, seed, tiny=(K <= 512)))
+    w, _ = S.svdq_pack_weights_calibrated(L.W, L.X, r, alphas=(0.5,), refine_iters=0,
+                                          bias_bits=L.b, to_device=False, gptq=True)
+    e = w.export()
+    W = oracle.bf16_bits_to_f64(L.W).T
+    a = oracle.calib_absmax(oracle.bf16_bits_to_f64(L.X))
+    lam = oracle.smoothing_lambda(a, np.max(np.abs(W), axis=1), 0.5)
+    assert np.array_equal(e["inv_lambda"].astype(np.float64), oracle.round_f32(1.0 / lam))
+    L1b = oracle.bf16_bits_to_f64(e["L1"])[:, :r]
+    L2b = oracle.bf16_bits_to_f64(e["L2"])[:r]
+    R, _, _ = oracle.residual_quantize(lam[:, None] * W, L1b, L2b)
+    codes, s_w = oracle.gptq_quantize_residual(R, oracle.gptq_hessian(L.X, e["inv_lambda"]))
+    assert np.array_equal(e["wq"], oracle.pack_nibbles(codes))
+    assert np.array_equal(e["s_w"].astype(np.float64), s_w)
+    w.free()
