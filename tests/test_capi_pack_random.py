@@ -111,3 +111,24 @@ def test_gptq_host_pack_two_level_parity(K, N, r, seed):
     assert np.array_equal(e["wq"], oracle.pack_nibbles(codes))
     assert np.array_equal(e["s_w"].astype(np.float64), s_w)
     w.free()
+
+
+@pytest.mark.parametrize("K,N,r,seed", [c for c in _gptq_cases(6, seed=101) if c[2] > 0][:4])
+def test_refined_host_pack_two_level_parity(K, N, r, seed):
+    """The calibrated pack with one alternating refinement: the library's
+    final (refined) factors give, through the oracle's residual
+    quantisation, the library's codes and scales bit for bit."""
+    L = synth.make_layer(synth.layer_spec(f"rf{seed}", 96, K, N, r, seed, tiny=(K <= 512)))
+    w, _ = S.svdq_pack_weights_calibrated(L.W, L.X, r, alphas=(0.5,), refine_iters=1,
+                                          bias_bits=L.b, to_device=False)
+    e = w.export()
+    W = oracle.bf16_bits_to_f64(L.W).T
+    a = oracle.calib_absmax(oracle.bf16_bits_to_f64(L.X))
+    lam = oracle.smoothing_lambda(a, np.max(np.abs(W), axis=1), 0.5)
+    Wt = lam[:, None] * W
+    L1b = oracle.bf16_bits_to_f64(e["L1"])[:, :r]
+    L2b = oracle.bf16_bits_to_f64(e["L2"])[:r]
+    _, codes, s_w = oracle.residual_quantize(Wt, L1b, L2b)
+    assert np.array_equal(e["wq"], oracle.pack_nibbles(codes))
+    assert np.array_equal(e["s_w"].astype(np.float64), s_w)
+    w.free()
