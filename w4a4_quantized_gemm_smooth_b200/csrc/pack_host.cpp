@@ -421,25 +421,32 @@ svdq_status gptq_factor(std::vector<double> H, int K, std::vector<double>& U) {
   mean /= K;
   for (int k = 0; k < K; ++k) H[(size_t)k * K + k] += 0.01 * mean;
   if (!cholesky_lower(H, K)) return SVDQ_ERR_NUMERIC;         // H = L L^T
-  // Linv = L^-1 (lower), column by column by forward substitution
-  std::vector<double> Linv((size_t)K * K, 0.0);
+  // Linv = L^-1 (lower), column by column by forward substitution; stored
+  // transposed (LinvT[c][i] = Linv[i][c]) so that every inner sum below runs
+  // over contiguous memory
+  std::vector<double> LinvT((size_t)K * K, 0.0);
 #pragma omp parallel for schedule(dynamic)
   for (int c = 0; c < K; ++c) {
+    double* lc = &LinvT[(size_t)c * K];
     for (int i = c; i < K; ++i) {
       double v = (i == c) ? 1.0 : 0.0;
-      for (int k = c; k < i; ++k) v -= H[(size_t)i * K + k] * Linv[(size_t)k * K + c];
-      Linv[(size_t)i * K + c] = v / H[(size_t)i * K + i];
+      const double* hi = &H[(size_t)i * K];
+      for (int k = c; k < i; ++k) v -= hi[k] * lc[k];
+      lc[i] = v / hi[i];
     }
   }
   // Hinv = Linv^T Linv (symmetric; lower triangle suffices for the next factor)
   std::vector<double> Hinv((size_t)K * K, 0.0);
 #pragma omp parallel for schedule(dynamic)
-  for (int i = 0; i < K; ++i)
+  for (int i = 0; i < K; ++i) {
+    const double* li = &LinvT[(size_t)i * K];
     for (int j = 0; j <= i; ++j) {
+      const double* lj = &LinvT[(size_t)j * K];
       double v = 0.0;
-      for (int k = i; k < K; ++k) v += Linv[(size_t)k * K + i] * Linv[(size_t)k * K + j];
+      for (int k = i; k < K; ++k) v += li[k] * lj[k];
       Hinv[(size_t)i * K + j] = v;
     }
+  }
   if (!cholesky_lower(Hinv, K)) return SVDQ_ERR_NUMERIC;       // Hinv = L2 L2^T
   U.assign((size_t)K * K, 0.0);
   for (int i = 0; i < K; ++i)
@@ -469,37 +476,63 @@ std::vector<double> gptq_hessian(int K, const uint16_t* X, int M, int ldx,
 // The residual R = W~ - L1b L2b, then GPTQ per output column (the columns
 // are independent): on entering a group of 64 the eq. 1 scale comes from the
 // updated group; channel k's error (w - q s) / U_kk moves the later channels
-// by U_kj.
+// by U_kj.  Columns are taken in batches of GPTQ_NB so that each row of U is
+// read once per batch (the loop over a batch's columns is innermost); every
+// column sees exactly the operations, in the same order, of a column-by-
+// column loop.
+constexpr int GPTQ_NB = 16;
 void gptq_residual(int K, int N, int rank, const std::vector<double>& U, Candidate& c) {
   const int G = K / SVDQ_GROUP;
   c.sw.assign((size_t)G * N, 0.0f);
   c.wq.assign((size_t)N * K / 2, 0);
+  const int nbat = (N + GPTQ_NB - 1) / GPTQ_NB;
 #pragma omp parallel for schedule(dynamic)
-  for (int n = 0; n < N; ++n) {
-    std::vector<double> r(K);
-    for (int k = 0; k < K; ++k) {
-      double v = c.Wt[(size_t)k * N + n];
-      for (int j = 0; j < rank; ++j)
-        v -= bf16_to_f64(c.L1[(size_t)k * rank + j]) * bf16_to_f64(c.L2[(size_t)j * N + n]);
-      r[k] = v;
-    }
-    std::vector<int8_t> q(K);
-    float s = 0.0f;
+  for (int bi = 0; bi < nbat; ++bi) {
+    const int n0 = bi * GPTQ_NB;
+    const int nb = N - n0 < GPTQ_NB ? N - n0 : GPTQ_NB;
+    std::vector<double> r((size_t)K * GPTQ_NB, 0.0);    // r[k][b]
+    for (int k = 0; k < K; ++k)
+      for (int b = 0; b < nb; ++b) {
+        double v = c.Wt[(size_t)k * N + n0 + b];
+        for (int j = 0; j < rank; ++j)
+          v -= bf16_to_f64(c.L1[(size_t)k * rank + j]) * bf16_to_f64(c.L2[(size_t)j * N + n0 + b]);
+        r[(size_t)k * GPTQ_NB + b] = v;
+      }
+    std::vector<int8_t> q((size_t)GPTQ_NB * K);
+    float s[GPTQ_NB] = {};
+    double err[GPTQ_NB] = {};
     for (int k = 0; k < K; ++k) {
       if (k % SVDQ_GROUP == 0) {
-        float m = 0.0f;
-        for (int i = 0; i < SVDQ_GROUP; ++i) m = std::fmax(m, std::fabs((float)r[k + i]));
-        s = m / 7.0f;
-        c.sw[(size_t)(k / SVDQ_GROUP) * N + n] = s;
+        for (int b = 0; b < nb; ++b) {
+          float m = 0.0f;
+          for (int i = 0; i < SVDQ_GROUP; ++i)
+            m = std::fmax(m, std::fabs((float)r[(size_t)(k + i) * GPTQ_NB + b]));
+          s[b] = m / 7.0f;
+          c.sw[(size_t)(k / SVDQ_GROUP) * N + n0 + b] = s[b];
+        }
       }
-      const int qk = s > 0.0f ? code_of((double)(float)r[k], (double)s) : 0;
-      q[k] = (int8_t)qk;
-      const double err = (r[k] - (double)qk * (double)s) / U[(size_t)k * K + k];
+      const double ukk = U[(size_t)k * K + k];
+      for (int b = 0; b < nb; ++b) {
+        const double rk = r[(size_t)k * GPTQ_NB + b];
+        const int qk = s[b] > 0.0f ? code_of((double)(float)rk, (double)s[b]) : 0;
+        q[(size_t)b * K + k] = (int8_t)qk;
+        err[b] = (rk - (double)qk * (double)s[b]) / ukk;
+      }
+      for (int b = nb; b < GPTQ_NB; ++b) err[b] = 0.0;
       const double* urow = &U[(size_t)k * K];
-      for (int j = k + 1; j < K; ++j) r[j] -= urow[j] * err;
+      for (int j = k + 1; j < K; ++j) {
+        const double u = urow[j];
+        double* rj = &r[(size_t)j * GPTQ_NB];
+#pragma omp simd
+        for (int b = 0; b < GPTQ_NB; ++b) rj[b] -= u * err[b];
+      }
     }
-    uint8_t* dst = &c.wq[(size_t)n * (K / 2)];
-    for (int b = 0; b < K / 2; ++b) dst[b] = (uint8_t)((q[2 * b] & 0xF) | ((q[2 * b + 1] & 0xF) << 4));
+    for (int b = 0; b < nb; ++b) {
+      uint8_t* dst = &c.wq[(size_t)(n0 + b) * (K / 2)];
+      const int8_t* qb = &q[(size_t)b * K];
+      for (int t = 0; t < K / 2; ++t)
+        dst[t] = (uint8_t)((qb[2 * t] & 0xF) | ((qb[2 * t + 1] & 0xF) << 4));
+    }
   }
 }
 
