@@ -568,7 +568,7 @@ def run_ours(args, spec):
                                             4.0 * bf16_burst)
     if extras and args.mlp_pair:
         line["cross_layer_fusion"] = _time_mlp_pair(S, flush, stream, args.steps)
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:      # at N = 1 only
         line["cpu_baseline"] = cpu_baseline(spec)
     if rank == 0:
         print(json.dumps(line), flush=True)
