@@ -2,23 +2,22 @@
 // 6.1, product side; eq. 7), warp-specialised for sm_100a.
 //
 // sm_100a tensor cores have no 4-bit integer kind, so the packed codes are
-// streamed by TMA into shared memory, expanded there to int8 (as 16 q, three
-// integer ops per 8 codes) and multiplied with tcgen05.mma.kind::i8 into
-// int32 TMEM accumulators, one per group of 64 K.  Each group's accumulator
-// is first set by a bf16 MMA (ones x 786432) to the fp32 value 12582912,
-// whose bit pattern is the int32 0x4B400000; the int8 MMAs then add 256 P_g
-// to those bits, so the word read back is exactly the float
-// 12582912 + 256 P_g (|256 P_g| <= 2^20).  The rescale is two fmas per
-// element and no int32 -> fp32 conversion: v = fma(word, s_w, c) with
-// c = -fl32(12582912 s_w) (one multiply per column pair, shared by the
-// thread's four rows), i.e. v = 256 P_g s_w rounded once after adding the
-// constant's own rounding residual (at most 0.75 s_w, about 1e-4 of a
-// typical term), then acc = fma(v, 2^-8 s_x, acc).  Only s_w is read from
-// shared memory: a broadcast 128-bit load costs four wavefronts whatever
-// the number of distinct addresses, so scale loads are the rescale's
-// largest shared-memory cost.  The low-rank term Z L2 is one more tensor-core
-// stage (kind::f16, bf16 operands, fp32 in TMEM) added unscaled; then the
-// bias (and GELU) are applied and Y is written once, as bf16, by TMA.
+// streamed by TMA into shared memory and expanded there to one byte per code
+// for tcgen05.mma.kind::f8f6f4 with E4M3 operands: a code q becomes the E4M3
+// number q * 2^-9, i.e. the byte sign << 7 | |q| (|q| <= 7 are the format's
+// subnormals m * 2^-9; |q| = 8 is its smallest normal 2^-6, bit pattern 0x08
+// again).  Every product is then an integer times 2^-18 and every sum of a
+// group of 64 is P_g 2^-18 with |P_g| <= 4096, so the fp32 TMEM accumulator
+// holds each group's integer partial exactly and needs no conversion.  The
+// activation codes arrive as two's-complement nibbles (the public layout);
+// the weight codes are stored on the device as sign-magnitude nibbles (a
+// layer with a code of -8, which only a subnormal scale can produce, keeps
+// two's complement and the longer conversion).  The device copy of the weight
+// scales holds s_w 2^18 (exact), so the rescale is plain fp32 arithmetic, two
+// operations per element and group: v = fl32(P_g s_w), acc = fl32(acc +
+// v s_x).  The low-rank term Z L2 is one more tensor-core stage (kind::f16,
+// bf16 operands, fp32 in TMEM) added unscaled; then the bias (and GELU) are
+// applied and Y is written once, as bf16, by TMA.
 //
 // The same kernel can instead hand its output to the next layer (MODE 4,
 // the cross-layer fusion): the epilogue quantises the bf16 tile with the
@@ -35,8 +34,8 @@
 //               slices of the low-rank stage (loaded straight into UMMA
 //               layout);
 //   warp 1      TMEM owner and MMA issuer (one thread);
-//   warps 2-7   expanders: packed nibbles -> int8 in the UMMA K-major
-//               layout (2-stage ring);
+//   warps 2-7   expanders: packed nibbles -> E4M3 bytes in the UMMA
+//               K-major layout (2-stage ring);
 //   warps 8-15  rescale + epilogue: warp w owns TMEM lanes 32 (w % 4).. and
 //               BN/2 columns; double-buffered TMEM lets group g+1 run on
 //               the tensor cores while group g is rescaled.
@@ -55,6 +54,8 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "gemm_common.cuh"
 #include "ptx.cuh"
 #include "quant_common.cuh"
@@ -69,9 +70,7 @@ constexpr int THREADS = 512;
 constexpr int N_EXP = 192;       // expanders: warps 2-7
 constexpr int RES_WARP0 = 8;     // rescale / epilogue: warps 8-15
 constexpr int N_RES_WARPS = 8;
-constexpr uint32_t MAGIC_BITS = 0x4B400000u;   // bits of 12582912.0f = 1.5 * 2^23
-constexpr uint16_t BF16_ONE = 0x3F80;          // 1.0
-constexpr uint16_t BF16_MAGIC16 = 0x4940;      // 786432 = 1.5 * 2^19; 16 of them make the bias
+constexpr float P_SCALE = 262144.0f;           // 2^18: a group's TMEM word times this is P_g
 // Register split after launch: the first two warpgroups (producer, MMA,
 // expanders) give registers to the two rescale warpgroups.
 // 256 * REG_LO + 256 * REG_HI
@@ -93,6 +92,7 @@ struct LinArgs {
   int epilogue;
   int tiles_n, num_tiles, tile_m0, tile_n0;
   int* err;
+  int b_twos;              // 1: weight codes in two's complement (else sign-magnitude)
   int sx_tma;              // 1: s_x rows are 16-byte aligned (M % 4 == 0), copy by TMA
   int32_t* P;              // partial dump (MODE 1)
   int row0, nrows, col0, ncols;
@@ -157,10 +157,7 @@ struct Lay {
   static constexpr int OFF_BIAS = OFF_SC + NS * SC_SLOT;   // per warp CW floats
   // MODE 4: the next layer's smoothing factors of the warp's columns
   static constexpr int OFF_ILAM = OFF_BIAS + N_RES_WARPS * CW * 4;
-  // constant operands of the accumulator-initialising bf16 MMA (K = 16)
-  static constexpr int INIT_A = BM * 32, INIT_B = BN * 32;
-  static constexpr int OFF_INIT = OFF_ILAM + N_RES_WARPS * CW * 4;
-  static constexpr int OFF_BAR = OFF_INIT + INIT_A + INIT_B;
+  static constexpr int OFF_BAR = OFF_ILAM + N_RES_WARPS * CW * 4;
   // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[NB],
   // tm_empty[NB], lr_full[NLR], lr_empty[NLR], xh_full
   static constexpr int N_BARS = 2 * NP + 2 * NE + 2 * NB + 2 * NLR + 1;
@@ -197,59 +194,79 @@ __device__ __forceinline__ void sts32u(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// 16 packed bytes (32 codes of one row: the first or second half of the
-// group) -> two 16-byte core-matrix rows at d and d + 128.
-// Each code q becomes the int8 16*q: the high nibble of a byte is already
-// 16*q in place (mask), the low nibble is moved up by 4 (a funnel rotate,
-// whose wrapped-around bits the mask removes).
-// Products are 256 q_x q_w, so the int32 group sum is 256 P_g (|256 P_g| <=
-// 2^20, exact); the factor 2^-8 is folded into the scale.
-__device__ __forceinline__ uint32_t rotl4(uint32_t x) {
-  uint32_t y;
-  asm("shf.l.wrap.b32 %0, %1, %1, 4;" : "=r"(y) : "r"(x));
-  return y;
+// Codes -> E4M3 bytes, four at a time (one byte each of a 32-bit word).
+// Two's complement: x holds four nibbles 0..15, y the same nibbles in the
+// high half of each byte (bit 7 = the code's sign).  A negative code q = x - 16
+// becomes (x ^ 0x8F) + 1 = 0x80 | (16 - x) = 0x80 | |q|, with no carry out of
+// its byte (|q| <= 8); the sign masks come from one byte permute in
+// sign-replicating mode.
+__device__ __forceinline__ uint32_t e4m3_twos(uint32_t x, uint32_t y) {
+  uint32_t m;
+  asm("prmt.b32 %0, %1, 0, 0xBA98;" : "=r"(m) : "r"(y));
+  return (x ^ (m & 0x8F8F8F8Fu)) + (m & 0x01010101u);
 }
-__device__ __forceinline__ void expand16(uint32_t src, uint32_t d) {
+// The low (even-k) and high (odd-k) nibbles of four packed bytes.
+template <bool TWOS>
+__device__ __forceinline__ uint32_t e4m3_lo(uint32_t w) {
+  if (TWOS) return e4m3_twos(w & 0x0F0F0F0Fu, w << 4);
+  return (w & 0x07070707u) | ((w << 4) & 0x80808080u);     // sign-magnitude: s << 7 | m
+}
+template <bool TWOS>
+__device__ __forceinline__ uint32_t e4m3_hi(uint32_t w) {
+  if (TWOS) return e4m3_twos((w >> 4) & 0x0F0F0F0Fu, w);
+  return ((w >> 4) & 0x07070707u) | (w & 0x80808080u);
+}
+// 16 packed bytes (32 codes of one row: the first or second half of the
+// group) -> two 16-byte core-matrix rows at d and d + 128.  Inside every 8
+// codes the even-k codes come first.
+template <bool TWOS>
+__device__ __forceinline__ void expand_e4m3(uint32_t src, uint32_t d) {
   const uint4 p = lds128u(src);
   uint4 o0, o1;
-  o0.x = rotl4(p.x) & 0xF0F0F0F0u;
-  o0.y = p.x & 0xF0F0F0F0u;
-  o0.z = rotl4(p.y) & 0xF0F0F0F0u;
-  o0.w = p.y & 0xF0F0F0F0u;
-  o1.x = rotl4(p.z) & 0xF0F0F0F0u;
-  o1.y = p.z & 0xF0F0F0F0u;
-  o1.z = rotl4(p.w) & 0xF0F0F0F0u;
-  o1.w = p.w & 0xF0F0F0F0u;
+  o0.x = e4m3_lo<TWOS>(p.x);
+  o0.y = e4m3_hi<TWOS>(p.x);
+  o0.z = e4m3_lo<TWOS>(p.y);
+  o0.w = e4m3_hi<TWOS>(p.y);
+  o1.x = e4m3_lo<TWOS>(p.z);
+  o1.y = e4m3_hi<TWOS>(p.z);
+  o1.z = e4m3_lo<TWOS>(p.w);
+  o1.w = e4m3_hi<TWOS>(p.w);
   sts128(d, o0);
   sts128(d + 128, o1);
 }
 
-// The expanders' share of one group: CNT rounds of 32 consecutive 16-byte
-// units starting at round R0.  Unit j of an operand is half (j >> 3) & 1 of
-// row 8 (j >> 4) + (j & 7), so each quarter-warp reads one half of eight
-// consecutive rows (eight distinct 16-byte bank groups under the 64-byte
-// swizzle) and writes 128 contiguous bytes.  Offsets are fixed per thread
-// and computed once.
-template <int BN, int CNT>
+// The expanders' share of one group: NA rounds of 32 consecutive 16-byte
+// units of A (activation codes) from round A0 and NB rounds of B (weight
+// codes) from round B0 of that operand.  Unit j of an operand is half
+// (j >> 3) & 1 of row 8 (j >> 4) + (j & 7), so each quarter-warp reads one
+// half of eight consecutive rows (eight distinct 16-byte bank groups under
+// the 64-byte swizzle) and writes 128 contiguous bytes.  Offsets are fixed
+// per thread and computed once.
+template <int BN, int NA, int NB>
 struct ExpandPlan {
+  static constexpr int CNT = NA + NB;
   uint32_t src[CNT], dst[CNT];
-  __device__ __forceinline__ ExpandPlan(int r0, int lane) {
+  __device__ __forceinline__ ExpandPlan(int a0, int b0, int lane) {
     using L = Lay<BN>;
 #pragma unroll
     for (int k = 0; k < CNT; ++k) {
-      const int u = 32 * (r0 + k) + lane;
-      const bool isa = u < BM * 2;
-      const int j = isa ? u : u - BM * 2;
+      const bool isa = k < NA;
+      const int j = 32 * (isa ? a0 + k : b0 + k - NA) + lane;
       const int hf = (j >> 3) & 1, row = ((j >> 4) << 3) | (j & 7);
       // group 0 of the stage; group 1 is chunk + 2, i.e. the offset ^ 32
       src[k] = (isa ? 0 : L::PK_A) + row * 64 + ((hf ^ ((row >> 1) & 3)) << 4);
       dst[k] = (isa ? 0 : L::EX_A) + (row >> 3) * 512 + (row & 7) * 16 + hf * 256;
     }
   }
-  // gsx = 32 * (group within the packed stage)
+  // gsx = 32 * (group within the packed stage); activation codes are two's
+  // complement, weight codes too when BTWOS
+  template <bool BTWOS>
   __device__ __forceinline__ void run(uint32_t pa, uint32_t ea, uint32_t gsx) const {
 #pragma unroll
-    for (int k = 0; k < CNT; ++k) expand16(pa + (src[k] ^ gsx), ea + dst[k]);
+    for (int k = 0; k < CNT; ++k) {
+      if (k < NA || BTWOS) expand_e4m3<true>(pa + (src[k] ^ gsx), ea + dst[k]);
+      else expand_e4m3<false>(pa + (src[k] ^ gsx), ea + dst[k]);
+    }
   }
 };
 
@@ -314,13 +331,6 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     mbar_init(xh_full, N_RES_WARPS);
     *abort_flag = 0;
     fence_mbarrier_init();
-  }
-  {
-    uint32_t* ia = reinterpret_cast<uint32_t*>(smem + L::OFF_INIT);
-    const uint32_t one2 = (uint32_t)BF16_ONE * 0x10001u, mag2 = (uint32_t)BF16_MAGIC16 * 0x10001u;
-    for (int i = tid; i < (L::INIT_A + L::INIT_B) / 4; i += THREADS)
-      ia[i] = (i < L::INIT_A / 4) ? one2 : mag2;
-    fence_proxy_async_smem();
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -421,10 +431,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     } else if (warp == 1) {
       // ---------------------------------------------------- MMA issuer
       if (lane == 0) {
-        const uint32_t id_i8 = idesc_i8(BM, BN), id_bf = idesc_bf16(BM, BN);
-        // the constant tiles hold one value each, so any layout descriptor works
-        const uint64_t init_ad = sdesc_kmajor_noswizzle(sbase + L::OFF_INIT, 128, 256);
-        const uint64_t init_bd = sdesc_kmajor_noswizzle(sbase + L::OFF_INIT + L::INIT_A, 128, 256);
+        const uint32_t id_f8 = idesc_e4m3(BM, BN), id_bf = idesc_bf16(BM, BN);
         uint32_t ite = 0, tb = 0, il = 0, ixh = 0;
         for (int wk = blockIdx.x; wk < p.num_tiles * p.splits; wk += gridDim.x) {
           const WorkItem wi = work_item(p, wk);
@@ -440,9 +447,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               const uint32_t ea = sbase + L::OFF_EX + s * L::EX_STAGE;
               const uint64_t ad = sdesc_kmajor_noswizzle(ea, 128, 512);
               const uint64_t bd = sdesc_kmajor_noswizzle(ea + L::EX_A, 128, 512);
-              mma_bf16(d, init_ad, init_bd, id_bf, 0u);   // D = 12582912.0f
-              mma_i8(d, ad, bd, id_i8, 1u);
-              mma_i8(d, ad + 16, bd + 16, id_i8, 1u);
+              mma_f8f6f4(d, ad, bd, id_f8, 0u);          // D = P_g 2^-18, K = 0..31
+              mma_f8f6f4(d, ad + 16, bd + 16, id_f8, 1u);  // K = 32..63
               mma_commit(ex_empty(s));
               ++ite;
             } else {
@@ -495,13 +501,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       __syncwarp();
     } else {
       // ---------------------------------------------------- expanders
-      // Warps 4 and 5 sit alone on their SM sub-partitions (with the producer
-      // and the MMA issuer); warps 2+6 and 3+7 share theirs.  Each
-      // sub-partition gets a quarter of the units, so the rescale warps next
-      // to them are slowed alike.
-      constexpr int ROUNDS = (BM + BN) * 2 / 32;
-      static_assert(ROUNDS % 8 == 0, "expander split");
-      auto expand_loop = [&](const auto& plan) {
+      auto expand_loop = [&](const auto& plan, auto btwos) {
+        constexpr bool BT = decltype(btwos)::value;
         uint32_t ist = 0, it = 0;            // packed stages, groups
         for (int wk = blockIdx.x; wk < p.num_tiles * p.splits; wk += gridDim.x) {
           const WorkItem wi = work_item(p, wk);
@@ -512,8 +513,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             for (int k = 0; k < ng; ++k, ++it) {
               const int se = it % NE;
               if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err)) return;
-              plan.run(sbase + L::OFF_PK + sp * L::PK_STAGE, sbase + L::OFF_EX + se * L::EX_STAGE,
-                       32u * k);
+              plan.template run<BT>(sbase + L::OFF_PK + sp * L::PK_STAGE,
+                                    sbase + L::OFF_EX + se * L::EX_STAGE, 32u * k);
               fence_proxy_async_smem();
               mbar_arrive(ex_full(se));
             }
@@ -521,13 +522,24 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
           }
         }
       };
+      auto expand_share = [&](const auto& plan) {
+        if (p.b_twos) expand_loop(plan, std::true_type{});
+        else expand_loop(plan, std::false_type{});
+      };
+      // Each SM sub-partition gets the same expansion cost: a round of A
+      // (two's-complement conversion) costs about twice a round of B
+      // (sign-magnitude).  Warps 4 and 5 sit alone on their sub-partitions
+      // (beside the producer and the MMA issuer) and take two rounds of A and
+      // a quarter of B each; warps 2, 6 and 3, 7 share theirs and take one
+      // round of A and an eighth of B each.
+      constexpr int AR = BM * 2 / 32, BR = BN * 2 / 32;
+      static_assert(AR == 8 && BR % 8 == 0, "expander split");
       if (warp == 4 || warp == 5) {
-        const ExpandPlan<BN, ROUNDS / 4> plan((warp - 4) * (ROUNDS / 4), lane);
-        expand_loop(plan);
+        const int i = warp - 4;
+        expand_share(ExpandPlan<BN, 2, BR / 4>(2 * i, (BR / 4) * i, lane));
       } else {
         const int slot_i = (warp & 3) - 2 + 2 * ((warp >> 2) & 1);   // warps 2,3,6,7 -> 0,1,2,3
-        const ExpandPlan<BN, ROUNDS / 8> plan(ROUNDS / 2 + slot_i * (ROUNDS / 8), lane);
-        expand_loop(plan);
+        expand_share(ExpandPlan<BN, 1, BR / 8>(4 + slot_i, BR / 2 + (BR / 8) * slot_i, lane));
       }
     }
   } else {
@@ -577,7 +589,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
           float2 sx2[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float v = lds32(slot + 4u * (32 * q + r0 + 8 * i)) * 0.00390625f;  // 2^-8 (exact)
+            const float v = lds32(slot + 4u * (32 * q + r0 + 8 * i));
             sx2[i] = make_float2(v, v);
           }
           const uint32_t swa = slot + 4u * (BM + h * CW) + 16u * pq;
@@ -606,14 +618,13 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
 #pragma unroll
               for (int bb = 0; bb < 2; ++bb) {
                 const float2 sw2 = bb ? make_float2(s4.z, s4.w) : make_float2(s4.x, s4.y);
-                const float2 cc2 = __fmul2_rn(sw2, make_float2(-SVDQ_ACC_BIAS, -SVDQ_ACC_BIAS));
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                   // register of row r0 + 8i: half (i >> 1), row (i & 1) of the 16-lane load
                   const uint32_t* wv = r + 8 * (i >> 1) + 4 * bb + 2 * (i & 1);
-                  // the word is the float SVDQ_ACC_BIAS + 256 P_g: v ~ 256 P_g s_w
-                  const float2 v = __ffma2_rn(make_float2(__uint_as_float(wv[0]), __uint_as_float(wv[1])),
-                                              sw2, cc2);
+                  // the word is P_g 2^-18 and sw2 holds s_w 2^18: v = fl32(P_g s_w)
+                  const float2 v = __fmul2_rn(make_float2(__uint_as_float(wv[0]), __uint_as_float(wv[1])),
+                                              sw2);
                   acc[i][2 * c + bb] = __ffma2_rn(v, sx2[i], acc[i][2 * c + bb]);
                 }
               }
@@ -632,7 +643,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               for (int j = 0; j < 16; ++j) {
                 const int jj = ncol0 + 16 * c + j - p.col0;
                 if (jj >= 0 && jj < p.ncols)
-                  p.P[((size_t)g * p.nrows + i) * p.ncols + jj] = ((int32_t)(r[j] - MAGIC_BITS)) >> 8;
+                  p.P[((size_t)g * p.nrows + i) * p.ncols + jj] =
+                      __float2int_rn(__uint_as_float(r[j]) * P_SCALE);   // exact
               }
             }
           }
@@ -917,6 +929,7 @@ bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* 
   a.tiles_n = (w->N + BN - 1) / BN;
   a.tile_m0 = 0; a.tile_n0 = 0;
   a.err = w->d_err;
+  a.b_twos = w->wq_twos ? 1 : 0;
   a.sx_tma = sx_tma ? 1 : 0;
   a.splits = 1;
   return true;
@@ -993,6 +1006,7 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
   a.rank = 0; a.rank_pad32 = 0; a.n_lr = 0; a.epilogue = 0;
   a.splits = 1;
   a.err = w->d_err;
+  a.b_twos = w->wq_twos ? 1 : 0;
   a.P = P; a.row0 = row0; a.nrows = nrows; a.col0 = col0; a.ncols = ncols;
   const int tm0 = row0 / BM, tm1 = (row0 + nrows - 1) / BM;
   const int tn0 = col0 / BN, tn1 = (col0 + ncols - 1) / BN;

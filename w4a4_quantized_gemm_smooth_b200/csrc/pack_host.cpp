@@ -220,12 +220,31 @@ svdq_status upload(svdq_weights* w, cudaStream_t st) {
     if ((s = dev_alloc_copy(&w->d_wq8, w->wq8.data(), (size_t)N * K, st))) return s;
     if ((s = dev_alloc_copy(&w->d_sw8, sw8p.data(), sw8p.size(), st))) return s;
   } else {
-    if ((s = dev_alloc_copy(&w->d_wq, w->wq.data(), (size_t)N * K / 2, st))) return s;
+    // device codes: sign-magnitude nibbles unless some code is -8
+    const size_t nb = (size_t)N * K / 2;
+    w->wq_twos = false;
+    for (size_t i = 0; i < nb && !w->wq_twos; ++i)
+      w->wq_twos = (w->wq[i] & 0x0F) == 0x08 || (w->wq[i] & 0xF0) == 0x80;
+    std::vector<uint8_t> wqd(w->wq);
+    if (!w->wq_twos) {
+      for (size_t i = 0; i < nb; ++i) {
+        uint8_t out = 0;
+        for (int h = 0; h < 2; ++h) {
+          const int q = (int)(int8_t)(uint8_t)(((w->wq[i] >> (4 * h)) & 0x0F) << 4) >> 4;
+          const uint8_t n = (uint8_t)((q < 0 ? 8 : 0) | (q < 0 ? -q : q));
+          out |= (uint8_t)(n << (4 * h));
+        }
+        wqd[i] = out;
+      }
+    }
+    if ((s = dev_alloc_copy(&w->d_wq, wqd.data(), nb, st))) return s;
     std::vector<float> swp((size_t)G * w->N16, 0.0f);
     for (int g = 0; g < G; ++g)
       for (int n = 0; n < N; ++n) {
         const int c = n & 15, pos = (n & ~15) + 4 * ((c & 7) >> 1) + 2 * (c >> 3) + (c & 1);
-        swp[(size_t)g * w->N16 + pos] = w->sw[(size_t)g * N + n];
+        const double v = (double)w->sw[(size_t)g * N + n];
+        if (!(v < SVDQ_SW_LIMIT)) return SVDQ_ERR_NUMERIC;
+        swp[(size_t)g * w->N16 + pos] = (float)std::ldexp(v, 18);   // exact
       }
     if ((s = dev_alloc_copy(&w->d_sw, swp.data(), swp.size(), st))) return s;
   }

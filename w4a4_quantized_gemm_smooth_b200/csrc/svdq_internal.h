@@ -20,8 +20,13 @@ struct svdq_weights {
   int format = SVDQ_FORMAT_W4A4;   // residual / activation number format
   // device copies (owned)
   float* d_inv_lambda = nullptr;   // [K]
-  uint8_t* d_wq = nullptr;         // [N][K/2] packed residual codes
-  // [G][N16], zero padded; inside each block of 16 columns, column
+  // [N][K/2] packed residual codes, two per byte (even k low); each nibble is
+  // sign << 3 | |q| (the GEMM's cheap E4M3 expansion), or the code in two's
+  // complement when the layer holds a -8 (wq_twos)
+  uint8_t* d_wq = nullptr;
+  bool wq_twos = false;
+  // [G][N16] weight scales times 2^18 (exact; the GEMM's group sums arrive as
+  // P_g 2^-18), zero padded; inside each block of 16 columns, column
   // 8b + 2p + e is stored at 4p + 2b + e, so that the rescale thread that owns
   // the column pairs 2p, 2p+1 of both 8-column halves reads them as one float4
   float* d_sw = nullptr;
@@ -51,10 +56,11 @@ struct svdq_weights {
   std::vector<double> sigma;       // [svd_rank + 1]
 };
 
-// The GEMM's int32 group accumulators start from the float 1.5 * 2^23 (bit
-// pattern 0x4B400000), so the word read back is the float SVDQ_ACC_BIAS +
-// 256 P_g; the rescale removes the bias with c = -fl32(SVDQ_ACC_BIAS s_w).
-constexpr float SVDQ_ACC_BIAS = 12582912.0f;
+// The W4A4 GEMM multiplies E4M3 operands holding q 2^-9 and receives each
+// group sum as P_g 2^-18; the device weight scales carry the factor 2^18.
+// Scales at or above this bound would overflow (a residual group maximum
+// above 7 * 2^110, about 9e33) and are rejected by the pack.
+constexpr double SVDQ_SW_LIMIT = 1.2980742146337069e33;   // 2^110
 
 // Device error word values.
 enum { SVDQ_DEVERR_NONE = 0, SVDQ_DEVERR_TIMEOUT = 1 };
