@@ -37,10 +37,13 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "svdq_linear effective TOPS (2MNK/s) at FLUX-like shapes; % int8 roofline"
+# minimum span of the clock record around the timed steps (seconds)
+CLOCK_WINDOW_S = 0.6
 
-# DRAM bytes (read + write) of one svdq_linear launch on this workload, from
-# the ncu capture summarised in profiles/svdq_linear_flux_qkv.md, valid only
-# for the kernel sources it was taken on (SHA-1 over the files below).
+# DRAM bytes (read + write) of one svdq_linear launch on this workload, from a
+# one-kernel, one-launch ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum), valid only for the kernel sources it was taken on
+# (SHA-1 over the files below); null otherwise.
 LINEAR_SOURCES = ("w4a4_quantized_gemm_smooth_b200/csrc/linear_ws.cu",
                   "w4a4_quantized_gemm_smooth_b200/csrc/gemm_common.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/ptx.cuh",
@@ -211,13 +214,24 @@ def cpu_oracle_step(st):
 
 
 def cpu_baseline(spec, reps=3):
+    """The oracle on the host's cores (BLAS threads as configured), and the
+    same sample on one thread."""
     st = cpu_oracle_setup(spec)
     cpu_oracle_step(st)
     ts = [cpu_oracle_step(st) for _ in range(reps)]
     t = statistics.median(ts)
     ops = 2.0 * st["rows"] * st["cols"] * st["K"]
-    return {"value": ops / t / 1e12, "unit": "TOPS", "cores": _blas_threads(),
-            "kind": "oracle", "sample": st["sample"], "seconds_per_sample": t}
+    out = {"value": ops / t / 1e12, "unit": "TOPS", "cores": _blas_threads(),
+           "kind": "oracle", "sample": st["sample"], "seconds_per_sample": t}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1, user_api="blas"):
+            t1 = cpu_oracle_step(st)
+        out["one_thread"] = {"value": ops / t1 / 1e12, "unit": "TOPS", "cores": 1,
+                             "seconds_per_sample": t1}
+    except Exception:
+        pass
+    return out
 
 
 def run_reference(args, spec):
@@ -251,37 +265,54 @@ def _to_dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def _time_steps(fn, steps, flush, stream):
-    """Per-step CUDA events (flush outside them); returns per-phase totals."""
+def _time_steps(fn, steps, flush, stream, per_step=False):
+    """Per-step CUDA events on the launching stream; `flush` (a buffer larger
+    than L2, or None for an L2-warm run) is written before every step,
+    outside the events.  Returns per-phase totals in ms, or per-step phase
+    times when per_step."""
     import torch
     evs = []
     for i in range(steps):
-        flush.fill_(i & 0xFF)
+        if flush is not None:
+            flush.fill_(i & 0xFF)
         marks = [torch.cuda.Event(enable_timing=True) for _ in range(fn.n_phases + 1)]
         fn(marks, stream)
         evs.append(marks)
     torch.cuda.synchronize()
-    tot = [0.0] * fn.n_phases
-    for marks in evs:
-        for j in range(fn.n_phases):
-            tot[j] += marks[j].elapsed_time(marks[j + 1])
-    return tot   # ms
+    rows = [[m[j].elapsed_time(m[j + 1]) for j in range(fn.n_phases)] for m in evs]
+    if per_step:
+        return rows
+    return [sum(r[j] for r in rows) for j in range(fn.n_phases)]   # ms
+
+
+def _dist_stats(xs):
+    """Median, 10th and 90th percentile (µs) of per-step times given in ms."""
+    v = np.asarray(xs, dtype=np.float64) * 1e3
+    return {"median_us": float(np.median(v)), "p10_us": float(np.percentile(v, 10)),
+            "p90_us": float(np.percentile(v, 90))}
 
 
 class _Step:
-    """quantize_act then linear, with an event between the two kernels."""
+    """quantize_act then linear, with an event between the two kernels.  With
+    a workspace the product is svdq_linear_splitk at the automatic split
+    (batches whose output tiles cannot fill the GPU)."""
     n_phases = 2
 
-    def __init__(self, S, w, X, bufs, epi):
+    def __init__(self, S, w, X, bufs, epi, workspace=None):
         self.S, self.w, self.X, self.epi = S, w, X, epi
         self.xq, self.s_x, self.Z, self.Y = bufs
+        self.ws = workspace
 
     def __call__(self, marks, stream):
         S = self.S
         marks[0].record(stream)
         S.svdq_quantize_act(self.w, self.X, self.xq, self.s_x, self.Z, stream)
         marks[1].record(stream)
-        S.svdq_linear(self.w, self.xq, self.s_x, self.Z, self.Y, self.epi, stream)
+        if self.ws is None:
+            S.svdq_linear(self.w, self.xq, self.s_x, self.Z, self.Y, self.epi, stream)
+        else:
+            S.svdq_linear_splitk(self.w, self.xq, self.s_x, self.Z, self.Y, self.ws, 0, self.epi,
+                                 stream)
         marks[2].record(stream)
 
 
@@ -417,7 +448,7 @@ def _time_mlp_pair(S, flush, stream, steps):
     return out
 
 
-def _time_e2e(S, w, Xh, Yh, Xd, bufs, epi, steps):
+def _time_e2e(S, w, Xh, Yh, Xd, bufs, epi, steps, workspace=None):
     """Public API end to end, as a serving loop: every step copies its X from
     pinned host memory to the device, runs svdq_quantize_act and svdq_linear,
     and copies its Y back to pinned host memory.  Uploads, compute and
@@ -447,7 +478,10 @@ def _time_e2e(S, w, Xh, Yh, Xd, bufs, epi, steps):
             comp.wait_event(ev_dn[b])          # Y of set b downloaded before it is rewritten
         S.svdq_quantize_act(w, Xd[b], xq, s_x, Z, comp)
         ev_xr[b].record(comp)
-        S.svdq_linear(w, xq, s_x, Z, Y, epi, comp)
+        if workspace is None:
+            S.svdq_linear(w, xq, s_x, Z, Y, epi, comp)
+        else:       # one compute stream: the split-K workspace is reused in order
+            S.svdq_linear_splitk(w, xq, s_x, Z, Y, workspace, 0, epi, comp)
         ev_cp[b].record(comp)
         down.wait_event(ev_cp[b])
         with torch.cuda.stream(down):
@@ -498,8 +532,16 @@ def run_ours(args, spec):
     bufs, bufs0 = lin.buffers(M), lin0.buffers(M)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
-    step = _Step(S, w, X, bufs, S.EPI_NONE)
-    step0 = _Step(S, w0, X, bufs0, S.EPI_NONE)
+    # split-K at the automatic split when the output tiles cannot fill the
+    # GPU (the library picks the split; 1 means the plain kernel)
+    splitk = S.svdq_linear_splitk_workspace(w, M, 0) > S.svdq_linear_splitk_workspace(w, M, 1)
+    wsb = wsb0 = None
+    if splitk:
+        wsb = torch.empty(S.svdq_linear_splitk_workspace(w, M, 0), dtype=torch.uint8, device="cuda")
+        wsb0 = torch.empty(S.svdq_linear_splitk_workspace(w0, M, 0), dtype=torch.uint8,
+                           device="cuda")
+    step = _Step(S, w, X, bufs, S.EPI_NONE, wsb)
+    step0 = _Step(S, w0, X, bufs0, S.EPI_NONE, wsb0)
     # e2e: two pinned host batches in, two out; two device buffer sets
     Xh = [torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
     for xh in Xh:
@@ -515,17 +557,34 @@ def run_ours(args, spec):
     time.sleep(0.2)                      # sampler up before the timed region
     barrier()
     clocks.mark("t0")
-    t_act, t_lin = _time_steps(step, args.steps, flush, stream)
+    t_wall0 = time.time()
+    rows = _time_steps(step, args.steps, flush, stream, per_step=True)
+    barrier()
+    clocks.mark("t_timed")
+    # clock window: untimed steps of the same workload until the sampled span
+    # reaches CLOCK_WINDOW_S, so that the clock record holds samples under
+    # this load even when the timed steps end within one sampling interval
+    n_more = 0
+    while time.time() - t_wall0 < CLOCK_WINDOW_S and n_more < 100000:
+        _time_steps(step, 8, flush, stream)
+        n_more += 8
     barrier()
     clocks.mark("t1")
     clk = clocks.stop()
+    if clk is not None:
+        clk["window"] = (f"the {args.steps} timed steps plus {n_more} untimed steps of the same "
+                         f"workload ({time.time() - t_wall0:.2f} s)")
     S.svdq_get_device_error(w)
+    t_act = sum(r[0] for r in rows)
+    t_lin = sum(r[1] for r in rows)
 
+    # L2-warm: the same steps without the flush
+    rows_warm = _time_steps(step, args.steps, None, stream, per_step=True)
     # same kernels without the low-rank branch (overhead), and end to end
     _time_steps(step0, 3, flush, stream)
     t_act0, t_lin0 = _time_steps(step0, args.steps, flush, stream)
-    _time_e2e(S, w, Xh, Yh, Xd, e2e_bufs, S.EPI_NONE, max(args.warmup, 3))
-    t_e2e = _time_e2e(S, w, Xh, Yh, Xd, e2e_bufs, S.EPI_NONE, args.steps)
+    _time_e2e(S, w, Xh, Yh, Xd, e2e_bufs, S.EPI_NONE, max(args.warmup, 3), wsb)
+    t_e2e = _time_e2e(S, w, Xh, Yh, Xd, e2e_bufs, S.EPI_NONE, args.steps, wsb)
     S.svdq_get_device_error(w0)
 
     tt = max_over_ranks([t_act + t_lin, t_lin, t_act, t_e2e], dist, "cuda")
@@ -556,6 +615,13 @@ def run_ours(args, spec):
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
+        "product": "svdq_linear_splitk (automatic split)" if splitk else "svdq_linear",
+        "variability": {"l2_flushed": {"act": _dist_stats([r[0] for r in rows]),
+                                       "linear": _dist_stats([r[1] for r in rows]),
+                                       "step": _dist_stats([r[0] + r[1] for r in rows])},
+                        "l2_warm": {"act": _dist_stats([r[0] for r in rows_warm]),
+                                    "linear": _dist_stats([r[1] for r in rows_warm]),
+                                    "step": _dist_stats([r[0] + r[1] for r in rows_warm])}},
     }
     # the comparisons below are single-GPU diagnostics, timed after the
     # headline steps; a multi-GPU run reports the headline only

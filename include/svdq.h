@@ -255,10 +255,14 @@ svdq_status svdq_linear_splitk(const svdq_weights* w, int M, const uint8_t* xq,
  * cudaMalloc, no allocating library).  The SVDQuant pages have no
  * counterpart; this exists for allocation-free callers.
  *
- * Same arguments and result bits as svdq_linear_splitk with the same
- * `splits` (0 = automatic).  The call clears the counters before its launch.
- * Requests whose workspace (svdq_linear_splitk_workspace) exceeds 16 MiB
- * are rejected with SVDQ_ERR_SHAPE; a single split needs no scratch.
+ * Same arguments as svdq_linear_splitk.  With an explicit `splits` the
+ * result bits equal svdq_linear_splitk's at that split count, and requests
+ * whose workspace (svdq_linear_splitk_workspace) exceeds 16 MiB are
+ * rejected with SVDQ_ERR_SHAPE.  With splits = 0 the automatic split is
+ * lowered, one step at a time, until its workspace fits in 16 MiB (down to
+ * a single split, which needs no scratch); the result bits then equal
+ * svdq_linear_splitk's at the split actually used.  The call clears the
+ * counters before its launch.
  * The scratch is shared by every call on the device: calls that overlap
  * in time (different streams, or handles used concurrently) race and
  * corrupt each other's results, so order them.  The first call on each
@@ -332,6 +336,24 @@ svdq_status svdq_get_device_error(const svdq_weights* w, cudaStream_t stream);
 svdq_status svdq_debug_partials(const svdq_weights* w, int M, const uint8_t* xq,
                                 int row0, int nrows, int col0, int ncols,
                                 int32_t* P, cudaStream_t stream);
+
+/*
+ * Test hook for the bounded device waits; no counterpart on the pages.
+ * Runs svdq_linear (no epilogue) with every device wait bounded by
+ * limit_us microseconds (1 .. 2,000,000) instead of the usual 2 s, while the
+ * TMA producer of the first CTA withholds its first stage of packed codes:
+ * nothing is copied for that stage, so the warps that wait on it give up
+ * after the bound, raise the handle's sticky error word and leave the
+ * kernel (every wait in it is bounded; the issuing thread waits for its own
+ * tensor-core operations before TMEM is freed).  The other CTAs finish
+ * normally.  Y is left partly unwritten.  svdq_get_device_error then
+ * returns SVDQ_ERR_DEVICE_TIMEOUT (and clears the word); the context and
+ * the handle stay usable.  Arguments as svdq_linear; SVDQ_ERR_INVALID_ARG
+ * for limit_us out of range.
+ */
+svdq_status svdq_debug_linear_stall(const svdq_weights* w, int M, const uint8_t* xq,
+                                    const float* s_x, const uint16_t* Z, uint16_t* Y,
+                                    int ldy, unsigned int limit_us, cudaStream_t stream);
 
 /*
  * ------------------------------------------------------------------------

@@ -39,15 +39,21 @@ def _cuda():
 
 
 def check_layer(spec, epilogue=S.EPI_NONE, rows_sample=None, partial_blocks=None,
-                svd=None, X_bits=None, ldy=None):
+                svd=None, X_bits=None, ldy=None, lora_scale=1.0):
     L = synth.make_layer(spec)
     Xb = L.X if X_bits is None else X_bits
     a = S.svdq_calib_absmax(Xb)
     w = S.svdq_pack_weights(L.W, a, spec.rank, bias_bits=L.b, lora_A_bits=L.A,
-                            lora_B_bits=L.B)
+                            lora_B_bits=L.B, lora_scale=lora_scale)
     p = oracle.pack_weights(L.W, a.astype(np.float64), spec.rank, bias_bits=L.b,
-                            lora_A_bits=L.A, lora_B_bits=L.B, svd=svd)
+                            lora_A_bits=L.A, lora_B_bits=L.B, lora_scale=lora_scale, svd=svd)
     e = w.export()
+    if spec.lora_rank:
+        # the adapter columns carry no sign ambiguity: bit-exact (eq. 13,
+        # the scale on the smoothed A side)
+        r0 = spec.rank
+        assert np.array_equal(oracle.bf16_bits_to_f64(e["L1"])[:, r0:], p["L1b"][:, r0:])
+        assert np.array_equal(oracle.bf16_bits_to_f64(e["L2"])[r0:], p["L2b"][r0:])
     # weights
     assert np.array_equal(e["inv_lambda"].astype(np.float64), p["inv_lambda"])
     assert np.array_equal(e["wq"], p["wq"])
@@ -117,9 +123,10 @@ def test_ragged_output_stride():
     check_layer(spec, ldy=200)
 
 
-def test_lora_branch():
+@pytest.mark.parametrize("lora_scale", [1.0, 0.3, -2.5])
+def test_lora_branch(lora_scale):
     spec = synth.layer_spec("lora", 256, 512, 384, 16, 21, lora_rank=16)
-    check_layer(spec)
+    check_layer(spec, lora_scale=lora_scale)
 
 
 def test_zero_rows_and_groups():

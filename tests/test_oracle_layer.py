@@ -221,3 +221,56 @@ def test_leading_svd_matches_full_svd(tiny):
     assert np.max(np.abs(q["sigma"] - p["sigma"]) / p["sigma"]) < 1e-12
     assert np.array_equal(np.abs(q["L1b"]), np.abs(p["L1b"]))
     assert np.array_equal(q["wq"], p["wq"]) and np.array_equal(q["s_w"], p["s_w"])
+
+
+def _lora_identity_err(p, X, W, A, B, b, s):
+    """Relative error between the unquantised two-branch layer built from the
+    stored factors (eq. 7 with quantisation off: [L1 | s D A] and [L2 ; B]
+    joined to the residual) and the adapted layer's definition X (W + s A B) + b
+    (eq. 13)."""
+    R = p["Wt"] - p["L1b"][:, :p["rank"] - A.shape[1]] @ p["L2b"][:p["rank"] - A.shape[1]]
+    y = oracle.two_branch_unquantized(X, p["lam"], p["L1b"], p["L2b"], R, b)
+    return _rel(y, X @ (W + float(np.float32(s)) * (A @ B)) + b)
+
+
+def _lora_placement_ok(p, lam, A, B, s, r):
+    """eq. 13 puts the adapter on the smoothed side: the stored low-rank
+    factors end with bf16(s D A) and with B unchanged."""
+    return (np.array_equal(p["L1b"][:, r:], oracle.round_bf16(lam[:, None] * A * float(np.float32(s))))
+            and np.array_equal(p["L2b"][r:], B))
+
+
+@pytest.mark.parametrize("scale", [0.3, 2.5, -0.75])
+def test_lora_scale_eq13(scale):
+    """LoRA scale s != 1: D (W + s A B) = D W + (s D A) B (eq. 13), the stored
+    factors hold s on the A side, and two planted mistakes fail the checks:
+    the scale applied to B instead, and the scale dropped."""
+    spec = synth.layer_spec("lora_s", 64, 256, 128, 8, 78, lora_rank=4, tiny=True)
+    L = synth.make_layer(spec)
+    X = oracle.bf16_bits_to_f64(L.X)
+    a = oracle.calib_absmax(X)
+    A = oracle.bf16_bits_to_f64(L.A) * 40.0          # an adapter term that matters
+    B = oracle.bf16_bits_to_f64(L.B) * 40.0
+    Ab, Bb = oracle.round_bf16_bits(A), oracle.round_bf16_bits(B)
+    A, B = oracle.bf16_bits_to_f64(Ab), oracle.bf16_bits_to_f64(Bb)
+    W = oracle.bf16_bits_to_f64(L.W).T
+    b = oracle.bf16_bits_to_f64(L.b)
+    p = oracle.pack_weights(L.W, a, 8, bias_bits=L.b, lora_A_bits=Ab, lora_B_bits=Bb,
+                            lora_scale=scale)
+    lam = p["lam"]
+    s32 = float(np.float32(scale))
+    assert _rel(lam[:, None] * (W + s32 * A @ B), p["Wt"] + (s32 * lam[:, None] * A) @ B) < 1e-12
+    assert _lora_placement_ok(p, lam, A, B, scale, 8)
+    # only the bf16 rounding of the factors separates the two (eq. 10 residual
+    # is taken against the stored SVD factors, so that part is exact)
+    err = _lora_identity_err(p, X, W, A, B, b, scale)
+    assert err < 2.0 ** -8, err
+    # mistake 1: the scale applied to B (same product, wrong placement)
+    bad = dict(p)
+    bad["L1b"] = np.hstack([p["L1b"][:, :8], oracle.round_bf16(lam[:, None] * A)])
+    bad["L2b"] = np.vstack([p["L2b"][:8], oracle.round_bf16(s32 * B)])
+    assert not _lora_placement_ok(bad, lam, A, B, scale, 8)
+    # mistake 2: the scale dropped (the layer no longer matches its definition)
+    drop = dict(p)
+    drop["L1b"] = np.hstack([p["L1b"][:, :8], oracle.round_bf16(lam[:, None] * A)])
+    assert _lora_identity_err(drop, X, W, A, B, b, scale) > 1e-2

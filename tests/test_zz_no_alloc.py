@@ -31,16 +31,37 @@ def _layer(M, K, N, r, seed):
     return w, xq, s_x, Z, Y
 
 
+SCRATCH = 16 << 20
+
+
+def _noalloc_split(w, M, splits):
+    """The split count svdq_linear_splitk_noalloc runs: an explicit one as
+    given; the automatic one lowered until its workspace fits the scratch."""
+    if splits:
+        return splits
+    ws_auto = S.svdq_linear_splitk_workspace(w, M, 0)
+    sp = next(s for s in range(1, 17) if S.svdq_linear_splitk_workspace(w, M, s) == ws_auto)
+    while sp > 1 and S.svdq_linear_splitk_workspace(w, M, sp) > SCRATCH:
+        sp -= 1
+    return sp
+
+
 @pytest.mark.parametrize("M,K,N,r,splits", [
     (256, 4608, 1152, 32, 0),     # automatic split (8 ranges), 9.4 MB of scratch
     (130, 320, 136, 24, 2),       # ragged, two ranges
     (1024, 1152, 4608, 32, 0),    # tiles fill the GPU: one split, no scratch
+    (256, 15360, 3072, 32, 0),    # 256-column tiles: the automatic 6 ranges need 18.9 MB; 5 fit
+    (128, 12288, 9216, 32, 0),    # 36 tiles x 4 ranges need 18.9 MB; 3 fit
 ])
 def test_noalloc_matches_splitk_twice(M, K, N, r, splits):
     assert torch.cuda.is_available()
     w, xq, s_x, Z, Y = _layer(M, K, N, r, 900 + M + r)
-    ws = torch.empty(S.svdq_linear_splitk_workspace(w, M, splits), dtype=torch.uint8, device="cuda")
-    S.svdq_linear_splitk(w, xq, s_x, Z, Y, ws, splits)
+    sp = _noalloc_split(w, M, splits)
+    if splits == 0 and S.svdq_linear_splitk_workspace(w, M, 0) > SCRATCH:
+        # a single split is the plain kernel and needs no scratch
+        assert sp == 1 or S.svdq_linear_splitk_workspace(w, M, sp) <= SCRATCH
+    ws = torch.empty(S.svdq_linear_splitk_workspace(w, M, sp), dtype=torch.uint8, device="cuda")
+    S.svdq_linear_splitk(w, xq, s_x, Z, Y, ws, sp)
     torch.cuda.synchronize()
     ref = _bits(Y).copy()
     Yn = torch.empty_like(Y)

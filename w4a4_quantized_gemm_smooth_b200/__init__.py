@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
         "svdq_linear": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _vp]),
         "svdq_get_device_error": (_i, [_vp, _vp]),
         "svdq_debug_partials": (_i, [_vp, _i, _vp, _i, _i, _i, _i, _vp, _vp]),
+        "svdq_debug_linear_stall": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, ctypes.c_uint, _vp]),
         "svdq_linear_splitk_workspace": (ctypes.c_size_t, [_vp, _i, _i]),
         "svdq_linear_splitk": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _vp,
                                     ctypes.c_size_t, _vp]),
@@ -411,6 +412,15 @@ def svdq_linear_nvfp4(w: Weights, xq, sfa, s_x, Z, Y, epilogue=EPI_NONE, stream=
 
 def svdq_get_device_error(w: Weights, stream=None):
     _check(lib().svdq_get_device_error(w.handle, _stream_ptr(stream)), "device")
+
+
+def svdq_debug_linear_stall(w: Weights, xq, s_x, Z, Y, limit_us=200, stream=None):
+    """Test hook: svdq_linear with every device wait bounded by limit_us and
+    the first CTA's first stage withheld (see include/svdq.h)."""
+    M = Y.shape[0]
+    _check(lib().svdq_debug_linear_stall(w.handle, M, _dev_ptr(xq), _dev_ptr(s_x), _dev_ptr(Z),
+                                         _dev_ptr(Y), Y.stride(0), ctypes.c_uint(int(limit_us)),
+                                         _stream_ptr(stream)), "svdq_debug_linear_stall")
 
 
 def svdq_debug_partials(w: Weights, M, xq, row0, nrows, col0, ncols, P, stream=None):

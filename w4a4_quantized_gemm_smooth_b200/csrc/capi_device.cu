@@ -149,6 +149,16 @@ svdq_status svdq_debug_partials(const svdq_weights* w, int M, const uint8_t* xq,
   return from_launch(svdq::launch_partials(w, M, xq, row0, nrows, col0, ncols, P, stream));
 }
 
+svdq_status svdq_debug_linear_stall(const svdq_weights* w, int M, const uint8_t* xq,
+                                    const float* s_x, const uint16_t* Z, uint16_t* Y, int ldy,
+                                    unsigned int limit_us, cudaStream_t stream) {
+  svdq_status s = check_linear(w, M, xq, s_x, Z, Y, ldy, SVDQ_EPI_NONE);
+  if (s != SVDQ_OK || M == 0) return s;
+  if (limit_us < 1 || limit_us > 2000000u) return SVDQ_ERR_INVALID_ARG;
+  return from_launch(svdq::launch_linear_stall(w, M, xq, s_x, Z, Y, ldy,
+                                               (uint64_t)limit_us * 1000u, stream));
+}
+
 svdq_status svdq_quantize_act_w8a8(const svdq_weights* w, int M, const uint16_t* X, int ldx,
                                    int8_t* xq, float* s_x, uint16_t* Z, cudaStream_t stream) {
   svdq_status s = check_handle_w8a8(w);

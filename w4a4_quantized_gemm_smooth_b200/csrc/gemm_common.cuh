@@ -16,16 +16,17 @@ namespace svdq {
 constexpr uint64_t LIMIT_NS = 2000000000ull;
 
 // Bounded wait: the thread sleeps in try_wait (up to 20 us per call) until
-// the phase completes; after LIMIT_NS, or when another thread of the CTA has
+// the phase completes; after limit_ns, or when another thread of the CTA has
 // given up, it returns false.
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
-                                              volatile int* abort_flag, int* err) {
+                                              volatile int* abort_flag, int* err,
+                                              uint64_t limit_ns = LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > LIMIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicExch(err, SVDQ_DEVERR_TIMEOUT);
       return false;

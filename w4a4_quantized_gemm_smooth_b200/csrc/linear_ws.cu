@@ -92,6 +92,8 @@ struct LinArgs {
   int epilogue;
   int tiles_n, num_tiles, tile_m0, tile_n0;
   int* err;
+  uint64_t limit_ns;       // bound on every wait (LIMIT_NS; shorter in the stall test)
+  int stall;               // test hook: CTA 0's producer withholds its first stage
   int b_twos;              // 1: weight codes in two's complement (else sign-magnitude)
   int sx_tma;              // 1: s_x rows are 16-byte aligned (M % 4 == 0), copy by TMA
   int32_t* P;              // partial dump (MODE 1)
@@ -159,8 +161,8 @@ struct Lay {
   static constexpr int OFF_ILAM = OFF_BIAS + N_RES_WARPS * CW * 4;
   static constexpr int OFF_BAR = OFF_ILAM + N_RES_WARPS * CW * 4;
   // barriers: pk_full[NP], pk_empty[NP], ex_full[NE], ex_empty[NE], tm_full[NB],
-  // tm_empty[NB], lr_full[NLR], lr_empty[NLR], xh_full
-  static constexpr int N_BARS = 2 * NP + 2 * NE + 2 * NB + 2 * NLR + 1;
+  // tm_empty[NB], lr_full[NLR], lr_empty[NLR], xh_full, mma_drain
+  static constexpr int N_BARS = 2 * NP + 2 * NE + 2 * NB + 2 * NLR + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;              // slack for 1024-B alignment
@@ -318,6 +320,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
   auto lr_full = [&](int s) { return bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + s); };
   auto lr_empty = [&](int s) { return bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + NLR + s); };
   const uint32_t xh_full = bar0 + 8u * (2 * NP + 2 * NE + 2 * NB + 2 * NLR);
+  const uint32_t mma_drain = xh_full + 8u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -329,6 +332,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     for (int b = 0; b < NB; ++b) { mbar_init(tm_full(b), 1); mbar_init(tm_empty(b), N_RES_WARPS); }
     for (int s = 0; s < NLR; ++s) { mbar_init(lr_full(s), 1); mbar_init(lr_empty(s), 1); }
     mbar_init(xh_full, N_RES_WARPS);
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -355,7 +359,14 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         for (int g = wi.g0; g < wi.g1; g += 2, ++it) {
           const int ng = wi.g1 - g < 2 ? 1 : 2;     // groups in this stage
           const int s = it % NP;
-          if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
+          if (!wait_or_abort(pk_empty(s), ((it / NP) & 1) ^ 1, abort_flag, p.err, p.limit_ns)) { alive = false; break; }
+          if (p.stall && it == 0 && blockIdx.x == 0) {
+            // test hook: the first stage is never filled, so its consumers'
+            // bounded waits run out (nothing is issued for it)
+            ig += ng;
+            __syncwarp();
+            continue;
+          }
           if (LAYER && !p.sx_tma) {
             // s_x rows not 16-byte aligned: 4-byte async copies by all lanes,
             // tracked by the stage's full barrier (raised before lane 0 arrives)
@@ -395,7 +406,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
         if (lane == 0) {
           for (int j = 0; j < (wi.lr ? p.n_lr : 0); ++j, ++il) {
             const int ls = il % NLR;
-            if (!wait_or_abort(lr_empty(ls), ((il / NLR) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
+            if (!wait_or_abort(lr_empty(ls), ((il / NLR) & 1) ^ 1, abort_flag, p.err, p.limit_ns)) { alive = false; break; }
             mbar_arrive_expect_tx(lr_full(ls), L::LR_SLOT);
             const uint32_t dst = sbase + L::OFF_LR + ls * L::LR_SLOT;
 #pragma unroll
@@ -409,7 +420,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
           // each, chunk c of 8 columns at c * rank2_pad * 16, row r at r * 16)
           for (int u = 0; FUSE && alive && u < p.n_l1; ++u, ++il) {
             const int ls = il % NLR;
-            if (!wait_or_abort(lr_empty(ls), ((il / NLR) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
+            if (!wait_or_abort(lr_empty(ls), ((il / NLR) & 1) ^ 1, abort_flag, p.err, p.limit_ns)) { alive = false; break; }
             mbar_arrive_expect_tx(lr_full(ls), (uint32_t)p.rank2_pad * 256u);
             const uint32_t dst = sbase + L::OFF_LR + ls * L::LR_SLOT;
 #pragma unroll 4
@@ -422,9 +433,10 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       // every issued copy has landed before the CTA exits
       if (lane == 0) {
         for (uint32_t k = (it > NP ? it - NP : 0); k < it; ++k)
-          mbar_wait_bounded(pk_full(k % NP), (k / NP) & 1, LIMIT_NS);
+          if (!(p.stall && k == 0 && blockIdx.x == 0))     // the withheld stage issued nothing
+            mbar_wait_bounded(pk_full(k % NP), (k / NP) & 1, p.limit_ns);
         for (uint32_t k = (il > NLR ? il - NLR : 0); k < il; ++k)
-          mbar_wait_bounded(lr_full(k % NLR), (k / NLR) & 1, LIMIT_NS);
+          mbar_wait_bounded(lr_full(k % NLR), (k / NLR) & 1, p.limit_ns);
       }
       cp_async_wait<0>();
       __syncwarp();
@@ -438,11 +450,11 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
           const bool lrs = wi.lr && p.n_lr > 0;
           for (int g = wi.g0; g < wi.g1 + (lrs ? 1 : 0); ++g) {
             const int b = tb % NB;
-            if (!wait_or_abort(tm_empty(b), ((tb / NB) & 1) ^ 1, abort_flag, p.err)) goto mma_done;
+            if (!wait_or_abort(tm_empty(b), ((tb / NB) & 1) ^ 1, abort_flag, p.err, p.limit_ns)) goto mma_done;
             const uint32_t d = tmem + b * BN;
             if (g < wi.g1) {
               const int s = ite % NE;
-              if (!wait_or_abort(ex_full(s), (ite / NE) & 1, abort_flag, p.err)) goto mma_done;
+              if (!wait_or_abort(ex_full(s), (ite / NE) & 1, abort_flag, p.err, p.limit_ns)) goto mma_done;
               tc_fence_after();
               const uint32_t ea = sbase + L::OFF_EX + s * L::EX_STAGE;
               const uint64_t ad = sdesc_kmajor_noswizzle(ea, 128, 512);
@@ -454,7 +466,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             } else {
               for (int j = 0; j < p.n_lr; ++j, ++il) {
                 const int ls = il % NLR;
-                if (!wait_or_abort(lr_full(ls), (il / NLR) & 1, abort_flag, p.err)) goto mma_done;
+                if (!wait_or_abort(lr_full(ls), (il / NLR) & 1, abort_flag, p.err, p.limit_ns)) goto mma_done;
                 tc_fence_after();
                 const uint32_t la = sbase + L::OFF_LR + ls * L::LR_SLOT;
                 // chunk c of the slice at c * rows * 16 bytes, row r at r * 16
@@ -471,14 +483,14 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             // the next layer's down-projection of this tile: x~ (bf16, written
             // by the epilogue) times its L1 rows, into the next TMEM buffer
             const int b = tb % NB;
-            if (!wait_or_abort(tm_empty(b), ((tb / NB) & 1) ^ 1, abort_flag, p.err)) goto mma_done;
-            if (!wait_or_abort(xh_full, ixh & 1, abort_flag, p.err)) goto mma_done;
+            if (!wait_or_abort(tm_empty(b), ((tb / NB) & 1) ^ 1, abort_flag, p.err, p.limit_ns)) goto mma_done;
+            if (!wait_or_abort(xh_full, ixh & 1, abort_flag, p.err, p.limit_ns)) goto mma_done;
             tc_fence_after();
             const uint32_t d = tmem + b * BN;
             const uint32_t id_z = idesc_bf16(BM, p.rank2_pad);
             for (int u = 0; u < p.n_l1; ++u, ++il) {
               const int ls = il % NLR;
-              if (!wait_or_abort(lr_full(ls), (il / NLR) & 1, abort_flag, p.err)) goto mma_done;
+              if (!wait_or_abort(lr_full(ls), (il / NLR) & 1, abort_flag, p.err, p.limit_ns)) goto mma_done;
               tc_fence_after();
               const uint32_t la = sbase + L::OFF_LR + ls * L::LR_SLOT;
               for (int j = 0; j < 8; ++j) {
@@ -496,7 +508,11 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             ++ixh;
           }
         }
-      mma_done:;
+      mma_done:
+        // every MMA this thread issued has completed before TMEM is freed,
+        // on the normal path and after an abort alike
+        mma_commit(mma_drain);
+        mbar_wait_bounded(mma_drain, 0, p.limit_ns);
       }
       __syncwarp();
     } else {
@@ -509,10 +525,10 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
           for (int g = wi.g0; g < wi.g1; g += 2, ++ist) {
             const int ng = wi.g1 - g < 2 ? 1 : 2;
             const int sp = ist % NP;
-            if (!wait_or_abort(pk_full(sp), (ist / NP) & 1, abort_flag, p.err)) return;
+            if (!wait_or_abort(pk_full(sp), (ist / NP) & 1, abort_flag, p.err, p.limit_ns)) return;
             for (int k = 0; k < ng; ++k, ++it) {
               const int se = it % NE;
-              if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err)) return;
+              if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err, p.limit_ns)) return;
               plan.template run<BT>(sbase + L::OFF_PK + sp * L::PK_STAGE,
                                     sbase + L::OFF_EX + se * L::EX_STAGE, 32u * k);
               fence_proxy_async_smem();
@@ -580,7 +596,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       for (int g = wi.g0; g < wi.g1; ++g, ++tb, ++gs) {
         const uint32_t slot = sbase + L::OFF_SC + (gs % L::NS) * L::SC_SLOT;
         const int b = tb % NB;
-        if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
         if (LAYER) {
@@ -656,7 +672,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       if (!ok || !LAYER) continue;
       if (wi.lr && p.n_lr > 0) {
         const int b = tb % NB;
-        if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ta = tmem + b * BN + h * CW + lane_off;
         uint32_t rb[2][16];
@@ -782,7 +798,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
           if (lane == 0) mbar_arrive(xh_full);
           // the tile's partial down-projection: 32x32b load, lane = row
           const int b = tb % NB;
-          if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!wait_or_abort(tm_full(b), (tb / NB) & 1, abort_flag, p.err, p.limit_ns)) { ok = false; break; }
           tc_fence_after();
           if (16 * h < p.rank2_pad) {
             uint32_t r[16];
@@ -929,6 +945,8 @@ bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* 
   a.tiles_n = (w->N + BN - 1) / BN;
   a.tile_m0 = 0; a.tile_n0 = 0;
   a.err = w->d_err;
+  a.limit_ns = LIMIT_NS;
+  a.stall = 0;
   a.b_twos = w->wq_twos ? 1 : 0;
   a.sx_tma = sx_tma ? 1 : 0;
   a.splits = 1;
@@ -953,6 +971,19 @@ cudaError_t launch_linear(const svdq_weights* w, int M, const uint8_t* xq, const
   LinMaps m;
   LinArgs a;
   if (!build_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, BN, m, a)) return cudaErrorInvalidValue;
+  const int tiles_m = (M + BM - 1) / BM;
+  return BN == 256 ? launch_ws<256, 0>(m, a, tiles_m, st) : launch_ws<128, 0>(m, a, tiles_m, st);
+}
+
+cudaError_t launch_linear_stall(const svdq_weights* w, int M, const uint8_t* xq,
+                                const float* s_x, const uint16_t* Z, uint16_t* Y, int ldy,
+                                uint64_t limit_ns, cudaStream_t st) {
+  const int BN = pick_bn(w->N);
+  LinMaps m;
+  LinArgs a;
+  if (!build_linear(w, M, xq, s_x, Z, Y, ldy, SVDQ_EPI_NONE, BN, m, a)) return cudaErrorInvalidValue;
+  a.limit_ns = limit_ns;
+  a.stall = 1;
   const int tiles_m = (M + BM - 1) / BM;
   return BN == 256 ? launch_ws<256, 0>(m, a, tiles_m, st) : launch_ws<128, 0>(m, a, tiles_m, st);
 }
@@ -1006,6 +1037,8 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
   a.rank = 0; a.rank_pad32 = 0; a.n_lr = 0; a.epilogue = 0;
   a.splits = 1;
   a.err = w->d_err;
+  a.limit_ns = LIMIT_NS;
+  a.stall = 0;
   a.b_twos = w->wq_twos ? 1 : 0;
   a.P = P; a.row0 = row0; a.nrows = nrows; a.col0 = col0; a.ncols = ncols;
   const int tm0 = row0 / BM, tm1 = (row0 + nrows - 1) / BM;

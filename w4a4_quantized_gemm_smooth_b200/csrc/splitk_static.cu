@@ -9,10 +9,11 @@
 
 namespace {
 
-// Scratch for the split-K partial tiles: 16 MiB per device, enough for the
-// automatic split of every batch whose output tiles cannot fill the GPU at
-// the review's PixArt-Sigma and FLUX widths (e.g. M = 256, N = 1152,
-// K = 4608: 9.4 MB).  Larger requests are rejected.
+// Scratch for the split-K partial tiles: 16 MiB per device.  An explicit
+// split count whose partial tiles need more is rejected; the automatic split
+// is lowered until its tiles fit (e.g. M = 256, K = 4608, N = 1152 keeps its
+// 8 ranges, 9.4 MB; M = 256, K = 15360, N = 3072 needs 18.9 MB at 6 ranges
+// and runs at 5, 15.7 MB).
 constexpr size_t kScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_splitk_scratch[kScratchBytes];
 
@@ -46,8 +47,10 @@ svdq_status svdq_linear_splitk_noalloc(const svdq_weights* w, int M, const uint8
                                        cudaStream_t stream) {
   svdq_status s = svdq::check_linear(w, M, xq, s_x, Z, Y, ldy, epilogue);
   if (s != SVDQ_OK || M == 0) return s;
-  const int sp = svdq::resolve_splits(w, M, splits);
+  int sp = svdq::resolve_splits(w, M, splits);
   if (sp < 1) return SVDQ_ERR_INVALID_ARG;
+  if (splits == 0)          // automatic: the largest split up to the choice that fits
+    while (sp > 1 && svdq::splitk_workspace(w, M, sp) > kScratchBytes) --sp;
   if (sp > 1 && svdq::splitk_workspace(w, M, sp) > kScratchBytes) return SVDQ_ERR_SHAPE;
   void* scratch = nullptr;
   if ((s = scratch_address(w->device, &scratch)) != SVDQ_OK) return s;

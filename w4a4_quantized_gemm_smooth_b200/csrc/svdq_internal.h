@@ -124,6 +124,11 @@ cudaError_t launch_linear_next(const svdq_weights* w, const svdq_weights* w2, in
                                const uint8_t* xq, const float* s_x, const uint16_t* Z,
                                int epilogue, uint8_t* xq2, float* s_x2, uint16_t* Z2,
                                float* zpart, cudaStream_t stream);
+// Test hook: launch_linear whose waits are bounded by limit_ns and whose CTA
+// 0 producer withholds its first stage (the consumers' waits run out).
+cudaError_t launch_linear_stall(const svdq_weights* w, int M, const uint8_t* xq,
+                                const float* s_x, const uint16_t* Z, uint16_t* Y, int ldy,
+                                uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq,
                             int row0, int nrows, int col0, int ncols,
                             int32_t* P, cudaStream_t stream);
