@@ -13,21 +13,25 @@
 // and stores Y by TMA.
 //
 // Persistent CTAs (one per SM), 128 x 128 tiles, static round-robin; 8 warps:
-//   warp 0    TMA producer: 128-K stages of A and B (one 64-byte-swizzled
-//             box each: 128 rows x 64 B) and the two 512-byte group-scale
+//   warp 0    TMA producer: 256-K stages of A and B (one 128-byte-swizzled
+//             box each: 128 rows x 128 B) and the four 512-byte group-scale
 //             atoms of A and of B (bulk copies); low-rank slices at tile end;
-//   warp 1    TMEM owner and MMA issuer: per stage two tcgen05.cp of each
-//             operand's atoms into TMEM and two block-scaled MMAs (K = 64);
+//   warp 1    TMEM owner and MMA issuer: per stage four tcgen05.cp of each
+//             operand's atoms into TMEM and four block-scaled MMAs (K = 64);
 //   warps 2-3 idle;
 //   warps 4-7 epilogue: warp w owns TMEM lanes 32 (w % 4)..; two 128-column
 //             accumulator buffers let tile t+1 accumulate while tile t is
 //             drained (the low-rank buffer is single: its stage comes at the
 //             end of a tile, after the previous tile's epilogue has read it).
-// TMEM: accumulators [0, 256), low-rank [256, 384), and one 16-column slot
+// The operand stream is bound by the L2 -> SM path (about 2700 cycles from
+// a stage's copy to its arrival at the measured rate): the widest rows the
+// copy engine takes (128 B) and four 36 KB stages in flight, with the
+// 256-K stage halving the per-stage round trips of a 128-K one.
+// TMEM: accumulators [0, 256), low-rank [256, 384), and one 32-column slot
 // of group scales per shared-memory stage [384, 512) (A: 4 columns per K
-// block, B: 4 columns per K block), so the scale copies of a stage never wait
-// for the MMAs of an earlier one: a slot is refilled only after its stage's
-// MMAs have completed (the stage's empty barrier).
+// block, then B), so the scale copies of a stage never wait for the MMAs of
+// an earlier one: a slot is refilled only after its stage's MMAs have
+// completed (the stage's empty barrier).
 // Every wait is bounded (the handle's error word is raised on expiry).
 #include "gemm_common.cuh"
 
@@ -54,10 +58,12 @@ struct F4Args {
 
 struct F4Lay {
   static constexpr int BM = F4_BM, BN = F4_BN;
-  static constexpr int ST_A = BM * 64, ST_B = BN * 64;       // 128 K of packed FP4
-  static constexpr int ST_SFA = 1024, ST_SFB = 1024;          // two 512-byte atoms each
+  static constexpr int KB = 4;                                // 64-K blocks per stage
+  static constexpr int ST_A = BM * 128, ST_B = BN * 128;     // 256 K of packed FP4
+  static constexpr int ST_SFA = KB * 512, ST_SFB = KB * 512;  // one 512-byte atom per K block
   static constexpr int STAGE = ST_A + ST_B + ST_SFA + ST_SFB;
-  static constexpr int NST = 8;          // also the TMEM scale slots (8 x 16 columns)
+  static constexpr int NST = 4;          // also the TMEM scale slots (4 x 32 columns)
+  static constexpr int SF_COLS = 32;
   static constexpr int NLR = 2;
   static constexpr int LR_SA = BM * 32, LR_SB = BN * 32, LR_SLOT = LR_SA + LR_SB;
   static constexpr int Y_BOX = 32 * 64 * 2;                   // 32 rows x 64 bf16
@@ -65,7 +71,9 @@ struct F4Lay {
   static constexpr int OFF_ST = 0;
   static constexpr int OFF_LR = OFF_ST + NST * STAGE;
   static constexpr int OFF_Y = OFF_LR + NLR * LR_SLOT;
-  static constexpr int OFF_BAR = OFF_Y + 4 * Y_WARP;
+  // per epilogue warp: the tile's 128 weight scales, then its 128 biases (fp32)
+  static constexpr int OFF_EPS = OFF_Y + 4 * Y_WARP;
+  static constexpr int OFF_BAR = OFF_EPS + 4 * 1024;
   // st_full[NST], st_empty[NST], tm_full[2], tm_empty[2], lr_full[NLR], lr_empty[NLR],
   // lrb_empty (low-rank TMEM buffer read by the epilogue)
   static constexpr int N_BARS = 2 * NST + 4 + 2 * NLR + 1;
@@ -89,7 +97,7 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 constexpr uint32_t TM_LR = 256;                    // low-rank accumulator
-constexpr uint32_t TM_SF = 384;                    // group-scale slots, 16 columns per stage
+constexpr uint32_t TM_SF = 384;                    // group-scale slots, 32 columns per stage
 
 // Instruction descriptor of the block-scaled FP4 MMA: E2M1 A and B (K-major),
 // UE4M3 scales, fp32 D, M = 128, N = 128, K = 64, scale ids 0.
@@ -100,14 +108,16 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);          // M / 16
 }
 
-// K-major operand as 64-byte rows with the 64-byte swizzle (see linear_w8a8).
-__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+// K-major operand as 128-byte rows with the 128-byte swizzle (8-row atoms of
+// 1 KB, stride 1 KB); the K block j of a row starts 32 j bytes in, i.e. the
+// descriptor's start address advances by 2 (16-byte units).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)1 << 16;
-  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)(1024 >> 4) << 32;
   d |= (uint64_t)1 << 46;
-  d |= (uint64_t)4 << 61;
+  d |= (uint64_t)2 << 61;
   return d;
 }
 
@@ -153,7 +163,8 @@ linear_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nst = (p.nkb + 1) / 2;            // 128-K stages per tile
+  constexpr int KB = L::KB;
+  const int nst = (p.nkb + KB - 1) / KB;      // 256-K stages per tile
 
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) { mbar_init(st_full(s), 1); mbar_init(st_empty(s), 1); }
@@ -183,11 +194,12 @@ linear_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
         for (int s = 0; s < nst; ++s, ++it) {
           const int st = it % NST;
           if (!wait_or_abort(st_empty(st), ((it / NST) & 1) ^ 1, abort_flag, p.err)) { alive = false; break; }
-          const int kb0 = 2 * s, nk = p.nkb - kb0 < 2 ? 1 : 2;
-          mbar_arrive_expect_tx(st_full(st), L::ST_A + L::ST_B + nk * 1024);
+          // K blocks [kb0, kb0 + nk); the boxes read zeros past the end of K
+          const int kb0 = KB * s, nk = p.nkb - kb0 < KB ? p.nkb - kb0 : KB;
+          mbar_arrive_expect_tx(st_full(st), L::ST_A + L::ST_B + 2 * nk * 512);
           const uint32_t dst = sbase + L::OFF_ST + st * L::STAGE;
-          tma_load_2d(dst, &tm_a, s * 64, m0, st_full(st));
-          tma_load_2d(dst + L::ST_A, &tm_b, s * 64, n0, st_full(st));
+          tma_load_2d(dst, &tm_a, s * 128, m0, st_full(st));
+          tma_load_2d(dst + L::ST_A, &tm_b, s * 128, n0, st_full(st));
           bulk_load(dst + L::ST_A + L::ST_B, p.sfa + ((size_t)mb * p.nkb + kb0) * 512, nk * 512,
                     st_full(st));
           bulk_load(dst + L::ST_A + L::ST_B + L::ST_SFA, p.sfb + ((size_t)(n0 / 128) * p.nkb + kb0) * 512,
@@ -236,17 +248,18 @@ linear_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
         tc_fence_after();
         const uint32_t sa = sbase + L::OFF_ST + st * L::STAGE;
         const uint32_t sb = sa + L::ST_A, ssfa = sb + L::ST_B, ssfb = ssfa + L::ST_SFA;
-        const int nk = p.nkb - 2 * s < 2 ? 1 : 2;
-        const uint32_t sf = tm + TM_SF + 16 * st;   // A: +4h, B: +8+4h
+        const int nk = p.nkb - KB * s < KB ? p.nkb - KB * s : KB;
+        const uint32_t sf = tm + TM_SF + L::SF_COLS * st;   // A: +4h, B: +16+4h
         if (elect_one()) {
           for (int h = 0; h < nk; ++h) {
             // this K block's scales: 4 TMEM columns per operand
             tmem_cp_sf(sf + 4 * h, ssfa + 512 * h);
-            tmem_cp_sf(sf + 8 + 4 * h, ssfb + 512 * h);
+            tmem_cp_sf(sf + 4 * KB + 4 * h, ssfb + 512 * h);
           }
+          const uint64_t ad = sdesc_sw128(sa), bd = sdesc_sw128(sb);
           for (int h = 0; h < nk; ++h)
-            mma_nvf4(d, sdesc_sw64(sa + 32 * h), sdesc_sw64(sb + 32 * h), id_f4,
-                     sf + 4 * h, sf + 8 + 4 * h, (s > 0 || h > 0) ? 1u : 0u);
+            mma_nvf4(d, ad + 2 * h, bd + 2 * h, id_f4, sf + 4 * h, sf + 4 * KB + 4 * h,
+                     (s > 0 || h > 0) ? 1u : 0u);
           mma_commit(st_empty(st));
         }
         __syncwarp();
@@ -276,16 +289,39 @@ linear_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
     const int q = warp & 3;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     uint8_t* ystage = smem + L::OFF_Y + q * L::Y_WARP;
+    // the tile's weight scales and biases, staged once per tile (zeros past N)
+    float* eps = reinterpret_cast<float*>(smem + L::OFF_EPS + q * 1024);
+    const uint32_t eps_sw = smem_u32(eps), eps_b = eps_sw + 512;
     const bool gelu = p.epilogue == SVDQ_EPI_GELU;
     uint32_t tb = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tb) {
       const int m0 = (t / p.tiles_n) * BM, n0 = (t % p.tiles_n) * BN;
       const int row = m0 + 32 * q + lane;
       const float sx = row < p.M ? __ldg(p.s_x + row) : 0.0f;
+      // columns n0 + 4 lane .. + 3, loaded before the accumulator is ready
+      const int nl = n0 + 4 * lane;
+      float4 w4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f), b4 = w4;
+      if (nl + 3 < p.N) {
+        w4 = __ldg(reinterpret_cast<const float4*>(p.s_w + nl));
+        const uint2 bb = __ldg(reinterpret_cast<const uint2*>(p.bias + nl));
+        b4 = make_float4(__uint_as_float(bb.x << 16), __uint_as_float(bb.x & 0xFFFF0000u),
+                         __uint_as_float(bb.y << 16), __uint_as_float(bb.y & 0xFFFF0000u));
+      } else {
+        float* wv = &w4.x;
+        float* bv = &b4.x;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (nl + e < p.N) {
+            wv[e] = __ldg(p.s_w + nl + e);
+            bv[e] = __uint_as_float((uint32_t)__ldg(p.bias + nl + e) << 16);
+          }
+      }
       const int b = tb & 1;
       if (!wait_or_abort(tm_full(b), (tb >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
       if (lane == 0) tma_store_wait_read0();
+      reinterpret_cast<float4*>(eps)[lane] = w4;
+      reinterpret_cast<float4*>(eps + 128)[lane] = b4;
       __syncwarp();
       const bool lr = p.n_lr > 0;
 #pragma unroll 1
@@ -295,13 +331,15 @@ linear_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
         if (lr) tmem_ld32(tmem + TM_LR + 32 * c + lane_off, z);
         tmem_wait_ld();
         uint32_t packed[16];
+        float4 sw4, bs4;
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const int n = n0 + 32 * c + j;
-          const float w0 = n < p.N ? __ldg(p.s_w + n) : 0.0f;
-          const float w1 = n + 1 < p.N ? __ldg(p.s_w + n + 1) : 0.0f;
-          float b0 = n < p.N ? __uint_as_float((uint32_t)__ldg(p.bias + n) << 16) : 0.0f;
-          float b1 = n + 1 < p.N ? __uint_as_float((uint32_t)__ldg(p.bias + n + 1) << 16) : 0.0f;
+          if ((j & 3) == 0) {
+            sw4 = lds128(eps_sw + 4u * (32 * c + j));     // same address in every lane
+            bs4 = lds128(eps_b + 4u * (32 * c + j));
+          }
+          const float w0 = (j & 2) ? sw4.z : sw4.x, w1 = (j & 2) ? sw4.w : sw4.y;
+          float b0 = (j & 2) ? bs4.z : bs4.x, b1 = (j & 2) ? bs4.w : bs4.y;
           if (lr) {
             b0 = __fadd_rn(__uint_as_float(z[j]), b0);
             b1 = __fadd_rn(__uint_as_float(z[j + 1]), b1);
@@ -362,10 +400,10 @@ cudaError_t launch_linear_nvfp4(const svdq_weights* w, int M, const uint8_t* xq,
     attr[dev] = true;
   }
   CUtensorMap ta, tb, ty, tz, tl;
-  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 64, L::BM,
-                CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map(&tb, w->d_wq4, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 64, L::BN,
-                CU_TENSOR_MAP_SWIZZLE_64B) ||
+  if (!make_map(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, M, w->K / 2, 128, L::BM,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tb, w->d_wq4, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->K / 2, w->N, w->K / 2, 128, L::BN,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->N, M, (uint64_t)ldy * 2, 64, 32,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
