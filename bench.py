@@ -48,8 +48,8 @@ LINEAR_SOURCES = ("w4a4_quantized_gemm_smooth_b200/csrc/linear_ws.cu",
                   "w4a4_quantized_gemm_smooth_b200/csrc/gemm_common.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/ptx.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/svdq_internal.h")
-LINEAR_TRAFFIC = {"sources_sha1": "86e314bfcfca76a8097ed75e947da04cee8198bd",
-                  "workload": "flux_qkv", "bytes": 24905216 + 28370176}
+LINEAR_TRAFFIC = {"sources_sha1": "3524f9aa0030e8b82b16843eb129154f5a427609",
+                  "workload": "flux_qkv", "bytes": 24867840 + 32785920}
 
 
 def _linear_traffic(workload):

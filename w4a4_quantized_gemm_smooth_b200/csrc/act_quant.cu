@@ -26,6 +26,13 @@
 // two xor-shuffles; codes regrouped into 8-byte stores by a 4 x 4 byte
 // transpose across the quad).
 //
+// Few tokens: when the 32-token blocks cannot fill the GPU, K is split over
+// a cluster of up to eight CTAs per token block (one K range each).  Codes
+// and scales are per group, so they need nothing more; each CTA sums its
+// warps' partial Z in shared memory, and after a cluster barrier CTA c sums,
+// for its share of the 32 rows, the partials of CTAs 0, 1, .. in order
+// through distributed shared memory (deterministic).
+//
 // The W8A8 comparator (review section 8, the eight-bit setting) runs the
 // same kernel with one int8 scale per token: the CTA streams its tokens
 // twice.  The first sweep takes each token's absmax of x~ and the
@@ -46,6 +53,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include "gemm_common.cuh"
 #include "ptx.cuh"
 #include "quant_common.cuh"
 #include "svdq_internal.h"
@@ -72,9 +80,29 @@ struct AqStage {
   static constexpr int BYTES = OFF_IL + GPS * 64 * 4;                 // multiple of 1024
   static constexpr int STAGES = (200 * 1024) / BYTES < 4 ? (200 * 1024) / BYTES : 4;
   static constexpr int RED = WARPS * 16 * NT * 8 * 4;                 // Z partials at the end
+  static constexpr int ZC = AQ_ROWS * NT * 8 * 4;                     // a CTA's partial Z (split K)
   static_assert(STAGES >= 2, "stage too large");
-  static_assert(RED <= STAGES * BYTES, "reduction buffer aliases the ring");
+  static_assert(RED + ZC <= STAGES * BYTES, "reduction buffers alias the ring");
 };
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of every CTA of the cluster (release / acquire at cluster scope).
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// fp32 at the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ float ld_cluster_f32(uint32_t saddr, uint32_t rank) {
+  uint32_t ra;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(saddr), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ float2 lds64(uint32_t addr) {
   float2 v;
@@ -254,7 +282,7 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
                  int M, int K, int rank,
                  uint8_t* __restrict__ xq, float* __restrict__ s_x,
                  uint16_t* __restrict__ Z, uint8_t* __restrict__ sfa,
-                 int* __restrict__ err) {
+                 int* __restrict__ err, int ksplit) {
   constexpr bool W8 = FMT != 0;                // two sweeps, one scale per token
   using ST = AqStage<NT>;
   constexpr int S = ST::STAGES;
@@ -268,9 +296,13 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
   const uint32_t ring = smem_u32(ring_p);
 
   const int tid = threadIdx.x, warp = tid >> 5, l = tid & 31;
-  const int row0 = blockIdx.x * AQ_ROWS;
+  // token block and K range (groups [g0, g1)) of this CTA; ksplit > 1 only
+  // for W4A4, and then, with a branch, the CTAs of a block form a cluster
+  const int row0 = (blockIdx.x / ksplit) * AQ_ROWS;
+  const int sp = blockIdx.x % ksplit;
   const int G = K / 64;
-  const int nstages = (G + AQ_GPS - 1) / AQ_GPS;
+  const int g0 = (int)((long long)sp * G / ksplit), g1 = (int)((long long)(sp + 1) * G / ksplit);
+  const int nstages = (g1 - g0 + AQ_GPS - 1) / AQ_GPS;
   const int nsweep = W8 ? 2 * nstages : nstages;      // W8: quantising sweep after the first
 
   if (tid == 0) {
@@ -303,17 +335,18 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
         if (*reinterpret_cast<volatile int*>(&abort_sh)) break;
         const bool second = c >= nstages;              // no L1 slices needed
         const int cc = second ? c - nstages : c;
-        const int ng = min(AQ_GPS, G - AQ_GPS * cc);
+        const int gb = g0 + AQ_GPS * cc;               // first group of the stage
+        const int ng = min(AQ_GPS, g1 - gb);
         const uint32_t fb = smem_u32(&full_bar[s]);
         const bool with_l1 = NT > 0 && !second;
         mbar_arrive_expect_tx(fb, ng * (AQ_XTILE + (with_l1 ? ST::L1_TILE : 0) + 256));
         const uint32_t st = ring + s * ST::BYTES;
         for (int g = 0; g < ng; ++g) {
-          const int col = (AQ_GPS * cc + g) * 64;
+          const int col = (gb + g) * 64;
           tma_load_2d(st + g * AQ_XTILE, &tm_x, col, row0, fb);
           if (with_l1) tma_load_2d(st + ST::OFF_L1 + g * ST::L1_TILE, &tm_l, col, 0, fb);
         }
-        bulk_load(st + ST::OFF_IL, inv_lambda + AQ_GPS * 64 * cc, ng * 256, fb);
+        bulk_load(st + ST::OFF_IL, inv_lambda + 64 * gb, ng * 256, fb);
       }
       // every issued copy lands before the CTA moves on
       for (int k = (c > S ? c - S : 0); k < c; ++k)
@@ -340,14 +373,14 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
         return false;
       }
       if (*reinterpret_cast<volatile int*>(&abort_sh)) return false;
-      const int grp = AQ_GPS * cc + gi;
-      if (FMT == 2 && second && grp < G) {
+      const int grp = g0 + AQ_GPS * cc + gi;
+      if (FMT == 2 && second && grp < g1) {
         const uint32_t st = ring + s * ST::BYTES;
         const int row = row0 + rl4, a = row >> 7, r = row & 127;
         nvfp4_row32(st + gi * AQ_XTILE + rl4 * 128, rl4, hh4, st + ST::OFF_IL + gi * 256, f4s, f4d6,
                     f4sc, f4tiny, row < M ? xq + (size_t)row * (K / 2) + grp * 32 + 16 * hh4 : nullptr,
                     sfa + ((size_t)a * G + grp) * 512 + 16 * (r & 31) + 4 * (r >> 5) + 2 * hh4);
-      } else if (grp < G) {
+      } else if (grp < g1) {
         const uint32_t st = ring + s * ST::BYTES;
         const uint32_t xt = st + gi * AQ_XTILE;
         // raw X in the A fragment layout: a[ks][0] row g8, cols 16ks+2q (+1);
@@ -515,13 +548,16 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
     }
   }
   __syncthreads();
-  if (abort_sh) return;
+  // Every thread reaches the cluster barriers below, also after an expired
+  // wait (the partials are then not used: the error word is raised).
+  const bool aborted = *reinterpret_cast<volatile int*>(&abort_sh) != 0;
+  if (aborted && (NT == 0 || ksplit == 1)) return;
 
   if constexpr (NT > 0) {
-    // sum the four group-warps of each token half; Z rows in bf16
+    // sum the group-warps of each token half; Z rows in bf16
     constexpr int RP = NT * 8;
     float* red = reinterpret_cast<float*>(ring_p);
-    if (warp < AQ_WARPS) {
+    if (!aborted && warp < AQ_WARPS) {
       float* rw = red + (size_t)warp * 16 * RP;
       const int q = l & 3, g8 = l >> 2;
 #pragma unroll
@@ -534,13 +570,41 @@ act_quant_kernel(const __grid_constant__ CUtensorMap tm_x,
       }
     }
     __syncthreads();
-    for (int idx = tid; idx < AQ_ROWS * rank; idx += AQ_THREADS) {
-      const int r = idx / rank, j = idx % rank, hb = r >> 4, r16 = r & 15;
-      float sum = 0.0f;
+    if (ksplit == 1) {
+      for (int idx = tid; idx < AQ_ROWS * rank; idx += AQ_THREADS) {
+        const int r = idx / rank, j = idx % rank, hb = r >> 4, r16 = r & 15;
+        float sum = 0.0f;
 #pragma unroll
-      for (int gw = 0; gw < AQ_GPS; ++gw) sum += red[(size_t)(2 * gw + hb) * 16 * RP + r16 * RP + j];
-      if (row0 + r < M)
-        Z[(size_t)(row0 + r) * rank + j] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+        for (int gw = 0; gw < AQ_GPS; ++gw) sum += red[(size_t)(2 * gw + hb) * 16 * RP + r16 * RP + j];
+        if (row0 + r < M)
+          Z[(size_t)(row0 + r) * rank + j] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+      }
+    } else {
+      // this CTA's partial [32][rank], then the cluster's sum in CTA order
+      float* zc = red + ST::RED / 4;
+      if (!aborted) {
+        for (int idx = tid; idx < AQ_ROWS * rank; idx += AQ_THREADS) {
+          const int r = idx / rank, j = idx % rank, hb = r >> 4, r16 = r & 15;
+          float sum = 0.0f;
+#pragma unroll
+          for (int gw = 0; gw < AQ_GPS; ++gw) sum += red[(size_t)(2 * gw + hb) * 16 * RP + r16 * RP + j];
+          zc[idx] = sum;
+        }
+      }
+      cluster_barrier();
+      if (!aborted) {
+        const uint32_t me = cluster_ctarank();
+        const int ra = (int)me * AQ_ROWS / ksplit, rb2 = ((int)me + 1) * AQ_ROWS / ksplit;
+        const uint32_t zc_s = smem_u32(zc);
+        for (int idx = ra * rank + tid; idx < rb2 * rank; idx += AQ_THREADS) {
+          const int r = idx / rank, j = idx % rank;
+          float sum = 0.0f;
+          for (int c = 0; c < ksplit; ++c) sum += ld_cluster_f32(zc_s + 4u * idx, (uint32_t)c);
+          if (row0 + r < M)
+            Z[(size_t)(row0 + r) * rank + j] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+        }
+      }
+      cluster_barrier();    // no CTA leaves while others read its partial
     }
   }
 }
@@ -593,10 +657,35 @@ cudaError_t launch_aq(const svdq_weights* w, int M, const uint16_t* X, int ldx,
     return cudaErrorInvalidValue;
   // NVFP4: cover whole 128-row blocks, so that every scale-atom row is written
   const int rows = FMT == 2 ? (M + 127) / 128 * 128 : M;
-  const dim3 grid((rows + AQ_ROWS - 1) / AQ_ROWS);
-  act_quant_kernel<NT, FMT><<<grid, ST::THREADS, dyn, st>>>(tx, tl, w->d_inv_lambda, M, w->K,
-                                                           w->rank, xq, s_x, Z, sfa, w->d_err);
-  return cudaGetLastError();
+  const int nrb = (rows + AQ_ROWS - 1) / AQ_ROWS;
+  // W4A4 with few token blocks: split K over up to eight CTAs per block
+  int ks = 1;
+  if (FMT == 0) {
+    ks = num_sms() / nrb;
+    ks = ks < 1 ? 1 : (ks > 8 ? 8 : ks);
+    if (ks > w->K / 64) ks = w->K / 64;
+  }
+  if (NT == 0 || ks == 1) {
+    act_quant_kernel<NT, FMT><<<dim3(nrb * ks), ST::THREADS, dyn, st>>>(
+        tx, tl, w->d_inv_lambda, M, w->K, w->rank, xq, s_x, Z, sfa, w->d_err, ks);
+    return cudaGetLastError();
+  }
+  // the CTAs of a token block form a cluster (their Z partials meet in
+  // distributed shared memory)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nrb * ks);
+  cfg.blockDim = dim3(ST::THREADS);
+  cfg.dynamicSmemBytes = dyn;
+  cfg.stream = st;
+  cudaLaunchAttribute attr_c[1];
+  attr_c[0].id = cudaLaunchAttributeClusterDimension;
+  attr_c[0].val.clusterDim.x = ks;
+  attr_c[0].val.clusterDim.y = 1;
+  attr_c[0].val.clusterDim.z = 1;
+  cfg.attrs = attr_c;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, act_quant_kernel<NT, FMT>, tx, tl, (const float*)w->d_inv_lambda, M,
+                            w->K, w->rank, xq, s_x, Z, sfa, (int*)w->d_err, ks);
 }
 
 template <int FMT>
