@@ -9,10 +9,16 @@
 // again).  Every product is then an integer times 2^-18 and every sum of a
 // group of 64 is P_g 2^-18 with |P_g| <= 4096, so the fp32 TMEM accumulator
 // holds each group's integer partial exactly and needs no conversion.  The
-// activation codes arrive as two's-complement nibbles (the public layout);
-// the weight codes are stored on the device as sign-magnitude nibbles (a
-// layer with a code of -8, which only a subnormal scale can produce, keeps
-// two's complement and the longer conversion).  The device copy of the weight
+// weight codes are stored on the device as sign-magnitude nibbles (a layer
+// with a code of -8, which only a subnormal scale can produce, keeps two's
+// complement and the longer conversion).  The activation codes arrive as
+// two's-complement nibbles (the public layout) and are expanded as u = q + 8
+// (the nibble with its top bit flipped, whose byte is exactly the E4M3
+// number u 2^-9: 0..7 subnormal, 8..15 the first binade), so that group's
+// MMAs sum P_g + 8 S_g with S_g = sum_k q_w.  A third MMA per group (K = 32)
+// adds the constant A slice (2^-6, 2^-3, 1, 0, ..) times the E4M3 digits
+// (d0, d1, d2, 0, ..) of -S_g = d0 + 8 d1 + 64 d2 (from the pack), i.e.
+// -8 S_g 2^-18, so the TMEM word is again exactly P_g 2^-18.  The device copy of the weight
 // scales holds s_w 2^18 (exact), so the rescale is plain fp32 arithmetic, two
 // operations per element and group: v = fl32(P_g s_w), acc = fl32(acc +
 // v s_x).  The low-rank term Z L2 is one more tensor-core stage (kind::f16,
@@ -137,7 +143,14 @@ struct Lay {
   // row r at r * 64 + 16 (c ^ ((r >> 1) & 3)); chunk 2 gs + hf is half hf
   // of group gs of the stage
   static constexpr int PK_A = BM * 64, PK_B = BN * 64, PK_STAGE = PK_A + PK_B;
-  static constexpr int EX_A = BM * 64, EX_B = BN * 64, EX_STAGE = EX_A + EX_B;
+  // expanded stage: A and B of one group, then the correction slice of B: one
+  // 16-byte row per column (digit bytes 0..3, the rest zero), read for both
+  // K halves of the K = 32 MMA (leading offset 0)
+  static constexpr int EX_A = BM * 64, EX_B = BN * 64, EX_X = BN * 16;
+  static constexpr int EX_STAGE = EX_A + EX_B + EX_X;
+  // the constant A slice of the correction MMA: 128 rows x 32 B (two 16-byte
+  // chunks), bytes 0..2 of each row 2^-6, 2^-3, 1, the rest zero
+  static constexpr int AX_BYTES = BM * 32;
   static constexpr int OFF_Y = 0;
   static constexpr int OFF_PK = OFF_Y + N_RES_WARPS * Y_WARP;
   static constexpr int OFF_EX = OFF_PK + NP * PK_STAGE;
@@ -146,15 +159,17 @@ struct Lay {
   // (four slots where shared memory allows: rank 64 in flight at once)
   static constexpr int NLR = BN == 256 ? 2 : 4;
   static constexpr int LR_SA = BM * 32, LR_SB = BN * 32, LR_SLOT = LR_SA + LR_SB;
-  static constexpr int OFF_LR = OFF_EX + NE * EX_STAGE;
-  // per-group scales: ring of 2 NP + NE + NB slots, each s_x[128] then
-  // s_w[BN], filled by the producer warp together with the packed codes.  The
+  static constexpr int OFF_AX = OFF_EX + NE * EX_STAGE;
+  static constexpr int OFF_LR = OFF_AX + AX_BYTES;
+  // per-group scales: ring of 2 NP + NE + NB slots, each s_x[128], s_w[BN]
+  // and the correction digits [BN] (one word per column), filled by the
+  // producer warp together with the packed codes.  The
   // producer writes the slots of groups j, j + 1 (stage k) once the expanders
   // released stage k - NP, i.e. expanded every group up to j - 2 NP + 1;
   // through the MMA and TMEM barriers the rescale of group j + 1 - 2 NP - NE
   // - NB, the previous owner of the last slot written, has then finished.
   static constexpr int NS = 2 * NP + NE + NB;
-  static constexpr int SC_SLOT = (BM + BN) * 4;
+  static constexpr int SC_SLOT = (BM + 2 * BN) * 4;
   static constexpr int OFF_SC = OFF_LR + NLR * LR_SLOT;
   static constexpr int OFF_BIAS = OFF_SC + NS * SC_SLOT;   // per warp CW floats
   // MODE 4: the next layer's smoothing factors of the warp's columns
@@ -195,6 +210,11 @@ __device__ __forceinline__ void row_group(const T (&src)[4][NP2], int sel, T (&a
 __device__ __forceinline__ void sts32u(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint32_t lds32u(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
 
 // Codes -> E4M3 bytes, four at a time (one byte each of a 32-bit word).
 // Two's complement: x holds four nibbles 0..15, y the same nibbles in the
@@ -218,6 +238,16 @@ __device__ __forceinline__ uint32_t e4m3_hi(uint32_t w) {
   if (TWOS) return e4m3_twos((w >> 4) & 0x0F0F0F0Fu, w);
   return ((w >> 4) & 0x07070707u) | (w & 0x80808080u);
 }
+// Activation codes as offset binary: the nibble with its top bit flipped is
+// u = q + 8 in 0..15, and the byte u is exactly the E4M3 number u 2^-9.
+__device__ __forceinline__ uint32_t e4m3_off_lo(uint32_t w) { return (w ^ 0x88888888u) & 0x0F0F0F0Fu; }
+__device__ __forceinline__ uint32_t e4m3_off_hi(uint32_t w) { return ((w ^ 0x88888888u) >> 4) & 0x0F0F0F0Fu; }
+__device__ __forceinline__ void expand_offset(uint32_t src, uint32_t d) {
+  const uint4 p = lds128u(src);
+  sts128(d, make_uint4(e4m3_off_lo(p.x), e4m3_off_hi(p.x), e4m3_off_lo(p.y), e4m3_off_hi(p.y)));
+  sts128(d + 128, make_uint4(e4m3_off_lo(p.z), e4m3_off_hi(p.z), e4m3_off_lo(p.w), e4m3_off_hi(p.w)));
+}
+
 // 16 packed bytes (32 codes of one row: the first or second half of the
 // group) -> two 16-byte core-matrix rows at d and d + 128.  Inside every 8
 // codes the even-k codes come first.
@@ -260,13 +290,14 @@ struct ExpandPlan {
       dst[k] = (isa ? 0 : L::EX_A) + (row >> 3) * 512 + (row & 7) * 16 + hf * 256;
     }
   }
-  // gsx = 32 * (group within the packed stage); activation codes are two's
-  // complement, weight codes too when BTWOS
+  // gsx = 32 * (group within the packed stage); activation codes become
+  // offset binary, weight codes sign-magnitude (two's complement when BTWOS)
   template <bool BTWOS>
   __device__ __forceinline__ void run(uint32_t pa, uint32_t ea, uint32_t gsx) const {
 #pragma unroll
     for (int k = 0; k < CNT; ++k) {
-      if (k < NA || BTWOS) expand_e4m3<true>(pa + (src[k] ^ gsx), ea + dst[k]);
+      if (k < NA) expand_offset(pa + (src[k] ^ gsx), ea + dst[k]);
+      else if (BTWOS) expand_e4m3<true>(pa + (src[k] ^ gsx), ea + dst[k]);
       else expand_e4m3<false>(pa + (src[k] ^ gsx), ea + dst[k]);
     }
   }
@@ -297,7 +328,8 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_l2,
                  const __grid_constant__ CUtensorMap tm_sx,
                  const __grid_constant__ CUtensorMap tm_sw,
-                 const __grid_constant__ CUtensorMap tm_l1, const LinArgs p) {
+                 const __grid_constant__ CUtensorMap tm_l1,
+                 const __grid_constant__ CUtensorMap tm_cs, const LinArgs p) {
   using L = Lay<BN>;
   constexpr bool LAYER = MODE != 1;
   constexpr bool SPLIT = MODE == 3;
@@ -340,6 +372,17 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
+  // the correction MMA's constant A slice (core matrix (r / 8, c) at
+  // (r / 8) 256 + c 128, row r % 8 at 16 (r % 8)) and the zero bytes of the
+  // B slices; both are read by the tensor core (async proxy)
+  for (int i = tid; i < L::AX_BYTES / 16; i += THREADS) {
+    const bool first = ((i >> 3) & 1) == 0;         // chunk 0 of its core matrix
+    sts128(sbase + L::OFF_AX + 16u * i, make_uint4(first ? 0x00382008u : 0u, 0u, 0u, 0u));
+  }
+  for (int se = 0; se < NE; ++se)
+    for (int i = tid; i < L::EX_X / 16; i += THREADS)
+      sts128(sbase + L::OFF_EX + se * L::EX_STAGE + L::EX_A + L::EX_B + 16u * i, make_uint4(0u, 0u, 0u, 0u));
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -383,20 +426,22 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
             __syncwarp();
           }
           if (lane == 0) {
+            // scales (the layer only) and the correction digits (every mode)
             const uint32_t scale_bytes =
-                LAYER ? ng * ((p.sx_tma ? BM * 4 : 0) + BN * 4) : 0;
+                ng * ((LAYER ? (p.sx_tma ? BM * 4 : 0) + BN * 4 : 0) + BN * 4);
             mbar_arrive_expect_tx(pk_full(s), L::PK_STAGE + scale_bytes);
             const uint32_t dst = sbase + L::OFF_PK + s * L::PK_STAGE;
             // one box per operand: packed bytes [32 g, 32 g + 64); a group
             // past the end of K reads as zeros and is not used
             tma_load_2d(dst, &tm_a, g * 32, m0, pk_full(s));
             tma_load_2d(dst + L::PK_A, &tm_b, g * 32, n0, pk_full(s));
-            if (LAYER) {
-              for (int k = 0; k < ng; ++k) {
-                const uint32_t slot = sbase + L::OFF_SC + ((ig + k) % L::NS) * L::SC_SLOT;
+            for (int k = 0; k < ng; ++k) {
+              const uint32_t slot = sbase + L::OFF_SC + ((ig + k) % L::NS) * L::SC_SLOT;
+              if (LAYER) {
                 if (p.sx_tma) tma_load_2d(slot, &tm_sx, m0, g + k, pk_full(s));
                 tma_load_2d(slot + 4 * BM, &tm_sw, n0, g + k, pk_full(s));
               }
+              tma_load_2d(slot + 4 * (BM + BN), &tm_cs, n0, g + k, pk_full(s));
             }
           }
           ig += ng;
@@ -444,6 +489,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       // ---------------------------------------------------- MMA issuer
       if (lane == 0) {
         const uint32_t id_f8 = idesc_e4m3(BM, BN), id_bf = idesc_bf16(BM, BN);
+        const uint64_t ax_desc = sdesc_kmajor_noswizzle(sbase + L::OFF_AX, 128, 256);
         uint32_t ite = 0, tb = 0, il = 0, ixh = 0;
         for (int wk = blockIdx.x; wk < p.num_tiles * p.splits; wk += gridDim.x) {
           const WorkItem wi = work_item(p, wk);
@@ -459,8 +505,10 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               const uint32_t ea = sbase + L::OFF_EX + s * L::EX_STAGE;
               const uint64_t ad = sdesc_kmajor_noswizzle(ea, 128, 512);
               const uint64_t bd = sdesc_kmajor_noswizzle(ea + L::EX_A, 128, 512);
-              mma_f8f6f4(d, ad, bd, id_f8, 0u);          // D = P_g 2^-18, K = 0..31
+              mma_f8f6f4(d, ad, bd, id_f8, 0u);          // D = (P_g + 8 S_g) 2^-18, K = 0..31
               mma_f8f6f4(d, ad + 16, bd + 16, id_f8, 1u);  // K = 32..63
+              // - 8 S_g 2^-18: the constant slice times the digits
+              mma_f8f6f4(d, ax_desc, sdesc_kmajor_noswizzle(ea + L::EX_A + L::EX_B, 0, 128), id_f8, 1u);
               mma_commit(ex_empty(s));
               ++ite;
             } else {
@@ -517,6 +565,9 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
       __syncwarp();
     } else {
       // ---------------------------------------------------- expanders
+      // warps 2, 3, 6, 7 also copy a quarter of each group's correction digits
+      // (one word per column) from the scale slot into the B correction slice
+      const int xq_i = (warp == 4 || warp == 5) ? -1 : (warp & 3) - 2 + 2 * ((warp >> 2) & 1);
       auto expand_loop = [&](const auto& plan, auto btwos) {
         constexpr bool BT = decltype(btwos)::value;
         uint32_t ist = 0, it = 0;            // packed stages, groups
@@ -531,6 +582,13 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
               if (!wait_or_abort(ex_empty(se), ((it / NE) & 1) ^ 1, abort_flag, p.err, p.limit_ns)) return;
               plan.template run<BT>(sbase + L::OFF_PK + sp * L::PK_STAGE,
                                     sbase + L::OFF_EX + se * L::EX_STAGE, 32u * k);
+              if (xq_i >= 0) {
+                const uint32_t cs = sbase + L::OFF_SC + (it % L::NS) * L::SC_SLOT + 4 * (BM + BN);
+                const uint32_t xs = sbase + L::OFF_EX + se * L::EX_STAGE + L::EX_A + L::EX_B;
+#pragma unroll
+                for (int r = xq_i * (BN / 4) + lane; r < (xq_i + 1) * (BN / 4); r += 32)
+                  sts32u(xs + 16u * r, lds32u(cs + 4u * r));
+              }
               fence_proxy_async_smem();
               mbar_arrive(ex_full(se));
             }
@@ -875,7 +933,7 @@ linear_ws_kernel(const __grid_constant__ CUtensorMap tm_a,
 // ------------------------------------------------------------------ host side
 
 struct LinMaps {
-  CUtensorMap ta, tb, ty, tz, tl, tsx, tsw, tl1;
+  CUtensorMap ta, tb, ty, tz, tl, tsx, tsw, tl1, tcs;
 };
 
 template <int BN, int MODE>
@@ -898,8 +956,14 @@ cudaError_t launch_ws(const LinMaps& m, LinArgs a, int tiles_m, cudaStream_t st)
   const int work = a.num_tiles * a.splits;
   const int grid = work < num_sms() ? work : num_sms();
   linear_ws_kernel<BN, MODE><<<grid, THREADS, L::ALLOC, st>>>(m.ta, m.tb, m.ty, m.tz, m.tl, m.tsx,
-                                                              m.tsw, m.tl1, a);
+                                                              m.tsw, m.tl1, m.tcs, a);
   return cudaGetLastError();
+}
+
+// The correction digits [G][N_pad], one 32-bit word per column: a {BN x 1} box.
+bool cs_map(const svdq_weights* w, int BN, LinMaps& m) {
+  return make_map(&m.tcs, w->d_wcs, CU_TENSOR_MAP_DATA_TYPE_UINT32, w->N_pad, w->G,
+                  (uint64_t)w->N_pad * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 int pick_bn(int N) {
@@ -929,7 +993,8 @@ bool build_linear(const svdq_weights* w, int M, const uint8_t* xq, const float* 
   if ((sx_tma && !make_map(&m.tsx, s_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, M, w->G,
                            (uint64_t)M * 4, BM, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
       !make_map(&m.tsw, w->d_sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->N16, w->G,
-                (uint64_t)w->N16 * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+                (uint64_t)w->N16 * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !cs_map(w, BN, m))
     return false;
   if (w->rank > 0 &&
       (!make_map(&m.tz, Z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->rank, M, (uint64_t)w->rank * 2, 8,
@@ -1032,6 +1097,7 @@ cudaError_t launch_partials(const svdq_weights* w, int M, const uint8_t* xq, int
                 CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   m.ty = m.tz = m.tl = m.tsx = m.tsw = m.tl1 = m.ta;
+  if (!cs_map(w, BN, m)) return cudaErrorInvalidValue;
   LinArgs a{};
   a.M = M; a.N = w->N; a.K = w->K; a.G = w->G;
   a.rank = 0; a.rank_pad32 = 0; a.n_lr = 0; a.epilogue = 0;

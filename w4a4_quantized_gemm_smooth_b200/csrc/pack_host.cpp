@@ -172,14 +172,15 @@ svdq_status dev_alloc_copy(T** dst, const T* src, size_t n, cudaStream_t st) {
 }
 
 void free_device(svdq_weights* w) {
-  cudaFree(w->d_inv_lambda); cudaFree(w->d_wq); cudaFree(w->d_sw);
+  cudaFree(w->d_inv_lambda); cudaFree(w->d_wq); cudaFree(w->d_sw); cudaFree(w->d_wcs);
   cudaFree(w->d_L1T); cudaFree(w->d_L2); cudaFree(w->d_L2T); cudaFree(w->d_bias);
   cudaFree(w->d_wq8); cudaFree(w->d_sw8);
   cudaFree(w->d_wq4); cudaFree(w->d_sfb4); cudaFree(w->d_sw4);
   cudaFree(w->d_err);
   w->d_wq8 = nullptr; w->d_sw8 = nullptr;
   w->d_wq4 = nullptr; w->d_sfb4 = nullptr; w->d_sw4 = nullptr;
-  w->d_inv_lambda = nullptr; w->d_wq = nullptr; w->d_sw = nullptr; w->d_L1T = nullptr;
+  w->d_inv_lambda = nullptr; w->d_wq = nullptr; w->d_sw = nullptr; w->d_wcs = nullptr;
+  w->d_L1T = nullptr;
   w->d_L2 = nullptr; w->d_L2T = nullptr; w->d_bias = nullptr; w->d_err = nullptr;
 }
 
@@ -247,6 +248,26 @@ svdq_status upload(svdq_weights* w, cudaStream_t st) {
         swp[(size_t)g * w->N16 + pos] = (float)std::ldexp(v, 18);   // exact
       }
     if ((s = dev_alloc_copy(&w->d_sw, swp.data(), swp.size(), st))) return s;
+    // per group and column: -sum_k q_w = d0 + 8 d1 + 64 d2 with d0, d1 in
+    // [-4, 3] (balanced base 8) and |d2| <= 8, each as the E4M3 byte of d 2^-9
+    std::vector<uint32_t> wcs((size_t)G * w->N_pad, 0u);
+    auto e4m3_int = [](int d) -> uint32_t { return (uint32_t)((d < 0 ? 0x80 : 0) | (d < 0 ? -d : d)); };
+    for (int n = 0; n < N; ++n)
+      for (int g = 0; g < G; ++g) {
+        int cs = 0;
+        for (int k = 64 * g; k < 64 * g + 64; ++k) {
+          const uint8_t b = w->wq[(size_t)n * (K / 2) + k / 2];
+          cs += (int)(int8_t)(uint8_t)(((b >> (4 * (k & 1))) & 0x0F) << 4) >> 4;
+        }
+        const int v = -cs;
+        const int d0 = ((v % 8) + 8 + 4) % 8 - 4;
+        const int v1 = (v - d0) / 8;
+        const int d1 = ((v1 % 8) + 8 + 4) % 8 - 4;
+        const int d2 = (v1 - d1) / 8;
+        if (d0 + 8 * d1 + 64 * d2 != v || d2 < -8 || d2 > 8) return SVDQ_ERR_NUMERIC;   // |cs| <= 512
+        wcs[(size_t)g * w->N_pad + n] = e4m3_int(d0) | (e4m3_int(d1) << 8) | (e4m3_int(d2) << 16);
+      }
+    if ((s = dev_alloc_copy(&w->d_wcs, wcs.data(), wcs.size(), st))) return s;
   }
   if ((s = dev_alloc_copy(&w->d_L1T, L1T.data(), L1T.size(), st))) return s;
   if ((s = dev_alloc_copy(&w->d_L2, L2p.data(), L2p.size(), st))) return s;

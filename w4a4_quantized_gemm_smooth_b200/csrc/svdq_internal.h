@@ -30,6 +30,12 @@ struct svdq_weights {
   // 8b + 2p + e is stored at 4p + 2b + e, so that the rescale thread that owns
   // the column pairs 2p, 2p+1 of both 8-column halves reads them as one float4
   float* d_sw = nullptr;
+  // [G][N_pad] per group and column, the E4M3 bytes (0..2) of the balanced
+  // base-8 digits d0 + 8 d1 + 64 d2 = -sum_k q_w over the group, zero padded.
+  // The GEMM takes the activation codes as q + 8 (offset binary, its cheapest
+  // expansion) and adds these digits times the constants 8, 64, 512 in one
+  // more K = 32 MMA, which restores the exact group sum.
+  uint32_t* d_wcs = nullptr;
   uint16_t* d_L1T = nullptr;       // [rank_pad][K] bf16, transposed L1
   uint16_t* d_L2 = nullptr;        // [rank_pad][N] bf16
   uint16_t* d_L2T = nullptr;       // [N_pad][rank_pad32] bf16, transposed L2
