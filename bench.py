@@ -48,8 +48,8 @@ LINEAR_SOURCES = ("w4a4_quantized_gemm_smooth_b200/csrc/linear_ws.cu",
                   "w4a4_quantized_gemm_smooth_b200/csrc/gemm_common.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/ptx.cuh",
                   "w4a4_quantized_gemm_smooth_b200/csrc/svdq_internal.h")
-LINEAR_TRAFFIC = {"sources_sha1": "3524f9aa0030e8b82b16843eb129154f5a427609",
-                  "workload": "flux_qkv", "bytes": 24867840 + 32785920}
+LINEAR_TRAFFIC = {"sources_sha1": "71e0331c3d32f46caa1e4d41ad4ec2feb02263b2",
+                  "workload": "flux_qkv", "bytes": 26641408 + 33591808}
 
 
 def _linear_traffic(workload):
