@@ -39,14 +39,18 @@ def _cuda():
 
 
 def check_layer(spec, epilogue=S.EPI_NONE, rows_sample=None, partial_blocks=None,
-                svd=None, X_bits=None, ldy=None, lora_scale=1.0):
+                svd=None, X_bits=None, ldy=None, lora_scale=1.0, W_bits=None, absmax=None,
+                pack_check=None):
     L = synth.make_layer(spec)
     Xb = L.X if X_bits is None else X_bits
-    a = S.svdq_calib_absmax(Xb)
-    w = S.svdq_pack_weights(L.W, a, spec.rank, bias_bits=L.b, lora_A_bits=L.A,
+    Wb = L.W if W_bits is None else W_bits
+    a = S.svdq_calib_absmax(Xb) if absmax is None else absmax
+    w = S.svdq_pack_weights(Wb, a, spec.rank, bias_bits=L.b, lora_A_bits=L.A,
                             lora_B_bits=L.B, lora_scale=lora_scale)
-    p = oracle.pack_weights(L.W, a.astype(np.float64), spec.rank, bias_bits=L.b,
+    p = oracle.pack_weights(Wb, a.astype(np.float64), spec.rank, bias_bits=L.b,
                             lora_A_bits=L.A, lora_B_bits=L.B, lora_scale=lora_scale, svd=svd)
+    if pack_check is not None:
+        pack_check(p)
     e = w.export()
     if spec.lora_rank:
         # the adapter columns carry no sign ambiguity: bit-exact (eq. 13,
@@ -127,6 +131,40 @@ def test_ragged_output_stride():
 def test_lora_branch(lora_scale):
     spec = synth.layer_spec("lora", 256, 512, 384, 16, 21, lora_rank=16)
     check_layer(spec, lora_scale=lora_scale)
+
+
+def test_weight_group_of_minus_eight_codes():
+    """A weight group whose residual codes are all -8.  Channels 64..127 get
+    smoothing factors of 2^-127 (activation statistic 2^-149 against a weight
+    of 2^105 in column 0), so column 1's weights of -2^-19 there become
+    residuals of -2^-146 = -8 s with the group scale s = fl32(2^-146 / 7) =
+    2^-149, the smallest fp32 subnormal (the clamp to [-8, 7] keeps -8).  The
+    layer then keeps two's-complement weight codes on the device, and the
+    GEMM's per-group correction for that group takes its largest digit
+    (-sum_k q_w = 512 = 64 * 8).  The activations of those channels are
+    +-2^-133 (bf16's smallest subnormal) times the factor 2^127, so the
+    partials there are non-zero."""
+    M, K, N = 256, 256, 256
+    spec = synth.layer_spec("minus8", M, K, N, 0, 91, tiny=True)
+    L = synth.make_layer(spec)
+    W = L.W.copy()
+    X = L.X.copy()
+    ch = slice(64, 128)
+    W[0, ch] = 0x7400                          # 2^105
+    W[1, ch] = 0xB600                          # -2^-19
+    X[:, ch] = 0
+    rng = np.random.default_rng(92)
+    pick = rng.random((M, 64)) < 0.3
+    X[:, ch] = np.where(pick, np.where(rng.random((M, 64)) < 0.5, 0x0001, 0x8001), 0).astype(X.dtype)
+    a = S.svdq_calib_absmax(X)
+    a[ch] = np.float32(2.0 ** -149)
+
+    def pack_check(p):
+        codes = p["wcodes"]
+        assert np.all(codes[1, ch] == -8), "the planted group is all -8"
+        assert p["s_w"][1, 1] == 2.0 ** -149
+    check_layer(spec, X_bits=X, W_bits=W, absmax=a, pack_check=pack_check,
+                partial_blocks=[(0, 256, 0, 256)])
 
 
 def test_zero_rows_and_groups():
