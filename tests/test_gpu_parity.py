@@ -122,6 +122,21 @@ def test_ragged_and_small_shapes(M, K, N, r):
     check_layer(spec, partial_blocks=[(0, M, 0, N), (M - 1, 1, N - 1, 1)])
 
 
+@pytest.mark.parametrize("M,K,r", [
+    (4773, 1152, 64),   # 150 token blocks, ragged last block, rank 64
+    (4773, 1152, 0),    # the same without a branch
+    (4800, 4608, 32),   # long K
+    (9472, 512, 16),    # 296 token blocks of a single stage each
+])
+def test_more_token_blocks_than_sms(M, K, r):
+    """More 32-token blocks than SMs (more than one wave of the activation
+    pass), the ragged last block included.  Every row's codes, scales and Z
+    are compared."""
+    spec = synth.layer_spec(f"p{M}_{K}_{r}", M, K, 128, r, 300 + M + K + r, tiny=True)
+    rows = np.sort(np.random.default_rng(M + K + r).choice(M, 192, replace=False))
+    check_layer(spec, rows_sample=rows, partial_blocks=[(M - 128, 128, 0, 128)])
+
+
 def test_ragged_output_stride():
     spec = synth.layer_spec("ldy", 96, 256, 196, 16, 7, tiny=True)
     check_layer(spec, ldy=200)
