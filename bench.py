@@ -492,6 +492,38 @@ def _time_e2e(S, w, Xh, Yh, Xd, bufs, epi, steps, workspace=None):
     return t0.elapsed_time(t1)   # ms
 
 
+def _time_e2e_host(S, w, Xh, Yh, epi, steps):
+    """Public API end to end through the C-ABI call with host buffers
+    (svdq_linear_host), as a serving loop: every step is one call that
+    copies its X from pinned host memory, runs both kernels and copies its Y
+    back to pinned host memory.  Steps rotate over len(Yh) streams, each with
+    its own device workspace and host Y, so one step's copies overlap the
+    other steps' copies and kernels; all copies of all steps lie inside the
+    timed region."""
+    import torch
+    M = Xh[0].shape[0]
+    n = len(Yh)
+    streams = [torch.cuda.Stream() for _ in range(n)]
+    wsp = [torch.empty(S.svdq_linear_host_workspace(w, M), dtype=torch.uint8, device="cuda")
+           for _ in range(n)]
+    cur = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    done = [torch.cuda.Event() for _ in range(n)]
+    torch.cuda.synchronize()
+    t0.record(cur)
+    for st in streams:
+        st.wait_event(t0)
+    for k in range(steps):
+        i = k % n
+        S.svdq_linear_host(w, Xh[k % len(Xh)], Yh[i], wsp[i], epi, streams[i])
+    for i in range(n):
+        done[i].record(streams[i])
+        cur.wait_event(done[i])
+    t1.record(cur)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1)   # ms
+
+
 def _act_bytes(M, K, r):
     """Algorithmic HBM bytes of one svdq_quantize_act launch: read X (bf16),
     write codes (K/2 per token), scales (4 per token-group) and Z (bf16),
@@ -583,8 +615,17 @@ def run_ours(args, spec):
     # same kernels without the low-rank branch (overhead), and end to end
     _time_steps(step0, 3, flush, stream)
     t_act0, t_lin0 = _time_steps(step0, args.steps, flush, stream)
-    _time_e2e(S, w, Xh, Yh, Xd, e2e_bufs, S.EPI_NONE, max(args.warmup, 3), wsb)
-    t_e2e = _time_e2e(S, w, Xh, Yh, Xd, e2e_bufs, S.EPI_NONE, args.steps, wsb)
+    if wsb is None:
+        # the C-ABI call with host buffers; three streams
+        e2e_api = "svdq_linear_host"
+        Yh3 = Yh + [torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)]
+        _time_e2e_host(S, w, Xh, Yh3, S.EPI_NONE, max(args.warmup, 3))
+        t_e2e = _time_e2e_host(S, w, Xh, Yh3, S.EPI_NONE, args.steps)
+    else:
+        # split-K product: device calls with the copies on their own streams
+        e2e_api = "svdq_quantize_act + svdq_linear_splitk, torch copies"
+        _time_e2e(S, w, Xh, Yh, Xd, e2e_bufs, S.EPI_NONE, max(args.warmup, 3), wsb)
+        t_e2e = _time_e2e(S, w, Xh, Yh, Xd, e2e_bufs, S.EPI_NONE, args.steps, wsb)
     S.svdq_get_device_error(w0)
 
     tt = max_over_ranks([t_act + t_lin, t_lin, t_act, t_e2e], dist, "cuda")
@@ -612,7 +653,8 @@ def run_ours(args, spec):
         "lowrank_overhead": {"linear": t_lin_ms / (t_lin0 / args.steps) - 1.0,
                              "layer": t_step_ms / ((t_act0 + t_lin0) / args.steps) - 1.0},
         "e2e": {"value": job_tops(ops, ws, t_e2e_ms * 1e-3), "unit": "TOPS",
-                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+                "api": e2e_api},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
         "product": "svdq_linear_splitk (automatic split)" if splitk else "svdq_linear",

@@ -219,6 +219,31 @@ svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq,
                         int ldy, int epilogue, cudaStream_t stream);
 
 /*
+ * The whole layer with its input and output in host memory (review section
+ * 6.1: the two fused kernels of the layer, here between a host-to-device
+ * copy of X and a device-to-host copy of Y).  Enqueues on `stream`, in
+ * order: the copy of X (host bf16 [M][ldx], ldx >= K) to the workspace,
+ * svdq_quantize_act, svdq_linear with `epilogue`, and the copy of Y to host
+ * bf16 [M][ldy], ldy >= N.  Returns once everything is enqueued; Y is valid
+ * after the stream has been synchronised.  Pinned host memory
+ * (cudaHostAlloc) lets the copies overlap other streams; pageable memory is
+ * accepted, and its copies then block the host.
+ * workspace: device memory, 16-byte aligned, at least
+ *         svdq_linear_host_workspace(w, M) bytes, owned by the caller; it
+ *         holds X, the codes, the scales, Z and Y on the device.  Calls
+ *         sharing a workspace must not overlap (same stream, or ordered by
+ *         events).
+ * Errors: as svdq_quantize_act and svdq_linear (nothing more is enqueued
+ * after the first failing step); SVDQ_ERR_INVALID_ARG for a null pointer,
+ * SVDQ_ERR_SHAPE for ldx < K, ldy < N or a workspace that is too small,
+ * SVDQ_ERR_CUDA if a copy cannot be enqueued.  M == 0 is a no-op.
+ */
+size_t svdq_linear_host_workspace(const svdq_weights* w, int M);
+svdq_status svdq_linear_host(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                             uint16_t* Y, int ldy, int epilogue, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Split-K form of svdq_linear for batches too small to fill the GPU with
  * output tiles (review section 9: PixArt-Sigma layers at a few hundred
  * tokens).  The K groups of every 128-row output tile are divided into

@@ -137,6 +137,36 @@ def test_more_token_blocks_than_sms(M, K, r):
     check_layer(spec, rows_sample=rows, partial_blocks=[(M - 128, 128, 0, 128)])
 
 
+def test_layer_from_host_buffers():
+    """svdq_linear_host: X read from host memory (pinned and pageable, row
+    stride above K), Y written to host memory (row stride above N, the
+    padding untouched); the same bits as the device calls on the same X."""
+    spec = synth.layer_spec("hostbuf", 333, 1152, 136, 32, 77, tiny=True)
+    L = synth.make_layer(spec)
+    a = S.svdq_calib_absmax(L.X)
+    w = S.svdq_pack_weights(L.W, a, spec.rank, bias_bits=L.b)
+    M, K, N = spec.M, spec.K, spec.N
+    X = to_dev(L.X)
+    for epi in (S.EPI_NONE, S.EPI_GELU):
+        Yref = S.SVDQLinear(w, epi).forward(X).cpu()
+        for pinned in (True, False):
+            Xh = torch.zeros((M, K + 64), dtype=torch.bfloat16, pin_memory=pinned)
+            Xh[:, :K] = X.cpu()
+            Yh = torch.full((M, N + 8), float("nan"), dtype=torch.bfloat16, pin_memory=pinned)
+            ws = torch.empty(S.svdq_linear_host_workspace(w, M), dtype=torch.uint8, device="cuda")
+            S.svdq_linear_host(w, Xh[:, :K], Yh[:, :N], ws, epi)
+            torch.cuda.synchronize()
+            S.svdq_get_device_error(w)
+            assert torch.equal(Yh[:, :N], Yref), (epi, pinned)
+            assert torch.isnan(Yh[:, N:].float()).all()
+    # a workspace one byte short is refused before anything is enqueued
+    short = torch.empty(S.svdq_linear_host_workspace(w, M) - 1, dtype=torch.uint8, device="cuda")
+    Yh = torch.empty((M, N), dtype=torch.bfloat16)
+    with pytest.raises(S.SVDQError):
+        S.svdq_linear_host(w, X.cpu(), Yh, short)
+    w.free()
+
+
 def test_ragged_output_stride():
     spec = synth.layer_spec("ldy", 96, 256, 196, 16, 7, tiny=True)
     check_layer(spec, ldy=200)

@@ -34,6 +34,7 @@ __all__ = [
     "FORMAT_W4A4", "FORMAT_W8A8", "FORMAT_NVFP4", "svdq_pack_weights_nvfp4",
     "svdq_quantize_act_nvfp4", "svdq_linear_nvfp4", "svdq_nvfp4_sf_bytes", "NVFP4Linear",
     "svdq_linear_quantize_next", "svdq_linear_quantize_next_workspace", "SVDQMLP",
+    "svdq_linear_host", "svdq_linear_host_workspace",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -111,6 +112,8 @@ def lib() -> ctypes.CDLL:
         "svdq_nvfp4_sf_bytes": (ctypes.c_size_t, [_i, _i]),
         "svdq_quantize_act_nvfp4": (_i, [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
         "svdq_linear_nvfp4": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp]),
+        "svdq_linear_host_workspace": (ctypes.c_size_t, [_vp, _i]),
+        "svdq_linear_host": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _vp, ctypes.c_size_t, _vp]),
         "svdq_linear_quantize_next_workspace": (ctypes.c_size_t, [_vp, _vp, _i]),
         "svdq_linear_quantize_next": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
                                            ctypes.c_size_t, _vp]),
@@ -295,6 +298,25 @@ def svdq_linear(w: Weights, xq, s_x, Z, Y, epilogue=EPI_NONE, stream=None):
     _check(lib().svdq_linear(w.handle, M, _dev_ptr(xq), _dev_ptr(s_x), _dev_ptr(Z),
                              _dev_ptr(Y), Y.stride(0), int(epilogue), _stream_ptr(stream)),
            "svdq_linear")
+
+
+def svdq_linear_host_workspace(w: Weights, M: int) -> int:
+    """Device workspace bytes of svdq_linear_host (0 for invalid arguments)."""
+    return int(lib().svdq_linear_host_workspace(w.handle, int(M)))
+
+
+def svdq_linear_host(w: Weights, X, Y, workspace, epilogue=EPI_NONE, stream=None):
+    """The layer from host memory: X CPU bf16 [M, K] (row stride X.stride(0)),
+    Y CPU bf16 [M, N] (row stride Y.stride(0)), both ideally pinned;
+    workspace: cuda tensor of at least svdq_linear_host_workspace(w, M)
+    bytes.  Enqueues the copies and both kernels on the stream; Y is valid
+    after it has been synchronised."""
+    M = X.shape[0]
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().svdq_linear_host(w.handle, M, _vp(X.data_ptr()), X.stride(0), _vp(Y.data_ptr()),
+                                  Y.stride(0), int(epilogue), _dev_ptr(workspace), nbytes,
+                                  _stream_ptr(stream)),
+           "svdq_linear_host")
 
 
 def svdq_linear_quantize_next_workspace(w: Weights, w_next: Weights, M: int) -> int:

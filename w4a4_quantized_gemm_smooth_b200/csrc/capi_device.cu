@@ -84,6 +84,63 @@ svdq_status svdq_linear(const svdq_weights* w, int M, const uint8_t* xq, const f
   return from_launch(svdq::launch_linear(w, M, xq, s_x, Z, Y, ldy, epilogue, stream));
 }
 
+// Device workspace of svdq_linear_host: X, codes, scales, Z and Y, each
+// starting on a 256-byte boundary; Y rows padded to a multiple of 8.
+struct HostLayerLayout {
+  size_t x, xq, sx, z, y, total;
+  int ldyd;
+};
+static HostLayerLayout host_layer_layout(const svdq_weights* w, int M) {
+  auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
+  const size_t m = (size_t)M, K = (size_t)w->K, N = (size_t)w->N, r = (size_t)w->rank;
+  HostLayerLayout L;
+  L.ldyd = (int)((N + 7) / 8 * 8);
+  L.x = 0;
+  L.xq = L.x + up(m * K * 2);
+  L.sx = L.xq + up(m * K / 2);
+  L.z = L.sx + up((K / 64) * m * 4);
+  L.y = L.z + up(m * r * 2);
+  L.total = L.y + up(m * (size_t)L.ldyd * 2);
+  return L;
+}
+
+size_t svdq_linear_host_workspace(const svdq_weights* w, int M) {
+  if (!w || M <= 0 || !w->d_wq) return 0;
+  return host_layer_layout(w, M).total;
+}
+
+svdq_status svdq_linear_host(const svdq_weights* w, int M, const uint16_t* X, int ldx,
+                             uint16_t* Y, int ldy, int epilogue, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+  svdq_status s = check_handle(w);
+  if (s != SVDQ_OK) return s;
+  if (M < 0 || ldx < w->K || ldy < w->N) return SVDQ_ERR_SHAPE;
+  if (epilogue != SVDQ_EPI_NONE && epilogue != SVDQ_EPI_GELU) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !Y || !workspace) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return SVDQ_ERR_ALIGNMENT;
+  const HostLayerLayout L = host_layer_layout(w, M);
+  if (workspace_bytes < L.total) return SVDQ_ERR_SHAPE;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint16_t* Xd = reinterpret_cast<uint16_t*>(base + L.x);
+  uint8_t* xq = base + L.xq;
+  float* sx = reinterpret_cast<float*>(base + L.sx);
+  uint16_t* Zd = w->rank > 0 ? reinterpret_cast<uint16_t*>(base + L.z) : nullptr;
+  uint16_t* Yd = reinterpret_cast<uint16_t*>(base + L.y);
+  const size_t K = (size_t)w->K, N = (size_t)w->N;
+  if (cudaMemcpy2DAsync(Xd, K * 2, X, (size_t)ldx * 2, K * 2, (size_t)M, cudaMemcpyHostToDevice,
+                        stream) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  s = svdq_quantize_act(w, M, Xd, w->K, xq, sx, Zd, stream);
+  if (s != SVDQ_OK) return s;
+  s = svdq_linear(w, M, xq, sx, Zd, Yd, L.ldyd, epilogue, stream);
+  if (s != SVDQ_OK) return s;
+  if (cudaMemcpy2DAsync(Y, (size_t)ldy * 2, Yd, (size_t)L.ldyd * 2, N * 2, (size_t)M,
+                        cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  return SVDQ_OK;
+}
+
 size_t svdq_linear_quantize_next_workspace(const svdq_weights* w, const svdq_weights* w_next,
                                            int M) {
   if (!w || !w_next || M <= 0 || !w->d_wq || !w_next->d_wq || w_next->K != w->N) return 0;
