@@ -69,6 +69,8 @@ def test_host_only_handle_is_rejected_by_hot_path_calls():
     assert lib.svdq_quantize_act(w.handle, 16, None, 128, None, None, None, None) == 1
     assert lib.svdq_linear(w.handle, 16, None, None, None, None, 64, 0, None) == 1
     assert lib.svdq_debug_partials(w.handle, 16, None, 0, 1, 0, 1, None, None) == 1
+    assert lib.svdq_linear_host(w.handle, 16, None, 128, None, 64, 0, None, 0, None) == 1
+    assert lib.svdq_linear_host_workspace(w.handle, 16) == 0
     w.free()
 
 
