@@ -208,7 +208,8 @@ svdq_status svdq_quantize_act(const svdq_weights* w, int M, const uint16_t* X,
 
 /*
  * Fused W4A4 product (review section 6.1, product side): one kernel computes
- *   P_g = sum_{k in g} q_x q_w       (int32, per group, on the tensor cores)
+ *   P_g = sum_{k in g} q_x q_w       (exact integer per group, formed on the
+ *                                     tensor cores; |P_g| <= 4096)
  *   acc = sum_g s_x[g][m] s_w[g][n] P_g            (fp32)
  *   Y   = bf16(epi(acc + Z L2 + b))                 written once
  * with epi = identity or GELU (exact-erf form in fp32).  Y is device bf16
